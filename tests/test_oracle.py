@@ -1,0 +1,294 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these checks retypes the oracle's own formula: they use closed forms,
+invariants, a hand-derived worked example, finite differences, an independent
+loop restatement, a library special case and the blockwise online-softmax
+recurrence the pages describe.  A final test plants mistakes in the oracle (on
+the CPU) and checks that the pins catch each one.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.attention as oa
+from oracle import (
+    attention_backward,
+    attention_forward,
+    attention_forward_rows,
+    attention_probs,
+    loop_attention_backward,
+    loop_attention_forward,
+    online_softmax_forward,
+)
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
+
+
+def randn(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+# ---------------------------------------------------------------- softmax normalisation
+@pytest.mark.parametrize("causal", [False, True])
+def test_probability_rows_sum_to_one(causal):
+    q, k = randn((2, 3, 37, 16), 1), randn((2, 3, 37, 16), 2)
+    P, _ = attention_probs(q, k, 0.25, causal)
+    np.testing.assert_allclose(P.sum(-1), 1.0, atol=1e-12)
+    assert np.all(P >= 0)
+    if causal:
+        upper = np.triu(np.ones((37, 37), dtype=bool), 1)
+        assert np.all(P[..., upper] == 0.0)
+
+
+# ---------------------------------------------------------------- O formula
+@pytest.mark.parametrize("causal", [False, True])
+def test_uniform_values_return_that_value(causal):
+    q, k = randn((1, 2, 29, 8), 3), randn((1, 2, 29, 8), 4)
+    row = randn((8,), 5)
+    v = np.broadcast_to(row, (1, 2, 29, 8)).copy()
+    O, _ = attention_forward(q, k, v, 1 / math.sqrt(8), causal)
+    np.testing.assert_allclose(O, v, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_single_dominant_logit_returns_its_value_row(causal):
+    n, d = 24, 6
+    jstar = 0 if causal else 17  # under causal every row must see the dominant key
+    q = np.zeros((n, d))
+    q[:, 0] = 1.0
+    k = 0.01 * randn((n, d), 6)
+    k[:, 0] = 0.0
+    k[jstar, 0] = 50.0
+    v = randn((n, d), 7)
+    O, L = attention_forward(q, k, v, 1.0, causal)
+    np.testing.assert_allclose(O, np.broadcast_to(v[jstar], O.shape), atol=n * math.exp(-49))
+    np.testing.assert_allclose(L, 50.0, atol=n * math.exp(-49))
+
+
+def test_noncausal_output_invariant_under_key_permutation():
+    q, k, v = randn((3, 41, 16), 8), randn((3, 41, 16), 9), randn((3, 41, 16), 10)
+    perm = np.random.default_rng(11).permutation(41)
+    O1, L1 = attention_forward(q, k, v, 0.3, False)
+    O2, L2 = attention_forward(q, k[:, perm], v[:, perm], 0.3, False)
+    np.testing.assert_allclose(O1, O2, atol=1e-12)
+    np.testing.assert_allclose(L1, L2, atol=1e-12)
+
+
+# ---------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("causal", [False, True])
+def test_single_token(causal):
+    q, k, v = randn((1, 5), 12), randn((1, 5), 13), randn((1, 5), 14)
+    O, L = attention_forward(q, k, v, 0.7, causal)
+    np.testing.assert_allclose(O, v, atol=1e-15)
+    np.testing.assert_allclose(L, [0.7 * float(np.dot(q[0], k[0]))], atol=1e-14)
+
+
+def test_causal_first_row_is_first_value():
+    q, k, v = randn((19, 4), 15), randn((19, 4), 16), randn((19, 4), 17)
+    O, L = attention_forward(q, k, v, 0.5, True)
+    np.testing.assert_allclose(O[0], v[0], atol=1e-15)
+    np.testing.assert_allclose(L[0], 0.5 * float(np.dot(q[0], k[0])), atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_queries_average_the_visible_values(causal):
+    n, d = 33, 7
+    q = np.zeros((n, d))
+    k, v = randn((n, d), 18), randn((n, d), 19)
+    O, L = attention_forward(q, k, v, 1.0, causal)
+    if causal:
+        expect = np.cumsum(v, axis=0) / np.arange(1, n + 1)[:, None]
+        lse = np.log(np.arange(1, n + 1))
+    else:
+        expect = np.broadcast_to(v.mean(0), (n, d))
+        lse = np.full(n, math.log(n))
+    np.testing.assert_allclose(O, expect, atol=1e-13)
+    np.testing.assert_allclose(L, lse, atol=1e-13)
+
+
+def test_golden_worked_examples():
+    cases = json.load(open(GOLDEN))["cases"]
+    for c in cases:
+        q, k, v = (np.array(c[n], dtype=np.float64) for n in ("q", "k", "v"))
+        O, L = attention_forward(q, k, v, c["scale"], c["causal"])
+        np.testing.assert_allclose(O, c["o"], atol=1e-14, err_msg=c["name"])
+        np.testing.assert_allclose(L, c["lse"], atol=1e-14, err_msg=c["name"])
+        if "do" in c:
+            do = np.array(c["do"])
+            dq, dk, dv, D = attention_backward(q, k, v, do, c["scale"], c["causal"], return_delta=True)
+            np.testing.assert_allclose(D, c["delta"], atol=1e-14, err_msg=c["name"])
+            np.testing.assert_allclose(dq, c["dq"], atol=1e-14, err_msg=c["name"])
+            np.testing.assert_allclose(dk, c["dk"], atol=1e-14, err_msg=c["name"])
+            np.testing.assert_allclose(dv, c["dv"], atol=1e-14, err_msg=c["name"])
+
+
+# ---------------------------------------------------------------- online recurrence
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("bq,bk", [(1, 1), (5, 3), (16, 16), (7, 40), (64, 13)])
+def test_online_softmax_recurrence_equals_definition(causal, bq, bk):
+    n, d = 37, 12
+    q, k, v = 2 * randn((n, d), 20), 2 * randn((n, d), 21), randn((n, d), 22)
+    O1, L1 = attention_forward(q, k, v, 0.4, causal)
+    O2, L2 = online_softmax_forward(q, k, v, 0.4, causal, bq, bk)
+    np.testing.assert_allclose(O2, O1, atol=1e-12)
+    np.testing.assert_allclose(L2, L1, atol=1e-12)
+
+
+# ---------------------------------------------------------------- loop restatement
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n,d", [(1, 3), (5, 4), (16, 8)])
+def test_loop_restatement_matches_numpy_oracle(causal, n, d):
+    q, k, v, do = (randn((n, d), s) for s in (23, 24, 25, 26))
+    O1, L1 = attention_forward(q, k, v, 0.6, causal)
+    O2, L2 = loop_attention_forward(q, k, v, 0.6, causal)
+    np.testing.assert_allclose(O1, O2, atol=1e-13)
+    np.testing.assert_allclose(L1, L2, atol=1e-13)
+    g1 = attention_backward(q, k, v, do, 0.6, causal)
+    g2 = loop_attention_backward(q, k, v, do, 0.6, causal)
+    for a, b in zip(g1, g2):
+        np.testing.assert_allclose(a, b, atol=1e-12)
+
+
+def test_row_sampler_matches_full_forward():
+    q, k, v = randn((50, 8), 27), randn((50, 8), 28), randn((50, 8), 29)
+    rows = [0, 1, 17, 48, 49]
+    for causal in (False, True):
+        O, L = attention_forward(q, k, v, 0.35, causal)
+        Or, Lr = attention_forward_rows(q, k, v, 0.35, causal, rows)
+        np.testing.assert_allclose(Or, O[rows], atol=1e-14)
+        np.testing.assert_allclose(Lr, L[rows], atol=1e-14)
+
+
+# ---------------------------------------------------------------- backward
+def _loss(q, k, v, do, scale, causal):
+    O, _ = attention_forward(q, k, v, scale, causal)
+    return float(np.sum(O * do))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n,d", [(1, 2), (5, 3), (8, 4)])
+def test_backward_matches_central_finite_differences(causal, n, d):
+    q, k, v, do = (randn((n, d), s) for s in (30, 31, 32, 33))
+    scale = 0.8
+    grads = attention_backward(q, k, v, do, scale, causal)
+    h = 1e-6
+    for which, g in zip(range(3), grads):
+        args = [q, k, v]
+        num = np.zeros_like(args[which])
+        for idx in np.ndindex(args[which].shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            num[idx] = (_loss(*plus, do, scale, causal) - _loss(*minus, do, scale, causal)) / (2 * h)
+        err = np.max(np.abs(num - g)) / max(1.0, np.max(np.abs(g)))
+        assert err <= 1e-6, (which, err)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_invariants(causal):
+    q, k, v, do = (randn((2, 45, 10), s) for s in (34, 35, 36, 37))
+    dq, dk, dv, D = attention_backward(q, k, v, do, 0.3, causal, return_delta=True)
+    # sum_j dV_j = sum_i dO_i  (rows of P sum to one)
+    np.testing.assert_allclose(dv.sum(-2), do.sum(-2), atol=1e-11)
+    # sum_j dK_j = 0  (rows of dS sum to zero)
+    np.testing.assert_allclose(dk.sum(-2), 0.0, atol=1e-11)
+    # D_i = sum_j P_ij dP_ij equals rowsum(dO * O)
+    O, _ = attention_forward(q, k, v, 0.3, causal)
+    np.testing.assert_allclose(D, np.sum(do * O, axis=-1), atol=1e-12)
+
+
+# ---------------------------------------------------------------- library special case
+@pytest.mark.parametrize("causal", [False, True])
+def test_agrees_with_torch_sdpa_math_path_fp64(causal):
+    torch = pytest.importorskip("torch")
+    import torch.nn.functional as F
+
+    q, k, v, do = (randn((2, 3, 31, 16), s) for s in (38, 39, 40, 41))
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    out = F.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=0.25)
+    out.backward(torch.tensor(do))
+    O, _ = attention_forward(q, k, v, 0.25, causal)
+    np.testing.assert_allclose(O, out.detach().numpy(), atol=1e-10)
+    dq, dk, dv = attention_backward(q, k, v, do, 0.25, causal)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-10)
+
+
+# ---------------------------------------------------------------- planted mistakes
+def _pins_pass() -> bool:
+    """A compact run of the pins above; False as soon as one fails."""
+    checks = [
+        test_golden_worked_examples,
+        lambda: test_causal_first_row_is_first_value(),
+        lambda: test_zero_queries_average_the_visible_values(True),
+        lambda: test_zero_queries_average_the_visible_values(False),
+        lambda: test_single_token(False),
+        lambda: test_online_softmax_recurrence_equals_definition(True, 5, 3),
+        lambda: test_probability_rows_sum_to_one(True),
+    ]
+    for c in checks:
+        try:
+            with np.errstate(all="ignore"):
+                c()
+        except AssertionError:
+            return False
+    return True
+
+
+def _bad_scores_no_scale(q2, k2, scale, causal):
+    return _orig_scores(q2, k2, 1.0, causal)
+
+
+def _bad_scores_strict_mask(q2, k2, scale, causal):
+    s = scale * (q2 @ k2.T)
+    if causal:
+        i = np.arange(s.shape[0])[:, None]
+        j = np.arange(s.shape[1])[None, :]
+        s = np.where(j >= i, -np.inf, s)  # hides the diagonal too
+    return s
+
+
+def _bad_scores_mask_transposed(q2, k2, scale, causal):
+    s = scale * (q2 @ k2.T)
+    if causal:
+        i = np.arange(s.shape[0])[:, None]
+        j = np.arange(s.shape[1])[None, :]
+        s = np.where(j < i, -np.inf, s)
+    return s
+
+
+def _bad_scores_transposed_operands(q2, k2, scale, causal):
+    return _orig_scores(k2, q2, scale, causal)
+
+
+def _bad_lse_log2(s):
+    m = np.max(s, axis=-1, keepdims=True)
+    return (m + np.log2(np.sum(np.exp(s - m), axis=-1, keepdims=True)))[..., 0]
+
+
+def _bad_lse_max_only(s):
+    return np.max(s, axis=-1)
+
+
+_orig_scores = oa._scores
+
+
+@pytest.mark.parametrize("name,attr,bad", [
+    ("dropped scale", "_scores", _bad_scores_no_scale),
+    ("diagonal masked", "_scores", _bad_scores_strict_mask),
+    ("mask transposed", "_scores", _bad_scores_mask_transposed),
+    ("Q and K swapped", "_scores", _bad_scores_transposed_operands),
+    ("log2 in LSE", "_lse_rows", _bad_lse_log2),
+    ("LSE without the sum", "_lse_rows", _bad_lse_max_only),
+])
+def test_pins_catch_planted_mistakes(monkeypatch, name, attr, bad):
+    assert _pins_pass(), "pins must pass on the unmodified oracle"
+    monkeypatch.setattr(oa, attr, bad)
+    assert not _pins_pass(), f"planted mistake not caught: {name}"
