@@ -1,0 +1,374 @@
+"""Benchmark: exact attention forward + backward on one B200 per process.
+
+A step is one pass of the whole hot path -- forward (fa_fwd) then backward
+(fa_bwd: preprocess, dK/dV kernel, dQ kernel) -- over the causal workload
+B=2, H=32, N=8192, d=128 (bf16 inputs, 1% of the keys of every head scaled by 8).
+The metric is TFLOPS with 4*B*H*N^2*d forward flops (halved under the causal
+mask) and 2.5x that for the backward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent
+replica of the workload on its own GPU (the method has no exchange step between
+GPUs); the value is the total work of all ranks over the slowest rank's time.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from exact_io_aware_91_b200 import inputs  # noqa: E402
+
+METRIC = "attention fwd/bwd TFLOPS (BF16, causal, N=8k, d=128) & % of B200 tensor peak"
+WORKLOAD = 3
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"bf16_tflops": d["bf16_tflops"], "bf16_tflops_sustained": d["bf16_tflops_sustained"],
+                "hbm_gbs": d["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- dist plumbing
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local) if backend == "nccl" else None)
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_teardown(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        try:
+            props = torch.cuda.get_device_properties(device)
+            self.gpu_id = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        except Exception:
+            self.gpu_id = str(device)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.05)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle baseline
+def oracle_head_step(inp_cpu: dict, w: inputs.Workload, b: int, h: int) -> None:
+    import oracle
+
+    q, k, v, do = (inp_cpu[n][b, h] for n in ("q", "k", "v", "do"))
+    oracle.attention_forward(q, k, v, w.scale, w.causal)
+    oracle.attention_backward(q, k, v, do, w.scale, w.causal)
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+
+        info = threadpoolctl.threadpool_info()
+        return int(max(i.get("num_threads", 1) for i in info)) if info else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(w: inputs.Workload, inp_cpu: dict, budget_s: float = 12.0) -> dict:
+    """The oracle, as it stands, on whole heads of the workload until ~budget_s of CPU work."""
+    per_head = (w.fwd_flops + w.bwd_flops) / (w.B * w.H)
+    heads, t0 = 0, time.perf_counter()
+    while True:
+        oracle_head_step(inp_cpu, w, heads // w.H % w.B, heads % w.H)
+        heads += 1
+        if time.perf_counter() - t0 > budget_s or heads >= w.B * w.H:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": per_head * heads / dt / 1e12, "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{heads} of {w.B * w.H} heads (fwd+bwd, fp64 numpy, S and P materialised), {dt:.1f} s"}
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    """--impl reference: the fp64 oracle timed on the host cores, one head per step."""
+    if rank != 0:
+        return
+    w = inputs.workload(WORKLOAD)
+    inp = inputs.make_inputs(w, device="cpu")
+    per_head = (w.fwd_flops + w.bwd_flops) / (w.B * w.H)
+    for i in range(args.warmup):
+        oracle_head_step(inp, w, 0, i % w.H)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_head_step(inp, w, (i // w.H) % w.B, i % w.H)
+    dt = time.perf_counter() - t0
+    value = per_head * args.steps / dt / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "step": "one (b, h) head of the workload, forward + backward"},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                         "sample": f"one head per step, {args.steps} steps"},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank: int, world: int, local: int) -> None:
+    from exact_io_aware_91_b200 import api
+
+    w = inputs.workload(WORKLOAD)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp_cpu = inputs.make_inputs(w, device="cpu")
+    q, k, v, do = (inp_cpu[n].to(dev) for n in ("q", "k", "v", "do"))
+    B, H, N, d = w.B, w.H, w.N, w.d
+    o = torch.empty_like(q)
+    res = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq = torch.empty((B, H, N, d), dtype=torch.float32, device=dev)
+    dk = torch.empty_like(dq)
+    dv = torch.empty_like(dq)
+    ws = torch.empty(api.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        api.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, o=o, lse=lse, o_resid=res)
+        api.fa_bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws, dq=dq, dk=dk, dv=dv,
+                   o_resid=res)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if api.fa_device_status() != api.FA_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    # ---- timed region: K steps, per-kernel events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(args.steps):
+        e = ev[s]
+        e[0].record(stream)
+        api.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, o=o, lse=lse, o_resid=res)
+        e[1].record(stream)
+        api.fa_bwd_set_phase_events((e[2], e[3]))
+        api.fa_bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws, dq=dq, dk=dk, dv=dv,
+                   o_resid=res)
+        api.fa_bwd_set_phase_events(None)
+        e[4].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(end)
+    total_ms_max = max_over_ranks(total_ms, world)
+    if api.fa_device_status() != api.FA_OK:
+        raise RuntimeError("device status not OK after the timed region")
+
+    phase = {"fwd": [], "bwd_pre": [], "bwd_dkdv": [], "bwd_dq": []}
+    for e in ev:
+        phase["fwd"].append(e[0].elapsed_time(e[1]))
+        phase["bwd_pre"].append(e[1].elapsed_time(e[2]))
+        phase["bwd_dkdv"].append(e[2].elapsed_time(e[3]))
+        phase["bwd_dq"].append(e[3].elapsed_time(e[4]))
+    mean = {kk: statistics.mean(vv) for kk, vv in phase.items()}
+
+    flops_step = w.fwd_flops + w.bwd_flops
+    ms_step = total_ms_max / args.steps
+    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    peaks = load_peaks()
+
+    # dominant kernel (largest mean time) and its algorithmic flops per launch
+    algo = {"fwd": w.fwd_flops,                  # QK^T and PV
+            "bwd_dkdv": 2.0 * w.fwd_flops,        # K Q^T, V dO^T, P^T dO, dS^T Q
+            "bwd_dq": 1.5 * w.fwd_flops}          # Q K^T, dO V^T, dS K
+    dom = max(("fwd", "bwd_dkdv", "bwd_dq"), key=lambda kk: mean[kk])
+    achieved = algo[dom] / (mean[dom] * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": args.traffic,
+                "peak_kind": f"{peaks['source']} bf16 dense matmul, sustained (kernel timed inside a long step)"}
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        h_in = {n: inp_cpu[n].pin_memory() for n in ("q", "k", "v", "do")}
+        h_out = {"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
+                 "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory(),
+                 "dq": torch.empty(dq.shape, dtype=dq.dtype).pin_memory(),
+                 "dk": torch.empty(dk.shape, dtype=dk.dtype).pin_memory(),
+                 "dv": torch.empty(dv.shape, dtype=dv.dtype).pin_memory()}
+        n_e2e = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            q.copy_(h_in["q"], non_blocking=True)
+            k.copy_(h_in["k"], non_blocking=True)
+            v.copy_(h_in["v"], non_blocking=True)
+            do.copy_(h_in["do"], non_blocking=True)
+            step()
+            for name, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+                h_out[name].copy_(t, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, world)
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+        e2e = {"value": flops_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, inp_cpu)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+                       "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (Q, K, V, dO, O 134 MB each > 126 MB)"},
+            "fwd_tflops": w.fwd_flops / (mean["fwd"] * 1e-3) / 1e12,
+            "bwd_tflops": w.bwd_flops / ((mean["bwd_pre"] + mean["bwd_dkdv"] + mean["bwd_dq"]) * 1e-3) / 1e12,
+            "kernel_ms": mean,
+            "frac_of_peak": {"measured_burst": value / world / peaks["bf16_tflops"],
+                             "measured_sustained": value / world / peaks["bf16_tflops_sustained"],
+                             "datasheet_2250": value / world / 2250.0},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch of the dominant kernel from an ncu capture (reported as-is)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        dist_teardown(world)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,193 @@
+"""Python binding of the C ABI in ``include/fa.h`` (argument marshalling only).
+
+Every function here has the name of the C entry point it calls.  PyTorch provides
+device memory and the current CUDA stream; all arithmetic happens in the CUDA
+kernels of ``libfa_b200.so``.  There is no fallback: if the library is missing
+or the device is not supported, the call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+from . import build as _build
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_MISALIGNED = 3
+FA_ERR_CUDA = 4
+FA_ERR_TIMEOUT = 5
+
+EXPORTS = ("fa_fwd", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_device_status",
+           "fa_bwd_set_phase_events", "fa_status_str")
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {status_str(status)} ({status})")
+        self.status = status
+
+
+_LIB = None
+
+
+def library() -> ctypes.CDLL:
+    """Load ``libfa_b200.so`` from the package directory (raises if it is not built)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = _build.LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m exact_io_aware_91_b200.build` "
+            "(there is no non-CUDA fallback)"
+        )
+    lib = ctypes.CDLL(path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_fwd.restype = i
+    lib.fa_fwd_f32.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_fwd_f32.restype = i
+    lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_bwd_workspace_size.restype = sz
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_bwd.restype = i
+    lib.fa_device_status.argtypes = [vp]
+    lib.fa_device_status.restype = i
+    lib.fa_bwd_set_phase_events.argtypes = [vp]
+    lib.fa_bwd_set_phase_events.restype = None
+    lib.fa_status_str.argtypes = [i]
+    lib.fa_status_str.restype = ctypes.c_char_p
+    _LIB = lib
+    return lib
+
+
+def status_str(status: int) -> str:
+    return library().fa_status_str(int(status)).decode()
+
+
+fa_status_str = status_str
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _check(fn: str, status: int) -> None:
+    if status != FA_OK:
+        raise FAError(fn, status)
+
+
+def _shape(q: torch.Tensor) -> tuple[int, int, int, int]:
+    if q.dim() != 4:
+        raise ValueError("expected a (B, H, N, d) tensor")
+    return tuple(int(x) for x in q.shape)  # type: ignore[return-value]
+
+
+def _same(*ts: torch.Tensor, dtype: torch.dtype, shape) -> None:
+    for t in ts:
+        if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"expected contiguous CUDA {dtype} tensors of shape {tuple(shape)}")
+
+
+def _scale(scale, d: int) -> float:
+    return float(1.0 / math.sqrt(d) if scale is None else scale)
+
+
+def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, scale: float | None = None,
+           o: torch.Tensor | None = None, lse: torch.Tensor | None = None, o_resid: torch.Tensor | None = None,
+           save_residual: bool = False, stream=None):
+    """Attention forward on bf16 (B, H, N, d) CUDA tensors.
+
+    Returns (o, lse), or (o, lse, o_resid) when ``save_residual`` (or ``o_resid``) is
+    given: the bf16 residual of O's final rounding, to be passed to ``fa_bwd``.
+    """
+    B, H, N, d = _shape(q)
+    _same(q, k, v, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if o_resid is None and save_residual:
+        o_resid = torch.empty_like(q)
+    _same(o, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if o_resid is not None:
+        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
+    st = library().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          None if o_resid is None else o_resid.data_ptr(), B, H, N, d, _scale(scale, d),
+                          int(bool(causal)), _stream_handle(stream))
+    _check("fa_fwd", st)
+    return (o, lse) if o_resid is None else (o, lse, o_resid)
+
+
+def fa_fwd_f32(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+               scale: float | None = None, stream=None):
+    """fp32 forward (no input rounding). Returns (o, lse)."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, dtype=torch.float32, shape=(B, H, N, d))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    st = library().fa_fwd_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N, d,
+                              _scale(scale, d), int(bool(causal)), _stream_handle(stream))
+    _check("fa_fwd_f32", st)
+    return o, lse
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(library().fa_bwd_workspace_size(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,
+           dq=None, dk=None, dv=None, o_resid=None, stream=None):
+    """dQ, dK, dV (fp32) of sum(O * dO). ``o_resid``: the forward's residual (recommended).
+
+    Returns (dq, dk, dv)."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, o, do, dtype=torch.bfloat16, shape=(B, H, N, d))
+    _same(lse, dtype=torch.float32, shape=(B, H, N))
+    if o_resid is not None:
+        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if dq is None:
+        dq = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    if dk is None:
+        dk = torch.empty_like(dq)
+    if dv is None:
+        dv = torch.empty_like(dq)
+    ws_bytes = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    st = library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                          None if o_resid is None else o_resid.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, _scale(scale, d),
+                          int(bool(causal)), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    _check("fa_bwd", st)
+    return dq, dk, dv
+
+
+def fa_device_status(stream=None) -> int:
+    """Synchronise and return the device status code (FA_OK, FA_ERR_TIMEOUT or FA_ERR_CUDA)."""
+    return int(library().fa_device_status(_stream_handle(stream)))
+
+
+_PHASE_EVENTS = None  # keeps the ctypes array alive while the hook is set
+
+
+def fa_bwd_set_phase_events(events=None) -> None:
+    """Profiling hook: record ``events[0]`` after the preprocess and ``events[1]`` after the
+    dK/dV kernel in every later ``fa_bwd`` of this thread (``torch.cuda.Event`` objects);
+    ``None`` turns it off."""
+    global _PHASE_EVENTS
+    if events is None:
+        _PHASE_EVENTS = None
+        library().fa_bwd_set_phase_events(None)
+        return
+    arr = (ctypes.c_void_p * 2)(events[0].cuda_event, events[1].cuda_event)
+    _PHASE_EVENTS = arr
+    library().fa_bwd_set_phase_events(ctypes.cast(arr, ctypes.c_void_p))

@@ -1,0 +1,290 @@
+// Host side of the C ABI declared in include/fa.h: argument checks, tensor-map
+// encoding, workspace carving and kernel launches.  No allocation happens here.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_internal.h"
+
+namespace fa {
+
+// The library's one piece of device state: an error word per device, written by
+// kernels that give up a bounded wait.
+__device__ int g_fa_err_word;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices];
+int g_cc_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 unsupported
+std::mutex g_mu;
+thread_local void* const* t_phase_events = nullptr;  // see fa_bwd_set_phase_events
+
+// Checks the current device (compute capability 10.0) and resolves its error word.
+fa_status device_setup(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_cc_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    g_cc_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  if (g_cc_ok[dev] < 0) return FA_ERR_UNSUPPORTED;
+  if (g_err_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_fa_err_word) != cudaSuccess) return FA_ERR_CUDA;
+    g_err_ptr[dev] = static_cast<int*>(ptr);
+  }
+  *dev_out = dev;
+  return FA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Shared validation of sizes/scalars.  Returns FA_OK and sets *empty when there is nothing to do.
+fa_status check_problem(int B, int H, int N, int d, float scale, int causal, bool* empty) {
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  *empty = (B == 0 || H == 0 || N == 0);
+  if (*empty) return FA_OK;
+  const long long BH = (long long)B * H;
+  // grid.x = work units <= 2^31-1; every TMA coordinate fits in int32; N padded to 128 fits in int
+  if (BH > (1LL << 24) || N > (1 << 30)) return FA_ERR_UNSUPPORTED;
+  const long long units = BH * ((N + 127) / 128);
+  if (units > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct BwdLayout {
+  size_t off_q16, off_k16, off_v16, off_do16, off_delta, off_lse2, total;
+  int Np;
+};
+
+BwdLayout bwd_layout(int B, int H, int N, int d) {
+  BwdLayout w{};
+  const size_t elems = (size_t)B * H * N * d;
+  const size_t t16 = align256(elems * 2);
+  w.Np = ((N + 127) / 128) * 128;
+  const size_t rows = align256((size_t)B * H * w.Np * 4);
+  w.off_q16 = 0;
+  w.off_k16 = t16;
+  w.off_v16 = 2 * t16;
+  w.off_do16 = 3 * t16;
+  w.off_delta = 4 * t16;
+  w.off_lse2 = 4 * t16 + rows;
+  w.total = 4 * t16 + 2 * rows;
+  return w;
+}
+
+}  // namespace
+
+int* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  return g_err_ptr[dev];
+}
+
+bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
+                  int box_cols, int box_rows, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * elem_bytes, (cuuint64_t)N * d * elem_bytes};
+  const cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_str(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
+                 int N, int d, float scale, int causal, fa_stream_t stream) {
+  bool empty = false;
+  fa_status st = check_problem(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(o_resid, 16))
+    return FA_ERR_MISALIGNED;
+  int dev = 0;
+  if ((st = device_setup(&dev)) != FA_OK) return st;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv, to;
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_tmap_3d(&tq, q, bf, 2, d, N, BH, 64, 128, true) || !make_tmap_3d(&tk, k, bf, 2, d, N, BH, 64, 128, true) ||
+      !make_tmap_3d(&tv, v, bf, 2, d, N, BH, 64, 128, true) || !make_tmap_3d(&to, o, bf, 2, d, N, BH, 64, 128, true))
+    return FA_ERR_CUDA;
+  FwdParams p{};
+  p.lse = lse;
+  p.o_resid = static_cast<__nv_bfloat16*>(o_resid);
+  p.N = N;
+  p.BH = BH;
+  p.n_pairs = (N + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.err = g_err_ptr[dev];
+  return launch_fwd_sm100(tq, tk, tv, to, p, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N,
+                     int d, float scale, int causal, fa_stream_t stream) {
+  bool empty = false;
+  fa_status st = check_problem(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(o, 4) || !aligned(lse, 4))
+    return FA_ERR_MISALIGNED;
+  int dev = 0;
+  if ((st = device_setup(&dev)) != FA_OK) return st;
+  return launch_fwd_f32(q, k, v, o, lse, B * H, N, d, scale, causal, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  bool empty = false;
+  if (check_problem(B, H, N, d, 1.0f, 0, &empty) != FA_OK || empty) return 0;
+  return bwd_layout(B, H, N, d).total;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* o_resid, const void* dout,
+                 const float* lse, float* dq, float* dk, float* dv, int B, int H, int N, int d, float scale,
+                 int causal, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  bool empty = false;
+  fa_status st = check_problem(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  const BwdLayout w = bwd_layout(B, H, N, d);
+  if (workspace_bytes < w.total) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(o_resid, 16) || !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(workspace, 256))
+    return FA_ERR_MISALIGNED;
+  int dev = 0;
+  if ((st = device_setup(&dev)) != FA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  BwdPreParams pp{};
+  pp.q = q;
+  pp.k = k;
+  pp.v = v;
+  pp.o = o;
+  pp.o_resid = o_resid;
+  pp.dout = dout;
+  pp.lse = lse;
+  pp.q16 = ws + w.off_q16;
+  pp.k16 = ws + w.off_k16;
+  pp.v16 = ws + w.off_v16;
+  pp.do16 = ws + w.off_do16;
+  pp.delta = reinterpret_cast<float*>(ws + w.off_delta);
+  pp.lse2 = reinterpret_cast<float*>(ws + w.off_lse2);
+  pp.N = N;
+  pp.Np = w.Np;
+  pp.BH = BH;
+  pp.d = d;
+  if (launch_bwd_pre(pp, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (t_phase_events != nullptr &&
+      cudaEventRecord(static_cast<cudaEvent_t>(t_phase_events[0]), s) != cudaSuccess)
+    return FA_ERR_CUDA;
+
+  const CUtensorMapDataType h = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap a_q, a_do, a_k, a_v;  // dK/dV kernel: 64-row Q/dO tiles, 128-row K/V tiles
+  CUtensorMap b_q, b_do, b_k, b_v;  // dQ kernel: 128-row Q/dO tiles, 64-row K/V tiles
+  if (!make_tmap_3d(&a_q, pp.q16, h, 2, d, N, BH, 64, 64, true) ||
+      !make_tmap_3d(&a_do, pp.do16, h, 2, d, N, BH, 64, 64, true) ||
+      !make_tmap_3d(&a_k, pp.k16, h, 2, d, N, BH, 64, 128, true) ||
+      !make_tmap_3d(&a_v, pp.v16, h, 2, d, N, BH, 64, 128, true) ||
+      !make_tmap_3d(&b_q, pp.q16, h, 2, d, N, BH, 64, 128, true) ||
+      !make_tmap_3d(&b_do, pp.do16, h, 2, d, N, BH, 64, 128, true) ||
+      !make_tmap_3d(&b_k, pp.k16, h, 2, d, N, BH, 64, 64, true) ||
+      !make_tmap_3d(&b_v, pp.v16, h, 2, d, N, BH, 64, 64, true))
+    return FA_ERR_CUDA;
+  BwdParams bp{};
+  bp.delta = pp.delta;
+  bp.lse2 = pp.lse2;
+  bp.dq = dq;
+  bp.dk = dk;
+  bp.dv = dv;
+  bp.N = N;
+  bp.Np = w.Np;
+  bp.BH = BH;
+  bp.scale = scale;
+  bp.scale_log2 = scale * 1.4426950408889634f;
+  bp.causal = causal;
+  bp.err = g_err_ptr[dev];
+  if (launch_bwd_dkdv_sm100(a_q, a_do, a_k, a_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (t_phase_events != nullptr &&
+      cudaEventRecord(static_cast<cudaEvent_t>(t_phase_events[1]), s) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (launch_bwd_dq_sm100(b_q, b_do, b_k, b_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+void fa_bwd_set_phase_events(void* const* events) { t_phase_events = events; }
+
+fa_status fa_device_status(fa_stream_t stream) {
+  int dev = 0;
+  fa_status st = device_setup(&dev);
+  if (st != FA_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fa_err_word, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_fa_err_word, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

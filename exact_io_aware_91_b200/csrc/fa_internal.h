@@ -1,0 +1,69 @@
+// Internal launch interface shared by the C-ABI host code and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace fa {
+
+struct FwdParams {
+  float* lse;        // (B*H, N) fp32, natural-log LSE of the scaled scores; may be null
+  __nv_bfloat16* o_resid;  // (B*H, N, d) bf16 residual O_fp32 - O_bf16; may be null
+  int N;             // sequence length (queries = keys)
+  int BH;            // B * H
+  int n_pairs;       // ceil(N / 256): work units per head (two 128-row query tiles each)
+  float scale_log2;  // softmax scale * log2(e)
+  int causal;
+  int* err;          // device error word
+};
+
+struct BwdPreParams {
+  const void* q;     // bf16 (BH, N, d)
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* o_resid;  // may be null: D then uses the bf16 O alone
+  const void* dout;
+  const float* lse;  // (BH, N)
+  void* q16;         // fp16 copies (BH, N, d)
+  void* k16;
+  void* v16;
+  void* do16;
+  float* delta;      // (BH, Np): rowsum(dO * O); 0 on padded rows
+  float* lse2;       // (BH, Np): LSE * log2(e); +inf on padded rows
+  int N, Np, BH, d;
+};
+
+struct BwdParams {
+  const float* delta;  // (BH, Np)
+  const float* lse2;   // (BH, Np)
+  float* dq;           // fp32 (BH, N, d)
+  float* dk;
+  float* dv;
+  int N, Np, BH;
+  float scale;         // softmax scale (applied to dQ and dK)
+  float scale_log2;    // scale * log2(e)
+  int causal;
+  int* err;
+};
+
+// Tensor maps are 3-D views (d, N, B*H) of a (B, H, N, d) tensor with the
+// 128-byte swizzle and a box of 64 columns x `box_rows` rows.
+bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
+                  int box_cols, int box_rows, bool swizzle128);
+
+cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t s);
+cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int BH, int N,
+                           int d, float scale, int causal, cudaStream_t s);
+cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t s);
+cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s);
+cudaError_t launch_bwd_dq_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                                const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s);
+
+int* device_error_word();  // address of the library's device error word on the current device
+
+}  // namespace fa

@@ -1,0 +1,418 @@
+// Forward pass of exact attention on sm_100a:
+//   O = softmax(scale * Q K^T + causal mask) V,  LSE = ln sum_j exp(scale * S_ij)
+//
+// The method ("Flash Attention uitgelegd: een uitgebreide gids", sections
+// "Tiling" and "Werkingsmechanisme"; "FlashAttention (EL)", sections "Tiling",
+// "Online computation of Softmax" and "Fusion of operations into one CUDA
+// kernel"): Q, K and V are cut into on-chip tiles, the softmax is applied
+// incrementally with a running row maximum and exp-sum, and the partial output
+// is rescaled as each K/V tile arrives, so the N x N score matrix never reaches
+// HBM.  One fused kernel writes only O (and the per-row LSE kept for the
+// backward pass).
+//
+// B200 design (not a translation of the pages' A100/H100 kernels):
+//   * one CTA = one work unit = two 128-row query tiles of one (b, h); the two
+//     tiles ping-pong on the tensor core so that the softmax of one overlaps the
+//     MMAs of the other ("overlapping GEMM + softmax", page "Flash Attention:
+//     Ako transformery ...", section 3, re-done for tcgen05);
+//   * warp 0 streams K/V tiles with TMA into a multi-stage shared-memory ring;
+//   * warp 1 issues tcgen05.mma: S_t = Q_t K_j^T into tensor memory (TMEM), and
+//     O_t += P_t V_j with P_t read straight from TMEM (it overwrites S_t there);
+//   * warps 2-3 convert each V tile to fp16 in shared memory (exact for bf16
+//     values of normal fp16 range) so that P is rounded to fp16 (11 significant
+//     bits) rather than bf16 (8) before the P V product;
+//   * warpgroups 1 and 2 (one per query tile, one thread per row) run the online
+//     softmax on S rows loaded from TMEM, write P back to TMEM as fp16 and, when
+//     the running maximum grows by more than 2^8, rescale O in TMEM; the row sum
+//     l adds up the fp16-rounded weights actually used in P V, so O = P V / l is
+//     an exact convex combination of the rounded weights;
+//   * the epilogue divides by the row sum, converts to bf16 and TMA-stores O, and
+//     optionally writes the bf16 residual O_fp32 - O_bf16 so that the backward
+//     pass can form rowsum(dO * O) from an fp32-accurate O.
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+template <int D>
+struct FwdLayout {
+  static constexpr int BM = 128;                 // query rows per tile
+  static constexpr int BN = 128;                 // keys per K/V tile
+  static constexpr int KCH = D / 64;             // 128-byte column chunks per row
+  static constexpr int BOX = 128 * 128;          // one 64-column x 128-row bf16 box (16 KB)
+  static constexpr int TILE = KCH * BOX;         // one 128 x D bf16 tile
+  static constexpr int STAGES = (D == 128) ? 4 : 8;
+  static constexpr int OFF_Q0 = 0;
+  static constexpr int OFF_Q1 = TILE;
+  static constexpr int OFF_KV = 2 * TILE;
+  static constexpr int OFF_BAR = OFF_KV + STAGES * TILE;
+  // barriers: q_full, kv_full[STAGES], kv_empty[STAGES], v_conv[STAGES], s_full[2], p_full[2],
+  // o_full[2], mma_done
+  static constexpr int BAR_Q = 0;
+  static constexpr int BAR_KV_FULL = 1;
+  static constexpr int BAR_KV_EMPTY = 1 + STAGES;
+  static constexpr int BAR_V_CONV = 1 + 2 * STAGES;
+  static constexpr int BAR_S_FULL = 1 + 3 * STAGES;
+  static constexpr int BAR_P_FULL = BAR_S_FULL + 2;
+  static constexpr int BAR_O_FULL = BAR_P_FULL + 2;
+  static constexpr int BAR_MMA_DONE = BAR_O_FULL + 2;
+  static constexpr int NBAR = BAR_MMA_DONE + 1;
+  static constexpr int OFF_TMEM_SLOT = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
+  static constexpr int BYTES = OFF_ABORT + 8;
+  static constexpr int SMEM_ALLOC = BYTES + 1024;  // slack to align the base to 1024 bytes
+  static constexpr uint32_t TMEM_COLS = 512;       // S0, S1 (128 each), O0, O1 (D each)
+  static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
+};
+
+constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 2-3 V to fp16, warps 4-7 / 8-11 softmax
+constexpr int kConvThreads = 64;
+static_assert(FwdLayout<128>::STAGES % 2 == 0 && FwdLayout<64>::STAGES % 2 == 0,
+              "K and V tiles must alternate over fixed ring stages");
+
+// Bounded wait used while draining copies on the way out: ignores the abort flag.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+  }
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                        const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + L::OFF_BAR + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_ABORT);
+  const WaitCtx wctx{abort_flag, p.err};
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: heaviest units first under the causal mask
+  const int L_idx = blockIdx.x;
+  const int pair = p.causal ? (p.n_pairs - 1 - L_idx / p.BH) : (L_idx / p.BH);
+  const int bh = L_idx % p.BH;
+  const int q_base0 = pair * 256;
+  const int q_base1 = q_base0 + 128;
+  const int n_kv = (p.N + 127) / 128;
+  const int n0 = p.causal ? min(n_kv, q_base0 / 128 + 1) : n_kv;
+  const int n1 = p.causal ? min(n_kv, q_base1 / 128 + 1) : n_kv;  // n1 >= n0
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(L::BAR_Q), 1);
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(bar(L::BAR_KV_FULL + s), 1);
+      mbar_init(bar(L::BAR_KV_EMPTY + s), 1);
+      mbar_init(bar(L::BAR_V_CONV + s), kConvThreads);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::BAR_S_FULL + t), 1);
+      mbar_init(bar(L::BAR_P_FULL + t), 128);
+      mbar_init(bar(L::BAR_O_FULL + t), 1);
+    }
+    mbar_init(bar(L::BAR_MMA_DONE), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(base + L::OFF_TMEM_SLOT, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_TMEM_SLOT);
+
+  if (warp == 0) {
+    // ===================================================== TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_o);
+      mbar_arrive_expect_tx(bar(L::BAR_Q), 2 * L::TILE);
+      for (int c = 0; c < L::KCH; ++c) {
+        tma_load_3d(base + L::OFF_Q0 + c * L::BOX, &tm_q, c * 64, q_base0, bh, bar(L::BAR_Q));
+        tma_load_3d(base + L::OFF_Q1 + c * L::BOX, &tm_q, c * 64, q_base1, bh, bar(L::BAR_Q));
+      }
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < n1 && ok; ++j) {
+        for (int which = 0; which < 2 && ok; ++which) {
+          const int st = issued % L::STAGES;
+          const uint32_t ph = (issued / L::STAGES) & 1;
+          ok = mbar_wait(bar(L::BAR_KV_EMPTY + st), ph ^ 1u, wctx);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(L::BAR_KV_FULL + st), L::TILE);
+          const CUtensorMap* m = which ? &tm_v : &tm_k;
+          for (int c = 0; c < L::KCH; ++c)
+            tma_load_3d(base + L::OFF_KV + st * L::TILE + c * L::BOX, m, c * 64, j * 128, bh,
+                        bar(L::BAR_KV_FULL + st));
+          ++issued;
+        }
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      drain_wait(bar(L::BAR_Q), 0);
+      const int first = issued > L::STAGES ? issued - L::STAGES : 0;
+      for (int i = first; i < issued; ++i)
+        drain_wait(bar(L::BAR_KV_FULL + (i % L::STAGES)), (i / L::STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    // ===================================================== MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = make_idesc(128, 128, true, false, false);
+      constexpr uint32_t idesc_pv = make_idesc(128, D, false, false, true);  // fp16 P (TMEM) x fp16 V
+      const uint32_t tS[2] = {tmem + L::T_S0, tmem + L::T_S1};
+      const uint32_t tO[2] = {tmem + L::T_O0, tmem + L::T_O1};
+      const uint32_t sQ[2] = {base + L::OFF_Q0, base + L::OFF_Q1};
+
+      auto issue_qk = [&](uint32_t d_tmem, uint32_t q_s, uint32_t k_s) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * L::BOX + (k & 3) * 32;
+          mma_ss(d_tmem, make_sdesc_sw128(q_s + off, 16, 1024), make_sdesc_sw128(k_s + off, 16, 1024), idesc_qk,
+                 k > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_s, bool acc) {
+#pragma unroll
+        for (int k = 0; k < L::BN / 16; ++k) {
+          mma_ts(d_tmem, p_tmem + k * 8, make_sdesc_sw128(v_s + k * 2048, L::BOX, 1024), idesc_pv,
+                 (acc || k > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = mbar_wait(bar(L::BAR_Q), 0, wctx);
+      tc_fence_after();
+      int prev_v_stage = 0;
+      for (int j = 0; j < n1 && ok; ++j) {
+        const int iK = 2 * j, iV = 2 * j + 1;
+        const int stK = iK % L::STAGES, stV = iV % L::STAGES;
+        const uint32_t sK = base + L::OFF_KV + stK * L::TILE;
+        const uint32_t sV = base + L::OFF_KV + stV * L::TILE;
+        if (!(ok = mbar_wait(bar(L::BAR_KV_FULL + stK), (iK / L::STAGES) & 1, wctx))) break;
+        tc_fence_after();
+        if (j < n0) {
+          issue_qk(tS[0], sQ[0], sK);
+          mma_commit(bar(L::BAR_S_FULL + 0));
+        }
+        if (j > 0) {  // O1 += P1 V_{j-1}
+          if (!(ok = mbar_wait(bar(L::BAR_P_FULL + 1), (j - 1) & 1, wctx))) break;
+          tc_fence_after();
+          issue_pv(tO[1], tS[1], base + L::OFF_KV + prev_v_stage * L::TILE, j - 1 > 0);
+          mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage));
+        }
+        issue_qk(tS[1], sQ[1], sK);
+        mma_commit(bar(L::BAR_S_FULL + 1));
+        mma_commit(bar(L::BAR_KV_EMPTY + stK));
+        if (!(ok = mbar_wait(bar(L::BAR_V_CONV + stV), (iV / L::STAGES) & 1, wctx))) break;
+        tc_fence_after();
+        if (j < n0) {  // O0 += P0 V_j
+          if (!(ok = mbar_wait(bar(L::BAR_P_FULL + 0), j & 1, wctx))) break;
+          tc_fence_after();
+          issue_pv(tO[0], tS[0], sV, j > 0);
+          if (j == n0 - 1) mma_commit(bar(L::BAR_O_FULL + 0));
+        }
+        prev_v_stage = stV;
+      }
+      if (ok) {  // O1 += P1 V_{n1-1}
+        ok = mbar_wait(bar(L::BAR_P_FULL + 1), (n1 - 1) & 1, wctx);
+        if (ok) {
+          tc_fence_after();
+          issue_pv(tO[1], tS[1], base + L::OFF_KV + prev_v_stage * L::TILE, n1 - 1 > 0);
+          mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage));
+          mma_commit(bar(L::BAR_O_FULL + 1));
+        }
+      }
+      // every MMA issued so far has finished before TMEM is released
+      mma_commit(bar(L::BAR_MMA_DONE));
+      drain_wait(bar(L::BAR_MMA_DONE), 0);
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ===================================================== V tiles: bf16 -> fp16 in place
+    const int ct = threadIdx.x - 64;  // 0..63
+    bool ok = true;
+    for (int j = 0; j < n1 && ok; ++j) {
+      const int iV = 2 * j + 1;
+      const int st = iV % L::STAGES;
+      if (!(ok = mbar_wait(bar(L::BAR_KV_FULL + st), (iV / L::STAGES) & 1, wctx))) break;
+      uint4* tile = reinterpret_cast<uint4*>(gbase + L::OFF_KV + st * L::TILE);
+#pragma unroll 4
+      for (int i = ct; i < L::TILE / 16; i += kConvThreads) {
+        uint4 u = tile[i];
+        uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+          w[e] = pack_f16(f.x, f.y);
+        }
+        tile[i] = u;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(L::BAR_V_CONV + st));
+    }
+  } else if (warp >= 4) {
+    // ===================================================== softmax warpgroups
+    const int t = (warp - 4) >> 2;        // query tile handled by this warpgroup
+    const int wq = (warp - 4) & 3;        // TMEM lane quarter
+    const int row = wq * 32 + lane;       // row inside the tile
+    const int q_base = t ? q_base1 : q_base0;
+    const int r = q_base + row;           // query index
+    const int n_t = t ? n1 : n0;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (t ? L::T_S1 : L::T_S0);
+    const uint32_t tO = tmem + lane_off + (t ? L::T_O1 : L::T_O0);
+    const float sl2 = p.scale_log2;
+
+    float m = -INFINITY;  // running max of scale*log2(e)*S (possibly stale by < 8)
+    float l = 0.f;        // running sum of 2^(scale*log2(e)*S - m)
+    bool ok = true;
+    for (int j = 0; j < n_t; ++j) {
+      if (!(ok = mbar_wait(bar(L::BAR_S_FULL + t), j & 1, wctx))) break;
+      tc_fence_after();
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tS + 32 * c, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(u[i]);
+      }
+      const int kb = j * 128;
+      const bool need_mask = (p.causal && kb + 127 > q_base) || (kb + 128 > p.N);
+      if (need_mask) {
+        const int lim = p.causal ? min(r, p.N - 1) : (p.N - 1);  // last visible key
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (kb + c > lim) x[c] = -INFINITY;
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      const float m_new = fmaxf(m, mx * sl2);
+      // keep a stale maximum while it is within 2^8 of the true one: exact in the end
+      // because O / l and the LSE use the same maximum
+      const float m_use = (m_new - m > 8.0f) ? m_new : m;
+      const float alpha = (m_use == m) ? 1.0f : ex2_approx(m - m_use);  // 0 on the first tile
+      const float neg_m = -m_use;
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) x[c] = ex2_approx(fmaf(x[c], sl2, neg_m));
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          pk[i] = pack_f16(x[64 * h + 2 * i], x[64 * h + 2 * i + 1]);
+          const float2 r = __half22float2(*reinterpret_cast<const __half2*>(&pk[i]));
+          sum += r.x + r.y;  // the weights P V really uses
+        }
+        tmem_st32(tS + 32 * h, pk);
+      }
+      l = fmaf(l, alpha, sum);
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        // the previous O += P V of this tile completed before S_j did (same issuing thread)
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld32(tO + 32 * c, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          tmem_st32(tO + 32 * c, u);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(L::BAR_P_FULL + t));
+      m = m_use;
+    }
+    // ---- epilogue: O / l -> bf16 -> swizzled staging (the Q tile's buffer) -> TMA store
+    if (ok) ok = mbar_wait(bar(L::BAR_O_FULL + t), 0, wctx);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const uint32_t stage = base + (t ? L::OFF_Q1 : L::OFF_Q0);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tO + 32 * c, u);
+        tmem_wait_ld();
+        uint32_t pk[16], rk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float a = __uint_as_float(u[2 * i]) * inv_l, b = __uint_as_float(u[2 * i + 1]) * inv_l;
+          pk[i] = pack_bf16(a, b);
+          const float2 ab = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
+          rk[i] = pack_bf16(a - ab.x, b - ab.y);
+        }
+        if (p.o_resid != nullptr && r < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o_resid + ((size_t)bh * p.N + r) * D + 32 * c);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            dst[q4] = make_uint4(rk[4 * q4], rk[4 * q4 + 1], rk[4 * q4 + 2], rk[4 * q4 + 3]);
+        }
+        const int box = (32 * c) / 64;
+        const int chunk0 = ((32 * c) % 64) / 8;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          st_shared_v4(stage + box * L::BOX + sw128_offset(row, chunk0 + q4), pk[4 * q4], pk[4 * q4 + 1],
+                       pk[4 * q4 + 2], pk[4 * q4 + 3]);
+      }
+      if (p.lse != nullptr && r < p.N) p.lse[(size_t)bh * p.N + r] = (m + __log2f(l)) * 0.69314718055994531f;
+      fence_proxy_async_smem();
+    }
+    named_bar_sync(1 + t, 128);
+    if (ok && row == 0) {
+      const uint32_t stage = base + (t ? L::OFF_Q1 : L::OFF_Q0);
+      for (int c = 0; c < L::KCH; ++c) tma_store_3d(&tm_o, c * 64, q_base, bh, stage + c * L::BOX);
+      bulk_commit_group();
+      bulk_wait_group_read0();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t s) {
+  const dim3 grid((unsigned)(p.n_pairs * p.BH));
+  if (d == 128) {
+    using L = FwdLayout<128>;
+    cudaError_t e = cudaFuncSetAttribute(fa_fwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    fa_fwd_sm100_kernel<128><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, to, p);
+  } else {
+    using L = FwdLayout<64>;
+    cudaError_t e = cudaFuncSetAttribute(fa_fwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    fa_fwd_sm100_kernel<64><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, to, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,151 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact IO-aware attention library
+ * (libfa_b200.so).
+ *
+ * The library computes exact scaled dot-product attention
+ *     O = softmax(scale * Q K^T + mask) V
+ * ("FlashAttention (EL)", section "Problem of standard attention", the attention
+ * formula) without ever writing the N x N score matrix to device memory: tiles of
+ * Q, K and V are staged on chip and the softmax is applied incrementally with a
+ * running row maximum and exp-sum ("FlashAttention (EL)", sections "Tiling" and
+ * "Online computation of Softmax"; "Flash Attention: Ako transformery zvladaju
+ * miliony tokenov", section 2).  The backward pass recomputes the probabilities
+ * from the saved per-row log-sum-exp instead of storing them ("Flash Attention
+ * uitgelegd: een uitgebreide gids", section "Recomputation").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense, row-major (B, H, N, d) with d innermost -- the layout of
+ *    the scaled_dot_product_attention call shown on "Flash Attention: Ako
+ *    transformery ...", section 6.  Per-row statistics (LSE) are (B, H, N).
+ *  - Q and K/V have the same sequence length N (square problem).
+ *  - causal = 1 masks key j for query i when j > i (query i sees keys 0..i, the
+ *    diagonal included); causal = 0 is full (bidirectional) attention.
+ *  - scale multiplies Q K^T before masking; callers normally pass 1/sqrt(d).
+ *  - LSE_i = ln sum_j exp(scale * S_ij) over the visible keys (natural log of the
+ *    scaled, masked scores), fp32.
+ *  - Every pointer is CALLER-OWNED DEVICE memory on the current CUDA device.  The
+ *    library allocates no memory and keeps no state between calls except one
+ *    device-resident error word per device (see fa_device_status).
+ *  - Calls are asynchronous on `stream` (NULL = the legacy default stream) and do
+ *    not synchronise.  Argument errors are detected on the host before anything
+ *    is launched; nothing is written then.
+ *  - B, H or N equal to 0 is an empty problem: FA_OK, nothing launched.
+ *  - Supported: d in {64, 128}; a B200-class GPU (compute capability 10.0).
+ *
+ * Thread safety: calls may be issued from several host threads; calls whose
+ * work overlaps on the GPU must not share output buffers or a workspace.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* fa_stream_t;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad scale/causal, workspace too small */
+  FA_ERR_UNSUPPORTED = 2, /* head dim not in {64,128}, sizes beyond limits, not a CC 10.0 device */
+  FA_ERR_MISALIGNED = 3,  /* a tensor base address is not 16-byte aligned (TMA requirement) */
+  FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
+  FA_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (reported by fa_device_status) */
+} fa_status;
+
+/*
+ * fa_fwd -- forward pass, bf16 in / bf16 out, on tensor cores.
+ *   q, k, v : const bf16 (B, H, N, d), 16-byte aligned.
+ *   o       : bf16 (B, H, N, d) output, 16-byte aligned; must not alias q, k, v.
+ *   lse     : fp32 (B, H, N) output (natural-log LSE, see above), or NULL to skip.
+ *   o_resid : bf16 (B, H, N, d) output or NULL: the residual O_fp32 - O_bf16 of
+ *             the final rounding of O.  A training forward passes it and hands it
+ *             to fa_bwd, which then forms rowsum(dO * O) from an fp32-accurate O
+ *             (the bf16 rounding of O alone costs the gradients up to ~0.2 of
+ *             absolute accuracy on sharply peaked softmax rows).
+ *   B, H, N : batch, heads, sequence length (>= 0).  d: head dim, 64 or 128.
+ *   scale   : finite, > 0.   causal: 0 or 1.   stream: CUDA stream.
+ * Q K^T is a bf16 product with fp32 accumulation; the probabilities are rounded
+ * to fp16 (round to nearest even) for the P V product, whose V operand is an
+ * exact fp16 copy of the bf16 V made on chip (|V| must stay below 65504); the row
+ * sums add up those rounded probabilities; O is rounded to bf16 once at the end.
+ * Returns FA_OK once the kernel is enqueued.
+ */
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B,
+                        int H, int N, int d, float scale, int causal, fa_stream_t stream);
+
+/*
+ * fa_fwd_f32 -- the same forward pass on fp32 inputs and outputs, computed
+ * entirely in fp32 on the CUDA cores (no input rounding).  Meant for small
+ * problems and checks; same arguments and rules as fa_fwd except dtypes, and
+ * pointers need only 4-byte alignment.
+ */
+FA_API fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N,
+                     int d, float scale, int causal, fa_stream_t stream);
+
+/*
+ * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for this
+ * problem (fp16 copies of Q, K, V, dO and two fp32 (B, H, N rounded up to 128)
+ * row vectors).  Returns 0 for an empty or invalid problem.
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_bwd -- backward pass: gradients of sum(O * dO) with respect to Q, K, V.
+ *   q, k, v, o, dout : const bf16 (B, H, N, d), 16-byte aligned; o, o_resid and
+ *                      lse are the outputs of fa_fwd on the same q, k, v, scale
+ *                      and causal.
+ *   o_resid          : const bf16 (B, H, N, d) residual from fa_fwd, or NULL
+ *                      (then rowsum(dO * O) uses the bf16 O alone: less accurate).
+ *   lse              : const fp32 (B, H, N).
+ *   dq, dk, dv       : fp32 (B, H, N, d) outputs, 16-byte aligned, not aliasing
+ *                      any input.  Overwritten (not accumulated into).
+ *   workspace        : device buffer of at least fa_bwd_workspace_size(B,H,N,d)
+ *                      bytes, 256-byte aligned, caller-owned; its contents on
+ *                      entry do not matter and on return are unspecified.
+ *   workspace_bytes  : its size.
+ * The probabilities are recomputed from LSE.  The tensor-core products run in
+ * fp16 on exact fp16 copies of the bf16 inputs (exact for |x| in [2^-14, 65504];
+ * larger magnitudes overflow), with fp32 accumulation; gradients are fp32.
+ */
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                        const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int N,
+                        int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                        fa_stream_t stream);
+
+/*
+ * fa_device_status -- synchronises `stream`, then reports whether any kernel of
+ * this library on the current device gave up a bounded wait since the last call
+ * (FA_ERR_TIMEOUT; the word is then cleared) or whether the CUDA context holds an
+ * error (FA_ERR_CUDA).  FA_OK otherwise.
+ */
+FA_API fa_status fa_device_status(fa_stream_t stream);
+
+/*
+ * fa_bwd_set_phase_events -- profiling hook.  With `events` pointing to two
+ * cudaEvent_t handles (created by the caller), every later fa_bwd call made from
+ * the same host thread records events[0] on its stream right after the
+ * preprocess kernel and events[1] right after the dK/dV kernel, so a caller that
+ * records its own events before and after the call can time each of the three
+ * backward kernels.  NULL turns the hook off.  The library keeps only the pointer.
+ */
+FA_API void fa_bwd_set_phase_events(void* const* events);
+
+/* Human-readable name of a status code (static string, never NULL). */
+FA_API const char* fa_status_str(fa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,122 @@
+"""Host-only checks of the C ABI: the library loads, exports every declared entry
+point, and rejects bad arguments before touching the GPU."""
+
+import os
+import re
+
+import pytest
+
+from exact_io_aware_91_b200 import api
+from exact_io_aware_91_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return api.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    assert sorted(declared_functions()) == sorted(api.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "FA_OK"), (1, "FA_ERR_INVALID_ARG"), (2, "FA_ERR_UNSUPPORTED"),
+                       (3, "FA_ERR_MISALIGNED"), (4, "FA_ERR_CUDA"), (5, "FA_ERR_TIMEOUT")]:
+        assert api.status_str(code) == name
+    assert api.status_str(99) == "FA_ERR_UNKNOWN"
+
+
+def _ws_expected(B, H, N, d):
+    a = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    Np = (N + 127) // 128 * 128
+    return 4 * a(B * H * N * d * 2) + 2 * a(B * H * Np * 4)
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1, 64), (4, 16, 2048, 128), (2, 32, 8192, 128), (1, 8, 131072, 128),
+                                   (3, 5, 1000, 64)])
+def test_workspace_size_is_linear_in_n(lib, shape):
+    assert api.fa_bwd_workspace_size(*shape) == _ws_expected(*shape)
+
+
+def test_workspace_size_of_empty_or_bad_problem_is_zero(lib):
+    assert api.fa_bwd_workspace_size(0, 1, 10, 64) == 0
+    assert api.fa_bwd_workspace_size(1, 1, 0, 64) == 0
+    assert api.fa_bwd_workspace_size(1, 1, 10, 96) == 0
+    assert api.fa_bwd_workspace_size(-1, 1, 10, 64) == 0
+
+
+# Fake device addresses: never dereferenced, because every call below is rejected
+# (or is empty) before anything is launched.
+A = 0x10000  # 16-byte (and 256-byte) aligned
+MIS = 0x10008
+
+
+def fwd(lib, q=A, k=A, v=A, o=A, lse=A, resid=None, B=1, H=1, N=16, d=64, scale=0.125, causal=0):
+    return lib.fa_fwd(q, k, v, o, lse, resid, B, H, N, d, scale, causal, None)
+
+
+def bwd(lib, ptr=A, ws=A, ws_bytes=1 << 40, B=1, H=1, N=16, d=64, scale=0.125, causal=0, dq=A, resid=A):
+    return lib.fa_bwd(ptr, ptr, ptr, ptr, resid, ptr, ptr, dq, ptr, ptr, B, H, N, d, scale, causal, ws, ws_bytes,
+                      None)
+
+
+def test_forward_argument_errors(lib):
+    assert fwd(lib, q=None) == api.FA_ERR_INVALID_ARG
+    assert fwd(lib, o=None) == api.FA_ERR_INVALID_ARG
+    assert fwd(lib, N=-1) == api.FA_ERR_INVALID_ARG
+    assert fwd(lib, scale=0.0) == api.FA_ERR_INVALID_ARG
+    assert fwd(lib, scale=float("nan")) == api.FA_ERR_INVALID_ARG
+    assert fwd(lib, scale=float("inf")) == api.FA_ERR_INVALID_ARG
+    assert fwd(lib, causal=2) == api.FA_ERR_INVALID_ARG
+    assert fwd(lib, d=96) == api.FA_ERR_UNSUPPORTED
+    assert fwd(lib, d=256) == api.FA_ERR_UNSUPPORTED
+    assert fwd(lib, q=MIS) == api.FA_ERR_MISALIGNED
+    assert fwd(lib, o=MIS) == api.FA_ERR_MISALIGNED
+    assert fwd(lib, lse=A + 2) == api.FA_ERR_MISALIGNED
+    assert fwd(lib, resid=A + 8) == api.FA_ERR_MISALIGNED
+    assert fwd(lib, B=1 << 25) == api.FA_ERR_UNSUPPORTED
+
+
+def test_empty_problems_are_no_ops(lib):
+    # nothing to compute: FA_OK even with null pointers, nothing launched
+    assert fwd(lib, q=None, k=None, v=None, o=None, lse=None, N=0) == api.FA_OK
+    assert fwd(lib, q=None, k=None, v=None, o=None, lse=None, B=0) == api.FA_OK
+    assert bwd(lib, ptr=None, ws=None, dq=None, resid=None, H=0) == api.FA_OK
+    assert lib.fa_fwd_f32(None, None, None, None, None, 1, 1, 0, 64, 0.125, 0, None) == api.FA_OK
+
+
+def test_backward_argument_errors(lib):
+    assert bwd(lib, ptr=None) == api.FA_ERR_INVALID_ARG
+    assert bwd(lib, ws=None) == api.FA_ERR_INVALID_ARG
+    assert bwd(lib, ws_bytes=_ws_expected(1, 1, 16, 64) - 1) == api.FA_ERR_INVALID_ARG
+    assert bwd(lib, d=32) == api.FA_ERR_UNSUPPORTED
+    assert bwd(lib, causal=-1) == api.FA_ERR_INVALID_ARG
+    assert bwd(lib, dq=MIS) == api.FA_ERR_MISALIGNED
+    assert bwd(lib, resid=MIS) == api.FA_ERR_MISALIGNED
+    assert bwd(lib, ws=A + 16) == api.FA_ERR_MISALIGNED  # workspace needs 256-byte alignment
+
+
+def test_f32_forward_argument_errors(lib):
+    assert lib.fa_fwd_f32(None, A, A, A, A, 1, 1, 8, 64, 0.125, 0, None) == api.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_f32(A + 2, A, A, A, A, 1, 1, 8, 64, 0.125, 0, None) == api.FA_ERR_MISALIGNED
+    assert lib.fa_fwd_f32(A, A, A, A, A, 1, 1, 8, 48, 0.125, 0, None) == api.FA_ERR_UNSUPPORTED
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-GPU path")
+def test_valid_call_without_a_gpu_fails_loudly(lib):
+    # all arguments valid: the call reaches the CUDA runtime, which has no device here
+    assert fwd(lib) == api.FA_ERR_CUDA
