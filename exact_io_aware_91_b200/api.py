@@ -188,6 +188,9 @@ def fa_bwd_set_phase_events(events=None) -> None:
         _PHASE_EVENTS = None
         library().fa_bwd_set_phase_events(None)
         return
+    for ev in events[:2]:
+        if not ev.cuda_event:  # torch creates the CUDA event lazily, on its first record
+            ev.record()
     arr = (ctypes.c_void_p * 2)(events[0].cuda_event, events[1].cuda_event)
     _PHASE_EVENTS = arr
     library().fa_bwd_set_phase_events(ctypes.cast(arr, ctypes.c_void_p))

@@ -233,7 +233,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   pp.BH = BH;
   pp.d = d;
   if (launch_bwd_pre(pp, s) != cudaSuccess) return FA_ERR_CUDA;
-  if (t_phase_events != nullptr &&
+  if (t_phase_events != nullptr && t_phase_events[0] != nullptr &&
       cudaEventRecord(static_cast<cudaEvent_t>(t_phase_events[0]), s) != cudaSuccess)
     return FA_ERR_CUDA;
 
@@ -263,7 +263,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   bp.causal = causal;
   bp.err = g_err_ptr[dev];
   if (launch_bwd_dkdv_sm100(a_q, a_do, a_k, a_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
-  if (t_phase_events != nullptr &&
+  if (t_phase_events != nullptr && t_phase_events[1] != nullptr &&
       cudaEventRecord(static_cast<cudaEvent_t>(t_phase_events[1]), s) != cudaSuccess)
     return FA_ERR_CUDA;
   if (launch_bwd_dq_sm100(b_q, b_do, b_k, b_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;

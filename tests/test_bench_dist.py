@@ -1,0 +1,57 @@
+"""The N > 1 plumbing of bench.py (replicas, barrier, max-over-ranks timing) on two
+gloo ranks on the CPU."""
+
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+
+    r, w, _ = bench.dist_setup(world)
+    try:
+        bench.barrier(w)
+        # each rank times a different amount of work: the job's time is the slowest rank's
+        t = bench.max_over_ranks(10.0 * (r + 1), w)
+        out.put((r, w, t))
+    finally:
+        bench.dist_teardown(w)
+
+
+@pytest.mark.timeout(120)
+def test_two_gloo_ranks_take_the_max_time():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(90)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    assert got == [(0, 2, 20.0), (1, 2, 20.0)]
+
+
+def test_single_rank_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    bench.barrier(1)
