@@ -23,8 +23,11 @@ FA_ERR_MISALIGNED = 3
 FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
 
-EXPORTS = ("fa_fwd", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_device_status",
+EXPORTS = ("fa_fwd", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_noalloc", "fa_device_status",
            "fa_bwd_set_phase_events", "fa_status_str")
+
+# Size of the scratch array fa_bwd_noalloc uses instead of a caller workspace.
+FA_BWD_NOALLOC_MAX_WORKSPACE = 64 << 20
 
 
 class FAError(RuntimeError):
@@ -57,6 +60,8 @@ def library() -> ctypes.CDLL:
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_bwd.restype = i
+    lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_bwd_noalloc.restype = i
     lib.fa_device_status.argtypes = [vp]
     lib.fa_device_status.restype = i
     lib.fa_bwd_set_phase_events.argtypes = [vp]
@@ -168,6 +173,26 @@ def fa_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None
                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, _scale(scale, d),
                           int(bool(causal)), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
     _check("fa_bwd", st)
+    return dq, dk, dv
+
+
+def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal: bool = False, scale: float | None = None,
+                   o_resid=None, stream=None):
+    """The backward pass without a workspace, for callers that cannot allocate device memory
+    when they run it: the C entry point uses a scratch array built into the library (64 MiB
+    per GPU, shared by all calls on that GPU, so overlapping calls race).  The caller passes
+    every input and the fp32 outputs dq, dk, dv; nothing is allocated here either."""
+    B, H, N, d = _shape(q)
+    _same(q, k, v, o, do, dtype=torch.bfloat16, shape=(B, H, N, d))
+    _same(lse, dtype=torch.float32, shape=(B, H, N))
+    _same(dq, dk, dv, dtype=torch.float32, shape=(B, H, N, d))
+    if o_resid is not None:
+        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
+    st = library().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  None if o_resid is None else o_resid.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                                  dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, _scale(scale, d),
+                                  int(bool(causal)), _stream_handle(stream))
+    _check("fa_bwd_noalloc", st)
     return dq, dk, dv
 
 

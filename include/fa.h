@@ -124,6 +124,35 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                         fa_stream_t stream);
 
 /*
+ * fa_bwd_noalloc -- the backward pass of fa_bwd for callers that cannot allocate
+ * device memory.  (The pages describe no such entry point; it is a service of this
+ * library.)  Some callers have no way to obtain a workspace at the moment they run
+ * the backward pass: a plugin's enqueue callback inside an engine that owns all
+ * device memory and forbids allocation there, or a latency-bound loop in which
+ * cudaMalloc (which may synchronise the device) is not acceptable.  This entry
+ * point takes the same arguments as fa_bwd minus the workspace and uses instead a
+ * scratch array compiled into the library: a file-scope device array of
+ * FA_BWD_NOALLOC_MAX_WORKSPACE bytes (64 MiB) that every GPU which loads the
+ * library holds until the process exits.  It calls no cudaMalloc, cudaFree or any
+ * other allocating routine.
+ *   - Problems whose fa_bwd_workspace_size() exceeds FA_BWD_NOALLOC_MAX_WORKSPACE are
+ *     rejected with FA_ERR_UNSUPPORTED before anything is launched (e.g. B*H*N*d up
+ *     to about 8 million elements fits).
+ *   - The first call on a device looks up the array's device address on that device
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the one array, which keeps whatever the last call
+ *     left in it.  Nothing in it needs to start at zero (each call overwrites every
+ *     byte it reads), but calls whose work overlaps on the GPU -- on different
+ *     streams, or from different host threads -- race on the array: serialise them.
+ * Results are identical to fa_bwd with a workspace of its own.
+ */
+#define FA_BWD_NOALLOC_MAX_WORKSPACE ((size_t)64 << 20)
+FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                                const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H,
+                                int N, int d, float scale, int causal, fa_stream_t stream);
+
+/*
  * fa_device_status -- synchronises `stream`, then reports whether any kernel of
  * this library on the current device gave up a bounded wait since the last call
  * (FA_ERR_TIMEOUT; the word is then cleared) or whether the CUDA context holds an
