@@ -28,6 +28,10 @@ namespace fa {
 namespace {
 
 constexpr int kThreads = 384;
+// registers per thread: 168 at launch (65536 / 384, rounded down to a multiple of 8);
+// warpgroup 0 (TMA, MMA) drops to 64 and the two compute warpgroups rise to 216
+constexpr uint32_t kRegsLaunch = 168, kRegsLow = 64, kRegsHigh = 216;
+static_assert(kRegsLow + 2 * kRegsHigh <= 3 * kRegsLaunch, "register split exceeds the launch budget");
 
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   uint64_t t0 = globaltimer_ns();
@@ -36,26 +40,24 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-// SS product D (+)= A * B^T over K = Dh, A rows in `a_box`-byte boxes, B rows in `b_box`-byte boxes.
-template <int Dh>
-__device__ __forceinline__ void issue_ss(uint32_t d_tmem, uint32_t a_s, uint32_t a_box, uint32_t b_s,
-                                         uint32_t b_box, uint32_t idesc) {
+// SS product D (+)= A * B^T over K = Dh; A rows in `a_box`-byte boxes, B rows in
+// `b_box`-byte boxes; the descriptors are prebuilt, each MMA adds a constant offset.
+template <int Dh, uint32_t a_box, uint32_t b_box>
+__device__ __forceinline__ void issue_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t issue) {
 #pragma unroll
-  for (int k = 0; k < Dh / 16; ++k) {
-    const uint32_t ka = (k >> 2) * a_box + (k & 3) * 32;
-    const uint32_t kb = (k >> 2) * b_box + (k & 3) * 32;
-    mma_ss(d_tmem, make_sdesc_sw128(a_s + ka, 16, 1024), make_sdesc_sw128(b_s + kb, 16, 1024), idesc,
-           k > 0 ? 1u : 0u);
-  }
+  for (int k = 0; k < Dh / 16; ++k)
+    mma_ss(d_tmem, sdesc_add(a_desc, (k >> 2) * a_box + (k & 3) * 32), sdesc_add(b_desc, (k >> 2) * b_box + (k & 3) * 32),
+           idesc, k > 0 ? 1u : 0u, issue);
 }
 
-// TS product D (+)= A[tmem] * B, K = `K` rows of B (MN-major, boxes of `b_box` bytes along N).
+// TS product D (+)= A[tmem] * B over K rows of B (MN-major descriptor prebuilt).
 template <int K>
-__device__ __forceinline__ void issue_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_s, uint32_t b_box,
-                                         uint32_t idesc, bool acc) {
+__device__ __forceinline__ void issue_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                         bool acc, uint32_t issue) {
 #pragma unroll
   for (int k = 0; k < K / 16; ++k)
-    mma_ts(d_tmem, a_tmem + k * 8, make_sdesc_sw128(b_s + k * 2048, b_box, 1024), idesc, (acc || k > 0) ? 1u : 0u);
+    mma_ts(d_tmem, a_tmem + k * 8, sdesc_add(b_desc, k * 2048), idesc, (acc || k > 0) ? 1u : 0u, issue);
 }
 
 // Write `ncols` fp32 columns of this thread's TMEM lane to global row `dst` (times `mult`).
@@ -120,9 +122,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wctx{abort_flag, p.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int BHi = p.BH;
-  const int j = blockIdx.x / BHi;  // key tile (small j = most work under the causal mask)
-  const int bh = blockIdx.x % BHi;
+  // head-major order (CTAs running together share Q / dO in L2); within a head the
+  // key tiles with the most work under the causal mask (small j) come first
+  const int n_kt = (p.N + 127) / 128;
+  const int bh = blockIdx.x / n_kt;
+  const int j = blockIdx.x % n_kt;
   const int nq = (p.N + 63) / 64;
   const int i_start = p.causal ? 2 * j : 0;
   const int n_it = nq - i_start;  // >= 1
@@ -152,15 +156,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_TMEM_SLOT);
 
   if (warp == 0) {
-    if (lane == 0) {
+    regs_dec<kRegsLow>();
+    {
+      const uint32_t leader = elect_one();  // the lane that issues async instructions
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_do);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(bar(L::BAR_KV), 2 * L::TILE_KV);
+      mbar_arrive_expect_tx(bar(L::BAR_KV), 2 * L::TILE_KV, leader);
       for (int c = 0; c < L::KCH; ++c) {
-        tma_load_3d(base + L::OFF_K + c * L::BOX_KV, &tm_k, c * 64, j * 128, bh, bar(L::BAR_KV));
-        tma_load_3d(base + L::OFF_V + c * L::BOX_KV, &tm_v, c * 64, j * 128, bh, bar(L::BAR_KV));
+        tma_load_3d(base + L::OFF_K + c * L::BOX_KV, &tm_k, c * 64, j * 128, bh, bar(L::BAR_KV), leader);
+        tma_load_3d(base + L::OFF_V + c * L::BOX_KV, &tm_v, c * 64, j * 128, bh, bar(L::BAR_KV), leader);
       }
       int issued = 0;
       for (int it = 0; it < n_it; ++it) {
@@ -169,14 +175,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int i = i_start + it;
         const uint32_t sb = base + L::OFF_STAGE + st * L::STAGE;
         const uint32_t fb = bar(L::BAR_Q_FULL + st);
-        mbar_arrive_expect_tx(fb, 2 * L::TILE_Q + 512);
+        mbar_arrive_expect_tx(fb, 2 * L::TILE_Q + 512, leader);
         for (int c = 0; c < L::KCH; ++c) {
-          tma_load_3d(sb + c * L::BOX_Q, &tm_q, c * 64, i * 64, bh, fb);
-          tma_load_3d(sb + L::TILE_Q + c * L::BOX_Q, &tm_do, c * 64, i * 64, bh, fb);
+          tma_load_3d(sb + c * L::BOX_Q, &tm_q, c * 64, i * 64, bh, fb, leader);
+          tma_load_3d(sb + L::TILE_Q + c * L::BOX_Q, &tm_do, c * 64, i * 64, bh, fb, leader);
         }
         const size_t roff = (size_t)bh * p.Np + (size_t)i * 64;
-        bulk_load(sb + 2 * L::TILE_Q, p.lse2 + roff, 256, fb);
-        bulk_load(sb + 2 * L::TILE_Q + 256, p.delta + roff, 256, fb);
+        bulk_load(sb + 2 * L::TILE_Q, p.lse2 + roff, 256, fb, leader);
+        bulk_load(sb + 2 * L::TILE_Q + 256, p.delta + roff, 256, fb, leader);
         ++issued;
       }
       drain_wait(bar(L::BAR_KV), 0);
@@ -185,17 +191,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(bar(L::BAR_Q_FULL + (it % L::STAGES)), (it / L::STAGES) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    regs_dec<kRegsLow>();
+    {
+      const uint32_t leader = elect_one();  // the lane that issues async instructions
       constexpr uint32_t idesc_s = make_idesc(128, 64, false, false, false);  // M=128 keys, N=64 queries
       constexpr uint32_t idesc_g = make_idesc(128, D, false, false, true);    // N=D, B MN-major
-      const uint32_t sK = base + L::OFF_K, sV = base + L::OFF_V;
-      auto stage_addr = [&](int it) { return base + L::OFF_STAGE + (it % L::STAGES) * L::STAGE; };
+      const uint64_t dK = make_sdesc_sw128(base + L::OFF_K, 16, 1024);
+      const uint64_t dV = make_sdesc_sw128(base + L::OFF_V, 16, 1024);
+      const uint64_t dStK = make_sdesc_sw128(base + L::OFF_STAGE, 16, 1024);        // Q / dO as K-major B
+      const uint64_t dStMN = make_sdesc_sw128(base + L::OFF_STAGE, L::BOX_Q, 1024);  // Q / dO as MN-major B
       auto issue_sdp = [&](int it) {
-        const uint32_t sb = stage_addr(it);
+        const uint32_t so = (it % L::STAGES) * L::STAGE;
         const uint32_t tb = tmem + L::T_BUF + 128 * (it & 1);
-        issue_ss<D>(tb, sK, L::BOX_KV, sb, L::BOX_Q, idesc_s);                // S^T  = K Q^T
-        issue_ss<D>(tb + 64, sV, L::BOX_KV, sb + L::TILE_Q, L::BOX_Q, idesc_s);  // dP^T = V dO^T
-        mma_commit(bar(L::BAR_SDP + (it & 1)));
+        issue_ss<D, L::BOX_KV, L::BOX_Q>(tb, dK, sdesc_add(dStK, so), idesc_s, leader);                     // S^T  = K Q^T
+        issue_ss<D, L::BOX_KV, L::BOX_Q>(tb + 64, dV, sdesc_add(dStK, so + L::TILE_Q), idesc_s, leader);    // dP^T = V dO^T
+        mma_commit(bar(L::BAR_SDP + (it & 1)), leader);
       };
       bool ok = mbar_wait(bar(L::BAR_KV), 0, wctx);
       if (ok) ok = mbar_wait(bar(L::BAR_Q_FULL + 0), 0, wctx);
@@ -213,17 +223,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = it & 1;
         if (!(ok = mbar_wait(bar(L::BAR_DS + b), (it >> 1) & 1, wctx))) break;
         tc_fence_after();
-        const uint32_t sb = stage_addr(it);
+        const uint32_t so = (it % L::STAGES) * L::STAGE;
         const uint32_t tb = tmem + L::T_BUF + 128 * b;
-        issue_ts<64>(tmem + L::T_DV, tb, sb + L::TILE_Q, L::BOX_Q, idesc_g, it > 0);  // dV += P^T dO
-        issue_ts<64>(tmem + L::T_DK, tb + 64, sb, L::BOX_Q, idesc_g, it > 0);         // dK += dS^T Q
-        mma_commit(bar(L::BAR_Q_EMPTY + (it % L::STAGES)));
+        issue_ts<64>(tmem + L::T_DV, tb, sdesc_add(dStMN, so + L::TILE_Q), idesc_g, it > 0, leader);  // dV += P^T dO
+        issue_ts<64>(tmem + L::T_DK, tb + 64, sdesc_add(dStMN, so), idesc_g, it > 0, leader);         // dK += dS^T Q
+        mma_commit(bar(L::BAR_Q_EMPTY + (it % L::STAGES)), leader);
       }
-      if (ok) mma_commit(bar(L::BAR_ACC));
-      mma_commit(bar(L::BAR_DONE));
+      if (ok) mma_commit(bar(L::BAR_ACC), leader);
+      mma_commit(bar(L::BAR_DONE), leader);
       drain_wait(bar(L::BAR_DONE), 0);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    regs_dec<kRegsLow>();  // warps 2-3: idle
+  } else {
+    regs_inc<kRegsHigh>();
     const int w = (warp - 4) >> 2;   // warpgroup: takes tiles it = w, w + 2, ...
     const int wq = (warp - 4) & 3;
     const int row = wq * 32 + lane;  // key row inside the tile
@@ -257,21 +270,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
       }
       const bool need_mask = p.causal && (i * 64 < j * 128 + 127);
+      const uint64_t sl2x2 = f2pack(sl2, sl2);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float pv = ex2_approx(fmaf(s[c], sl2, -lse2[c]));
-        if (need_mask && (i * 64 + c < key)) pv = 0.f;
-        s[c] = pv;
-        dp[c] = pv * (dp[c] - delta[c]);
-      }
-      {
-        uint32_t pk[32];
+      for (int g = 0; g < 64; g += 16) {  // 16 query columns at a time: 8 packed words of P^T and dS^T
+        uint32_t pk_p[8], pk_ds[8];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_f16(s[2 * c], s[2 * c + 1]);
-        tmem_st32(tb, pk);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_f16(dp[2 * c], dp[2 * c + 1]);
-        tmem_st32(tb + 64, pk);
+        for (int c = g; c < g + 16; c += 4) {
+          // per-query LSE and D are broadcast reads of the stage's vectors (16 bytes at a time)
+          const float4 L4 = *reinterpret_cast<const float4*>(lse2 + c);
+          const float4 D4 = *reinterpret_cast<const float4*>(delta + c);
+          float t0, t1, t2, t3;
+          f2unpack(ffma2(f2pack(s[c], s[c + 1]), sl2x2, f2pack(-L4.x, -L4.y)), t0, t1);
+          f2unpack(ffma2(f2pack(s[c + 2], s[c + 3]), sl2x2, f2pack(-L4.z, -L4.w)), t2, t3);
+          float p0 = ex2_approx(t0), p1 = ex2_approx(t1), p2 = ex2_approx(t2), p3 = ex2_approx(t3);
+          if (need_mask) {
+            if (i * 64 + c < key) p0 = 0.f;
+            if (i * 64 + c + 1 < key) p1 = 0.f;
+            if (i * 64 + c + 2 < key) p2 = 0.f;
+            if (i * 64 + c + 3 < key) p3 = 0.f;
+          }
+          float d0, d1, d2, d3;
+          f2unpack(fmul2(f2pack(p0, p1), fsub2(f2pack(dp[c], dp[c + 1]), f2pack(D4.x, D4.y))), d0, d1);
+          f2unpack(fmul2(f2pack(p2, p3), fsub2(f2pack(dp[c + 2], dp[c + 3]), f2pack(D4.z, D4.w))), d2, d3);
+          pk_p[(c - g) / 2] = pack_f16(p0, p1);
+          pk_p[(c - g) / 2 + 1] = pack_f16(p2, p3);
+          pk_ds[(c - g) / 2] = pack_f16(d0, d1);
+          pk_ds[(c - g) / 2 + 1] = pack_f16(d2, d3);
+        }
+        tmem_st8(tb + g / 2, pk_p);
+        tmem_st8(tb + 64 + g / 2, pk_ds);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -340,8 +367,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int nq = (p.N + 127) / 128;
   const int nk = (p.N + 63) / 64;
-  const int qt = p.causal ? (nq - 1 - (int)(blockIdx.x / p.BH)) : (int)(blockIdx.x / p.BH);
-  const int bh = blockIdx.x % p.BH;
+  // head-major order (CTAs running together share K / V in L2); within a head the
+  // query tiles with the most work under the causal mask come first
+  const int bh = blockIdx.x / nq;
+  const int qt = p.causal ? (nq - 1 - (int)(blockIdx.x % nq)) : (int)(blockIdx.x % nq);
   const int n_it = p.causal ? min(nk, (qt * 128 + 127) / 64 + 1) : nk;  // key tiles 0..n_it-1
 
   if (threadIdx.x == 0) {
@@ -369,15 +398,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_TMEM_SLOT);
 
   if (warp == 0) {
-    if (lane == 0) {
+    regs_dec<kRegsLow>();
+    {
+      const uint32_t leader = elect_one();  // the lane that issues async instructions
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_do);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(bar(L::BAR_Q), 2 * L::TILE_Q);
+      mbar_arrive_expect_tx(bar(L::BAR_Q), 2 * L::TILE_Q, leader);
       for (int c = 0; c < L::KCH; ++c) {
-        tma_load_3d(base + L::OFF_Q + c * L::BOX_Q, &tm_q, c * 64, qt * 128, bh, bar(L::BAR_Q));
-        tma_load_3d(base + L::OFF_DO + c * L::BOX_Q, &tm_do, c * 64, qt * 128, bh, bar(L::BAR_Q));
+        tma_load_3d(base + L::OFF_Q + c * L::BOX_Q, &tm_q, c * 64, qt * 128, bh, bar(L::BAR_Q), leader);
+        tma_load_3d(base + L::OFF_DO + c * L::BOX_Q, &tm_do, c * 64, qt * 128, bh, bar(L::BAR_Q), leader);
       }
       int issued = 0;
       for (int it = 0; it < n_it; ++it) {
@@ -385,10 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(bar(L::BAR_KV_EMPTY + st), ((it / L::STAGES) & 1) ^ 1u, wctx)) break;
         const uint32_t sb = base + L::OFF_STAGE + st * L::STAGE;
         const uint32_t fb = bar(L::BAR_KV_FULL + st);
-        mbar_arrive_expect_tx(fb, 2 * L::TILE_K);
+        mbar_arrive_expect_tx(fb, 2 * L::TILE_K, leader);
         for (int c = 0; c < L::KCH; ++c) {
-          tma_load_3d(sb + c * L::BOX_K, &tm_k, c * 64, it * 64, bh, fb);
-          tma_load_3d(sb + L::TILE_K + c * L::BOX_K, &tm_v, c * 64, it * 64, bh, fb);
+          tma_load_3d(sb + c * L::BOX_K, &tm_k, c * 64, it * 64, bh, fb, leader);
+          tma_load_3d(sb + L::TILE_K + c * L::BOX_K, &tm_v, c * 64, it * 64, bh, fb, leader);
         }
         ++issued;
       }
@@ -398,17 +429,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(bar(L::BAR_KV_FULL + (it % L::STAGES)), (it / L::STAGES) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    regs_dec<kRegsLow>();
+    {
+      const uint32_t leader = elect_one();  // the lane that issues async instructions
       constexpr uint32_t idesc_s = make_idesc(128, 64, false, false, false);  // M=128 queries, N=64 keys
       constexpr uint32_t idesc_g = make_idesc(128, D, false, false, true);
-      const uint32_t sQ = base + L::OFF_Q, sDO = base + L::OFF_DO;
-      auto stage_addr = [&](int it) { return base + L::OFF_STAGE + (it % L::STAGES) * L::STAGE; };
+      const uint64_t dQd = make_sdesc_sw128(base + L::OFF_Q, 16, 1024);
+      const uint64_t dDO = make_sdesc_sw128(base + L::OFF_DO, 16, 1024);
+      const uint64_t dStK = make_sdesc_sw128(base + L::OFF_STAGE, 16, 1024);        // K / V as K-major B
+      const uint64_t dStMN = make_sdesc_sw128(base + L::OFF_STAGE, L::BOX_K, 1024);  // K as MN-major B
       auto issue_sdp = [&](int it) {
-        const uint32_t sb = stage_addr(it);
+        const uint32_t so = (it % L::STAGES) * L::STAGE;
         const uint32_t tb = tmem + L::T_BUF + 128 * (it & 1);
-        issue_ss<D>(tb, sQ, L::BOX_Q, sb, L::BOX_K, idesc_s);                  // S  = Q K^T
-        issue_ss<D>(tb + 64, sDO, L::BOX_Q, sb + L::TILE_K, L::BOX_K, idesc_s);  // dP = dO V^T
-        mma_commit(bar(L::BAR_SDP + (it & 1)));
+        issue_ss<D, L::BOX_Q, L::BOX_K>(tb, dQd, sdesc_add(dStK, so), idesc_s, leader);                    // S  = Q K^T
+        issue_ss<D, L::BOX_Q, L::BOX_K>(tb + 64, dDO, sdesc_add(dStK, so + L::TILE_K), idesc_s, leader);   // dP = dO V^T
+        mma_commit(bar(L::BAR_SDP + (it & 1)), leader);
       };
       bool ok = mbar_wait(bar(L::BAR_Q), 0, wctx);
       if (ok) ok = mbar_wait(bar(L::BAR_KV_FULL + 0), 0, wctx);
@@ -427,14 +462,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(bar(L::BAR_DS + b), (it >> 1) & 1, wctx))) break;
         tc_fence_after();
         const uint32_t tb = tmem + L::T_BUF + 128 * b;
-        issue_ts<64>(tmem + L::T_DQ, tb, stage_addr(it), L::BOX_K, idesc_g, it > 0);  // dQ += dS K
-        mma_commit(bar(L::BAR_KV_EMPTY + (it % L::STAGES)));
+        issue_ts<64>(tmem + L::T_DQ, tb, sdesc_add(dStMN, (it % L::STAGES) * L::STAGE), idesc_g, it > 0, leader);  // dQ += dS K
+        mma_commit(bar(L::BAR_KV_EMPTY + (it % L::STAGES)), leader);
       }
-      if (ok) mma_commit(bar(L::BAR_ACC));
-      mma_commit(bar(L::BAR_DONE));
+      if (ok) mma_commit(bar(L::BAR_ACC), leader);
+      mma_commit(bar(L::BAR_DONE), leader);
       drain_wait(bar(L::BAR_DONE), 0);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    regs_dec<kRegsLow>();  // warps 2-3: idle
+  } else {
+    regs_inc<kRegsHigh>();
     const int w = (warp - 4) >> 2;
     const int wq = (warp - 4) & 3;
     const int row = wq * 32 + lane;
@@ -469,16 +507,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int kb = it * 64;
       const bool need_mask = (p.causal && kb + 63 > qt * 128) || (kb + 64 > p.N);
+      const uint64_t sl2x2 = f2pack(sl2, sl2), nl2 = f2pack(-lse2, -lse2), dd = f2pack(delta, delta);
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        float p0 = ex2_approx(fmaf(s[2 * c], sl2, -lse2));
-        float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, -lse2));
+        float t0, t1;
+        f2unpack(ffma2(f2pack(s[2 * c], s[2 * c + 1]), sl2x2, nl2), t0, t1);
+        float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
         if (need_mask) {
           if (kb + 2 * c > lim) p0 = 0.f;
           if (kb + 2 * c + 1 > lim) p1 = 0.f;
         }
-        pk[c] = pack_f16(p0 * (dp[2 * c] - delta), p1 * (dp[2 * c + 1] - delta));
+        float d0, d1;
+        f2unpack(fmul2(f2pack(p0, p1), fsub2(f2pack(dp[2 * c], dp[2 * c + 1]), dd)), d0, d1);
+        pk[c] = pack_f16(d0, d1);
       }
       tmem_st32(tb, pk);
       tmem_wait_st();

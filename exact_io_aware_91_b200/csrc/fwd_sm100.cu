@@ -101,10 +101,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: heaviest units first under the causal mask
+  // ---- work unit: head-major (CTAs running together share K/V in L2), heaviest
+  // query tiles of each head first under the causal mask
   const int L_idx = blockIdx.x;
-  const int pair = p.causal ? (p.n_pairs - 1 - L_idx / p.BH) : (L_idx / p.BH);
-  const int bh = L_idx % p.BH;
+  const int bh = L_idx / p.n_pairs;
+  const int pair = p.causal ? (p.n_pairs - 1 - L_idx % p.n_pairs) : (L_idx % p.n_pairs);
   const int q_base0 = pair * 256;
   const int q_base1 = q_base0 + 128;
   const int n_kv = (p.N + 127) / 128;
@@ -139,15 +140,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ===================================================== TMA producer
-    if (lane == 0) {
+    {
+      const uint32_t leader = elect_one();  // the lane that issues async instructions
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_o);
-      mbar_arrive_expect_tx(bar(L::BAR_Q), 2 * L::TILE);
+      mbar_arrive_expect_tx(bar(L::BAR_Q), 2 * L::TILE, leader);
       for (int c = 0; c < L::KCH; ++c) {
-        tma_load_3d(base + L::OFF_Q0 + c * L::BOX, &tm_q, c * 64, q_base0, bh, bar(L::BAR_Q));
-        tma_load_3d(base + L::OFF_Q1 + c * L::BOX, &tm_q, c * 64, q_base1, bh, bar(L::BAR_Q));
+        tma_load_3d(base + L::OFF_Q0 + c * L::BOX, &tm_q, c * 64, q_base0, bh, bar(L::BAR_Q), leader);
+        tma_load_3d(base + L::OFF_Q1 + c * L::BOX, &tm_q, c * 64, q_base1, bh, bar(L::BAR_Q), leader);
       }
       int issued = 0;
       bool ok = true;
@@ -157,11 +159,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ph = (issued / L::STAGES) & 1;
           ok = mbar_wait(bar(L::BAR_KV_EMPTY + st), ph ^ 1u, wctx);
           if (!ok) break;
-          mbar_arrive_expect_tx(bar(L::BAR_KV_FULL + st), L::TILE);
+          mbar_arrive_expect_tx(bar(L::BAR_KV_FULL + st), L::TILE, leader);
           const CUtensorMap* m = which ? &tm_v : &tm_k;
           for (int c = 0; c < L::KCH; ++c)
             tma_load_3d(base + L::OFF_KV + st * L::TILE + c * L::BOX, m, c * 64, j * 128, bh,
-                        bar(L::BAR_KV_FULL + st));
+                        bar(L::BAR_KV_FULL + st), leader);
           ++issued;
         }
       }
@@ -173,27 +175,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ===================================================== MMA issuer
-    if (lane == 0) {
+    {
+      const uint32_t leader = elect_one();  // the lane that issues async instructions
       constexpr uint32_t idesc_qk = make_idesc(128, 128, true, false, false);
       constexpr uint32_t idesc_pv = make_idesc(128, D, false, false, true);  // fp16 P (TMEM) x fp16 V
       const uint32_t tS[2] = {tmem + L::T_S0, tmem + L::T_S1};
       const uint32_t tO[2] = {tmem + L::T_O0, tmem + L::T_O1};
       const uint32_t sQ[2] = {base + L::OFF_Q0, base + L::OFF_Q1};
 
-      auto issue_qk = [&](uint32_t d_tmem, uint32_t q_s, uint32_t k_s) {
+      // descriptors are built once; each MMA only adds a constant byte offset
+      const uint64_t dQ[2] = {make_sdesc_sw128(sQ[0], 16, 1024), make_sdesc_sw128(sQ[1], 16, 1024)};
+      const uint64_t dKV0 = make_sdesc_sw128(base + L::OFF_KV, 16, 1024);       // K-major (K tiles)
+      const uint64_t dV0 = make_sdesc_sw128(base + L::OFF_KV, L::BOX, 1024);    // MN-major (V tiles)
+      auto issue_qk = [&](uint32_t d_tmem, uint64_t q_desc, int stage) {
+        const uint64_t k_desc = sdesc_add(dKV0, stage * L::TILE);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * L::BOX + (k & 3) * 32;
-          mma_ss(d_tmem, make_sdesc_sw128(q_s + off, 16, 1024), make_sdesc_sw128(k_s + off, 16, 1024), idesc_qk,
-                 k > 0 ? 1u : 0u);
+          mma_ss(d_tmem, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, k > 0 ? 1u : 0u, leader);
         }
       };
-      auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_s, bool acc) {
+      auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, int stage, bool acc) {
+        const uint64_t v_desc = sdesc_add(dV0, stage * L::TILE);
 #pragma unroll
-        for (int k = 0; k < L::BN / 16; ++k) {
-          mma_ts(d_tmem, p_tmem + k * 8, make_sdesc_sw128(v_s + k * 2048, L::BOX, 1024), idesc_pv,
-                 (acc || k > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < L::BN / 16; ++k)
+          mma_ts(d_tmem, p_tmem + k * 8, sdesc_add(v_desc, k * 2048), idesc_pv, (acc || k > 0) ? 1u : 0u, leader);
       };
 
       bool ok = mbar_wait(bar(L::BAR_Q), 0, wctx);
@@ -202,30 +208,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n1 && ok; ++j) {
         const int iK = 2 * j, iV = 2 * j + 1;
         const int stK = iK % L::STAGES, stV = iV % L::STAGES;
-        const uint32_t sK = base + L::OFF_KV + stK * L::TILE;
-        const uint32_t sV = base + L::OFF_KV + stV * L::TILE;
         if (!(ok = mbar_wait(bar(L::BAR_KV_FULL + stK), (iK / L::STAGES) & 1, wctx))) break;
         tc_fence_after();
         if (j < n0) {
-          issue_qk(tS[0], sQ[0], sK);
-          mma_commit(bar(L::BAR_S_FULL + 0));
+          issue_qk(tS[0], dQ[0], stK);
+          mma_commit(bar(L::BAR_S_FULL + 0), leader);
         }
         if (j > 0) {  // O1 += P1 V_{j-1}
           if (!(ok = mbar_wait(bar(L::BAR_P_FULL + 1), (j - 1) & 1, wctx))) break;
           tc_fence_after();
-          issue_pv(tO[1], tS[1], base + L::OFF_KV + prev_v_stage * L::TILE, j - 1 > 0);
-          mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage));
+          issue_pv(tO[1], tS[1], prev_v_stage, j - 1 > 0);
+          mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage), leader);
         }
-        issue_qk(tS[1], sQ[1], sK);
-        mma_commit(bar(L::BAR_S_FULL + 1));
-        mma_commit(bar(L::BAR_KV_EMPTY + stK));
+        issue_qk(tS[1], dQ[1], stK);
+        mma_commit(bar(L::BAR_S_FULL + 1), leader);
+        mma_commit(bar(L::BAR_KV_EMPTY + stK), leader);
         if (!(ok = mbar_wait(bar(L::BAR_V_CONV + stV), (iV / L::STAGES) & 1, wctx))) break;
         tc_fence_after();
         if (j < n0) {  // O0 += P0 V_j
           if (!(ok = mbar_wait(bar(L::BAR_P_FULL + 0), j & 1, wctx))) break;
           tc_fence_after();
-          issue_pv(tO[0], tS[0], sV, j > 0);
-          if (j == n0 - 1) mma_commit(bar(L::BAR_O_FULL + 0));
+          issue_pv(tO[0], tS[0], stV, j > 0);
+          if (j == n0 - 1) mma_commit(bar(L::BAR_O_FULL + 0), leader);
         }
         prev_v_stage = stV;
       }
@@ -233,13 +237,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(bar(L::BAR_P_FULL + 1), (n1 - 1) & 1, wctx);
         if (ok) {
           tc_fence_after();
-          issue_pv(tO[1], tS[1], base + L::OFF_KV + prev_v_stage * L::TILE, n1 - 1 > 0);
-          mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage));
-          mma_commit(bar(L::BAR_O_FULL + 1));
+          issue_pv(tO[1], tS[1], prev_v_stage, n1 - 1 > 0);
+          mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage), leader);
+          mma_commit(bar(L::BAR_O_FULL + 1), leader);
         }
       }
       // every MMA issued so far has finished before TMEM is released
-      mma_commit(bar(L::BAR_MMA_DONE));
+      mma_commit(bar(L::BAR_MMA_DONE), leader);
       drain_wait(bar(L::BAR_MMA_DONE), 0);
     }
   } else if (warp == 2 || warp == 3) {
@@ -301,30 +305,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (kb + c > lim) x[c] = -INFINITY;
       }
-      float mx = x[0];
+      // row max: four independent 3-input max chains
+      float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      for (int c = 4; c < 124; c += 8) {
+        a0 = max3f(a0, x[c], x[c + 1]);
+        a1 = max3f(a1, x[c + 2], x[c + 3]);
+        a2 = max3f(a2, x[c + 4], x[c + 5]);
+        a3 = max3f(a3, x[c + 6], x[c + 7]);
+      }
+      a0 = max3f(a0, x[124], x[125]);
+      a1 = max3f(a1, x[126], x[127]);
+      const float mx = max3f(fmaxf(a0, a1), a2, a3);
       const float m_new = fmaxf(m, mx * sl2);
       // keep a stale maximum while it is within 2^8 of the true one: exact in the end
       // because O / l and the LSE use the same maximum
       const float m_use = (m_new - m > 8.0f) ? m_new : m;
       const float alpha = (m_use == m) ? 1.0f : ex2_approx(m - m_use);  // 0 on the first tile
       const float neg_m = -m_use;
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = ex2_approx(fmaf(x[c], sl2, neg_m));
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;  // sums of the fp16-rounded weights
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          pk[i] = pack_f16(x[64 * h + 2 * i], x[64 * h + 2 * i + 1]);
-          const float2 r = __half22float2(*reinterpret_cast<const __half2*>(&pk[i]));
-          sum += r.x + r.y;  // the weights P V really uses
+        for (int i = 0; i < 32; i += 2) {
+          float* e = &x[64 * h + 2 * i];
+          fma2(e[0], e[1], sl2, neg_m);
+          fma2(e[2], e[3], sl2, neg_m);
+          pk[i] = pack_f16(ex2_approx(e[0]), ex2_approx(e[1]));
+          pk[i + 1] = pack_f16(ex2_approx(e[2]), ex2_approx(e[3]));
+          add_f16x2_to_f32(s0, s1, pk[i]);
+          add_f16x2_to_f32(s2, s3, pk[i + 1]);
         }
         tmem_st32(tS + 32 * h, pk);
       }
-      l = fmaf(l, alpha, sum);
+      l = fmaf(l, alpha, (s0 + s1) + (s2 + s3));
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
         // the previous O += P V of this tile completed before S_j did (same issuing thread)
 #pragma unroll 1
