@@ -23,9 +23,7 @@
 //     bits) rather than bf16 (8) before the P V product;
 //   * warpgroups 1 and 2 (one per query tile, one thread per row) run the online
 //     softmax on S rows loaded from TMEM, write P back to TMEM as fp16 and, when
-//     the running maximum grows by more than 2^8, rescale O in TMEM; the row sum
-//     l adds up the fp16-rounded weights actually used in P V, so O = P V / l is
-//     an exact convex combination of the rounded weights;
+//     the running maximum grows by more than 2^8, rescale O in TMEM;
 //   * the epilogue divides by the row sum, converts to bf16 and TMA-stores O, and
 //     optionally writes the bf16 residual O_fp32 - O_bf16 so that the backward
 //     pass can form rowsum(dO * O) from an fp32-accurate O.
@@ -67,7 +65,17 @@ struct FwdLayout {
 };
 
 constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 2-3 V to fp16, warps 4-7 / 8-11 softmax
+// registers per thread: 168 at launch (65536 / 384, rounded down to a multiple of 8);
+// warpgroup 0 (TMA, MMA, V conversion) drops to 64, the softmax warpgroups rise to 216
+constexpr uint32_t kRegsLaunch = 168, kRegsLow = 64, kRegsHigh = 216;
+static_assert(kRegsLow + 2 * kRegsHigh <= 3 * kRegsLaunch, "register split exceeds the launch budget");
 constexpr int kConvThreads = 64;
+#ifndef FA_EXP_FMA_PER8
+#define FA_EXP_FMA_PER8 0
+#endif
+// element pairs out of every 8 whose exponentials run on the FMA pipe (even, 0..8)
+constexpr int kExpFmaPer8 = FA_EXP_FMA_PER8;
+static_assert(kExpFmaPer8 % 2 == 0 && kExpFmaPer8 >= 0 && kExpFmaPer8 <= 8, "pairs are taken two at a time");
 static_assert(FwdLayout<128>::STAGES % 2 == 0 && FwdLayout<64>::STAGES % 2 == 0,
               "K and V tiles must alternate over fixed ring stages");
 
@@ -140,6 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ===================================================== TMA producer
+    regs_dec<kRegsLow>();
     {
       const uint32_t leader = elect_one();  // the lane that issues async instructions
       prefetch_tmap(&tm_q);
@@ -175,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ===================================================== MMA issuer
+    regs_dec<kRegsLow>();
     {
       const uint32_t leader = elect_one();  // the lane that issues async instructions
       constexpr uint32_t idesc_qk = make_idesc(128, 128, true, false, false);
@@ -248,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2 || warp == 3) {
     // ===================================================== V tiles: bf16 -> fp16 in place
+    regs_dec<kRegsLow>();
     const int ct = threadIdx.x - 64;  // 0..63
     bool ok = true;
     for (int j = 0; j < n1 && ok; ++j) {
@@ -271,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // ===================================================== softmax warpgroups
+    regs_inc<kRegsHigh>();
     const int t = (warp - 4) >> 2;        // query tile handled by this warpgroup
     const int wq = (warp - 4) & 3;        // TMEM lane quarter
     const int row = wq * 32 + lane;       // row inside the tile
@@ -323,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_use = (m_new - m > 8.0f) ? m_new : m;
       const float alpha = (m_use == m) ? 1.0f : ex2_approx(m - m_use);  // 0 on the first tile
       const float neg_m = -m_use;
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;  // sums of the fp16-rounded weights
+      uint64_t sa = 0, sb = 0;  // packed fp32 partial row sums (0.0f, 0.0f)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
@@ -332,13 +344,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           float* e = &x[64 * h + 2 * i];
           fma2(e[0], e[1], sl2, neg_m);
           fma2(e[2], e[3], sl2, neg_m);
-          pk[i] = pack_f16(ex2_approx(e[0]), ex2_approx(e[1]));
-          pk[i + 1] = pack_f16(ex2_approx(e[2]), ex2_approx(e[3]));
-          add_f16x2_to_f32(s0, s1, pk[i]);
-          add_f16x2_to_f32(s2, s3, pk[i + 1]);
+          // kExpFmaPer8 of every 8 element pairs take 2^x on the FMA pipe, the rest on MUFU
+          if ((i & 7) < 2 * (kExpFmaPer8 / 2)) {
+            exp2_fma_pipe(e[0], e[1]);
+            exp2_fma_pipe(e[2], e[3]);
+            pk[i] = pack_f16(e[0], e[1]);
+            pk[i + 1] = pack_f16(e[2], e[3]);
+          } else {
+            e[0] = ex2_approx(e[0]);
+            e[1] = ex2_approx(e[1]);
+            e[2] = ex2_approx(e[2]);
+            e[3] = ex2_approx(e[3]);
+            pk[i] = pack_f16(e[0], e[1]);
+            pk[i + 1] = pack_f16(e[2], e[3]);
+          }
+          asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sa) : "l"(f2pack(e[0], e[1])));
+          asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sb) : "l"(f2pack(e[2], e[3])));
         }
         tmem_st32(tS + 32 * h, pk);
       }
+      float s0, s1, s2, s3;
+      f2unpack(sa, s0, s1);
+      f2unpack(sb, s2, s3);
       l = fmaf(l, alpha, (s0 + s1) + (s2 + s3));
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
         // the previous O += P V of this tile completed before S_j did (same issuing thread)

@@ -78,7 +78,7 @@ typedef enum {
  * Q K^T is a bf16 product with fp32 accumulation; the probabilities are rounded
  * to fp16 (round to nearest even) for the P V product, whose V operand is an
  * exact fp16 copy of the bf16 V made on chip (|V| must stay below 65504); the row
- * sums add up those rounded probabilities; O is rounded to bf16 once at the end.
+ * sums are fp32; O is rounded to bf16 once at the end.
  * Returns FA_OK once the kernel is enqueued.
  */
 FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B,
