@@ -238,16 +238,11 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     return FA_ERR_CUDA;
 
   const CUtensorMapDataType h = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  CUtensorMap a_q, a_do, a_k, a_v;  // dK/dV kernel: 64-row Q/dO tiles, 128-row K/V tiles
-  CUtensorMap b_q, b_do, b_k, b_v;  // dQ kernel: 128-row Q/dO tiles, 64-row K/V tiles
-  if (!make_tmap_3d(&a_q, pp.q16, h, 2, d, N, BH, 64, 64, true) ||
-      !make_tmap_3d(&a_do, pp.do16, h, 2, d, N, BH, 64, 64, true) ||
-      !make_tmap_3d(&a_k, pp.k16, h, 2, d, N, BH, 64, 128, true) ||
-      !make_tmap_3d(&a_v, pp.v16, h, 2, d, N, BH, 64, 128, true) ||
-      !make_tmap_3d(&b_q, pp.q16, h, 2, d, N, BH, 64, 128, true) ||
-      !make_tmap_3d(&b_do, pp.do16, h, 2, d, N, BH, 64, 128, true) ||
-      !make_tmap_3d(&b_k, pp.k16, h, 2, d, N, BH, 64, 64, true) ||
-      !make_tmap_3d(&b_v, pp.v16, h, 2, d, N, BH, 64, 64, true))
+  CUtensorMap t_q, t_do, t_k, t_v;  // 128-row boxes, shared by the dK/dV and dQ kernels
+  if (!make_tmap_3d(&t_q, pp.q16, h, 2, d, N, BH, 64, 128, true) ||
+      !make_tmap_3d(&t_do, pp.do16, h, 2, d, N, BH, 64, 128, true) ||
+      !make_tmap_3d(&t_k, pp.k16, h, 2, d, N, BH, 64, 128, true) ||
+      !make_tmap_3d(&t_v, pp.v16, h, 2, d, N, BH, 64, 128, true))
     return FA_ERR_CUDA;
   BwdParams bp{};
   bp.delta = pp.delta;
@@ -262,11 +257,11 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   bp.scale_log2 = scale * 1.4426950408889634f;
   bp.causal = causal;
   bp.err = g_err_ptr[dev];
-  if (launch_bwd_dkdv_sm100(a_q, a_do, a_k, a_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_dkdv_sm100(t_q, t_do, t_k, t_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
   if (t_phase_events != nullptr && t_phase_events[1] != nullptr &&
       cudaEventRecord(static_cast<cudaEvent_t>(t_phase_events[1]), s) != cudaSuccess)
     return FA_ERR_CUDA;
-  if (launch_bwd_dq_sm100(b_q, b_do, b_k, b_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_dq_sm100(t_q, t_do, t_k, t_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
 }
 
