@@ -37,6 +37,27 @@ METRIC = "attention fwd/bwd TFLOPS (BF16, causal, N=8k, d=128) & % of B200 tenso
 WORKLOAD = 3  # the metric's workload; --workload picks another one for profiling only
 
 
+def recorded_traffic(kernel: str, workload_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    import hashlib
+
+    short = {"causal_b2_h32_n8192_d128_spiky": "causal_b2_h32_n8192_d128"}.get(workload_name)
+    if short is None:
+        return None
+    path = os.path.join(ROOT, "profiles", f"traffic_{short}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "exact_io_aware_91_b200", "csrc", rec["source"])
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+            return None  # the kernel changed since the counters were taken
+    return rec["bytes"]
+
+
 def load_peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -283,7 +304,8 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     achieved = algo[dom] / (mean[dom] * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": args.traffic,
+                "frac": achieved / peak,
+                "traffic": args.traffic if args.traffic is not None else recorded_traffic(dom, w.name),
                 "peak_kind": f"{peaks['source']} bf16 dense matmul, sustained (kernel timed inside a long step)"}
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
