@@ -146,11 +146,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wctx{abort_flag, p.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // head-major order (CTAs running together share Q / dO in L2); within a head the
-  // key tiles with the most work under the causal mask (small j) come first
+  // heaviest first within groups of heads (see unit_order): under the causal mask the
+  // first key tiles of a head meet the most query tiles
   const int n_kt = (p.N + 127) / 128;
-  const int bh = blockIdx.x / n_kt;
-  const int j = blockIdx.x % n_kt;  // key tile
+  int bh, j;  // head, key tile
+  unit_order((int)blockIdx.x, n_kt, p.BH, p.head_group, bh, j);
   const int i_start = p.causal ? j : 0;
   const int n_it = n_kt - i_start;  // 128-query steps, >= 1
 
@@ -409,10 +409,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wctx{abort_flag, p.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // head-major order; within a head the query tiles with the most work come first
+  // heaviest first within groups of heads (see unit_order): under the causal mask the
+  // last query tiles of a head meet the most key tiles
   const int nq = (p.N + 127) / 128;
-  const int bh = blockIdx.x / nq;
-  const int qt = p.causal ? (nq - 1 - (int)(blockIdx.x % nq)) : (int)(blockIdx.x % nq);
+  int bh, rank;
+  unit_order((int)blockIdx.x, nq, p.BH, p.head_group, bh, rank);
+  const int qt = p.causal ? (nq - 1 - rank) : rank;
   const int n_it = p.causal ? qt + 1 : nq;  // 128-key steps
 
   if (threadIdx.x == 0) {

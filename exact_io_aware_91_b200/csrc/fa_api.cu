@@ -166,6 +166,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.N = N;
   p.BH = BH;
   p.n_pairs = (N + 255) / 256;
+  p.head_group = head_group_size(BH, N, d, kFwdGroupBytes);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal;
   p.err = g_err_ptr[dev];
@@ -253,6 +254,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   bp.N = N;
   bp.Np = w.Np;
   bp.BH = BH;
+  bp.head_group = head_group_size(BH, N, d, kBwdGroupBytes);
   bp.scale = scale;
   bp.scale_log2 = scale * 1.4426950408889634f;
   bp.causal = causal;

@@ -14,6 +14,7 @@ struct FwdParams {
   int N;             // sequence length (queries = keys)
   int BH;            // B * H
   int n_pairs;       // ceil(N / 256): work units per head (two 128-row query tiles each)
+  int head_group;    // heads per group in the CTA order (unit_order)
   float scale_log2;  // softmax scale * log2(e)
   int causal;
   int* err;          // device error word
@@ -43,6 +44,7 @@ struct BwdParams {
   float* dk;
   float* dv;
   int N, Np, BH;
+  int head_group;      // heads per group in the CTA order (unit_order)
   float scale;         // softmax scale (applied to dQ and dK)
   float scale_log2;    // scale * log2(e)
   int causal;
@@ -51,6 +53,19 @@ struct BwdParams {
 
 // Tensor maps are 3-D views (d, N, B*H) of a (B, H, N, d) tensor with the
 // 128-byte swizzle and a box of 64 columns x `box_rows` rows.
+// Heads per group in the CTA order: as many heads as keep the streamed operand pair
+// (K and V in the forward and dQ kernels, Q and dO in the dK/dV kernel; 4 * N * d bytes
+// per head) within `budget` bytes of L2.  Measured on B200 (N = 2048 and 8192, d = 128):
+// the forward runs best with 16 MB groups, the backward with 8 MB.
+constexpr unsigned long long kFwdGroupBytes = 16ull << 20;
+constexpr unsigned long long kBwdGroupBytes = 8ull << 20;
+inline int head_group_size(int BH, int N, int d, unsigned long long budget) {
+  const unsigned long long per_head = 4ull * (unsigned long long)N * (unsigned long long)d;
+  unsigned long long g = budget / (per_head ? per_head : 1ull);
+  if (g < 1ull) g = 1ull;
+  return g > (unsigned long long)BH ? BH : (int)g;
+}
+
 bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
                   int box_cols, int box_rows, bool swizzle128);
 

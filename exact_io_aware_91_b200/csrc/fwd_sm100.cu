@@ -45,14 +45,16 @@ struct FwdLayout {
   static constexpr int OFF_Q1 = TILE;
   static constexpr int OFF_KV = 2 * TILE;
   static constexpr int OFF_BAR = OFF_KV + STAGES * TILE;
-  // barriers: q_full, kv_full[STAGES], kv_empty[STAGES], v_conv[STAGES], s_full[2], p_full[2],
-  // o_full[2], mma_done
+  // barriers: q_full, kv_full[STAGES], kv_empty[STAGES], v_conv[STAGES], s_full[2], p_half[2],
+  // p_full[2], o_full[2], mma_done
   static constexpr int BAR_Q = 0;
   static constexpr int BAR_KV_FULL = 1;
   static constexpr int BAR_KV_EMPTY = 1 + STAGES;
   static constexpr int BAR_V_CONV = 1 + 2 * STAGES;
   static constexpr int BAR_S_FULL = 1 + 3 * STAGES;
-  static constexpr int BAR_P_FULL = BAR_S_FULL + 2;
+  static constexpr int BAR_P_HALF = BAR_S_FULL + 2;  // P for keys 0..63 of the tile is in TMEM
+  static constexpr int BAR_P_FULL = BAR_P_HALF + 2;
+  static_assert(BAR_P_FULL == BAR_P_HALF + 2, "the softmax arrives on BAR_P_HALF + t + 2 * half");
   static constexpr int BAR_O_FULL = BAR_P_FULL + 2;
   static constexpr int BAR_MMA_DONE = BAR_O_FULL + 2;
   static constexpr int NBAR = BAR_MMA_DONE + 1;
@@ -109,11 +111,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: head-major (CTAs running together share K/V in L2), heaviest
-  // query tiles of each head first under the causal mask
-  const int L_idx = blockIdx.x;
-  const int bh = L_idx / p.n_pairs;
-  const int pair = p.causal ? (p.n_pairs - 1 - L_idx % p.n_pairs) : (L_idx % p.n_pairs);
+  // ---- work unit: heaviest first within groups of heads (see unit_order); under the
+  // causal mask the last query tiles of a head carry the most work
+  int bh, rank;
+  unit_order((int)blockIdx.x, p.n_pairs, p.BH, p.head_group, bh, rank);
+  const int pair = p.causal ? (p.n_pairs - 1 - rank) : rank;
   const int q_base0 = pair * 256;
   const int q_base1 = q_base0 + 128;
   const int n_kv = (p.N + 127) / 128;
@@ -131,6 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::BAR_S_FULL + t), 1);
+      mbar_init(bar(L::BAR_P_HALF + t), 128);
       mbar_init(bar(L::BAR_P_FULL + t), 128);
       mbar_init(bar(L::BAR_O_FULL + t), 1);
     }
@@ -205,11 +208,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(d_tmem, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, k > 0 ? 1u : 0u, leader);
         }
       };
-      auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, int stage, bool acc) {
+      // O += P V over keys [64 * part, 64 * part + 64) of the tile
+      auto issue_pv_half = [&](uint32_t d_tmem, uint32_t p_tmem, int stage, bool acc, int part) {
         const uint64_t v_desc = sdesc_add(dV0, stage * L::TILE);
 #pragma unroll
-        for (int k = 0; k < L::BN / 16; ++k)
+        for (int kk = 0; kk < L::BN / 32; ++kk) {
+          const int k = part * (L::BN / 32) + kk;
           mma_ts(d_tmem, p_tmem + k * 8, sdesc_add(v_desc, k * 2048), idesc_pv, (acc || k > 0) ? 1u : 0u, leader);
+        }
+      };
+      // the first half of the product starts while the softmax still computes the second half of P
+      auto issue_pv = [&](int t, uint32_t d_tmem, uint32_t p_tmem, int stage, bool acc, uint32_t parity) -> bool {
+        if (!mbar_wait(bar(L::BAR_P_HALF + t), parity, wctx)) return false;
+        tc_fence_after();
+        issue_pv_half(d_tmem, p_tmem, stage, acc, 0);
+        if (!mbar_wait(bar(L::BAR_P_FULL + t), parity, wctx)) return false;
+        tc_fence_after();
+        issue_pv_half(d_tmem, p_tmem, stage, acc, 1);
+        return true;
       };
 
       bool ok = mbar_wait(bar(L::BAR_Q), 0, wctx);
@@ -225,9 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(bar(L::BAR_S_FULL + 0), leader);
         }
         if (j > 0) {  // O1 += P1 V_{j-1}
-          if (!(ok = mbar_wait(bar(L::BAR_P_FULL + 1), (j - 1) & 1, wctx))) break;
-          tc_fence_after();
-          issue_pv(tO[1], tS[1], prev_v_stage, j - 1 > 0);
+          if (!(ok = issue_pv(1, tO[1], tS[1], prev_v_stage, j - 1 > 0, (j - 1) & 1))) break;
           mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage), leader);
         }
         issue_qk(tS[1], dQ[1], stK);
@@ -236,18 +250,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(bar(L::BAR_V_CONV + stV), (iV / L::STAGES) & 1, wctx))) break;
         tc_fence_after();
         if (j < n0) {  // O0 += P0 V_j
-          if (!(ok = mbar_wait(bar(L::BAR_P_FULL + 0), j & 1, wctx))) break;
-          tc_fence_after();
-          issue_pv(tO[0], tS[0], stV, j > 0);
+          if (!(ok = issue_pv(0, tO[0], tS[0], stV, j > 0, j & 1))) break;
           if (j == n0 - 1) mma_commit(bar(L::BAR_O_FULL + 0), leader);
         }
         prev_v_stage = stV;
       }
       if (ok) {  // O1 += P1 V_{n1-1}
-        ok = mbar_wait(bar(L::BAR_P_FULL + 1), (n1 - 1) & 1, wctx);
+        ok = issue_pv(1, tO[1], tS[1], prev_v_stage, n1 - 1 > 0, (n1 - 1) & 1);
         if (ok) {
-          tc_fence_after();
-          issue_pv(tO[1], tS[1], prev_v_stage, n1 - 1 > 0);
           mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage), leader);
           mma_commit(bar(L::BAR_O_FULL + 1), leader);
         }
@@ -301,13 +311,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = mbar_wait(bar(L::BAR_S_FULL + t), j & 1, wctx))) break;
       tc_fence_after();
       float x[128];
+      {
+        uint32_t u[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t u[32];
-        tmem_ld32(tS + 32 * c, u);
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, u[c]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(u[i]);
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(u[c][i]);
       }
       const int kb = j * 128;
       const bool need_mask = (p.causal && kb + 127 > q_base) || (kb + 128 > p.N);
@@ -335,6 +347,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_use = (m_new - m > 8.0f) ? m_new : m;
       const float alpha = (m_use == m) ? 1.0f : ex2_approx(m - m_use);  // 0 on the first tile
       const float neg_m = -m_use;
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        // rescale O before this tile's P V starts; the previous O += P V of this tile
+        // completed before S_j did (same issuing thread, in-order tensor pipe)
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld32(tO + 32 * c, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          tmem_st32(tO + 32 * c, u);
+        }
+      }
       uint64_t sa = 0, sb = 0;  // packed fp32 partial row sums (0.0f, 0.0f)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -362,26 +387,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sb) : "l"(f2pack(e[2], e[3])));
         }
         tmem_st32(tS + 32 * h, pk);
+        // first half of P (and any rescale of O) visible to the tensor core: its half of P V
+        // can start while the second half is computed
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::BAR_P_HALF + t + 2 * h));  // BAR_P_FULL = BAR_P_HALF + 2
       }
       float s0, s1, s2, s3;
       f2unpack(sa, s0, s1);
       f2unpack(sb, s2, s3);
       l = fmaf(l, alpha, (s0 + s1) + (s2 + s3));
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        // the previous O += P V of this tile completed before S_j did (same issuing thread)
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld32(tO + 32 * c, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st32(tO + 32 * c, u);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(L::BAR_P_FULL + t));
       m = m_use;
     }
     // ---- epilogue: O / l -> bf16 -> swizzled staging (the Q tile's buffer) -> TMA store

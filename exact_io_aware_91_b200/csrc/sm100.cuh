@@ -111,6 +111,23 @@ __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// ----------------------------------------------------------------- work order
+// CTA index -> (head, rank) where rank 0 is the unit with the most work.  Heads are taken
+// in groups of `group`; inside a group the units go heaviest first, interleaved over the
+// group's heads.  The hardware hands out CTAs roughly in index order, so the lightest units
+// of each group come last (short tail), while the CTAs resident at any time read the K/V
+// (or Q/dO) of one group of heads, sized by the host to stay in L2.  group = 1 is plain
+// head-major order.
+__device__ __forceinline__ void unit_order(int cta, int per_head, int n_heads, int group, int& head, int& rank) {
+  const int per_group = group * per_head;
+  const int g = cta / per_group;
+  const int g0 = g * group;
+  const int gs = min(group, n_heads - g0);  // heads in this group (the last may be smaller)
+  const int r = cta - g * per_group;        // every earlier group is full
+  rank = r / gs;
+  head = g0 + r % gs;
+}
+
 // ----------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -330,21 +347,20 @@ __device__ __forceinline__ void add_f16x2_to_f32(float& s0, float& s1, uint32_t 
       : "+f"(s0), "+f"(s1)
       : "r"(h));
 }
-// 2^x for a pair of values on the FMA pipe instead of the MUFU unit (which is the
-// softmax's throughput limit on sm_100a).  Method: round-to-nearest range
-// reduction x = j + f, j integer, f in [-1/2, 1/2] (the 1.5 * 2^23 shifter trick:
-// adding it leaves round(x) in the low mantissa bits), 2^f by a degree-4 polynomial
-// fitted here for minimum relative error on [-1/2, 1/2] (max relative error
-// 2.7e-6 in fp32 Horner form, far below the fp16 rounding P gets next), and 2^j
+// 2^x for a pair of values on the FMA pipe instead of the MUFU unit (16 exponentials
+// per clock per SM, the softmax's throughput limit on sm_100a).  Method: round-to-
+// nearest range reduction x = j + f, j integer, f in [-1/2, 1/2] (adding 1.5 * 2^23
+// leaves round(x) in the low mantissa bits), 2^f by a degree-3 polynomial fitted for
+// minimum relative error on [-1/2, 1/2] (max relative error 7.5e-5 in fp32 Horner form,
+// below the 2^-11 rounding that P gets next when it is packed to fp16), and 2^j
 // applied by adding j to the exponent field.  Inputs are clamped to >= -126 so the
 // scaled result stays a normal float (2^-126 becomes 0 once rounded to fp16); the
 // largest input the softmax produces is 8 (a stale running maximum).
 constexpr float kExp2Shifter = 12582912.0f;  // 1.5 * 2^23
-constexpr float kExp2C0 = 0.9999992847442627f;
-constexpr float kExp2C1 = 0.6931217908859253f;
-constexpr float kExp2C2 = 0.240247443318367f;
-constexpr float kExp2C3 = 0.05591786280274391f;
-constexpr float kExp2C4 = 0.009570101276040077f;
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111400127411f;
+constexpr float kExp2C3 = 0.0551716685295105f;
 __device__ __forceinline__ void exp2_fma_pipe(float& a, float& b) {
   a = fmaxf(a, -126.0f);
   b = fmaxf(b, -126.0f);
@@ -355,8 +371,7 @@ __device__ __forceinline__ void exp2_fma_pipe(float& a, float& b) {
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(t), "l"(shifter));
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(f));
   auto splat = [](float c) { return ((uint64_t)__float_as_uint(c) << 32) | __float_as_uint(c); };
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(splat(kExp2C4)), "l"(f), "l"(splat(kExp2C3)));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(splat(kExp2C2)));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(splat(kExp2C3)), "l"(f), "l"(splat(kExp2C2)));
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(splat(kExp2C1)));
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(splat(kExp2C0)));
   float p0, p1, t0, t1;
@@ -365,7 +380,6 @@ __device__ __forceinline__ void exp2_fma_pipe(float& a, float& b) {
   a = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
   b = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
-
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
