@@ -18,4 +18,7 @@ from .attention import (  # noqa: F401
     online_softmax_forward,
     loop_attention_forward,
     loop_attention_backward,
+    kv_head_of,
+    attention_forward_gqa,
+    attention_backward_gqa,
 )

@@ -31,6 +31,15 @@ Sources (titles of the web pages this method is described on):
 LSE (the per-row log-sum-exp that the forward saves for the backward) is the
 natural log of the row sum of exp of the scaled, masked scores.
 
+Grouped-query and multi-query attention ("Flash Attention: Ako transformery
+zvladaju miliony tokenov", section "5. Limity a co dalej", and "FlashAttention
+(EL)", the closing list of extensions, name GQA/MQA support without defining
+it).  Reading taken: H query heads share H_kv key/value heads (H a multiple of
+H_kv; H_kv = 1 is MQA), query head h reads key/value head h // (H / H_kv) --
+consecutive query heads form a group -- and each head's attention is the
+definition above.  The gradients of a shared K or V are the sums of the
+per-query-head gradients over its group (the chain rule through the sharing).
+
 Parity pins: every function here is pinned by ``tests/test_oracle.py``
 (closed forms, invariants, finite differences, a hand-computed worked example,
 a library special case and a brute-force loop restatement).
@@ -50,6 +59,9 @@ __all__ = [
     "online_softmax_forward",
     "loop_attention_forward",
     "loop_attention_backward",
+    "kv_head_of",
+    "attention_forward_gqa",
+    "attention_backward_gqa",
 ]
 
 
@@ -287,3 +299,65 @@ def loop_attention_backward(q, k, v, do, scale: float, causal: bool):
                 dQ[i][c] += scale * ds * kf[j][c]
                 dK[j][c] += scale * ds * qf[i][c]
     return np.array(dQ), np.array(dK), np.array(dV)
+
+
+# ---------------------------------------------------------------- grouped-query attention
+def kv_head_of(h: int, n_heads: int, n_kv_heads: int) -> int:
+    """Key/value head read by query head h: consecutive groups of H / H_kv query heads."""
+    return h // (n_heads // n_kv_heads)
+
+
+def _check_gqa_shapes(q, k, v):
+    if q.ndim != 4 or k.ndim != 4 or v.ndim != 4:
+        raise ValueError("grouped-query attention takes (B, H, N, d) arrays")
+    B, H, N, _ = q.shape
+    if k.shape[:3] != (B, k.shape[1], N) or v.shape[:3] != k.shape[:3] or k.shape[1] == 0 or H % k.shape[1]:
+        raise ValueError("K and V need (B, H_kv, N, .) with H a multiple of H_kv")
+
+
+def attention_forward_gqa(q, k, v, scale: float, causal: bool):
+    """O and LSE of grouped-query attention, one query head at a time.
+
+    q: (B, H, N, d); k, v: (B, H_kv, N, d).  Returns O (B, H, N, d_v), LSE (B, H, N).
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    _check_gqa_shapes(q, k, v)
+    B, H, N, _ = q.shape
+    Hkv = k.shape[1]
+    O = np.empty((B, H, N, v.shape[3]))
+    L = np.empty((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            g = kv_head_of(h, H, Hkv)
+            s = _scores(q[b, h], k[b, g], scale, causal)
+            lse = _lse_rows(s)
+            O[b, h] = np.exp(s - lse[:, None]) @ v[b, g]
+            L[b, h] = lse
+    return O, L
+
+
+def attention_backward_gqa(q, k, v, do, scale: float, causal: bool):
+    """dQ (B, H, N, d), dK and dV (B, H_kv, N, d) of L = sum(O * dO) for grouped-query attention.
+
+    Per query head the gradients are those of the plain definition (see
+    ``attention_backward``); a shared key/value head accumulates the dK and dV of
+    every query head of its group.
+    """
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    _check_gqa_shapes(q, k, v)
+    B, H, N, _ = q.shape
+    Hkv = k.shape[1]
+    dq = np.empty_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            g = kv_head_of(h, H, Hkv)
+            s = _scores(q[b, h], k[b, g], scale, causal)
+            p = np.exp(s - _lse_rows(s)[:, None])
+            dp = do[b, h] @ v[b, g].T
+            ds = p * (dp - np.sum(p * dp, axis=-1)[:, None])
+            dq[b, h] = scale * (ds @ k[b, g])
+            dk[b, g] += scale * (ds.T @ q[b, h])
+            dv[b, g] += p.T @ do[b, h]
+    return dq, dk, dv

@@ -18,6 +18,8 @@ import oracle
 import oracle.attention as oa
 from oracle import (
     attention_backward,
+    attention_backward_gqa,
+    attention_forward_gqa,
     attention_forward,
     attention_forward_rows,
     attention_probs,
@@ -292,3 +294,88 @@ def test_pins_catch_planted_mistakes(monkeypatch, name, attr, bad):
     assert _pins_pass(), "pins must pass on the unmodified oracle"
     monkeypatch.setattr(oa, attr, bad)
     assert not _pins_pass(), f"planted mistake not caught: {name}"
+
+
+# ---------------------------------------------------------------- grouped-query attention
+def _cumulative_mean(v):
+    """Row i: mean of rows 0..i (the closed form of causal attention with zero queries)."""
+    return np.cumsum(v, axis=-2) / np.arange(1, v.shape[-2] + 1)[:, None]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (6, 1), (6, 3)])
+def test_gqa_zero_queries_average_their_group_values(causal, H, Hkv):
+    # Q = 0: every score is 0, so query head h averages the visible rows of V[h // (H / Hkv)]
+    B, N, d = 2, 13, 5
+    q = np.zeros((B, H, N, d))
+    k, v = randn((B, Hkv, N, d), 60), randn((B, Hkv, N, d), 61)
+    O, L = attention_forward_gqa(q, k, v, 0.5, causal)
+    for h in range(H):
+        g = h // (H // Hkv)
+        want = _cumulative_mean(v[:, g]) if causal else np.broadcast_to(v[:, g].mean(-2, keepdims=True), (B, N, d))
+        np.testing.assert_allclose(O[:, h], want, atol=1e-13)
+        want_l = np.log(np.arange(1, N + 1)) if causal else np.full(N, math.log(N))
+        np.testing.assert_allclose(L[:, h], np.broadcast_to(want_l, (B, N)), atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("H,Hkv", [(4, 1), (4, 2), (6, 3), (3, 3)])
+def test_gqa_agrees_with_torch_sdpa_enable_gqa_fp64(causal, H, Hkv):
+    torch = pytest.importorskip("torch")
+    import torch.nn.functional as F
+
+    q, do = randn((2, H, 23, 8), 62), randn((2, H, 23, 8), 63)
+    k, v = randn((2, Hkv, 23, 8), 64), randn((2, Hkv, 23, 8), 65)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    out = F.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=0.3, enable_gqa=True)
+    out.backward(torch.tensor(do))
+    O, _ = attention_forward_gqa(q, k, v, 0.3, causal)
+    np.testing.assert_allclose(O, out.detach().numpy(), atol=1e-10)
+    dq, dk, dv = attention_backward_gqa(q, k, v, do, 0.3, causal)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-10)
+
+
+def _gqa_loss(q, k, v, do, scale, causal):
+    O, _ = attention_forward_gqa(q, k, v, scale, causal)
+    return float(np.sum(O * do))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_backward_matches_central_finite_differences(causal):
+    q, do = randn((1, 4, 5, 3), 66), randn((1, 4, 5, 3), 67)
+    k, v = randn((1, 2, 5, 3), 68), randn((1, 2, 5, 3), 69)
+    scale = 0.7
+    grads = attention_backward_gqa(q, k, v, do, scale, causal)
+    h = 1e-6
+    for which, g in zip(range(3), grads):
+        args = [q, k, v]
+        num = np.zeros_like(args[which])
+        for idx in np.ndindex(args[which].shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            num[idx] = (_gqa_loss(*plus, do, scale, causal) - _gqa_loss(*minus, do, scale, causal)) / (2 * h)
+        err = np.max(np.abs(num - g)) / max(1.0, np.max(np.abs(g)))
+        assert err <= 1e-6, (which, err)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_backward_invariants(causal):
+    H, Hkv = 6, 2
+    q, do = randn((2, H, 19, 7), 70), randn((2, H, 19, 7), 71)
+    k, v = randn((2, Hkv, 19, 7), 72), randn((2, Hkv, 19, 7), 73)
+    dq, dk, dv = attention_backward_gqa(q, k, v, do, 0.4, causal)
+    # rows of each head's dS sum to zero; rows of its P sum to one
+    np.testing.assert_allclose(dk.sum(-2), 0.0, atol=1e-11)
+    group_do = do.reshape(2, Hkv, H // Hkv, 19, 7).sum(axis=(2, 3))
+    np.testing.assert_allclose(dv.sum(-2), group_do, atol=1e-11)
+
+
+def test_gqa_pin_catches_a_wrong_group_mapping(monkeypatch):
+    # interleaved groups (h % H_kv) instead of consecutive ones
+    monkeypatch.setattr(oa, "kv_head_of", lambda h, n_heads, n_kv_heads: h % n_kv_heads)
+    with pytest.raises(AssertionError):
+        test_gqa_zero_queries_average_their_group_values(True, 4, 2)
