@@ -38,6 +38,12 @@ constexpr uint32_t kRegsLaunch = 168, kRegsLow = 64, kRegsHigh = 216;
 static_assert(kRegsLow + 2 * kRegsHigh <= 3 * kRegsLaunch, "register split exceeds the launch budget");
 
 constexpr int kBox = 128 * 128;  // one 64-column x 128-row fp16 box (16 KB)
+#ifndef FA_DKDV_EXP_FMA_PER16
+#define FA_DKDV_EXP_FMA_PER16 8
+#endif
+// exponentials out of every 16 of the dK/dV kernel's P^T that run on the FMA pipe (multiple of 4)
+constexpr int kDkdvExpFmaPer16 = FA_DKDV_EXP_FMA_PER16;
+static_assert(kDkdvExpFmaPer16 % 4 == 0 && kDkdvExpFmaPer16 >= 0 && kDkdvExpFmaPer16 <= 16, "groups of four");
 
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   uint64_t t0 = globaltimer_ns();
@@ -68,6 +74,19 @@ __device__ __forceinline__ void issue_ts_split(uint32_t d_tmem, uint32_t a_regio
   for (int k = 0; k < 8; ++k) {
     const uint32_t a = a_region + (k < 4 ? 8 * k : 64 + 8 * (k - 4));
     mma_ts(d_tmem, a, sdesc_add(b_desc, k * 2048), idesc, (acc || k > 0) ? 1u : 0u, issue);
+  }
+}
+
+// Half of the TS product above: part 0 takes K rows {0..31, 64..95} (the first 32 columns
+// each compute warpgroup writes), part 1 the rest.  `first` marks the product's first MMA
+// (which overwrites D).
+__device__ __forceinline__ void issue_ts_split_part(uint32_t d_tmem, uint32_t a_region, uint64_t b_desc,
+                                                    uint32_t idesc, bool first, int part, uint32_t issue) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int k = (i & 1) + 2 * part + 4 * (i >> 1);  // part 0: 0 1 4 5, part 1: 2 3 6 7
+    const uint32_t a = a_region + (k < 4 ? 8 * k : 64 + 8 * (k - 4));
+    mma_ts(d_tmem, a, sdesc_add(b_desc, k * 2048), idesc, (first && i == 0) ? 0u : 1u, issue);
   }
 }
 
@@ -123,7 +142,8 @@ struct DkdvLayout {
   static constexpr int BAR_DS_READY = 12;
   static constexpr int BAR_ACC = 13;
   static constexpr int BAR_DONE = 14;
-  static constexpr int NBAR = 15;
+  static constexpr int BAR_P_HALF = 15;   // first 32 of each warpgroup's 64 P^T columns written
+  static constexpr int NBAR = 16;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
   static constexpr int SMEM_ALLOC = OFF_ABORT + 8 + 1024;
@@ -166,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(L::BAR_S), 1);
     mbar_init(bar(L::BAR_DP), 1);
     mbar_init(bar(L::BAR_P_READY), 256);
+    mbar_init(bar(L::BAR_P_HALF), 256);
     mbar_init(bar(L::BAR_DS_READY), 256);
     mbar_init(bar(L::BAR_ACC), 1);
     mbar_init(bar(L::BAR_DONE), 1);
@@ -246,9 +267,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int it = 0; it < n_it && ok; ++it) {
       const int s = it & 1;
       const uint32_t so = s * L::TILE;
+      // dV += P^T dO in two halves: the first starts while the second half of P^T is computed
+      if (!(ok = mbar_wait(bar(L::BAR_P_HALF), it & 1, wctx))) break;
+      tc_fence_after();
+      issue_ts_split_part(tmem + L::T_DV, tmem + L::T_S, sdesc_add(dDOmn, so), idesc_g, it == 0, 0, leader);
       if (!(ok = mbar_wait(bar(L::BAR_P_READY), it & 1, wctx))) break;
       tc_fence_after();
-      issue_ts_split(tmem + L::T_DV, tmem + L::T_S, sdesc_add(dDOmn, so), idesc_g, it > 0, leader);  // dV += P^T dO
+      issue_ts_split_part(tmem + L::T_DV, tmem + L::T_S, sdesc_add(dDOmn, so), idesc_g, false, 1, leader);
       mma_commit(bar(L::BAR_DO_EMPTY + s), leader);
       if (it + 1 < n_it) {
         const int s1 = (it + 1) & 1;
@@ -307,10 +332,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           float t0, t1, t2, t3;
           f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, f2pack(-L4.x, -L4.y)), t0, t1);
           f2unpack(ffma2(f2pack(pr[c + 2], pr[c + 3]), sl2x2, f2pack(-L4.z, -L4.w)), t2, t3);
-          pr[c] = ex2_approx(t0);
-          pr[c + 1] = ex2_approx(t1);
-          pr[c + 2] = ex2_approx(t2);
-          pr[c + 3] = ex2_approx(t3);
+          if ((c - g) < kDkdvExpFmaPer16) {
+            // both warpgroups run this phase at once, so the MUFU unit is the limit: part of
+            // the exponentials go to the FMA pipe
+            exp2_fma_pipe(t0, t1);
+            exp2_fma_pipe(t2, t3);
+            pr[c] = t0;
+            pr[c + 1] = t1;
+            pr[c + 2] = t2;
+            pr[c + 3] = t3;
+          } else {
+            pr[c] = ex2_approx(t0);
+            pr[c + 1] = ex2_approx(t1);
+            pr[c + 2] = ex2_approx(t2);
+            pr[c + 3] = ex2_approx(t3);
+          }
           if (need_mask) {
             if (q0 + c < key) pr[c] = 0.f;
             if (q0 + c + 1 < key) pr[c + 1] = 0.f;
@@ -321,6 +357,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[(c - g) / 2 + 1] = pack_f16(pr[c + 2], pr[c + 3]);
         }
         tmem_st8(tS + g / 2, pk);
+        if (g == 16) {  // columns 0..31 of this warpgroup done: the first half of dV may start
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(L::BAR_P_HALF));
+        }
       }
       tmem_wait_st();
       tc_fence_before();
