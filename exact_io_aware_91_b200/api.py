@@ -23,8 +23,8 @@ FA_ERR_MISALIGNED = 3
 FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
 
-EXPORTS = ("fa_fwd", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_noalloc", "fa_device_status",
-           "fa_bwd_set_phase_events", "fa_status_str")
+EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_gqa_workspace_size",
+           "fa_bwd_gqa", "fa_bwd_noalloc", "fa_device_status", "fa_bwd_set_phase_events", "fa_status_str")
 
 # Size of the scratch array fa_bwd_noalloc uses instead of a caller workspace.
 FA_BWD_NOALLOC_MAX_WORKSPACE = 64 << 20
@@ -54,12 +54,18 @@ def library() -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_fwd.restype = i
+    lib.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    lib.fa_fwd_gqa.restype = i
     lib.fa_fwd_f32.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_fwd_f32.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_bwd.restype = i
+    lib.fa_bwd_gqa_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_bwd_gqa_workspace_size.restype = sz
+    lib.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_bwd_gqa.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_bwd_noalloc.restype = i
     lib.fa_device_status.argtypes = [vp]
@@ -132,6 +138,41 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Fal
     return (o, lse) if o_resid is None else (o, lse, o_resid)
 
 
+def _gqa_heads(q: torch.Tensor, k: torch.Tensor) -> int:
+    if k.dim() != 4 or k.shape[0] != q.shape[0] or k.shape[2:] != q.shape[2:]:
+        raise ValueError("k, v must be (B, H_kv, N, d) with q's B, N and d")
+    h_kv = int(k.shape[1])
+    if h_kv < 1 or q.shape[1] % h_kv:
+        raise ValueError("the query head count must be a multiple of the key/value head count")
+    return h_kv
+
+
+def fa_fwd_gqa(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+               scale: float | None = None, o: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+               o_resid: torch.Tensor | None = None, save_residual: bool = False, stream=None):
+    """Grouped-query / multi-query forward: q (B, H, N, d), k and v (B, H_kv, N, d) bf16.
+
+    Query head h reads key/value head h // (H // H_kv).  Returns like ``fa_fwd``."""
+    B, H, N, d = _shape(q)
+    H_kv = _gqa_heads(q, k)
+    _same(q, dtype=torch.bfloat16, shape=(B, H, N, d))
+    _same(k, v, dtype=torch.bfloat16, shape=(B, H_kv, N, d))
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if o_resid is None and save_residual:
+        o_resid = torch.empty_like(q)
+    _same(o, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if o_resid is not None:
+        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
+    st = library().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                              None if o_resid is None else o_resid.data_ptr(), B, H, H_kv, N, d, _scale(scale, d),
+                              int(bool(causal)), _stream_handle(stream))
+    _check("fa_fwd_gqa", st)
+    return (o, lse) if o_resid is None else (o, lse, o_resid)
+
+
 def fa_fwd_f32(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
                scale: float | None = None, stream=None):
     """fp32 forward (no input rounding). Returns (o, lse)."""
@@ -173,6 +214,39 @@ def fa_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None
                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, _scale(scale, d),
                           int(bool(causal)), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
     _check("fa_bwd", st)
+    return dq, dk, dv
+
+
+def fa_bwd_gqa_workspace_size(B: int, H: int, H_kv: int, N: int, d: int) -> int:
+    return int(library().fa_bwd_gqa_workspace_size(B, H, H_kv, N, d))
+
+
+def fa_bwd_gqa(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,
+               dq=None, dk=None, dv=None, o_resid=None, stream=None):
+    """Grouped-query backward: dq (B, H, N, d); dk, dv (B, H_kv, N, d), summed over each group."""
+    B, H, N, d = _shape(q)
+    H_kv = _gqa_heads(q, k)
+    _same(q, o, do, dtype=torch.bfloat16, shape=(B, H, N, d))
+    _same(k, v, dtype=torch.bfloat16, shape=(B, H_kv, N, d))
+    _same(lse, dtype=torch.float32, shape=(B, H, N))
+    if o_resid is not None:
+        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if dq is None:
+        dq = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    if dk is None:
+        dk = torch.empty((B, H_kv, N, d), dtype=torch.float32, device=q.device)
+    if dv is None:
+        dv = torch.empty_like(dk)
+    _same(dq, dtype=torch.float32, shape=(B, H, N, d))
+    _same(dk, dv, dtype=torch.float32, shape=(B, H_kv, N, d))
+    ws_bytes = fa_bwd_gqa_workspace_size(B, H, H_kv, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    st = library().fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              None if o_resid is None else o_resid.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N, d, _scale(scale, d),
+                              int(bool(causal)), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    _check("fa_bwd_gqa", st)
     return dq, dk, dv
 
 

@@ -3,7 +3,8 @@
 //            with O = O_bf16 + residual when the forward's residual is given,
 //            i.e. the forward's fp32 O, so that D does not carry O's bf16 rounding
 //   lse2_i = LSE_i * log2(e)               (so the kernels form P = 2^(s*scale*log2e - lse2))
-//   q16, k16, v16, do16 = fp16 copies of the bf16 inputs
+//   q16, k16, v16, do16 = fp16 copies of the bf16 inputs (k16 / v16 for the first BH_kv
+//   heads only: with grouped-query attention K and V have fewer heads than Q)
 // Rows N..Np-1 of D / lse2 are padding for the 64/128-row tiles: D = 0 and
 // lse2 = +inf, which makes every probability of a padded query exactly 0.
 //
@@ -53,15 +54,17 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
   if (real) {
     const size_t off = ((size_t)bh * p.N + i) * D + (size_t)sub * 8;  // element offset
     const uint4 vq = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + off);
-    const uint4 vk = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.k) + off);
-    const uint4 vv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.v) + off);
     const uint4 vo = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + off);
     const uint4 vd = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) + off);
     float fq[8], fk[8], fv[8], fo[8], fd[8];
     *reinterpret_cast<uint4*>(static_cast<__half*>(p.q16) + off) = bf16x8_to_f16x8(vq, fq);
-    *reinterpret_cast<uint4*>(static_cast<__half*>(p.k16) + off) = bf16x8_to_f16x8(vk, fk);
-    *reinterpret_cast<uint4*>(static_cast<__half*>(p.v16) + off) = bf16x8_to_f16x8(vv, fv);
     *reinterpret_cast<uint4*>(static_cast<__half*>(p.do16) + off) = bf16x8_to_f16x8(vd, fd);
+    if (bh < p.BH_kv) {  // key/value rows share the (head, row) index space of the first BH_kv heads
+      const uint4 vk = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.k) + off);
+      const uint4 vv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.v) + off);
+      *reinterpret_cast<uint4*>(static_cast<__half*>(p.k16) + off) = bf16x8_to_f16x8(vk, fk);
+      *reinterpret_cast<uint4*>(static_cast<__half*>(p.v16) + off) = bf16x8_to_f16x8(vv, fv);
+    }
     bf16x8_to_f16x8(vo, fo);
     if (p.o_resid != nullptr) {
       float fr[8];

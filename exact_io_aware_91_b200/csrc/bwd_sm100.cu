@@ -169,10 +169,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // heaviest first within groups of heads (see unit_order): under the causal mask the
   // first key tiles of a head meet the most query tiles
   const int n_kt = (p.N + 127) / 128;
-  int bh, j;  // head, key tile
-  unit_order((int)blockIdx.x, n_kt, p.BH, p.head_group, bh, j);
+  int bh, j;  // key/value head, key tile
+  unit_order((int)blockIdx.x, n_kt, p.BH / p.H * p.H_kv, p.head_group_kv, bh, j);
   const int i_start = p.causal ? j : 0;
-  const int n_it = n_kt - i_start;  // 128-query steps, >= 1
+  const int n_q = n_kt - i_start;          // 128-query tiles per query head, >= 1
+  const int n_it = (p.H / p.H_kv) * n_q;   // steps: every query tile of every query head of the group
+  // step it: query head q_head_of(bh, it / n_q), query tile i_start + it % n_q
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -218,20 +220,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int it = 0; it < n_it; ++it) {
       const int s = it & 1;
       const uint32_t ph = ((it >> 1) & 1) ^ 1u;
-      const int i = i_start + it;
+      const int i = i_start + it % n_q;
+      const int bhq = q_head_of(bh, it / n_q, p.H, p.H_kv);
       if (!mbar_wait(bar(L::BAR_Q_EMPTY + s), ph, wctx)) break;
       const uint32_t fq = bar(L::BAR_Q_FULL + s);
       mbar_arrive_expect_tx(fq, L::TILE + 1024, leader);
       for (int c = 0; c < L::KCH; ++c)
-        tma_load_3d(base + L::OFF_Q + s * L::TILE + c * kBox, &tm_q, c * 64, i * 128, bh, fq, leader);
-      const size_t roff = (size_t)bh * p.Np + (size_t)i * 128;
+        tma_load_3d(base + L::OFF_Q + s * L::TILE + c * kBox, &tm_q, c * 64, i * 128, bhq, fq, leader);
+      const size_t roff = (size_t)bhq * p.Np + (size_t)i * 128;
       bulk_load(base + L::OFF_LD + s * 1024, p.lse2 + roff, 512, fq, leader);
       bulk_load(base + L::OFF_LD + s * 1024 + 512, p.delta + roff, 512, fq, leader);
       if (!mbar_wait(bar(L::BAR_DO_EMPTY + s), ph, wctx)) break;
       const uint32_t fd = bar(L::BAR_DO_FULL + s);
       mbar_arrive_expect_tx(fd, L::TILE, leader);
       for (int c = 0; c < L::KCH; ++c)
-        tma_load_3d(base + L::OFF_DO + s * L::TILE + c * kBox, &tm_do, c * 64, i * 128, bh, fd, leader);
+        tma_load_3d(base + L::OFF_DO + s * L::TILE + c * kBox, &tm_do, c * 64, i * 128, bhq, fd, leader);
       ++issued;
     }
     drain_wait(bar(L::BAR_KV), 0);
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t sl2x2 = f2pack(sl2, sl2);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int i = i_start + it;
+      const int i = i_start + it % n_q;  // query tile of this step
       const float* lse2 = reinterpret_cast<const float*>(gbase + L::OFF_LD + (it & 1) * 1024) + 64 * w;
       const float* delta = lse2 + 128;
       const int q0 = i * 128 + 64 * w;  // first query of this warpgroup's columns
@@ -455,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nq = (p.N + 127) / 128;
   int bh, rank;
   unit_order((int)blockIdx.x, nq, p.BH, p.head_group, bh, rank);
+  const int bh_kv = kv_head_of(bh, p.H, p.H_kv);  // the key/value head this query head reads
   const int qt = p.causal ? (nq - 1 - rank) : rank;
   const int n_it = p.causal ? qt + 1 : nq;  // 128-key steps
 
@@ -504,13 +508,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(bar(L::BAR_K_EMPTY + sk), ((it / 3) & 1) ^ 1u, wctx)) break;
       mbar_arrive_expect_tx(bar(L::BAR_K_FULL + sk), L::TILE, leader);
       for (int c = 0; c < L::KCH; ++c)
-        tma_load_3d(base + L::OFF_K + sk * L::TILE + c * kBox, &tm_k, c * 64, it * 128, bh, bar(L::BAR_K_FULL + sk),
-                    leader);
+        tma_load_3d(base + L::OFF_K + sk * L::TILE + c * kBox, &tm_k, c * 64, it * 128, bh_kv,
+                    bar(L::BAR_K_FULL + sk), leader);
       if (!mbar_wait(bar(L::BAR_V_EMPTY + sv), ((it >> 1) & 1) ^ 1u, wctx)) break;
       mbar_arrive_expect_tx(bar(L::BAR_V_FULL + sv), L::TILE, leader);
       for (int c = 0; c < L::KCH; ++c)
-        tma_load_3d(base + L::OFF_V + sv * L::TILE + c * kBox, &tm_v, c * 64, it * 128, bh, bar(L::BAR_V_FULL + sv),
-                    leader);
+        tma_load_3d(base + L::OFF_V + sv * L::TILE + c * kBox, &tm_v, c * 64, it * 128, bh_kv,
+                    bar(L::BAR_V_FULL + sv), leader);
       ++issued;
     }
     drain_wait(bar(L::BAR_Q), 0);
@@ -663,7 +667,7 @@ cudaError_t launch_one(Kern kern, dim3 grid, const CUtensorMap& a, const CUtenso
 
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                                   const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s) {
-  const dim3 grid((unsigned)(((p.N + 127) / 128) * p.BH));
+  const dim3 grid((unsigned)(((p.N + 127) / 128) * (p.BH / p.H * p.H_kv)));  // key tiles x key/value heads
   if (d == 128)
     return launch_one<DkdvLayout<128>>(fa_bwd_dkdv_sm100_kernel<128>, grid, tq, tdo, tk, tv, p, s);
   return launch_one<DkdvLayout<64>>(fa_bwd_dkdv_sm100_kernel<64>, grid, tq, tdo, tk, tv, p, s);

@@ -65,8 +65,10 @@ fa_status device_setup(int* dev_out) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // Shared validation of sizes/scalars.  Returns FA_OK and sets *empty when there is nothing to do.
-fa_status check_problem(int B, int H, int N, int d, float scale, int causal, bool* empty) {
-  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+// H_kv: key/value heads (H for plain multi-head attention); H must be a multiple of it.
+fa_status check_problem(int B, int H, int H_kv, int N, int d, float scale, int causal, bool* empty) {
+  if (B < 0 || H < 0 || N < 0 || H_kv < 0) return FA_ERR_INVALID_ARG;
+  if (H > 0 && (H_kv < 1 || H % H_kv != 0)) return FA_ERR_INVALID_ARG;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
@@ -87,19 +89,21 @@ struct BwdLayout {
   int Np;
 };
 
-BwdLayout bwd_layout(int B, int H, int N, int d) {
+// Workspace: fp16 copies of Q and dO (B*H heads) and of K and V (B*H_kv heads), then
+// D and LSE*log2(e) per query row padded to a multiple of 128 rows.
+BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d) {
   BwdLayout w{};
-  const size_t elems = (size_t)B * H * N * d;
-  const size_t t16 = align256(elems * 2);
+  const size_t t16 = align256((size_t)B * H * N * d * 2);
+  const size_t t16kv = align256((size_t)B * H_kv * N * d * 2);
   w.Np = ((N + 127) / 128) * 128;
   const size_t rows = align256((size_t)B * H * w.Np * 4);
   w.off_q16 = 0;
-  w.off_k16 = t16;
-  w.off_v16 = 2 * t16;
-  w.off_do16 = 3 * t16;
-  w.off_delta = 4 * t16;
-  w.off_lse2 = 4 * t16 + rows;
-  w.total = 4 * t16 + 2 * rows;
+  w.off_do16 = t16;
+  w.off_k16 = 2 * t16;
+  w.off_v16 = 2 * t16 + t16kv;
+  w.off_delta = 2 * t16 + 2 * t16kv;
+  w.off_lse2 = w.off_delta + rows;
+  w.total = w.off_lse2 + rows;
   return w;
 }
 
@@ -145,8 +149,13 @@ const char* fa_status_str(fa_status s) {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
                  int N, int d, float scale, int causal, fa_stream_t stream) {
+  return fa_fwd_gqa(q, k, v, o, lse, o_resid, B, H, H, N, d, scale, causal, stream);
+}
+
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
+                     int H_kv, int N, int d, float scale, int causal, fa_stream_t stream) {
   bool empty = false;
-  fa_status st = check_problem(B, H, N, d, scale, causal, &empty);
+  fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
   if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
@@ -154,19 +163,23 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     return FA_ERR_MISALIGNED;
   int dev = 0;
   if ((st = device_setup(&dev)) != FA_OK) return st;
-  const int BH = B * H;
+  const int BH = B * H, BH_kv = B * H_kv;
   CUtensorMap tq, tk, tv, to;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!make_tmap_3d(&tq, q, bf, 2, d, N, BH, 64, 128, true) || !make_tmap_3d(&tk, k, bf, 2, d, N, BH, 64, 128, true) ||
-      !make_tmap_3d(&tv, v, bf, 2, d, N, BH, 64, 128, true) || !make_tmap_3d(&to, o, bf, 2, d, N, BH, 64, 128, true))
+  if (!make_tmap_3d(&tq, q, bf, 2, d, N, BH, 64, 128, true) ||
+      !make_tmap_3d(&tk, k, bf, 2, d, N, BH_kv, 64, 128, true) ||
+      !make_tmap_3d(&tv, v, bf, 2, d, N, BH_kv, 64, 128, true) || !make_tmap_3d(&to, o, bf, 2, d, N, BH, 64, 128, true))
     return FA_ERR_CUDA;
   FwdParams p{};
   p.lse = lse;
   p.o_resid = static_cast<__nv_bfloat16*>(o_resid);
   p.N = N;
   p.BH = BH;
+  p.H = H;
+  p.H_kv = H_kv;
   p.n_pairs = (N + 255) / 256;
-  p.head_group = head_group_size(BH, N, d, kFwdGroupBytes);
+  // K and V bytes per query head: a group of H / H_kv query heads shares them
+  p.head_group = head_group_size(BH, 4ull * N * d / (H / H_kv), kFwdGroupBytes);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal;
   p.err = g_err_ptr[dev];
@@ -178,7 +191,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N,
                      int d, float scale, int causal, fa_stream_t stream) {
   bool empty = false;
-  fa_status st = check_problem(B, H, N, d, scale, causal, &empty);
+  fa_status st = check_problem(B, H, H, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
   if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(o, 4) || !aligned(lse, 4))
@@ -191,20 +204,30 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, f
              : FA_ERR_CUDA;
 }
 
-size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) { return fa_bwd_gqa_workspace_size(B, H, H, N, d); }
+
+size_t fa_bwd_gqa_workspace_size(int B, int H, int H_kv, int N, int d) {
   bool empty = false;
-  if (check_problem(B, H, N, d, 1.0f, 0, &empty) != FA_OK || empty) return 0;
-  return bwd_layout(B, H, N, d).total;
+  if (check_problem(B, H, H_kv, N, d, 1.0f, 0, &empty) != FA_OK || empty) return 0;
+  return bwd_layout(B, H, H_kv, N, d).total;
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* o_resid, const void* dout,
                  const float* lse, float* dq, float* dk, float* dv, int B, int H, int N, int d, float scale,
                  int causal, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  return fa_bwd_gqa(q, k, v, o, o_resid, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, workspace,
+                    workspace_bytes, stream);
+}
+
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                     const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int H_kv,
+                     int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                     fa_stream_t stream) {
   bool empty = false;
-  fa_status st = check_problem(B, H, N, d, scale, causal, &empty);
+  fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
-  const BwdLayout w = bwd_layout(B, H, N, d);
+  const BwdLayout w = bwd_layout(B, H, H_kv, N, d);
   if (workspace_bytes < w.total) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
       !aligned(o_resid, 16) || !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(workspace, 256))
@@ -212,7 +235,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   int dev = 0;
   if ((st = device_setup(&dev)) != FA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int BH = B * H;
+  const int BH = B * H, BH_kv = B * H_kv, group = H / H_kv;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
 
   BwdPreParams pp{};
@@ -232,6 +255,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   pp.N = N;
   pp.Np = w.Np;
   pp.BH = BH;
+  pp.BH_kv = BH_kv;
   pp.d = d;
   if (launch_bwd_pre(pp, s) != cudaSuccess) return FA_ERR_CUDA;
   if (t_phase_events != nullptr && t_phase_events[0] != nullptr &&
@@ -242,8 +266,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   CUtensorMap t_q, t_do, t_k, t_v;  // 128-row boxes, shared by the dK/dV and dQ kernels
   if (!make_tmap_3d(&t_q, pp.q16, h, 2, d, N, BH, 64, 128, true) ||
       !make_tmap_3d(&t_do, pp.do16, h, 2, d, N, BH, 64, 128, true) ||
-      !make_tmap_3d(&t_k, pp.k16, h, 2, d, N, BH, 64, 128, true) ||
-      !make_tmap_3d(&t_v, pp.v16, h, 2, d, N, BH, 64, 128, true))
+      !make_tmap_3d(&t_k, pp.k16, h, 2, d, N, BH_kv, 64, 128, true) ||
+      !make_tmap_3d(&t_v, pp.v16, h, 2, d, N, BH_kv, 64, 128, true))
     return FA_ERR_CUDA;
   BwdParams bp{};
   bp.delta = pp.delta;
@@ -254,7 +278,12 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   bp.N = N;
   bp.Np = w.Np;
   bp.BH = BH;
-  bp.head_group = head_group_size(BH, N, d, kBwdGroupBytes);
+  bp.H = H;
+  bp.H_kv = H_kv;
+  // dQ orders query heads (K and V bytes per query head shared by the group); dK/dV orders
+  // key/value heads (Q and dO of the whole group per key/value head)
+  bp.head_group = head_group_size(BH, 4ull * N * d / group, kBwdGroupBytes);
+  bp.head_group_kv = head_group_size(BH_kv, 4ull * N * d * group, kBwdGroupBytes);
   bp.scale = scale;
   bp.scale_log2 = scale * 1.4426950408889634f;
   bp.causal = causal;

@@ -12,7 +12,8 @@ struct FwdParams {
   float* lse;        // (B*H, N) fp32, natural-log LSE of the scaled scores; may be null
   __nv_bfloat16* o_resid;  // (B*H, N, d) bf16 residual O_fp32 - O_bf16; may be null
   int N;             // sequence length (queries = keys)
-  int BH;            // B * H
+  int BH;            // B * H (query heads)
+  int H, H_kv;       // query heads and key/value heads per batch entry (H a multiple of H_kv)
   int n_pairs;       // ceil(N / 256): work units per head (two 128-row query tiles each)
   int head_group;    // heads per group in the CTA order (unit_order)
   float scale_log2;  // softmax scale * log2(e)
@@ -35,6 +36,7 @@ struct BwdPreParams {
   float* delta;      // (BH, Np): rowsum(dO * O); 0 on padded rows
   float* lse2;       // (BH, Np): LSE * log2(e); +inf on padded rows
   int N, Np, BH, d;
+  int BH_kv;         // B * H_kv: rows of k / v / k16 / v16 (<= BH)
 };
 
 struct BwdParams {
@@ -44,7 +46,9 @@ struct BwdParams {
   float* dk;
   float* dv;
   int N, Np, BH;
-  int head_group;      // heads per group in the CTA order (unit_order)
+  int H, H_kv;         // query heads and key/value heads per batch entry (H a multiple of H_kv)
+  int head_group;      // query heads per group in the dQ kernel's CTA order (unit_order)
+  int head_group_kv;   // key/value heads per group in the dK/dV kernel's CTA order
   float scale;         // softmax scale (applied to dQ and dK)
   float scale_log2;    // scale * log2(e)
   int causal;
@@ -54,13 +58,12 @@ struct BwdParams {
 // Tensor maps are 3-D views (d, N, B*H) of a (B, H, N, d) tensor with the
 // 128-byte swizzle and a box of 64 columns x `box_rows` rows.
 // Heads per group in the CTA order: as many heads as keep the streamed operand pair
-// (K and V in the forward and dQ kernels, Q and dO in the dK/dV kernel; 4 * N * d bytes
-// per head) within `budget` bytes of L2.  Measured on B200 (N = 2048 and 8192, d = 128):
+// (K and V in the forward and dQ kernels, Q and dO in the dK/dV kernel; `per_head`
+// bytes per head of the CTA order) within `budget` bytes of L2.  Measured on B200 (N = 2048 and 8192, d = 128):
 // the forward runs best with 16 MB groups, the backward with 8 MB.
 constexpr unsigned long long kFwdGroupBytes = 16ull << 20;
 constexpr unsigned long long kBwdGroupBytes = 8ull << 20;
-inline int head_group_size(int BH, int N, int d, unsigned long long budget) {
-  const unsigned long long per_head = 4ull * (unsigned long long)N * (unsigned long long)d;
+inline int head_group_size(int BH, unsigned long long per_head, unsigned long long budget) {
   unsigned long long g = budget / (per_head ? per_head : 1ull);
   if (g < 1ull) g = 1ull;
   return g > (unsigned long long)BH ? BH : (int)g;

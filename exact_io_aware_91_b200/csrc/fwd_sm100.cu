@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int bh, rank;
   unit_order((int)blockIdx.x, p.n_pairs, p.BH, p.head_group, bh, rank);
   const int pair = p.causal ? (p.n_pairs - 1 - rank) : rank;
+  const int bh_kv = kv_head_of(bh, p.H, p.H_kv);  // the key/value head this query head reads
   const int q_base0 = pair * 256;
   const int q_base1 = q_base0 + 128;
   const int n_kv = (p.N + 127) / 128;
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar(L::BAR_KV_FULL + st), L::TILE, leader);
           const CUtensorMap* m = which ? &tm_v : &tm_k;
           for (int c = 0; c < L::KCH; ++c)
-            tma_load_3d(base + L::OFF_KV + st * L::TILE + c * L::BOX, m, c * 64, j * 128, bh,
+            tma_load_3d(base + L::OFF_KV + st * L::TILE + c * L::BOX, m, c * 64, j * 128, bh_kv,
                         bar(L::BAR_KV_FULL + st), leader);
           ++issued;
         }

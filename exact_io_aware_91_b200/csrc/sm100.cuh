@@ -128,6 +128,17 @@ __device__ __forceinline__ void unit_order(int cta, int per_head, int n_heads, i
   head = g0 + r % gs;
 }
 
+// Grouped-query attention: consecutive groups of H / H_kv query heads share one
+// key/value head.  Head indices here run over batch x heads.
+__device__ __forceinline__ int kv_head_of(int bh, int H, int H_kv) {
+  const int b = bh / H;
+  return b * H_kv + (bh - b * H) / (H / H_kv);
+}
+__device__ __forceinline__ int q_head_of(int bh_kv, int g, int H, int H_kv) {
+  const int b = bh_kv / H_kv;
+  return b * H + (bh_kv - b * H_kv) * (H / H_kv) + g;
+}
+
 // ----------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -73,24 +73,26 @@ def _draw(shape, dist: str, g: torch.Generator) -> torch.Tensor:
 
 def make_qkv(B: int, H: int, N: int, d: int, *, dtype=torch.bfloat16, dist: str = "normal",
              spiky_frac: float = 0.0, backward: bool = True, seed: int = 0,
-             device: str | torch.device = "cpu") -> dict:
+             device: str | torch.device = "cpu", kv_heads: int | None = None) -> dict:
     """Draw q, k, v (and do when ``backward``) on the host from one seeded generator.
 
     Values are drawn in fp32 and then cast to ``dtype`` (round to nearest even).
     With ``spiky_frac`` > 0, for each (b, h) a seeded set of ceil(spiky_frac * N)
     key rows is multiplied by 8 in fp32 before the cast (x8 is exact in bf16),
-    which makes many softmax rows nearly one-hot.
+    which makes many softmax rows nearly one-hot.  ``kv_heads`` (grouped-query
+    attention) gives k and v that many heads instead of H.
     """
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     shape = (B, H, N, d)
+    kv_shape = (B, H if kv_heads is None else kv_heads, N, d)
     q = _draw(shape, dist, g)
-    k = _draw(shape, dist, g)
-    v = _draw(shape, dist, g)
+    k = _draw(kv_shape, dist, g)
+    v = _draw(kv_shape, dist, g)
     if spiky_frac > 0.0:
         n_spiky = int(math.ceil(spiky_frac * N))
         for b in range(B):
-            for h in range(H):
+            for h in range(kv_shape[1]):
                 idx = torch.randperm(N, generator=g)[:n_spiky]
                 k[b, h, idx, :] *= 8.0
     out = {"q": q, "k": k, "v": v}

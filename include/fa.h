@@ -56,7 +56,8 @@ typedef struct CUstream_st* fa_stream_t;
 
 typedef enum {
   FA_OK = 0,
-  FA_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad scale/causal, workspace too small */
+  FA_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad scale/causal, H not a multiple of
+                             H_kv, workspace too small */
   FA_ERR_UNSUPPORTED = 2, /* head dim not in {64,128}, sizes beyond limits, not a CC 10.0 device */
   FA_ERR_MISALIGNED = 3,  /* a tensor base address is not 16-byte aligned (TMA requirement) */
   FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
@@ -83,6 +84,21 @@ typedef enum {
  */
 FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B,
                         int H, int N, int d, float scale, int causal, fa_stream_t stream);
+
+/*
+ * fa_fwd_gqa -- fa_fwd for grouped-query / multi-query attention ("Flash
+ * Attention: Ako transformery ...", section 5, and "FlashAttention (EL)", the list
+ * of extensions, name GQA/MQA support; the grouping below is the reading taken).
+ *   q, o, o_resid : (B, H, N, d) as in fa_fwd;  lse: (B, H, N).
+ *   k, v          : const bf16 (B, H_kv, N, d), 16-byte aligned.
+ *   H_kv          : key/value heads, >= 1, H a multiple of H_kv (H_kv = 1: MQA,
+ *                   H_kv = H: plain multi-head attention, identical to fa_fwd).
+ * Query head h of batch entry b attends with key/value head h / (H / H_kv) of the
+ * same batch entry (consecutive groups of H / H_kv query heads share one K/V head).
+ * Everything else (precision, alignment, errors, asynchrony) as fa_fwd.
+ */
+FA_API fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B,
+                            int H, int H_kv, int N, int d, float scale, int causal, fa_stream_t stream);
 
 /*
  * fa_fwd_f32 -- the same forward pass on fp32 inputs and outputs, computed
@@ -122,6 +138,26 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                         const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int N,
                         int d, float scale, int causal, void* workspace, size_t workspace_bytes,
                         fa_stream_t stream);
+
+/*
+ * fa_bwd_gqa_workspace_size / fa_bwd_gqa -- fa_bwd for grouped-query attention
+ * (grouping as in fa_fwd_gqa).
+ *   q, o, o_resid, dout, dq : (B, H, N, d);  lse: (B, H, N).
+ *   k, v                    : const bf16 (B, H_kv, N, d).
+ *   dk, dv                  : fp32 (B, H_kv, N, d) outputs: the gradient of a shared
+ *                             key/value head is the sum over the query heads of its
+ *                             group.  Overwritten (not accumulated into).
+ *   workspace               : at least fa_bwd_gqa_workspace_size(B, H, H_kv, N, d)
+ *                             bytes (fp16 copies of Q and dO with H heads, of K and
+ *                             V with H_kv heads, and the two fp32 row vectors).
+ * With H_kv = H both are identical to fa_bwd_workspace_size / fa_bwd.  Everything
+ * else as fa_bwd.
+ */
+FA_API size_t fa_bwd_gqa_workspace_size(int B, int H, int H_kv, int N, int d);
+FA_API fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                            const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H,
+                            int H_kv, int N, int d, float scale, int causal, void* workspace,
+                            size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fa_bwd_noalloc -- the backward pass of fa_bwd for callers that cannot allocate

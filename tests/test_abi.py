@@ -52,6 +52,36 @@ def test_workspace_size_is_linear_in_n(lib, shape):
     assert api.fa_bwd_workspace_size(*shape) == _ws_expected(*shape)
 
 
+def _ws_expected_gqa(B, H, Hkv, N, d):
+    a = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    Np = (N + 127) // 128 * 128
+    return 2 * a(B * H * N * d * 2) + 2 * a(B * Hkv * N * d * 2) + 2 * a(B * H * Np * 4)
+
+
+@pytest.mark.parametrize("shape", [(1, 4, 1, 1, 64), (2, 32, 8, 8192, 128), (1, 8, 1, 131072, 128),
+                                   (3, 6, 3, 1000, 64), (2, 16, 16, 2048, 128)])
+def test_gqa_workspace_size(lib, shape):
+    B, H, Hkv, N, d = shape
+    assert api.fa_bwd_gqa_workspace_size(*shape) == _ws_expected_gqa(*shape)
+    if H == Hkv:
+        assert api.fa_bwd_gqa_workspace_size(*shape) == api.fa_bwd_workspace_size(B, H, N, d)
+
+
+def test_gqa_head_counts_are_checked(lib):
+    assert api.fa_bwd_gqa_workspace_size(1, 6, 4, 64, 64) == 0  # 6 is not a multiple of 4
+    assert api.fa_bwd_gqa_workspace_size(1, 6, 0, 64, 64) == 0
+    fwd_gqa = lambda H, Hkv: lib.fa_fwd_gqa(A, A, A, A, A, None, 1, H, Hkv, 16, 64, 0.125, 0, None)  # noqa: E731
+    assert fwd_gqa(6, 4) == api.FA_ERR_INVALID_ARG
+    assert fwd_gqa(6, 0) == api.FA_ERR_INVALID_ARG
+    assert fwd_gqa(6, -3) == api.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_gqa(None, None, None, None, None, None, 1, 0, 0, 16, 64, 0.125, 0, None) == api.FA_OK
+    bwd_gqa = lambda H, Hkv: lib.fa_bwd_gqa(A, A, A, A, A, A, A, A, A, A, 1, H, Hkv, 16, 64, 0.125, 0, A,  # noqa: E731
+                                             1 << 40, None)
+    assert bwd_gqa(8, 3) == api.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_gqa(A, A, A, A, A, A, A, A, A, A, 1, 8, 2, 16, 64, 0.125, 0, A,
+                          _ws_expected_gqa(1, 8, 2, 16, 64) - 1, None) == api.FA_ERR_INVALID_ARG
+
+
 def test_workspace_size_of_empty_or_bad_problem_is_zero(lib):
     assert api.fa_bwd_workspace_size(0, 1, 10, 64) == 0
     assert api.fa_bwd_workspace_size(1, 1, 0, 64) == 0

@@ -87,6 +87,47 @@ def test_batched_heads_are_independent():
     assert_grads(r["grads"], oracle.attention_backward(q, k, v, do, r["scale"], True))
 
 
+# ------------------------------------------------------------------ grouped-query attention
+GQA = [(B, H, Hkv, N, d, c) for (B, H, Hkv) in ((1, 4, 2), (2, 6, 1), (1, 8, 8), (1, 6, 3))
+       for N, d in ((300, 128), (257, 64)) for c in (False, True)]
+
+
+@pytest.mark.parametrize("B,H,Hkv,N,d,causal", GQA)
+def test_gqa_fwd_bwd(B, H, Hkv, N, d, causal):
+    inp = inputs.make_qkv(B, H, N, d, seed=H * 31 + Hkv * 7 + N + causal, kv_heads=Hkv, device="cuda")
+    q, k, v, do = (inp[n] for n in ("q", "k", "v", "do"))
+    scale = 1.0 / np.sqrt(d)
+    o, lse, res = api.fa_fwd_gqa(q, k, v, causal=causal, scale=scale, save_residual=True)
+    grads = api.fa_bwd_gqa(q, k, v, o, do, lse, causal=causal, scale=scale, o_resid=res)
+    torch.cuda.synchronize()
+    tag = f"B={B} H={H} Hkv={Hkv} N={N} d={d} causal={causal}"
+    O, L = oracle.attention_forward_gqa(q, k, v, scale, causal)
+    assert_fwd(o, lse, O, L, tag)
+    assert_grads(grads, oracle.attention_backward_gqa(q, k, v, do, scale, causal), tag)
+    if Hkv == H:  # the grouped entry points with H_kv = H are plain multi-head attention
+        o2, lse2, res2 = api.fa_fwd(q, k, v, causal=causal, scale=scale, save_residual=True)
+        g2 = api.fa_bwd(q, k, v, o2, do, lse2, causal=causal, scale=scale, o_resid=res2)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o2) and torch.equal(lse, lse2)
+        for a, b in zip(grads, g2):
+            assert torch.equal(a, b)
+
+
+def test_gqa_long_spiky_matches_oracle_rows():
+    # a long grouped problem with peaked softmax rows: all of dK/dV of one key/value head
+    # against the oracle, which materialises N x N per query head
+    B, H, Hkv, N, d = 1, 4, 1, 4096, 128
+    inp = inputs.make_qkv(B, H, N, d, seed=77, spiky_frac=0.01, kv_heads=Hkv, device="cuda")
+    q, k, v, do = (inp[n] for n in ("q", "k", "v", "do"))
+    scale = 1.0 / np.sqrt(d)
+    o, lse, res = api.fa_fwd_gqa(q, k, v, causal=True, scale=scale, save_residual=True)
+    grads = api.fa_bwd_gqa(q, k, v, o, do, lse, causal=True, scale=scale, o_resid=res)
+    torch.cuda.synchronize()
+    O, L = oracle.attention_forward_gqa(q, k, v, scale, True)
+    assert_fwd(o, lse, O, L, "MQA N=4096 spiky")
+    assert_grads(grads, oracle.attention_backward_gqa(q, k, v, do, scale, True), "MQA N=4096 spiky")
+
+
 # ------------------------------------------------------------------ the five workloads
 def test_workload1_fp32_forward():
     w = inputs.workload(1)
