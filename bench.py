@@ -167,7 +167,9 @@ class ClockSampler:
 def oracle_head_step(inp_cpu: dict, w: inputs.Workload, b: int, h: int) -> None:
     import oracle
 
-    q, k, v, do = (inp_cpu[n][b, h] for n in ("q", "k", "v", "do"))
+    g = h // (inp_cpu["q"].shape[1] // inp_cpu["k"].shape[1])  # key/value head (grouped-query runs)
+    q, do = inp_cpu["q"][b, h], inp_cpu["do"][b, h]
+    k, v = inp_cpu["k"][b, g], inp_cpu["v"][b, g]
     oracle.attention_forward(q, k, v, w.scale, w.causal)
     oracle.attention_backward(q, k, v, do, w.scale, w.causal)
 
@@ -232,22 +234,31 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     if not w.backward:
         raise SystemExit("bench.py times forward + backward: pick a workload with a backward pass")
     dev = torch.device("cuda", torch.cuda.current_device())
-    inp_cpu = inputs.make_inputs(w, device="cpu")
-    q, k, v, do = (inp_cpu[n].to(dev) for n in ("q", "k", "v", "do"))
     B, H, N, d = w.B, w.H, w.N, w.d
+    Hkv = H if args.kv_heads is None else args.kv_heads
+    if Hkv < 1 or H % Hkv:
+        raise SystemExit(f"--kv-heads must divide H = {H}")
+    name = w.name if Hkv == H else f"{w.name}_gqa_h{H}_hkv{Hkv}"
+    inp_cpu = inputs.make_qkv(B, H, N, d, dtype=w.dtype, dist=w.dist, spiky_frac=w.spiky_frac, backward=True,
+                              seed=w.seed, kv_heads=None if Hkv == H else Hkv)
+    q, k, v, do = (inp_cpu[n].to(dev) for n in ("q", "k", "v", "do"))
     o = torch.empty_like(q)
     res = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     dq = torch.empty((B, H, N, d), dtype=torch.float32, device=dev)
-    dk = torch.empty_like(dq)
-    dv = torch.empty_like(dq)
-    ws = torch.empty(api.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    dk = torch.empty((B, Hkv, N, d), dtype=torch.float32, device=dev)
+    dv = torch.empty_like(dk)
+    ws = torch.empty(api.fa_bwd_gqa_workspace_size(B, H, Hkv, N, d), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    if Hkv == H:
+        fwd_call, bwd_call = api.fa_fwd, api.fa_bwd
+    else:
+        fwd_call, bwd_call = api.fa_fwd_gqa, api.fa_bwd_gqa
 
     def step():
-        api.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, o=o, lse=lse, o_resid=res)
-        api.fa_bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws, dq=dq, dk=dk, dv=dv,
-                   o_resid=res)
+        fwd_call(q, k, v, causal=w.causal, scale=w.scale, o=o, lse=lse, o_resid=res)
+        bwd_call(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws, dq=dq, dk=dk, dv=dv,
+                 o_resid=res)
 
     for _ in range(args.warmup):
         step()
@@ -267,11 +278,11 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     for s in range(args.steps):
         e = ev[s]
         e[0].record(stream)
-        api.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, o=o, lse=lse, o_resid=res)
+        fwd_call(q, k, v, causal=w.causal, scale=w.scale, o=o, lse=lse, o_resid=res)
         e[1].record(stream)
         api.fa_bwd_set_phase_events((e[2], e[3]))
-        api.fa_bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws, dq=dq, dk=dk, dv=dv,
-                   o_resid=res)
+        bwd_call(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws, dq=dq, dk=dk, dv=dv,
+                 o_resid=res)
         api.fa_bwd_set_phase_events(None)
         e[4].record(stream)
     end.record(stream)
@@ -305,7 +316,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     peak = peaks["bf16_tflops_sustained"]
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak,
-                "traffic": args.traffic if args.traffic is not None else recorded_traffic(dom, w.name),
+                "traffic": args.traffic if args.traffic is not None else recorded_traffic(dom, name),
                 "peak_kind": f"{peaks['source']} bf16 dense matmul, sustained (kernel timed inside a long step)"}
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
@@ -353,7 +364,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+            "config": {"workload": name, "B": B, "H": H, "H_kv": Hkv, "N": N, "d": d, "causal": w.causal,
                        "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
                        "l2": ("inputs larger than L2 (Q, K, V, dO, O 134 MB each > 126 MB)" if w.N * w.B * w.H >= 2 ** 19
                    else "small workload: inputs may stay in L2")},
@@ -382,6 +393,8 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[2, 3, 5],
                     help="workload index (3 = the metric's; others for profiling runs)")
+    ap.add_argument("--kv-heads", type=int, default=None,
+                    help="grouped-query run: K/V with this many heads (fa_fwd_gqa / fa_bwd_gqa); default H")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the dominant kernel from an ncu capture (reported as-is)")
     args = ap.parse_args()

@@ -90,7 +90,37 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
   }
 }
 
+// dK, dV of grouped-query attention when one key/value head's query heads were split
+// over several CTAs: out[e] = sum over splits of part[split][e], in a fixed order.
+__global__ void __launch_bounds__(256) fa_bwd_kv_reduce_kernel(const float4* __restrict__ dk_part,
+                                                              const float4* __restrict__ dv_part,
+                                                              float4* __restrict__ dk, float4* __restrict__ dv,
+                                                              long long n4, int splits) {
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += (long long)gridDim.x * blockDim.x) {
+    float4 a = dk_part[e], b = dv_part[e];
+    for (int s = 1; s < splits; ++s) {
+      const float4 x = dk_part[(long long)s * n4 + e], y = dv_part[(long long)s * n4 + e];
+      a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+      b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+    }
+    dk[e] = a;
+    dv[e] = b;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_bwd_kv_reduce(const float* dk_part, const float* dv_part, float* dk, float* dv, long long elems,
+                                 int splits, cudaStream_t s) {
+  const long long n4 = elems / 4;  // d is a multiple of 4
+  long long blocks = (n4 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  fa_bwd_kv_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(dk_part),
+                                                           reinterpret_cast<const float4*>(dv_part),
+                                                           reinterpret_cast<float4*>(dk),
+                                                           reinterpret_cast<float4*>(dv), n4, splits);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t s) {
   const long long rows = (long long)p.BH * p.Np;

@@ -169,12 +169,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // heaviest first within groups of heads (see unit_order): under the causal mask the
   // first key tiles of a head meet the most query tiles
   const int n_kt = (p.N + 127) / 128;
-  int bh, j;  // key/value head, key tile
-  unit_order((int)blockIdx.x, n_kt, p.BH / p.H * p.H_kv, p.head_group_kv, bh, j);
+  int bh, rank;  // key/value head, rank of (key tile, split) within the head
+  unit_order((int)blockIdx.x, n_kt * p.kv_split, p.BH / p.H * p.H_kv, p.head_group_kv, bh, rank);
+  const int j = rank / p.kv_split;         // key tile
+  const int sp = rank % p.kv_split;        // which share of the group's query heads
+  const int g_per = p.H / p.H_kv / p.kv_split;  // query heads handled by this CTA
   const int i_start = p.causal ? j : 0;
   const int n_q = n_kt - i_start;          // 128-query tiles per query head, >= 1
-  const int n_it = (p.H / p.H_kv) * n_q;   // steps: every query tile of every query head of the group
-  // step it: query head q_head_of(bh, it / n_q), query tile i_start + it % n_q
+  const int n_it = g_per * n_q;            // steps: every query tile of each of this CTA's query heads
+  // step it: query head q_head_of(bh, sp * g_per + it / n_q), query tile i_start + it % n_q
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -221,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = it & 1;
       const uint32_t ph = ((it >> 1) & 1) ^ 1u;
       const int i = i_start + it % n_q;
-      const int bhq = q_head_of(bh, it / n_q, p.H, p.H_kv);
+      const int bhq = q_head_of(bh, sp * g_per + it / n_q, p.H, p.H_kv);
       if (!mbar_wait(bar(L::BAR_Q_EMPTY + s), ph, wctx)) break;
       const uint32_t fq = bar(L::BAR_Q_FULL + s);
       mbar_arrive_expect_tx(fq, L::TILE + 1024, leader);
@@ -397,7 +400,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       // warpgroup 0 writes dV, warpgroup 1 writes scale * dK (rows past N are padding)
-      float* dst = (key < p.N) ? ((w == 0 ? p.dv : p.dk) + ((size_t)bh * p.N + key) * D) : nullptr;
+      // with the group split over several CTAs each writes its partial sums for the reduction
+      const size_t row_index = p.kv_split == 1 ? (size_t)bh * p.N + key
+                                                : ((size_t)sp * (p.BH / p.H * p.H_kv) + bh) * p.N + key;
+      float* out = p.kv_split == 1 ? (w == 0 ? p.dv : p.dk) : (w == 0 ? p.dv_part : p.dk_part);
+      float* dst = (key < p.N) ? (out + row_index * D) : nullptr;
       store_rows_f32<D>(tmem + lane_off + (w == 0 ? L::T_DV : L::T_DK), dst, w == 0 ? 1.0f : p.scale);
     }
   }
@@ -667,7 +674,8 @@ cudaError_t launch_one(Kern kern, dim3 grid, const CUtensorMap& a, const CUtenso
 
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                                   const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s) {
-  const dim3 grid((unsigned)(((p.N + 127) / 128) * (p.BH / p.H * p.H_kv)));  // key tiles x key/value heads
+  // key tiles x key/value heads x group splits
+  const dim3 grid((unsigned)(((p.N + 127) / 128) * (p.BH / p.H * p.H_kv) * p.kv_split));
   if (d == 128)
     return launch_one<DkdvLayout<128>>(fa_bwd_dkdv_sm100_kernel<128>, grid, tq, tdo, tk, tv, p, s);
   return launch_one<DkdvLayout<64>>(fa_bwd_dkdv_sm100_kernel<64>, grid, tq, tdo, tk, tv, p, s);

@@ -85,14 +85,30 @@ fa_status check_problem(int B, int H, int H_kv, int N, int d, float scale, int c
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct BwdLayout {
-  size_t off_q16, off_k16, off_v16, off_do16, off_delta, off_lse2, total;
+  size_t off_q16, off_k16, off_v16, off_do16, off_delta, off_lse2, off_dk_part, off_dv_part, total;
   int Np;
+  int kv_split;
 };
 
+// Grouped-query attention with few key/value heads leaves the dK/dV kernel (one CTA per
+// key/value head and key tile) with too few, very unequal CTAs: then each group's query
+// heads are split over kv_split CTAs -- the smallest divisor of the group size that gives at
+// least four CTAs per SM -- whose partial sums a reduction kernel adds up.
+constexpr long long kDkdvMinUnits = 4 * 148;
+int kv_split_for(int B, int H, int H_kv, int N) {
+  const int group = H / H_kv;
+  const long long units = (long long)B * H_kv * ((N + 127) / 128);
+  for (int s = 1; s < group; ++s)
+    if (group % s == 0 && units * s >= kDkdvMinUnits) return s;
+  return group;
+}
+
 // Workspace: fp16 copies of Q and dO (B*H heads) and of K and V (B*H_kv heads), then
-// D and LSE*log2(e) per query row padded to a multiple of 128 rows.
+// D and LSE*log2(e) per query row padded to a multiple of 128 rows, then (only when the
+// group is split, see kv_split_for) fp32 partial dK and dV per split.
 BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d) {
   BwdLayout w{};
+  w.kv_split = kv_split_for(B, H, H_kv, N);
   const size_t t16 = align256((size_t)B * H * N * d * 2);
   const size_t t16kv = align256((size_t)B * H_kv * N * d * 2);
   w.Np = ((N + 127) / 128) * 128;
@@ -103,7 +119,10 @@ BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d) {
   w.off_v16 = 2 * t16 + t16kv;
   w.off_delta = 2 * t16 + 2 * t16kv;
   w.off_lse2 = w.off_delta + rows;
-  w.total = w.off_lse2 + rows;
+  w.off_dk_part = w.off_lse2 + rows;
+  const size_t part = w.kv_split > 1 ? align256((size_t)w.kv_split * B * H_kv * N * d * 4) : 0;
+  w.off_dv_part = w.off_dk_part + part;
+  w.total = w.off_dv_part + part;
   return w;
 }
 
@@ -283,12 +302,18 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
   // dQ orders query heads (K and V bytes per query head shared by the group); dK/dV orders
   // key/value heads (Q and dO of the whole group per key/value head)
   bp.head_group = head_group_size(BH, 4ull * N * d / group, kBwdGroupBytes);
-  bp.head_group_kv = head_group_size(BH_kv, 4ull * N * d * group, kBwdGroupBytes);
+  bp.head_group_kv = head_group_size(BH_kv, 4ull * N * d * (group / w.kv_split), kBwdGroupBytes);
+  bp.kv_split = w.kv_split;
+  bp.dk_part = w.kv_split > 1 ? reinterpret_cast<float*>(ws + w.off_dk_part) : nullptr;
+  bp.dv_part = w.kv_split > 1 ? reinterpret_cast<float*>(ws + w.off_dv_part) : nullptr;
   bp.scale = scale;
   bp.scale_log2 = scale * 1.4426950408889634f;
   bp.causal = causal;
   bp.err = g_err_ptr[dev];
   if (launch_bwd_dkdv_sm100(t_q, t_do, t_k, t_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (w.kv_split > 1 &&
+      launch_bwd_kv_reduce(bp.dk_part, bp.dv_part, dk, dv, (long long)BH_kv * N * d, w.kv_split, s) != cudaSuccess)
+    return FA_ERR_CUDA;
   if (t_phase_events != nullptr && t_phase_events[1] != nullptr &&
       cudaEventRecord(static_cast<cudaEvent_t>(t_phase_events[1]), s) != cudaSuccess)
     return FA_ERR_CUDA;

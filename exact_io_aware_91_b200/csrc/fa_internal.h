@@ -49,6 +49,9 @@ struct BwdParams {
   int H, H_kv;         // query heads and key/value heads per batch entry (H a multiple of H_kv)
   int head_group;      // query heads per group in the dQ kernel's CTA order (unit_order)
   int head_group_kv;   // key/value heads per group in the dK/dV kernel's CTA order
+  int kv_split;        // CTAs sharing one (key/value head, key tile): each takes H/H_kv/kv_split query heads
+  float* dk_part;      // with kv_split > 1: fp32 (kv_split, B*H_kv, N, d) partial dK (scaled) and dV,
+  float* dv_part;      //   summed into dk / dv by launch_bwd_kv_reduce; unused when kv_split == 1
   float scale;         // softmax scale (applied to dQ and dK)
   float scale_log2;    // scale * log2(e)
   int causal;
@@ -74,6 +77,8 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int 
 
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t s);
+cudaError_t launch_bwd_kv_reduce(const float* dk_part, const float* dv_part, float* dk, float* dv,
+                                 long long elems, int splits, cudaStream_t s);
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int BH, int N,
                            int d, float scale, int causal, cudaStream_t s);
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t s);

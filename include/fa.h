@@ -149,7 +149,11 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
  *                             group.  Overwritten (not accumulated into).
  *   workspace               : at least fa_bwd_gqa_workspace_size(B, H, H_kv, N, d)
  *                             bytes (fp16 copies of Q and dO with H heads, of K and
- *                             V with H_kv heads, and the two fp32 row vectors).
+ *                             V with H_kv heads, the two fp32 row vectors and, when
+ *                             B * H_kv * ceil(N / 128) < 592, fp32 partial dK and dV
+ *                             for the CTAs that split a group's query heads; their
+ *                             sum is formed in a fixed order: results are
+ *                             deterministic).
  * With H_kv = H both are identical to fa_bwd_workspace_size / fa_bwd.  Everything
  * else as fa_bwd.
  */
