@@ -3,6 +3,7 @@
 //            with O = O_bf16 + residual when the forward's residual is given,
 //            i.e. the forward's fp32 O, so that D does not carry O's bf16 rounding
 //   lse2_i = LSE_i * log2(e)               (so the kernels form P = 2^(s*scale*log2e - lse2))
+//   counters         = 0: the work counters of the persistent backward kernels that follow
 //   q16, k16, v16, do16 = fp16 copies of the bf16 inputs (k16 / v16 for the first BH_kv
 //   heads only: with grouped-query attention K and V have fewer heads than Q)
 // Rows N..Np-1 of D / lse2 are padding for the 64/128-row tiles: D = 0 and
@@ -49,6 +50,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
   const int bh = valid_slot ? (int)(row_global / p.Np) : 0;
   const int i = valid_slot ? (int)(row_global % p.Np) : 0;
   const bool real = valid_slot && i < p.N;
+
+  if (blockIdx.x == 0 && threadIdx.x < kNumCounters) p.counters[threadIdx.x] = 0u;
 
   float dsum = 0.f;
   if (real) {

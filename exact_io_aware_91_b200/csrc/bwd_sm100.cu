@@ -90,22 +90,59 @@ __device__ __forceinline__ void issue_ts_split_part(uint32_t d_tmem, uint32_t a_
   }
 }
 
-// Write NC fp32 columns of this thread's TMEM lane to global row `dst` (times `mult`).
+// Coalesced store of a warp's rows: lane l holds NC fp32 values of row `row0 + l` (times
+// `mult`) to be written at dst_base + (row0 + l) * ld.  One lane per row would make each
+// store instruction touch 32 rows (32 cache lines); instead each 8-lane group transposes
+// its 8 x 8 block of float4 (per 32-column chunk) with three xor-shuffle butterfly stages,
+// after which store instruction i writes row 8g + i of every group g with 8 consecutive
+// lanes: four full 128-byte lines per instruction.  Rows >= n_rows are not written.
 template <int NC>
-__device__ __forceinline__ void store_rows_f32(uint32_t t_row, float* dst, float mult) {
-#pragma unroll 1
-  for (int c = 0; c < NC / 32; ++c) {
-    uint32_t u[32];
-    tmem_ld32(t_row + 32 * c, u);
-    tmem_wait_ld();
-    if (dst != nullptr) {
-      float4* out = reinterpret_cast<float4*>(dst + 32 * c);
+__device__ __forceinline__ void warp_store_rows_f32(const float (&v)[NC], float* dst_base, size_t ld, int row0,
+                                                    int n_rows, float mult) {
+  static_assert(NC % 32 == 0, "32-column chunks");
+  const int lane = threadIdx.x & 31;
+  const int gl = lane & 7;       // lane inside its group of 8
+  const int gbase = lane & ~7;   // first row (relative to row0) of this group
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        out[i] = make_float4(__uint_as_float(u[4 * i]) * mult, __uint_as_float(u[4 * i + 1]) * mult,
-                             __uint_as_float(u[4 * i + 2]) * mult, __uint_as_float(u[4 * i + 3]) * mult);
+  for (int ch = 0; ch < NC / 32; ++ch) {
+    float4 a[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      a[m] = make_float4(v[32 * ch + 4 * m] * mult, v[32 * ch + 4 * m + 1] * mult, v[32 * ch + 4 * m + 2] * mult,
+                         v[32 * ch + 4 * m + 3] * mult);
+    // after the stage with distance s, position m of lane l holds what position m ^ s of lane
+    // l ^ s held, wherever bit s of m differs from bit s of l: three stages transpose the block
+#pragma unroll
+    for (int s = 1; s < 8; s <<= 1) {
+      const bool hi = (gl & s) != 0;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        if (m & s) continue;
+        const float4 send = hi ? a[m] : a[m | s];
+        float4 recv;
+        recv.x = __shfl_xor_sync(0xffffffffu, send.x, s);
+        recv.y = __shfl_xor_sync(0xffffffffu, send.y, s);
+        recv.z = __shfl_xor_sync(0xffffffffu, send.z, s);
+        recv.w = __shfl_xor_sync(0xffffffffu, send.w, s);
+        if (hi)
+          a[m] = recv;
+        else
+          a[m | s] = recv;
+      }
+    }
+    // lane gl now holds columns [32 ch + 4 gl, +4) of rows gbase + i in a[i]
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = row0 + gbase + i;
+      if (r < n_rows) *reinterpret_cast<float4*>(dst_base + (size_t)r * ld + 32 * ch + 4 * gl) = a[i];
     }
   }
+}
+
+template <int N>
+__device__ __forceinline__ float (&acc_lo_view(float (&a)[N]))[64] {
+  static_assert(N >= 64, "needs 64 entries");
+  return *reinterpret_cast<float(*)[64]>(&a[0]);
 }
 
 // Load 64 fp32 columns of this thread's TMEM lane (two 32-column loads, one wait).
@@ -399,13 +436,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = mbar_wait(bar(L::BAR_ACC), 0, wctx);
     if (ok) {
       tc_fence_after();
-      // warpgroup 0 writes dV, warpgroup 1 writes scale * dK (rows past N are padding)
       // with the group split over several CTAs each writes its partial sums for the reduction
-      const size_t row_index = p.kv_split == 1 ? (size_t)bh * p.N + key
-                                                : ((size_t)sp * (p.BH / p.H * p.H_kv) + bh) * p.N + key;
-      float* out = p.kv_split == 1 ? (w == 0 ? p.dv : p.dk) : (w == 0 ? p.dv_part : p.dk_part);
-      float* dst = (key < p.N) ? (out + row_index * D) : nullptr;
-      store_rows_f32<D>(tmem + lane_off + (w == 0 ? L::T_DV : L::T_DK), dst, w == 0 ? 1.0f : p.scale);
+      const size_t head_off = p.kv_split == 1 ? (size_t)bh * p.N * D
+                                              : ((size_t)sp * (p.BH / p.H * p.H_kv) + bh) * p.N * D;
+      float* out = (p.kv_split == 1 ? (w == 0 ? p.dv : p.dk) : (w == 0 ? p.dv_part : p.dk_part)) + head_off;
+      float acc[D];
+      const uint32_t t_acc = tmem + lane_off + (w == 0 ? L::T_DV : L::T_DK);
+      if constexpr (D == 128) {
+        float hi[64];
+        tmem_ld64(t_acc, acc_lo_view(acc));
+        tmem_ld64(t_acc + 64, hi);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) acc[64 + c] = hi[c];
+      } else {
+        tmem_ld64(t_acc, acc_lo_view(acc));
+      }
+      // warpgroup 0 writes dV, warpgroup 1 writes scale * dK (rows past N are padding)
+      warp_store_rows_f32<D>(acc, out, D, j * 128 + wq * 32, p.N, w == 0 ? 1.0f : p.scale);
     }
   }
 
@@ -427,7 +474,7 @@ struct DqLayout {
   static constexpr int OFF_K = 2 * TILE;  // three K buffers
   static constexpr int OFF_V = 5 * TILE;  // two V buffers
   static constexpr int OFF_BAR = 7 * TILE;
-  static constexpr int BAR_Q = 0;
+  static constexpr int BAR_Q = 0;        // Q and dO of a unit landed
   static constexpr int BAR_K_FULL = 1;   // [3]
   static constexpr int BAR_K_EMPTY = 4;  // [3]
   static constexpr int BAR_V_FULL = 7;   // [2]
@@ -435,16 +482,29 @@ struct DqLayout {
   static constexpr int BAR_S = 11;       // [2]
   static constexpr int BAR_DP = 13;
   static constexpr int BAR_DS = 14;      // [2]
-  static constexpr int BAR_ACC = 16;
+  static constexpr int BAR_ACC = 16;     // a unit's dQ complete in TMEM
   static constexpr int BAR_DONE = 17;
-  static constexpr int NBAR = 18;
-  static constexpr int OFF_TMEM_SLOT = OFF_BAR + NBAR * 8;
+  static constexpr int BAR_Q_EMPTY = 18; // the MMAs reading a unit's Q and dO have completed
+  static constexpr int BAR_DQ_FREE = 19; // the epilogue has read a unit's dQ out of TMEM
+  static constexpr int BAR_UNIT_FULL = 20;   // [2] next work unit index published
+  static constexpr int BAR_UNIT_EMPTY = 22;  // [2] ... and read by the MMA warp and both warpgroups
+  static constexpr int NBAR = 24;
+  static constexpr int OFF_UNIT = OFF_BAR + NBAR * 8;  // int[2]: work unit ring
+  static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
   static constexpr int SMEM_ALLOC = OFF_ABORT + 8 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0, T_DP = 256, T_DQ = 384;  // S buffer b at T_S + 128 b
 };
 
+// Persistent dQ kernel: one CTA per SM takes work units one after another, so that one
+// unit's epilogue and the next unit's loads and first MMAs overlap instead of paying a CTA
+// launch, barrier and TMEM set-up and a pipeline fill per unit.  Units are handed out
+// dynamically in the order of unit_order (heaviest first within L2-sized head groups): the
+// producer warp takes the next index from a global counter (zeroed by the preprocess
+// kernel) and publishes it to the other roles through a two-slot ring in shared memory;
+// an index >= the unit count means "no more work".  Ring positions (K, V, S, dS, dP) count
+// steps across units; per-unit barriers (Q, Q_EMPTY, ACC, DQ_FREE) count units.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -463,15 +523,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   // heaviest first within groups of heads (see unit_order): under the causal mask the
   // last query tiles of a head meet the most key tiles
   const int nq = (p.N + 127) / 128;
-  int bh, rank;
-  unit_order((int)blockIdx.x, nq, p.BH, p.head_group, bh, rank);
-  const int bh_kv = kv_head_of(bh, p.H, p.H_kv);  // the key/value head this query head reads
-  const int qt = p.causal ? (nq - 1 - rank) : rank;
-  const int n_it = p.causal ? qt + 1 : nq;  // 128-key steps
+  const int n_units = nq * p.BH;
+  struct Unit {
+    int bh, bh_kv, qt, n_it;
+  };
+  auto unit_of = [&](int u) -> Unit {
+    Unit x;
+    int rank;
+    unit_order(u, nq, p.BH, p.head_group, x.bh, rank);
+    x.bh_kv = kv_head_of(x.bh, p.H, p.H_kv);  // the key/value head this query head reads
+    x.qt = p.causal ? (nq - 1 - rank) : rank;
+    x.n_it = p.causal ? x.qt + 1 : nq;        // 128-key steps
+    return x;
+  };
+
+  int* unit_ring = reinterpret_cast<int*>(gbase + L::OFF_UNIT);
+  // index of the k-th unit of this CTA (all roles call it in the same order, k = 0, 1, ...)
+  auto next_unit = [&](int k, bool& ok) -> int {
+    const int slot = k & 1;
+    ok = mbar_wait(bar(L::BAR_UNIT_FULL + slot), (k >> 1) & 1, wctx);
+    const int u = ok ? *reinterpret_cast<volatile int*>(unit_ring + slot) : n_units;
+    return u;
+  };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(bar(L::BAR_Q), 1);
+    mbar_init(bar(L::BAR_Q_EMPTY), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::BAR_UNIT_FULL + s), 1);
+      mbar_init(bar(L::BAR_UNIT_EMPTY + s), 1 + 256);
+    }
     for (int s = 0; s < 3; ++s) {
       mbar_init(bar(L::BAR_K_FULL + s), 1);
       mbar_init(bar(L::BAR_K_EMPTY + s), 1);
@@ -484,6 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(L::BAR_DP), 1);
     mbar_init(bar(L::BAR_ACC), 1);
+    mbar_init(bar(L::BAR_DQ_FREE), 256);
     mbar_init(bar(L::BAR_DONE), 1);
     fence_barrier_init();
   }
@@ -504,31 +587,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_do);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
-    mbar_arrive_expect_tx(bar(L::BAR_Q), 2 * L::TILE, leader);
-    for (int c = 0; c < L::KCH; ++c) {
-      tma_load_3d(base + L::OFF_Q + c * kBox, &tm_q, c * 64, qt * 128, bh, bar(L::BAR_Q), leader);
-      tma_load_3d(base + L::OFF_DO + c * kBox, &tm_do, c * 64, qt * 128, bh, bar(L::BAR_Q), leader);
+    int T = 0;   // K/V tiles issued (ring position, across units)
+    int uc = 0;  // units started
+    int q_issued = 0;
+    bool ok = true;
+    for (;; ++uc) {
+      // take the next unit and publish it (slot free once every consumer read unit uc - 2)
+      if (uc >= 2 && !(ok = mbar_wait(bar(L::BAR_UNIT_EMPTY + (uc & 1)), ((uc - 2) >> 1) & 1, wctx))) break;
+      int u = 0;
+      if (lane == 0) u = (int)atomicAdd(p.dq_counter, 1u);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (lane == 0) {
+        unit_ring[uc & 1] = u < n_units ? u : n_units;
+        mbar_arrive(bar(L::BAR_UNIT_FULL + (uc & 1)));
+      }
+      __syncwarp();
+      if (u >= n_units) break;
+      const Unit x = unit_of(u);
+      // Q, dO of this unit overwrite the previous unit's once its last S and dP MMAs are done
+      if (uc > 0 && !(ok = mbar_wait(bar(L::BAR_Q_EMPTY), (uc - 1) & 1, wctx))) break;
+      mbar_arrive_expect_tx(bar(L::BAR_Q), 2 * L::TILE, leader);
+      for (int c = 0; c < L::KCH; ++c) {
+        tma_load_3d(base + L::OFF_Q + c * kBox, &tm_q, c * 64, x.qt * 128, x.bh, bar(L::BAR_Q), leader);
+        tma_load_3d(base + L::OFF_DO + c * kBox, &tm_do, c * 64, x.qt * 128, x.bh, bar(L::BAR_Q), leader);
+      }
+      ++q_issued;
+      for (int it = 0; it < x.n_it; ++it, ++T) {
+        const int sk = T % 3, sv = T & 1;
+        if (!(ok = mbar_wait(bar(L::BAR_K_EMPTY + sk), ((T / 3) & 1) ^ 1u, wctx))) break;
+        mbar_arrive_expect_tx(bar(L::BAR_K_FULL + sk), L::TILE, leader);
+        for (int c = 0; c < L::KCH; ++c)
+          tma_load_3d(base + L::OFF_K + sk * L::TILE + c * kBox, &tm_k, c * 64, it * 128, x.bh_kv,
+                      bar(L::BAR_K_FULL + sk), leader);
+        if (!(ok = mbar_wait(bar(L::BAR_V_EMPTY + sv), ((T >> 1) & 1) ^ 1u, wctx))) {
+          ++T;  // the K tile of this step was issued
+          break;
+        }
+        mbar_arrive_expect_tx(bar(L::BAR_V_FULL + sv), L::TILE, leader);
+        for (int c = 0; c < L::KCH; ++c)
+          tma_load_3d(base + L::OFF_V + sv * L::TILE + c * kBox, &tm_v, c * 64, it * 128, x.bh_kv,
+                      bar(L::BAR_V_FULL + sv), leader);
+      }
     }
-    int issued = 0;
-    for (int it = 0; it < n_it; ++it) {
-      const int sk = it % 3, sv = it & 1;
-      if (!mbar_wait(bar(L::BAR_K_EMPTY + sk), ((it / 3) & 1) ^ 1u, wctx)) break;
-      mbar_arrive_expect_tx(bar(L::BAR_K_FULL + sk), L::TILE, leader);
-      for (int c = 0; c < L::KCH; ++c)
-        tma_load_3d(base + L::OFF_K + sk * L::TILE + c * kBox, &tm_k, c * 64, it * 128, bh_kv,
-                    bar(L::BAR_K_FULL + sk), leader);
-      if (!mbar_wait(bar(L::BAR_V_EMPTY + sv), ((it >> 1) & 1) ^ 1u, wctx)) break;
-      mbar_arrive_expect_tx(bar(L::BAR_V_FULL + sv), L::TILE, leader);
-      for (int c = 0; c < L::KCH; ++c)
-        tma_load_3d(base + L::OFF_V + sv * L::TILE + c * kBox, &tm_v, c * 64, it * 128, bh_kv,
-                    bar(L::BAR_V_FULL + sv), leader);
-      ++issued;
-    }
-    drain_wait(bar(L::BAR_Q), 0);
-    for (int it = (issued > 3 ? issued - 3 : 0); it < issued; ++it)
-      drain_wait(bar(L::BAR_K_FULL + it % 3), (it / 3) & 1);
-    for (int it = (issued > 2 ? issued - 2 : 0); it < issued; ++it)
-      drain_wait(bar(L::BAR_V_FULL + (it & 1)), (it >> 1) & 1);
+    // drain: every issued copy has landed before the CTA may exit
+    if (q_issued > 0) drain_wait(bar(L::BAR_Q), (q_issued - 1) & 1);
+    for (int t = (T > 3 ? T - 3 : 0); t < T; ++t) drain_wait(bar(L::BAR_K_FULL + t % 3), (t / 3) & 1);
+    for (int t = (T > 2 ? T - 2 : 0); t < T; ++t) drain_wait(bar(L::BAR_V_FULL + (t & 1)), (t >> 1) & 1);
   } else if (warp == 1) {
     // ===================================================== MMA issuer
     regs_dec<kRegsLow>();
@@ -540,52 +644,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dKk = make_sdesc_sw128(base + L::OFF_K, 16, 1024);      // K as K-major B
     const uint64_t dVk = make_sdesc_sw128(base + L::OFF_V, 16, 1024);      // V as K-major B
     const uint64_t dKmn = make_sdesc_sw128(base + L::OFF_K, kBox, 1024);   // K as MN-major B
-    auto issue_s = [&](int it) {  // S(it) = Q K_it^T into S buffer it & 1
-      issue_ss<D>(tmem + L::T_S + 128 * (it & 1), dQd, sdesc_add(dKk, (it % 3) * L::TILE), idesc_s, leader);
-      mma_commit(bar(L::BAR_S + (it & 1)), leader);
+    int T0 = 0;  // global step index of the current unit's step 0
+    // S(t) = Q K_t^T into S buffer t & 1 (t global)
+    auto issue_s = [&](int t) -> bool {
+      if (!mbar_wait(bar(L::BAR_K_FULL + t % 3), (t / 3) & 1, wctx)) return false;
+      tc_fence_after();
+      issue_ss<D>(tmem + L::T_S + 128 * (t & 1), dQd, sdesc_add(dKk, (t % 3) * L::TILE), idesc_s, leader);
+      mma_commit(bar(L::BAR_S + (t & 1)), leader);
+      return true;
     };
-    auto issue_dp = [&](int it) {  // dP(it) = dO V_it^T
-      issue_ss<D>(tmem + L::T_DP, dDO, sdesc_add(dVk, (it & 1) * L::TILE), idesc_s, leader);
+    // dP(t) = dO V_t^T
+    auto issue_dp = [&](int t) -> bool {
+      if (!mbar_wait(bar(L::BAR_V_FULL + (t & 1)), (t >> 1) & 1, wctx)) return false;
+      tc_fence_after();
+      issue_ss<D>(tmem + L::T_DP, dDO, sdesc_add(dVk, (t & 1) * L::TILE), idesc_s, leader);
       mma_commit(bar(L::BAR_DP), leader);
-      mma_commit(bar(L::BAR_V_EMPTY + (it & 1)), leader);
+      mma_commit(bar(L::BAR_V_EMPTY + (t & 1)), leader);
+      return true;
     };
-    bool ok = mbar_wait(bar(L::BAR_Q), 0, wctx);
-    if (ok) ok = mbar_wait(bar(L::BAR_K_FULL + 0), 0, wctx);
-    if (ok) {
+    bool ok = true;
+    for (int uc = 0;; ++uc) {
+      const int u = next_unit(uc, ok);
+      if (lane == 0) mbar_arrive(bar(L::BAR_UNIT_EMPTY + (uc & 1)));
+      if (!ok || u >= n_units) break;
+      const int n = unit_of(u).n_it;
+      if (!(ok = mbar_wait(bar(L::BAR_Q), uc & 1, wctx))) break;
       tc_fence_after();
-      issue_s(0);
-      ok = mbar_wait(bar(L::BAR_V_FULL + 0), 0, wctx);
-    }
-    if (ok) {
-      tc_fence_after();
-      issue_dp(0);
-      if (n_it > 1) {
-        ok = mbar_wait(bar(L::BAR_K_FULL + 1), 0, wctx);
-        if (ok) {
+      if (!(ok = issue_s(T0))) break;
+      if (!(ok = issue_dp(T0))) break;
+      if (n > 1 && !(ok = issue_s(T0 + 1))) break;
+      // the last MMAs that read this unit's Q / dO: S(n-1) and dP(n-1)
+      if (n == 1) mma_commit(bar(L::BAR_Q_EMPTY), leader);
+      for (int it = 0; it < n && ok; ++it) {
+        const int t = T0 + it;
+        const int b = t & 1;
+        if (!(ok = mbar_wait(bar(L::BAR_DS + b), (t >> 1) & 1, wctx))) break;
+        tc_fence_after();
+        // the first dQ MMA of a unit overwrites the accumulator: the previous unit's epilogue
+        // must have read it out of TMEM
+        if (it == 0 && uc > 0) {
+          if (!(ok = mbar_wait(bar(L::BAR_DQ_FREE), (uc - 1) & 1, wctx))) break;
           tc_fence_after();
-          issue_s(1);
         }
+        issue_ts_split(tmem + L::T_DQ, tmem + L::T_S + 128 * b, sdesc_add(dKmn, (t % 3) * L::TILE), idesc_g, it > 0,
+                       leader);  // dQ += dS K
+        mma_commit(bar(L::BAR_K_EMPTY + t % 3), leader);
+        if (it + 1 < n && !(ok = issue_dp(t + 1))) break;
+        if (it + 2 < n && !(ok = issue_s(t + 2))) break;
+        if (it + 2 == n) mma_commit(bar(L::BAR_Q_EMPTY), leader);  // S(n-1), dP(n-1) issued
       }
+      if (ok) mma_commit(bar(L::BAR_ACC), leader);
+      T0 += n;
     }
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int b = it & 1;
-      if (!(ok = mbar_wait(bar(L::BAR_DS + b), (it >> 1) & 1, wctx))) break;
-      tc_fence_after();
-      issue_ts_split(tmem + L::T_DQ, tmem + L::T_S + 128 * b, sdesc_add(dKmn, (it % 3) * L::TILE), idesc_g, it > 0,
-                     leader);  // dQ += dS K
-      mma_commit(bar(L::BAR_K_EMPTY + it % 3), leader);
-      if (it + 1 < n_it) {
-        if (!(ok = mbar_wait(bar(L::BAR_V_FULL + ((it + 1) & 1)), ((it + 1) >> 1) & 1, wctx))) break;
-        tc_fence_after();
-        issue_dp(it + 1);
-      }
-      if (it + 2 < n_it) {
-        if (!(ok = mbar_wait(bar(L::BAR_K_FULL + (it + 2) % 3), ((it + 2) / 3) & 1, wctx))) break;
-        tc_fence_after();
-        issue_s(it + 2);
-      }
-    }
-    if (ok) mma_commit(bar(L::BAR_ACC), leader);
     mma_commit(bar(L::BAR_DONE), leader);
     drain_wait(bar(L::BAR_DONE), 0);
   } else if (warp < 4) {
@@ -596,60 +706,96 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int w = (warp - 4) >> 2;   // key columns [64 w, 64 w + 64) of every step
     const int wq = (warp - 4) & 3;
     const int row = wq * 32 + lane;
-    const int r = qt * 128 + row;    // query index
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const float sl2 = p.scale_log2;
-    const size_t prow = (size_t)bh * p.Np + r;  // r < Np always (Np is a multiple of 128)
-    const float lse2 = p.lse2[prow];
-    const float delta = p.delta[prow];
-    const int lim = p.causal ? min(r, p.N - 1) : (p.N - 1);  // last visible key
-    const uint64_t sl2x2 = f2pack(sl2, sl2), nl2 = f2pack(-lse2, -lse2), dd = f2pack(delta, delta);
+    const uint64_t sl2x2 = f2pack(sl2, sl2);
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int b = it & 1;
-      const uint32_t tS = tmem + lane_off + L::T_S + 128 * b + 64 * w;
-      const int k0 = it * 128 + 64 * w;  // first key of this warpgroup's columns
-      const bool need_mask = (p.causal && k0 + 63 > qt * 128) || (k0 + 64 > p.N);
-      if (!(ok = mbar_wait(bar(L::BAR_S + b), (it >> 1) & 1, wctx))) break;
-      tc_fence_after();
-      float pr[64];
-      tmem_ld64(tS, pr);
-#pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        float t0, t1;
-        f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, nl2), t0, t1);
-        pr[c] = ex2_approx(t0);
-        pr[c + 1] = ex2_approx(t1);
-        if (need_mask) {
-          if (k0 + c > lim) pr[c] = 0.f;
-          if (k0 + c + 1 > lim) pr[c + 1] = 0.f;
-        }
-      }
-      if (!(ok = mbar_wait(bar(L::BAR_DP), it & 1, wctx))) break;
-      tc_fence_after();
-      float dp[64];
-      tmem_ld64(tmem + lane_off + L::T_DP + 64 * w, dp);
-#pragma unroll
-      for (int g = 0; g < 64; g += 16) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int c = g; c < g + 16; c += 2) {
-          float d0, d1;
-          f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(f2pack(dp[c], dp[c + 1]), dd)), d0, d1);
-          pk[(c - g) / 2] = pack_f16(d0, d1);
-        }
-        tmem_st8(tS + g / 2, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(L::BAR_DS + b));
+    int T0 = 0;
+    // this row's lse2 and delta, loaded one unit ahead (during the previous unit's epilogue)
+    float lse2 = 0.f, delta = 0.f;
+    int u = next_unit(0, ok);
+    mbar_arrive(bar(L::BAR_UNIT_EMPTY + 0));
+    if (ok && u < n_units) {
+      const Unit x0 = unit_of(u);
+      const size_t prow = (size_t)x0.bh * p.Np + x0.qt * 128 + row;  // < BH * Np (Np is a multiple of 128)
+      lse2 = p.lse2[prow];
+      delta = p.delta[prow];
     }
-    if (ok) ok = mbar_wait(bar(L::BAR_ACC), 0, wctx);
-    if (ok) {
+    for (int uc = 0; ok && u < n_units; ++uc) {
+      const Unit x = unit_of(u);
+      const int r = x.qt * 128 + row;  // query index
+      const int lim = p.causal ? min(r, p.N - 1) : (p.N - 1);  // last visible key
+      const uint64_t nl2 = f2pack(-lse2, -lse2), dd = f2pack(delta, delta);
+      for (int it = 0; it < x.n_it; ++it) {
+        const int t = T0 + it;
+        const int b = t & 1;
+        const uint32_t tS = tmem + lane_off + L::T_S + 128 * b + 64 * w;
+        const int k0 = it * 128 + 64 * w;  // first key of this warpgroup's columns
+        const bool need_mask = (p.causal && k0 + 63 > x.qt * 128) || (k0 + 64 > p.N);
+        if (!(ok = mbar_wait(bar(L::BAR_S + b), (t >> 1) & 1, wctx))) break;
+        tc_fence_after();
+        float pr[64];
+        tmem_ld64(tS, pr);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float t0, t1;
+          f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, nl2), t0, t1);
+          pr[c] = ex2_approx(t0);
+          pr[c + 1] = ex2_approx(t1);
+          if (need_mask) {
+            if (k0 + c > lim) pr[c] = 0.f;
+            if (k0 + c + 1 > lim) pr[c + 1] = 0.f;
+          }
+        }
+        if (!(ok = mbar_wait(bar(L::BAR_DP), t & 1, wctx))) break;
+        tc_fence_after();
+        float dp[64];
+        tmem_ld64(tmem + lane_off + L::T_DP + 64 * w, dp);
+#pragma unroll
+        for (int g = 0; g < 64; g += 16) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int c = g; c < g + 16; c += 2) {
+            float d0, d1;
+            f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(f2pack(dp[c], dp[c + 1]), dd)), d0, d1);
+            pk[(c - g) / 2] = pack_f16(d0, d1);
+          }
+          tmem_st8(tS + g / 2, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::BAR_DS + b));
+      }
+      if (!ok) break;
+      if (!(ok = mbar_wait(bar(L::BAR_ACC), uc & 1, wctx))) break;
       tc_fence_after();
-      // each warpgroup writes half of the columns of scale * dQ
-      float* dst = (r < p.N) ? (p.dq + ((size_t)bh * p.N + r) * D + w * (D / 2)) : nullptr;
-      store_rows_f32<D / 2>(tmem + lane_off + L::T_DQ + w * (D / 2), dst, p.scale);
+      // each warpgroup writes half of the columns of scale * dQ: read them out of TMEM,
+      // release the accumulator to the next unit, then store
+      float acc[D / 2];
+      if constexpr (D == 128) {
+        tmem_ld64(tmem + lane_off + L::T_DQ + w * 64, acc);
+      } else {
+        uint32_t uu[32];
+        tmem_ld32(tmem + lane_off + L::T_DQ + w * 32, uu);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) acc[c] = __uint_as_float(uu[c]);
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::BAR_DQ_FREE));
+      const int u_next = next_unit(uc + 1, ok);  // published long before: the producer runs ahead
+      mbar_arrive(bar(L::BAR_UNIT_EMPTY + ((uc + 1) & 1)));
+      if (ok && u_next < n_units) {  // prefetch the next unit's row statistics
+        const Unit xn = unit_of(u_next);
+        const size_t prow = (size_t)xn.bh * p.Np + xn.qt * 128 + row;
+        lse2 = p.lse2[prow];
+        delta = p.delta[prow];
+      }
+      // this warp's 32 query rows, columns [w D/2, (w + 1) D/2) of scale * dQ
+      warp_store_rows_f32<D / 2>(acc, p.dq + (size_t)x.bh * p.N * D + w * (D / 2), D, x.qt * 128 + wq * 32, p.N,
+                                 p.scale);
+      T0 += x.n_it;
+      u = u_next;
     }
   }
 
@@ -683,7 +829,9 @@ cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tdo,
 
 cudaError_t launch_bwd_dq_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                                 const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s) {
-  const dim3 grid((unsigned)(((p.N + 127) / 128) * p.BH));
+  // persistent: one CTA per SM (at most one per work unit)
+  const long long units = (long long)((p.N + 127) / 128) * p.BH;
+  const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
   if (d == 128) return launch_one<DqLayout<128>>(fa_bwd_dq_sm100_kernel<128>, grid, tq, tdo, tk, tv, p, s);
   return launch_one<DqLayout<64>>(fa_bwd_dq_sm100_kernel<64>, grid, tq, tdo, tk, tv, p, s);
 }

@@ -37,6 +37,7 @@ constexpr int kMaxDevices = 64;
 int* g_err_ptr[kMaxDevices];
 int g_cc_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 unsupported
 std::mutex g_mu;
+int g_num_sms[kMaxDevices] = {};  // multiprocessor count per device (persistent grids)
 thread_local void* const* t_phase_events = nullptr;  // see fa_bwd_set_phase_events
 
 // Checks the current device (compute capability 10.0) and resolves its error word.
@@ -53,6 +54,9 @@ fa_status device_setup(int* dev_out) {
     g_cc_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
   }
   if (g_cc_ok[dev] < 0) return FA_ERR_UNSUPPORTED;
+  if (g_num_sms[dev] == 0 &&
+      cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
   if (g_err_ptr[dev] == nullptr) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_fa_err_word) != cudaSuccess) return FA_ERR_CUDA;
@@ -85,7 +89,7 @@ fa_status check_problem(int B, int H, int H_kv, int N, int d, float scale, int c
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct BwdLayout {
-  size_t off_q16, off_k16, off_v16, off_do16, off_delta, off_lse2, off_dk_part, off_dv_part, total;
+  size_t off_q16, off_k16, off_v16, off_do16, off_delta, off_lse2, off_dk_part, off_dv_part, off_counters, total;
   int Np;
   int kv_split;
 };
@@ -105,7 +109,8 @@ int kv_split_for(int B, int H, int H_kv, int N) {
 
 // Workspace: fp16 copies of Q and dO (B*H heads) and of K and V (B*H_kv heads), then
 // D and LSE*log2(e) per query row padded to a multiple of 128 rows, then (only when the
-// group is split, see kv_split_for) fp32 partial dK and dV per split.
+// group is split, see kv_split_for) fp32 partial dK and dV per split, then 256 bytes for the
+// work counters of the persistent kernels.
 BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d) {
   BwdLayout w{};
   w.kv_split = kv_split_for(B, H, H_kv, N);
@@ -122,7 +127,8 @@ BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d) {
   w.off_dk_part = w.off_lse2 + rows;
   const size_t part = w.kv_split > 1 ? align256((size_t)w.kv_split * B * H_kv * N * d * 4) : 0;
   w.off_dv_part = w.off_dk_part + part;
-  w.total = w.off_dv_part + part;
+  w.off_counters = w.off_dv_part + part;
+  w.total = w.off_counters + 256;
   return w;
 }
 
@@ -275,6 +281,7 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
   pp.Np = w.Np;
   pp.BH = BH;
   pp.BH_kv = BH_kv;
+  pp.counters = reinterpret_cast<unsigned*>(ws + w.off_counters);
   pp.d = d;
   if (launch_bwd_pre(pp, s) != cudaSuccess) return FA_ERR_CUDA;
   if (t_phase_events != nullptr && t_phase_events[0] != nullptr &&
@@ -304,6 +311,8 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
   bp.head_group = head_group_size(BH, 4ull * N * d / group, kBwdGroupBytes);
   bp.head_group_kv = head_group_size(BH_kv, 4ull * N * d * (group / w.kv_split), kBwdGroupBytes);
   bp.kv_split = w.kv_split;
+  bp.num_sms = g_num_sms[dev];
+  bp.dq_counter = pp.counters;
   bp.dk_part = w.kv_split > 1 ? reinterpret_cast<float*>(ws + w.off_dk_part) : nullptr;
   bp.dv_part = w.kv_split > 1 ? reinterpret_cast<float*>(ws + w.off_dv_part) : nullptr;
   bp.scale = scale;

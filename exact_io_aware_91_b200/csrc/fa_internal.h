@@ -21,6 +21,8 @@ struct FwdParams {
   int* err;          // device error word
 };
 
+constexpr int kNumCounters = 2;  // [0] dQ kernel, [1] reserved
+
 struct BwdPreParams {
   const void* q;     // bf16 (BH, N, d)
   const void* k;
@@ -37,6 +39,7 @@ struct BwdPreParams {
   float* lse2;       // (BH, Np): LSE * log2(e); +inf on padded rows
   int N, Np, BH, d;
   int BH_kv;         // B * H_kv: rows of k / v / k16 / v16 (<= BH)
+  unsigned* counters;  // work counters of the persistent kernels, zeroed here (kNumCounters)
 };
 
 struct BwdParams {
@@ -52,6 +55,8 @@ struct BwdParams {
   int kv_split;        // CTAs sharing one (key/value head, key tile): each takes H/H_kv/kv_split query heads
   float* dk_part;      // with kv_split > 1: fp32 (kv_split, B*H_kv, N, d) partial dK (scaled) and dV,
   float* dv_part;      //   summed into dk / dv by launch_bwd_kv_reduce; unused when kv_split == 1
+  int num_sms;         // multiprocessors of the device (grid of the persistent kernels)
+  unsigned* dq_counter;  // work units handed out so far by the persistent dQ kernel (zeroed by the preprocess)
   float scale;         // softmax scale (applied to dQ and dK)
   float scale_log2;    // scale * log2(e)
   int causal;

@@ -111,8 +111,9 @@ FA_API fa_status fa_fwd_f32(const float* q, const float* k, const float* v, floa
 
 /*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for this
- * problem (fp16 copies of Q, K, V, dO and two fp32 (B, H, N rounded up to 128)
- * row vectors).  Returns 0 for an empty or invalid problem.
+ * problem (fp16 copies of Q, K, V, dO, two fp32 (B, H, N rounded up to 128) row
+ * vectors and 256 bytes of work counters).  Returns 0 for an empty or invalid
+ * problem.
  */
 FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 

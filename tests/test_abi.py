@@ -43,7 +43,7 @@ def test_status_strings(lib):
 def _ws_expected(B, H, N, d):
     a = lambda x: (x + 255) // 256 * 256  # noqa: E731
     Np = (N + 127) // 128 * 128
-    return 4 * a(B * H * N * d * 2) + 2 * a(B * H * Np * 4)
+    return 4 * a(B * H * N * d * 2) + 2 * a(B * H * Np * 4) + 256  # + work counters
 
 
 @pytest.mark.parametrize("shape", [(1, 1, 1, 64), (4, 16, 2048, 128), (2, 32, 8192, 128), (1, 8, 131072, 128),
@@ -59,7 +59,7 @@ def _ws_expected_gqa(B, H, Hkv, N, d):
     group, units = H // Hkv, B * Hkv * ((N + 127) // 128)
     split = next((s for s in range(1, group) if group % s == 0 and units * s >= 4 * 148), group)
     part = 2 * a(split * B * Hkv * N * d * 4) if split > 1 else 0
-    return 2 * a(B * H * N * d * 2) + 2 * a(B * Hkv * N * d * 2) + 2 * a(B * H * Np * 4) + part
+    return 2 * a(B * H * N * d * 2) + 2 * a(B * Hkv * N * d * 2) + 2 * a(B * H * Np * 4) + part + 256
 
 
 @pytest.mark.parametrize("shape", [(1, 4, 1, 1, 64), (2, 32, 8, 8192, 128), (1, 8, 1, 131072, 128),
