@@ -91,51 +91,19 @@ __device__ __forceinline__ void issue_ts_split_part(uint32_t d_tmem, uint32_t a_
 }
 
 // Coalesced store of a warp's rows: lane l holds NC fp32 values of row `row0 + l` (times
-// `mult`) to be written at dst_base + (row0 + l) * ld.  One lane per row would make each
-// store instruction touch 32 rows (32 cache lines); instead each 8-lane group transposes
-// its 8 x 8 block of float4 (per 32-column chunk) with three xor-shuffle butterfly stages,
-// after which store instruction i writes row 8g + i of every group g with 8 consecutive
-// lanes: four full 128-byte lines per instruction.  Rows >= n_rows are not written.
+// `mult`) to be written at dst_base + (row0 + l) * ld (in floats); see warp_store_rows_128b.
 template <int NC>
 __device__ __forceinline__ void warp_store_rows_f32(const float (&v)[NC], float* dst_base, size_t ld, int row0,
                                                     int n_rows, float mult) {
   static_assert(NC % 32 == 0, "32-column chunks");
-  const int lane = threadIdx.x & 31;
-  const int gl = lane & 7;       // lane inside its group of 8
-  const int gbase = lane & ~7;   // first row (relative to row0) of this group
 #pragma unroll
   for (int ch = 0; ch < NC / 32; ++ch) {
-    float4 a[8];
+    uint4 a[8];
 #pragma unroll
     for (int m = 0; m < 8; ++m)
-      a[m] = make_float4(v[32 * ch + 4 * m] * mult, v[32 * ch + 4 * m + 1] * mult, v[32 * ch + 4 * m + 2] * mult,
-                         v[32 * ch + 4 * m + 3] * mult);
-    // after the stage with distance s, position m of lane l holds what position m ^ s of lane
-    // l ^ s held, wherever bit s of m differs from bit s of l: three stages transpose the block
-#pragma unroll
-    for (int s = 1; s < 8; s <<= 1) {
-      const bool hi = (gl & s) != 0;
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        if (m & s) continue;
-        const float4 send = hi ? a[m] : a[m | s];
-        float4 recv;
-        recv.x = __shfl_xor_sync(0xffffffffu, send.x, s);
-        recv.y = __shfl_xor_sync(0xffffffffu, send.y, s);
-        recv.z = __shfl_xor_sync(0xffffffffu, send.z, s);
-        recv.w = __shfl_xor_sync(0xffffffffu, send.w, s);
-        if (hi)
-          a[m] = recv;
-        else
-          a[m | s] = recv;
-      }
-    }
-    // lane gl now holds columns [32 ch + 4 gl, +4) of rows gbase + i in a[i]
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = row0 + gbase + i;
-      if (r < n_rows) *reinterpret_cast<float4*>(dst_base + (size_t)r * ld + 32 * ch + 4 * gl) = a[i];
-    }
+      a[m] = make_uint4(__float_as_uint(v[32 * ch + 4 * m] * mult), __float_as_uint(v[32 * ch + 4 * m + 1] * mult),
+                        __float_as_uint(v[32 * ch + 4 * m + 2] * mult), __float_as_uint(v[32 * ch + 4 * m + 3] * mult));
+    warp_store_rows_128b(a, reinterpret_cast<uint8_t*>(dst_base + 32 * ch), ld * sizeof(float), row0, n_rows);
   }
 }
 

@@ -406,31 +406,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.0f / l;
       const uint32_t stage = base + (t ? L::OFF_Q1 : L::OFF_Q0);
+      // 64-column chunks: O / l rounded to bf16 goes to the swizzled staging tile (one 64-column
+      // TMA box); the bf16 residual goes straight to global memory, coalesced across the warp
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(tO + 32 * c, u);
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t u0[32], u1[32];
+        tmem_ld32(tO + 64 * c, u0);
+        tmem_ld32(tO + 64 * c + 32, u1);
         tmem_wait_ld();
-        uint32_t pk[16], rk[16];
+        uint32_t pk[32], rk[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = __uint_as_float(u[2 * i]) * inv_l, b = __uint_as_float(u[2 * i + 1]) * inv_l;
+        for (int i = 0; i < 32; ++i) {
+          const uint32_t* uu = i < 16 ? u0 : u1;
+          const int k = 2 * (i & 15);
+          const float a = __uint_as_float(uu[k]) * inv_l, b = __uint_as_float(uu[k + 1]) * inv_l;
           pk[i] = pack_bf16(a, b);
           const float2 ab = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
           rk[i] = pack_bf16(a - ab.x, b - ab.y);
         }
-        if (p.o_resid != nullptr && r < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o_resid + ((size_t)bh * p.N + r) * D + 32 * c);
+        if (p.o_resid != nullptr) {
+          uint4 ra[8];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            dst[q4] = make_uint4(rk[4 * q4], rk[4 * q4 + 1], rk[4 * q4 + 2], rk[4 * q4 + 3]);
+          for (int q4 = 0; q4 < 8; ++q4) ra[q4] = make_uint4(rk[4 * q4], rk[4 * q4 + 1], rk[4 * q4 + 2], rk[4 * q4 + 3]);
+          warp_store_rows_128b(ra, reinterpret_cast<uint8_t*>(p.o_resid + (size_t)bh * p.N * D + 64 * c), D * 2,
+                               q_base + wq * 32, p.N);
         }
-        const int box = (32 * c) / 64;
-        const int chunk0 = ((32 * c) % 64) / 8;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          st_shared_v4(stage + box * L::BOX + sw128_offset(row, chunk0 + q4), pk[4 * q4], pk[4 * q4 + 1],
-                       pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        for (int q4 = 0; q4 < 8; ++q4)
+          st_shared_v4(stage + c * L::BOX + sw128_offset(row, q4), pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2],
+                       pk[4 * q4 + 3]);
       }
       if (p.lse != nullptr && r < p.N) p.lse[(size_t)bh * p.N + r] = (m + __log2f(l)) * 0.69314718055994531f;
       fence_proxy_async_smem();

@@ -111,6 +111,45 @@ __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// ----------------------------------------------------------------- coalesced row stores
+// Lane l of a warp holds 128 bytes (a[0..7], 16 bytes each) of row `row0 + l`, to be written
+// at dst + (row0 + l) * ld_bytes.  One lane per row would make every store instruction touch
+// 32 rows (32 cache lines); instead each 8-lane group transposes its 8 x 8 block of 16-byte
+// units with three xor-shuffle butterfly stages (after the stage with distance s, position m
+// of lane l holds what position m ^ s of lane l ^ s held, wherever bit s of m differs from
+// bit s of l), after which store instruction i writes row 8g + i of every group g with 8
+// consecutive lanes: four full 128-byte lines per instruction.  Rows >= n_rows are skipped.
+__device__ __forceinline__ void warp_store_rows_128b(uint4 (&a)[8], uint8_t* dst, size_t ld_bytes, int row0,
+                                                     int n_rows) {
+  const int lane = threadIdx.x & 31;
+  const int gl = lane & 7;      // lane inside its group of 8
+  const int gbase = lane & ~7;  // first row (relative to row0) of this group
+#pragma unroll
+  for (int s = 1; s < 8; s <<= 1) {
+    const bool hi = (gl & s) != 0;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      if (m & s) continue;
+      const uint4 send = hi ? a[m] : a[m | s];
+      uint4 recv;
+      recv.x = __shfl_xor_sync(0xffffffffu, send.x, s);
+      recv.y = __shfl_xor_sync(0xffffffffu, send.y, s);
+      recv.z = __shfl_xor_sync(0xffffffffu, send.z, s);
+      recv.w = __shfl_xor_sync(0xffffffffu, send.w, s);
+      if (hi)
+        a[m] = recv;
+      else
+        a[m | s] = recv;
+    }
+  }
+  // lane gl now holds bytes [16 gl, 16 gl + 16) of rows gbase + i in a[i]
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = row0 + gbase + i;
+    if (r < n_rows) *reinterpret_cast<uint4*>(dst + (size_t)r * ld_bytes + 16 * gl) = a[i];
+  }
+}
+
 // ----------------------------------------------------------------- work order
 // CTA index -> (head, rank) where rank 0 is the unit with the most work.  Heads are taken
 // in groups of `group`; inside a group the units go heaviest first, interleaved over the
