@@ -250,10 +250,12 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     dv = torch.empty_like(dk)
     ws = torch.empty(api.fa_bwd_gqa_workspace_size(B, H, Hkv, N, d), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    if Hkv == H:
-        fwd_call, bwd_call = api.fa_fwd, api.fa_bwd
-    else:
-        fwd_call, bwd_call = api.fa_fwd_gqa, api.fa_bwd_gqa
+    # forward with a workspace: V converted to fp16 in one streaming pass, then the kernel
+    fws = torch.empty(api.fa_fwd_workspace_size(B, Hkv, N, d), dtype=torch.uint8, device=dev)
+    bwd_call = api.fa_bwd if Hkv == H else api.fa_bwd_gqa
+
+    def fwd_call(q, k, v, **kw):
+        return api.fa_fwd_ws(q, k, v, workspace=fws, **kw)
 
     def step():
         fwd_call(q, k, v, causal=w.causal, scale=w.scale, o=o, lse=lse, o_resid=res)
@@ -377,7 +379,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": 5 * args.steps,  # V conversion + forward, preprocess, dK/dV, dQ
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)

@@ -23,7 +23,7 @@ FA_ERR_MISALIGNED = 3
 FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
 
-EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_gqa_workspace_size",
+EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_workspace_size", "fa_fwd_ws", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_gqa_workspace_size",
            "fa_bwd_gqa", "fa_bwd_noalloc", "fa_device_status", "fa_bwd_set_phase_events", "fa_status_str")
 
 # Size of the scratch array fa_bwd_noalloc uses instead of a caller workspace.
@@ -56,6 +56,10 @@ def library() -> ctypes.CDLL:
     lib.fa_fwd.restype = i
     lib.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     lib.fa_fwd_gqa.restype = i
+    lib.fa_fwd_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_fwd_workspace_size.restype = sz
+    lib.fa_fwd_ws.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_fwd_ws.restype = i
     lib.fa_fwd_f32.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_fwd_f32.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
@@ -170,6 +174,37 @@ def fa_fwd_gqa(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool =
                               None if o_resid is None else o_resid.data_ptr(), B, H, H_kv, N, d, _scale(scale, d),
                               int(bool(causal)), _stream_handle(stream))
     _check("fa_fwd_gqa", st)
+    return (o, lse) if o_resid is None else (o, lse, o_resid)
+
+
+def fa_fwd_workspace_size(B: int, H_kv: int, N: int, d: int) -> int:
+    return int(library().fa_fwd_workspace_size(B, H_kv, N, d))
+
+
+def fa_fwd_ws(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+              scale: float | None = None, o: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+              o_resid: torch.Tensor | None = None, save_residual: bool = False, workspace=None, stream=None):
+    """Forward with a workspace (V converted to fp16 in one pass before the kernel); k, v may
+    have fewer heads than q (grouped-query).  Returns like ``fa_fwd``."""
+    B, H, N, d = _shape(q)
+    H_kv = _gqa_heads(q, k)
+    _same(q, dtype=torch.bfloat16, shape=(B, H, N, d))
+    _same(k, v, dtype=torch.bfloat16, shape=(B, H_kv, N, d))
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if o_resid is None and save_residual:
+        o_resid = torch.empty_like(q)
+    _same(o, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if o_resid is not None:
+        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if workspace is None:
+        workspace = torch.empty(max(fa_fwd_workspace_size(B, H_kv, N, d), 1), dtype=torch.uint8, device=q.device)
+    st = library().fa_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                             None if o_resid is None else o_resid.data_ptr(), B, H, H_kv, N, d, _scale(scale, d),
+                             int(bool(causal)), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    _check("fa_fwd_ws", st)
     return (o, lse) if o_resid is None else (o, lse, o_resid)
 
 

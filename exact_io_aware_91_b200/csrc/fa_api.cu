@@ -177,23 +177,35 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   return fa_fwd_gqa(q, k, v, o, lse, o_resid, B, H, H, N, d, scale, causal, stream);
 }
 
-fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
-                     int H_kv, int N, int d, float scale, int causal, fa_stream_t stream) {
+namespace {
+// Shared body of fa_fwd_gqa (V converted on chip) and fa_fwd_ws (V converted to fp16 into
+// the workspace by a streaming pass first).
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
+                   int H_kv, int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                   fa_stream_t stream) {
   bool empty = false;
   fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
   if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
-      !aligned(o_resid, 16))
+      !aligned(o_resid, 16) || !aligned(workspace, 256))
     return FA_ERR_MISALIGNED;
+  const size_t v16_bytes = align256((size_t)B * H_kv * N * d * 2);
+  if (workspace != nullptr && workspace_bytes < v16_bytes) return FA_ERR_INVALID_ARG;
   int dev = 0;
   if ((st = device_setup(&dev)) != FA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int BH = B * H, BH_kv = B * H_kv;
+  if (workspace != nullptr && launch_fwd_v16(v, workspace, (long long)BH_kv * N * d, s) != cudaSuccess)
+    return FA_ERR_CUDA;
   CUtensorMap tq, tk, tv, to;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const bool v16 = workspace != nullptr;
   if (!make_tmap_3d(&tq, q, bf, 2, d, N, BH, 64, 128, true) ||
       !make_tmap_3d(&tk, k, bf, 2, d, N, BH_kv, 64, 128, true) ||
-      !make_tmap_3d(&tv, v, bf, 2, d, N, BH_kv, 64, 128, true) || !make_tmap_3d(&to, o, bf, 2, d, N, BH, 64, 128, true))
+      !make_tmap_3d(&tv, v16 ? workspace : v, v16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : bf, 2, d, N, BH_kv, 64, 128,
+                    true) ||
+      !make_tmap_3d(&to, o, bf, 2, d, N, BH, 64, 128, true))
     return FA_ERR_CUDA;
   FwdParams p{};
   p.lse = lse;
@@ -208,9 +220,30 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal;
   p.err = g_err_ptr[dev];
-  return launch_fwd_sm100(tq, tk, tv, to, p, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? FA_OK
-             : FA_ERR_CUDA;
+  return launch_fwd_sm100(tq, tk, tv, to, p, d, v16, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+}  // namespace
+
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
+                     int H_kv, int N, int d, float scale, int causal, fa_stream_t stream) {
+  return fwd_impl(q, k, v, o, lse, o_resid, B, H, H_kv, N, d, scale, causal, nullptr, 0, stream);
+}
+
+size_t fa_fwd_workspace_size(int B, int H_kv, int N, int d) {
+  bool empty = false;
+  if (check_problem(B, H_kv, H_kv, N, d, 1.0f, 0, &empty) != FA_OK || empty) return 0;
+  return align256((size_t)B * H_kv * N * d * 2);
+}
+
+fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
+                    int H_kv, int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                    fa_stream_t stream) {
+  if (workspace == nullptr) {
+    bool empty = false;
+    const fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty);
+    return (st != FA_OK || empty) ? st : FA_ERR_INVALID_ARG;
+  }
+  return fwd_impl(q, k, v, o, lse, o_resid, B, H, H_kv, N, d, scale, causal, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N,

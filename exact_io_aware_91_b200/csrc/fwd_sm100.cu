@@ -94,7 +94,10 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-template <int D>
+// kVf16: V arrives already converted to fp16 (fa_fwd_ws converts it in a streaming pass
+// first); warps 2-3 then have nothing to do, and the softmax warps sharing their SM
+// sub-partitions run as fast as the others.
+template <int D, bool kVf16>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -248,7 +251,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_qk(tS[1], dQ[1], stK);
         mma_commit(bar(L::BAR_S_FULL + 1), leader);
         mma_commit(bar(L::BAR_KV_EMPTY + stK), leader);
-        if (!(ok = mbar_wait(bar(L::BAR_V_CONV + stV), (iV / L::STAGES) & 1, wctx))) break;
+        if (kVf16) {
+          if (!(ok = mbar_wait(bar(L::BAR_KV_FULL + stV), (iV / L::STAGES) & 1, wctx))) break;
+        } else {
+          if (!(ok = mbar_wait(bar(L::BAR_V_CONV + stV), (iV / L::STAGES) & 1, wctx))) break;
+        }
         tc_fence_after();
         if (j < n0) {  // O0 += P0 V_j
           if (!(ok = issue_pv(0, tO[0], tS[0], stV, j > 0, j & 1))) break;
@@ -267,6 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar(L::BAR_MMA_DONE), leader);
       drain_wait(bar(L::BAR_MMA_DONE), 0);
     }
+  } else if ((warp == 2 || warp == 3) && kVf16) {
+    regs_dec<kRegsLow>();  // V is fp16 already: nothing to convert
   } else if (warp == 2 || warp == 3) {
     // ===================================================== V tiles: bf16 -> fp16 in place
     regs_dec<kRegsLow>();
@@ -458,22 +467,47 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t s) {
+namespace {
+template <int D, bool kVf16>
+cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                         const FwdParams& p, cudaStream_t s) {
+  using L = FwdLayout<D>;
   const dim3 grid((unsigned)(p.n_pairs * p.BH));
-  if (d == 128) {
-    using L = FwdLayout<128>;
-    cudaError_t e = cudaFuncSetAttribute(fa_fwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         L::SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    fa_fwd_sm100_kernel<128><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, to, p);
-  } else {
-    using L = FwdLayout<64>;
-    cudaError_t e = cudaFuncSetAttribute(fa_fwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         L::SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    fa_fwd_sm100_kernel<64><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, to, p);
+  cudaError_t e = cudaFuncSetAttribute(fa_fwd_sm100_kernel<D, kVf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       L::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  fa_fwd_sm100_kernel<D, kVf16><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, to, p);
+  return cudaGetLastError();
+}
+
+// V (bf16) -> fp16 copy, 8 elements per 16-byte access (exact for |v| in [2^-14, 65504]).
+__global__ void __launch_bounds__(256) fa_fwd_v16_kernel(const uint4* __restrict__ v, uint4* __restrict__ v16,
+                                                         long long n8) {
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n8; e += (long long)gridDim.x * blockDim.x) {
+    uint4 u = v[e];
+    uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      w[i] = pack_f16(f.x, f.y);
+    }
+    v16[e] = u;
   }
+}
+}  // namespace
+
+cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& to, const FwdParams& p, int d, bool v_is_f16, cudaStream_t s) {
+  if (d == 128)
+    return v_is_f16 ? launch_fwd_t<128, true>(tq, tk, tv, to, p, s) : launch_fwd_t<128, false>(tq, tk, tv, to, p, s);
+  return v_is_f16 ? launch_fwd_t<64, true>(tq, tk, tv, to, p, s) : launch_fwd_t<64, false>(tq, tk, tv, to, p, s);
+}
+
+cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, cudaStream_t s) {
+  const long long n8 = elems / 8;  // d is a multiple of 8
+  long long blocks = (n8 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  fa_fwd_v16_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8);
   return cudaGetLastError();
 }
 

@@ -101,6 +101,24 @@ FA_API fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o
                             int H, int H_kv, int N, int d, float scale, int causal, fa_stream_t stream);
 
 /*
+ * fa_fwd_workspace_size / fa_fwd_ws -- the forward pass of fa_fwd_gqa (H_kv = H for
+ * plain multi-head attention) with a caller workspace, used to run the V operand's
+ * bf16 -> fp16 conversion as one streaming pass before the attention kernel instead of
+ * inside it (fa_fwd / fa_fwd_gqa convert each V tile on chip, on two warps that share
+ * SM sub-partitions with half of the softmax warps).  Results are identical to fa_fwd_gqa.
+ *   workspace       : device buffer of at least fa_fwd_workspace_size(B, H_kv, N, d)
+ *                     bytes (an fp16 copy of V), 256-byte aligned, caller-owned; contents
+ *                     on entry do not matter, unspecified on return.  NULL is an error.
+ *   workspace_bytes : its size.
+ * fa_fwd_workspace_size returns 0 for an empty or invalid problem.  Everything else as
+ * fa_fwd_gqa.
+ */
+FA_API size_t fa_fwd_workspace_size(int B, int H_kv, int N, int d);
+FA_API fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B,
+                           int H, int H_kv, int N, int d, float scale, int causal, void* workspace,
+                           size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fa_fwd_f32 -- the same forward pass on fp32 inputs and outputs, computed
  * entirely in fp32 on the CUDA cores (no input rounding).  Meant for small
  * problems and checks; same arguments and rules as fa_fwd except dtypes, and

@@ -86,6 +86,21 @@ def test_gqa_head_counts_are_checked(lib):
                           _ws_expected_gqa(1, 8, 2, 16, 64) - 1, None) == api.FA_ERR_INVALID_ARG
 
 
+def test_forward_workspace(lib):
+    a = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert api.fa_fwd_workspace_size(2, 8, 8192, 128) == a(2 * 8 * 8192 * 128 * 2)
+    assert api.fa_fwd_workspace_size(1, 1, 300, 64) == a(300 * 64 * 2)
+    assert api.fa_fwd_workspace_size(0, 8, 100, 64) == 0
+    assert api.fa_fwd_workspace_size(1, 1, 100, 96) == 0
+    ws = lambda ptr=A, n=1 << 40, H=4, Hkv=2: lib.fa_fwd_ws(A, A, A, A, A, None, 1, H, Hkv, 16, 64, 0.125, 0,  # noqa: E731
+                                                            ptr, n, None)
+    assert ws(ptr=None) == api.FA_ERR_INVALID_ARG
+    assert ws(n=api.fa_fwd_workspace_size(1, 2, 16, 64) - 1) == api.FA_ERR_INVALID_ARG
+    assert ws(ptr=A + 16) == api.FA_ERR_MISALIGNED
+    assert ws(H=6, Hkv=4) == api.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_ws(None, None, None, None, None, None, 1, 4, 2, 0, 64, 0.125, 0, None, 0, None) == api.FA_OK
+
+
 def test_workspace_size_of_empty_or_bad_problem_is_zero(lib):
     assert api.fa_bwd_workspace_size(0, 1, 10, 64) == 0
     assert api.fa_bwd_workspace_size(1, 1, 0, 64) == 0

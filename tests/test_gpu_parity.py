@@ -113,6 +113,21 @@ def test_gqa_fwd_bwd(B, H, Hkv, N, d, causal):
             assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("B,H,Hkv,N,d,causal", [(1, 2, 2, 300, 128, True), (1, 2, 2, 257, 64, False),
+                                                (2, 4, 1, 1000, 128, True), (1, 6, 3, 129, 64, True)])
+def test_forward_with_workspace_matches_on_chip_conversion(B, H, Hkv, N, d, causal):
+    # fa_fwd_ws (V converted to fp16 by a separate pass) == fa_fwd_gqa (converted on chip), bit for bit
+    inp = inputs.make_qkv(B, H, N, d, seed=N + H + Hkv, kv_heads=Hkv, backward=False, device="cuda")
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    scale = 1.0 / np.sqrt(d)
+    o1, l1, r1 = api.fa_fwd_gqa(q, k, v, causal=causal, scale=scale, save_residual=True)
+    o2, l2, r2 = api.fa_fwd_ws(q, k, v, causal=causal, scale=scale, save_residual=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2) and torch.equal(r1, r2)
+    O, L = oracle.attention_forward_gqa(q, k, v, scale, causal)
+    assert_fwd(o2, l2, O, L, f"fa_fwd_ws B={B} H={H} Hkv={Hkv} N={N} d={d} causal={causal}")
+
+
 def test_gqa_long_spiky_matches_oracle_rows():
     # a long grouped problem with peaked softmax rows: all of dK/dV of one key/value head
     # against the oracle, which materialises N x N per query head
