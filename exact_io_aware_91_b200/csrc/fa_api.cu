@@ -191,12 +191,14 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
       !aligned(o_resid, 16) || !aligned(workspace, 256))
     return FA_ERR_MISALIGNED;
   const size_t v16_bytes = align256((size_t)B * H_kv * N * d * 2);
-  if (workspace != nullptr && workspace_bytes < v16_bytes) return FA_ERR_INVALID_ARG;
+  if (workspace != nullptr && workspace_bytes < v16_bytes + 256) return FA_ERR_INVALID_ARG;
   int dev = 0;
   if ((st = device_setup(&dev)) != FA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int BH = B * H, BH_kv = B * H_kv;
-  if (workspace != nullptr && launch_fwd_v16(v, workspace, (long long)BH_kv * N * d, s) != cudaSuccess)
+  unsigned* counter = workspace != nullptr ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + v16_bytes)
+                                           : nullptr;
+  if (workspace != nullptr && launch_fwd_v16(v, workspace, (long long)BH_kv * N * d, counter, s) != cudaSuccess)
     return FA_ERR_CUDA;
   CUtensorMap tq, tk, tv, to;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -209,7 +211,10 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     return FA_ERR_CUDA;
   FwdParams p{};
   p.lse = lse;
+  p.o = static_cast<__nv_bfloat16*>(o);
   p.o_resid = static_cast<__nv_bfloat16*>(o_resid);
+  p.counter = counter;
+  p.num_sms = g_num_sms[dev];
   p.N = N;
   p.BH = BH;
   p.H = H;
@@ -220,7 +225,10 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal;
   p.err = g_err_ptr[dev];
-  return launch_fwd_sm100(tq, tk, tv, to, p, d, v16, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  // with a workspace: the persistent kernel (work counter in the workspace); without: one CTA
+  // per unit, V converted on chip
+  const cudaError_t e = v16 ? launch_fwd_persist_sm100(tq, tk, tv, p, d, s) : launch_fwd_sm100(tq, tk, tv, to, p, d, s);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 }  // namespace
 
@@ -232,7 +240,7 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float
 size_t fa_fwd_workspace_size(int B, int H_kv, int N, int d) {
   bool empty = false;
   if (check_problem(B, H_kv, H_kv, N, d, 1.0f, 0, &empty) != FA_OK || empty) return 0;
-  return align256((size_t)B * H_kv * N * d * 2);
+  return align256((size_t)B * H_kv * N * d * 2) + 256;  // fp16 V, then the work counter
 }
 
 fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,

@@ -10,6 +10,9 @@ namespace fa {
 
 struct FwdParams {
   float* lse;        // (B*H, N) fp32, natural-log LSE of the scaled scores; may be null
+  __nv_bfloat16* o;  // (B*H, N, d) bf16 output (the persistent kernel stores it directly)
+  unsigned* counter; // persistent kernel: work units handed out so far (zeroed by the V conversion)
+  int num_sms;       // persistent kernel: grid size
   __nv_bfloat16* o_resid;  // (B*H, N, d) bf16 residual O_fp32 - O_bf16; may be null
   int N;             // sequence length (queries = keys)
   int BH;            // B * H (query heads)
@@ -81,8 +84,10 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int 
                   int box_cols, int box_rows, bool swizzle128);
 
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& to, const FwdParams& p, int d, bool v_is_f16, cudaStream_t s);
-cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, cudaStream_t s);
+                             const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t s);
+cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, cudaStream_t s);
+cudaError_t launch_fwd_persist_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                     const FwdParams& p, int d, cudaStream_t s);
 cudaError_t launch_bwd_kv_reduce(const float* dk_part, const float* dv_part, float* dk, float* dv,
                                  long long elems, int splits, cudaStream_t s);
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int BH, int N,

@@ -94,10 +94,110 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-// kVf16: V arrives already converted to fp16 (fa_fwd_ws converts it in a streaming pass
-// first); warps 2-3 then have nothing to do, and the softmax warps sharing their SM
-// sub-partitions run as fast as the others.
-template <int D, bool kVf16>
+// One online-softmax step of a query tile (one thread per row): S_j from TMEM, mask,
+// running maximum (kept while within 2^8 of the true one), O rescaled in TMEM when the
+// maximum moves, P = 2^(scale*log2(e)*S - m) written back over S as fp16 in two halves
+// (the tensor core starts on the first half's P V while the second half is computed).
+// Returns false if a bounded wait gave up.
+template <int D>
+__device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS, uint32_t tO, uint32_t bar_s_full,
+                                                 uint32_t s_parity, uint32_t bar_p_half, uint32_t bar_p_full, int j,
+                                                 int q_base, int r, float& m, float& l, const WaitCtx& wctx) {
+  const float sl2 = p.scale_log2;
+  if (!mbar_wait(bar_s_full, s_parity, wctx)) return false;
+    tc_fence_after();
+    float x[128];
+    {
+      uint32_t u[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, u[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(u[c][i]);
+    }
+    const int kb = j * 128;
+    const bool need_mask = (p.causal && kb + 127 > q_base) || (kb + 128 > p.N);
+    if (need_mask) {
+      const int lim = p.causal ? min(r, p.N - 1) : (p.N - 1);  // last visible key
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        if (kb + c > lim) x[c] = -INFINITY;
+    }
+    // row max: four independent 3-input max chains
+    float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
+#pragma unroll
+    for (int c = 4; c < 124; c += 8) {
+      a0 = max3f(a0, x[c], x[c + 1]);
+      a1 = max3f(a1, x[c + 2], x[c + 3]);
+      a2 = max3f(a2, x[c + 4], x[c + 5]);
+      a3 = max3f(a3, x[c + 6], x[c + 7]);
+    }
+    a0 = max3f(a0, x[124], x[125]);
+    a1 = max3f(a1, x[126], x[127]);
+    const float mx = max3f(fmaxf(a0, a1), a2, a3);
+    const float m_new = fmaxf(m, mx * sl2);
+    // keep a stale maximum while it is within 2^8 of the true one: exact in the end
+    // because O / l and the LSE use the same maximum
+    const float m_use = (m_new - m > 8.0f) ? m_new : m;
+    const float alpha = (m_use == m) ? 1.0f : ex2_approx(m - m_use);  // 0 on the first tile
+    const float neg_m = -m_use;
+    if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+      // rescale O before this tile's P V starts; the previous O += P V of this tile
+      // completed before S_j did (same issuing thread, in-order tensor pipe)
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tO + 32 * c, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+        tmem_st32(tO + 32 * c, u);
+      }
+    }
+    uint64_t sa = 0, sb = 0;  // packed fp32 partial row sums (0.0f, 0.0f)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        float* e = &x[64 * h + 2 * i];
+        fma2(e[0], e[1], sl2, neg_m);
+        fma2(e[2], e[3], sl2, neg_m);
+        // kExpFmaPer8 of every 8 element pairs take 2^x on the FMA pipe, the rest on MUFU
+        if ((i & 7) < 2 * (kExpFmaPer8 / 2)) {
+          exp2_fma_pipe(e[0], e[1]);
+          exp2_fma_pipe(e[2], e[3]);
+          pk[i] = pack_f16(e[0], e[1]);
+          pk[i + 1] = pack_f16(e[2], e[3]);
+        } else {
+          e[0] = ex2_approx(e[0]);
+          e[1] = ex2_approx(e[1]);
+          e[2] = ex2_approx(e[2]);
+          e[3] = ex2_approx(e[3]);
+          pk[i] = pack_f16(e[0], e[1]);
+          pk[i + 1] = pack_f16(e[2], e[3]);
+        }
+        asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sa) : "l"(f2pack(e[0], e[1])));
+        asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sb) : "l"(f2pack(e[2], e[3])));
+      }
+      tmem_st32(tS + 32 * h, pk);
+      // first half of P (and any rescale of O) visible to the tensor core: its half of P V
+      // can start while the second half is computed
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(h == 0 ? bar_p_half : bar_p_full);
+    }
+    float s0, s1, s2, s3;
+    f2unpack(sa, s0, s1);
+    f2unpack(sb, s2, s3);
+    l = fmaf(l, alpha, (s0 + s1) + (s2 + s3));
+    m = m_use;
+  return true;
+}
+
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -251,11 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_qk(tS[1], dQ[1], stK);
         mma_commit(bar(L::BAR_S_FULL + 1), leader);
         mma_commit(bar(L::BAR_KV_EMPTY + stK), leader);
-        if (kVf16) {
-          if (!(ok = mbar_wait(bar(L::BAR_KV_FULL + stV), (iV / L::STAGES) & 1, wctx))) break;
-        } else {
-          if (!(ok = mbar_wait(bar(L::BAR_V_CONV + stV), (iV / L::STAGES) & 1, wctx))) break;
-        }
+        if (!(ok = mbar_wait(bar(L::BAR_V_CONV + stV), (iV / L::STAGES) & 1, wctx))) break;
         tc_fence_after();
         if (j < n0) {  // O0 += P0 V_j
           if (!(ok = issue_pv(0, tO[0], tS[0], stV, j > 0, j & 1))) break;
@@ -274,8 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar(L::BAR_MMA_DONE), leader);
       drain_wait(bar(L::BAR_MMA_DONE), 0);
     }
-  } else if ((warp == 2 || warp == 3) && kVf16) {
-    regs_dec<kRegsLow>();  // V is fp16 already: nothing to convert
   } else if (warp == 2 || warp == 3) {
     // ===================================================== V tiles: bf16 -> fp16 in place
     regs_dec<kRegsLow>();
@@ -312,102 +406,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + (t ? L::T_S1 : L::T_S0);
     const uint32_t tO = tmem + lane_off + (t ? L::T_O1 : L::T_O0);
-    const float sl2 = p.scale_log2;
 
     float m = -INFINITY;  // running max of scale*log2(e)*S (possibly stale by < 8)
     float l = 0.f;        // running sum of 2^(scale*log2(e)*S - m)
     bool ok = true;
     for (int j = 0; j < n_t; ++j) {
-      if (!(ok = mbar_wait(bar(L::BAR_S_FULL + t), j & 1, wctx))) break;
-      tc_fence_after();
-      float x[128];
-      {
-        uint32_t u[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, u[c]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(u[c][i]);
-      }
-      const int kb = j * 128;
-      const bool need_mask = (p.causal && kb + 127 > q_base) || (kb + 128 > p.N);
-      if (need_mask) {
-        const int lim = p.causal ? min(r, p.N - 1) : (p.N - 1);  // last visible key
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (kb + c > lim) x[c] = -INFINITY;
-      }
-      // row max: four independent 3-input max chains
-      float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
-#pragma unroll
-      for (int c = 4; c < 124; c += 8) {
-        a0 = max3f(a0, x[c], x[c + 1]);
-        a1 = max3f(a1, x[c + 2], x[c + 3]);
-        a2 = max3f(a2, x[c + 4], x[c + 5]);
-        a3 = max3f(a3, x[c + 6], x[c + 7]);
-      }
-      a0 = max3f(a0, x[124], x[125]);
-      a1 = max3f(a1, x[126], x[127]);
-      const float mx = max3f(fmaxf(a0, a1), a2, a3);
-      const float m_new = fmaxf(m, mx * sl2);
-      // keep a stale maximum while it is within 2^8 of the true one: exact in the end
-      // because O / l and the LSE use the same maximum
-      const float m_use = (m_new - m > 8.0f) ? m_new : m;
-      const float alpha = (m_use == m) ? 1.0f : ex2_approx(m - m_use);  // 0 on the first tile
-      const float neg_m = -m_use;
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        // rescale O before this tile's P V starts; the previous O += P V of this tile
-        // completed before S_j did (same issuing thread, in-order tensor pipe)
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld32(tO + 32 * c, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st32(tO + 32 * c, u);
-        }
-      }
-      uint64_t sa = 0, sb = 0;  // packed fp32 partial row sums (0.0f, 0.0f)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float* e = &x[64 * h + 2 * i];
-          fma2(e[0], e[1], sl2, neg_m);
-          fma2(e[2], e[3], sl2, neg_m);
-          // kExpFmaPer8 of every 8 element pairs take 2^x on the FMA pipe, the rest on MUFU
-          if ((i & 7) < 2 * (kExpFmaPer8 / 2)) {
-            exp2_fma_pipe(e[0], e[1]);
-            exp2_fma_pipe(e[2], e[3]);
-            pk[i] = pack_f16(e[0], e[1]);
-            pk[i + 1] = pack_f16(e[2], e[3]);
-          } else {
-            e[0] = ex2_approx(e[0]);
-            e[1] = ex2_approx(e[1]);
-            e[2] = ex2_approx(e[2]);
-            e[3] = ex2_approx(e[3]);
-            pk[i] = pack_f16(e[0], e[1]);
-            pk[i + 1] = pack_f16(e[2], e[3]);
-          }
-          asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sa) : "l"(f2pack(e[0], e[1])));
-          asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sb) : "l"(f2pack(e[2], e[3])));
-        }
-        tmem_st32(tS + 32 * h, pk);
-        // first half of P (and any rescale of O) visible to the tensor core: its half of P V
-        // can start while the second half is computed
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(L::BAR_P_HALF + t + 2 * h));  // BAR_P_FULL = BAR_P_HALF + 2
-      }
-      float s0, s1, s2, s3;
-      f2unpack(sa, s0, s1);
-      f2unpack(sb, s2, s3);
-      l = fmaf(l, alpha, (s0 + s1) + (s2 + s3));
-      m = m_use;
+      if (!(ok = fwd_softmax_step<D>(p, tS, tO, bar(L::BAR_S_FULL + t), j & 1, bar(L::BAR_P_HALF + t),
+                                     bar(L::BAR_P_FULL + t), j, q_base, r, m, l, wctx)))
+        break;
     }
     // ---- epilogue: O / l -> bf16 -> swizzled staging (the Q tile's buffer) -> TMA store
     if (ok) ok = mbar_wait(bar(L::BAR_O_FULL + t), 0, wctx);
@@ -468,21 +474,351 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 namespace {
-template <int D, bool kVf16>
+// ============================================================================ persistent
+// Persistent forward (fa_fwd_ws): one CTA per SM takes work units (pairs of 128-row query
+// tiles) one after another from a work counter in the caller's workspace (zeroed by the V
+// conversion pass), in the order of unit_order; the producer warp takes each index and
+// publishes it to the other roles through a two-slot ring in shared memory (an index >=
+// the unit count means "no more work").  The next unit's Q loads and first Q K^T products
+// overlap the previous unit's last steps and epilogue.  V is fp16 already.  K/V ring
+// positions count loads across units, the per-tile barriers (S_FULL, P_HALF, P_FULL)
+// count that tile's steps across units, and the per-unit barriers (Q_FULL, Q_EMPTY,
+// O_FULL, O_FREE) count units.  O and the residual are stored straight from registers
+// (coalesced by warp_store_rows_128b): the Q buffers are reloaded for the next unit and
+// cannot serve as the output staging tile.
+template <int D>
+struct FwdPLayout {
+  static constexpr int KCH = D / 64;
+  static constexpr int BOX = 128 * 128;
+  static constexpr int TILE = KCH * BOX;
+  static constexpr int STAGES = (D == 128) ? 4 : 8;
+  static constexpr int OFF_Q0 = 0;
+  static constexpr int OFF_Q1 = TILE;
+  static constexpr int OFF_KV = 2 * TILE;
+  static constexpr int OFF_BAR = OFF_KV + STAGES * TILE;
+  static constexpr int BAR_Q_FULL = 0;
+  static constexpr int BAR_Q_EMPTY = 1;
+  static constexpr int BAR_KV_FULL = 2;
+  static constexpr int BAR_KV_EMPTY = 2 + STAGES;
+  static constexpr int BAR_S_FULL = 2 + 2 * STAGES;  // [2]
+  static constexpr int BAR_P_HALF = BAR_S_FULL + 2;  // [2]
+  static constexpr int BAR_P_FULL = BAR_P_HALF + 2;  // [2]
+  static constexpr int BAR_O_FULL = BAR_P_FULL + 2;  // [2]
+  static constexpr int BAR_O_FREE = BAR_O_FULL + 2;  // [2] a tile's epilogue has read O out of TMEM
+  static constexpr int BAR_UNIT_FULL = BAR_O_FREE + 2;   // [2]
+  static constexpr int BAR_UNIT_EMPTY = BAR_UNIT_FULL + 2;  // [2]
+  static constexpr int BAR_MMA_DONE = BAR_UNIT_EMPTY + 2;
+  static constexpr int NBAR = BAR_MMA_DONE + 1;
+  static constexpr int OFF_UNIT = OFF_BAR + NBAR * 8;  // int[2]
+  static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
+  static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
+  static constexpr int SMEM_ALLOC = OFF_ABORT + 8 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_persist_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdPLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + L::OFF_BAR + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_ABORT);
+  const WaitCtx wctx{abort_flag, p.err};
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int n_units = p.n_pairs * p.BH;
+  const int n_kv = (p.N + 127) / 128;
+  struct Unit {
+    int bh, bh_kv, q_base0, n0, n1;
+  };
+  auto unit_of = [&](int u) -> Unit {
+    Unit x;
+    int rank;
+    unit_order(u, p.n_pairs, p.BH, p.head_group, x.bh, rank);
+    const int pair = p.causal ? (p.n_pairs - 1 - rank) : rank;
+    x.bh_kv = kv_head_of(x.bh, p.H, p.H_kv);
+    x.q_base0 = pair * 256;
+    x.n0 = p.causal ? min(n_kv, x.q_base0 / 128 + 1) : n_kv;
+    x.n1 = p.causal ? min(n_kv, x.q_base0 / 128 + 2) : n_kv;  // n1 >= n0
+    return x;
+  };
+  int* unit_ring = reinterpret_cast<int*>(gbase + L::OFF_UNIT);
+  auto next_unit = [&](int k, bool& ok) -> int {  // index of this CTA's k-th unit
+    const int slot = k & 1;
+    ok = mbar_wait(bar(L::BAR_UNIT_FULL + slot), (k >> 1) & 1, wctx);
+    return ok ? *reinterpret_cast<volatile int*>(unit_ring + slot) : n_units;
+  };
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(L::BAR_Q_FULL), 1);
+    mbar_init(bar(L::BAR_Q_EMPTY), 1);
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(bar(L::BAR_KV_FULL + s), 1);
+      mbar_init(bar(L::BAR_KV_EMPTY + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::BAR_S_FULL + t), 1);
+      mbar_init(bar(L::BAR_P_HALF + t), 128);
+      mbar_init(bar(L::BAR_P_FULL + t), 128);
+      mbar_init(bar(L::BAR_O_FULL + t), 1);
+      mbar_init(bar(L::BAR_O_FREE + t), 128);
+      mbar_init(bar(L::BAR_UNIT_FULL + t), 1);
+      mbar_init(bar(L::BAR_UNIT_EMPTY + t), 1 + 256);
+    }
+    mbar_init(bar(L::BAR_MMA_DONE), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(base + L::OFF_TMEM_SLOT, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_TMEM_SLOT);
+
+  if (warp == 0) {
+    // ===================================================== TMA producer + work distribution
+    regs_dec<kRegsLow>();
+    const uint32_t leader = elect_one();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    int issued = 0, q_issued = 0;
+    bool ok = true;
+    for (int uc = 0;; ++uc) {
+      // the ring slot is free once every consumer has read unit uc - 2
+      if (uc >= 2 && !(ok = mbar_wait(bar(L::BAR_UNIT_EMPTY + (uc & 1)), ((uc - 2) >> 1) & 1, wctx))) break;
+      int u = 0;
+      if (lane == 0) u = (int)atomicAdd(p.counter, 1u);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (lane == 0) {
+        unit_ring[uc & 1] = u < n_units ? u : n_units;
+        mbar_arrive(bar(L::BAR_UNIT_FULL + (uc & 1)));
+      }
+      __syncwarp();
+      if (u >= n_units) break;
+      const Unit x = unit_of(u);
+      // this unit's Q tiles replace the previous unit's once its last Q K^T products completed
+      if (uc > 0 && !(ok = mbar_wait(bar(L::BAR_Q_EMPTY), (uc - 1) & 1, wctx))) break;
+      mbar_arrive_expect_tx(bar(L::BAR_Q_FULL), 2 * L::TILE, leader);
+      for (int c = 0; c < L::KCH; ++c) {
+        tma_load_3d(base + L::OFF_Q0 + c * L::BOX, &tm_q, c * 64, x.q_base0, x.bh, bar(L::BAR_Q_FULL), leader);
+        tma_load_3d(base + L::OFF_Q1 + c * L::BOX, &tm_q, c * 64, x.q_base0 + 128, x.bh, bar(L::BAR_Q_FULL),
+                    leader);
+      }
+      ++q_issued;
+      for (int j = 0; j < x.n1 && ok; ++j) {
+        for (int which = 0; which < 2; ++which) {
+          const int st = issued % L::STAGES;
+          if (!(ok = mbar_wait(bar(L::BAR_KV_EMPTY + st), ((issued / L::STAGES) & 1) ^ 1u, wctx))) break;
+          mbar_arrive_expect_tx(bar(L::BAR_KV_FULL + st), L::TILE, leader);
+          const CUtensorMap* m = which ? &tm_v : &tm_k;
+          for (int c = 0; c < L::KCH; ++c)
+            tma_load_3d(base + L::OFF_KV + st * L::TILE + c * L::BOX, m, c * 64, j * 128, x.bh_kv,
+                        bar(L::BAR_KV_FULL + st), leader);
+          ++issued;
+        }
+      }
+      if (!ok) break;
+    }
+    // drain: every issued copy has landed before the CTA may exit
+    if (q_issued > 0) drain_wait(bar(L::BAR_Q_FULL), (q_issued - 1) & 1);
+    for (int i = (issued > L::STAGES ? issued - L::STAGES : 0); i < issued; ++i)
+      drain_wait(bar(L::BAR_KV_FULL + (i % L::STAGES)), (i / L::STAGES) & 1);
+  } else if (warp == 1) {
+    // ===================================================== MMA issuer
+    regs_dec<kRegsLow>();
+    const uint32_t leader = elect_one();
+    constexpr uint32_t idesc_qk = make_idesc(128, 128, true, false, false);
+    constexpr uint32_t idesc_pv = make_idesc(128, D, false, false, true);  // fp16 P (TMEM) x fp16 V
+    const uint32_t tS[2] = {tmem + L::T_S0, tmem + L::T_S1};
+    const uint32_t tO[2] = {tmem + L::T_O0, tmem + L::T_O1};
+    const uint64_t dQ[2] = {make_sdesc_sw128(base + L::OFF_Q0, 16, 1024), make_sdesc_sw128(base + L::OFF_Q1, 16, 1024)};
+    const uint64_t dKV0 = make_sdesc_sw128(base + L::OFF_KV, 16, 1024);     // K-major (K tiles)
+    const uint64_t dV0 = make_sdesc_sw128(base + L::OFF_KV, L::BOX, 1024);  // MN-major (V tiles)
+    auto issue_qk = [&](uint32_t d_tmem, uint64_t q_desc, int stage) {
+      const uint64_t k_desc = sdesc_add(dKV0, stage * L::TILE);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * L::BOX + (k & 3) * 32;
+        mma_ss(d_tmem, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, k > 0 ? 1u : 0u, leader);
+      }
+    };
+    auto issue_pv_half = [&](uint32_t d_tmem, uint32_t p_tmem, int stage, bool acc, int part) {
+      const uint64_t v_desc = sdesc_add(dV0, stage * L::TILE);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int k = part * 4 + kk;
+        mma_ts(d_tmem, p_tmem + k * 8, sdesc_add(v_desc, k * 2048), idesc_pv, (acc || k > 0) ? 1u : 0u, leader);
+      }
+    };
+    int L0 = 0, G0 = 0, G1 = 0;  // K/V loads and tile steps of the previous units
+    bool ok = true;
+    // O_t += P_t V (tile t's local step jt, K/V stage st); before a unit's first product
+    // into O_t the previous unit's epilogue must have read O_t out of TMEM
+    auto issue_pv = [&](int t, int jt, int stage, int uc) -> bool {
+      if (jt == 0 && uc > 0) {
+        if (!mbar_wait(bar(L::BAR_O_FREE + t), (uc - 1) & 1, wctx)) return false;
+        tc_fence_after();
+      }
+      const uint32_t ph = ((t ? G1 : G0) + jt) & 1;
+      if (!mbar_wait(bar(L::BAR_P_HALF + t), ph, wctx)) return false;
+      tc_fence_after();
+      issue_pv_half(tO[t], tS[t], stage, jt > 0, 0);
+      if (!mbar_wait(bar(L::BAR_P_FULL + t), ph, wctx)) return false;
+      tc_fence_after();
+      issue_pv_half(tO[t], tS[t], stage, jt > 0, 1);
+      return true;
+    };
+    for (int uc = 0; ok; ++uc) {
+      const int u = next_unit(uc, ok);
+      if (lane == 0) mbar_arrive(bar(L::BAR_UNIT_EMPTY + (uc & 1)));
+      if (!ok || u >= n_units) break;
+      const Unit x = unit_of(u);
+      if (!(ok = mbar_wait(bar(L::BAR_Q_FULL), uc & 1, wctx))) break;
+      tc_fence_after();
+      int prev_v_stage = 0;
+      for (int j = 0; j < x.n1 && ok; ++j) {
+        const int iK = L0 + 2 * j, iV = iK + 1;
+        const int stK = iK % L::STAGES, stV = iV % L::STAGES;
+        if (!(ok = mbar_wait(bar(L::BAR_KV_FULL + stK), (iK / L::STAGES) & 1, wctx))) break;
+        tc_fence_after();
+        if (j < x.n0) {
+          issue_qk(tS[0], dQ[0], stK);
+          mma_commit(bar(L::BAR_S_FULL + 0), leader);
+        }
+        if (j > 0) {  // O1 += P1 V_{j-1}
+          if (!(ok = issue_pv(1, j - 1, prev_v_stage, uc))) break;
+          mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage), leader);
+        }
+        issue_qk(tS[1], dQ[1], stK);
+        mma_commit(bar(L::BAR_S_FULL + 1), leader);
+        mma_commit(bar(L::BAR_KV_EMPTY + stK), leader);
+        if (j == x.n1 - 1) mma_commit(bar(L::BAR_Q_EMPTY), leader);  // the unit's last Q K^T
+        if (!(ok = mbar_wait(bar(L::BAR_KV_FULL + stV), (iV / L::STAGES) & 1, wctx))) break;
+        tc_fence_after();
+        if (j < x.n0) {  // O0 += P0 V_j
+          if (!(ok = issue_pv(0, j, stV, uc))) break;
+          if (j == x.n0 - 1) mma_commit(bar(L::BAR_O_FULL + 0), leader);
+        }
+        prev_v_stage = stV;
+      }
+      if (!ok) break;
+      if (!(ok = issue_pv(1, x.n1 - 1, prev_v_stage, uc))) break;  // O1 += P1 V_{n1-1}
+      mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage), leader);
+      mma_commit(bar(L::BAR_O_FULL + 1), leader);
+      L0 += 2 * x.n1;
+      G0 += x.n0;
+      G1 += x.n1;
+    }
+    // every MMA issued so far has finished before TMEM is released
+    mma_commit(bar(L::BAR_MMA_DONE), leader);
+    drain_wait(bar(L::BAR_MMA_DONE), 0);
+  } else if (warp < 4) {
+    regs_dec<kRegsLow>();  // warps 2-3: idle (V is fp16 already)
+  } else {
+    // ===================================================== softmax warpgroups
+    regs_inc<kRegsHigh>();
+    const int t = (warp - 4) >> 2;   // query tile handled by this warpgroup
+    const int wq = (warp - 4) & 3;   // TMEM lane quarter
+    const int row = wq * 32 + lane;  // row inside the tile
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (t ? L::T_S1 : L::T_S0);
+    const uint32_t tO = tmem + lane_off + (t ? L::T_O1 : L::T_O0);
+    bool ok = true;
+    int G = 0;  // this tile's steps in the previous units
+    int u = next_unit(0, ok);
+    mbar_arrive(bar(L::BAR_UNIT_EMPTY + 0));
+    for (int uc = 0; ok && u < n_units; ++uc) {
+      const Unit x = unit_of(u);
+      const int q_base = x.q_base0 + 128 * t;
+      const int r = q_base + row;  // query index
+      const int n_t = t ? x.n1 : x.n0;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < n_t; ++j) {
+        if (!(ok = fwd_softmax_step<D>(p, tS, tO, bar(L::BAR_S_FULL + t), (G + j) & 1, bar(L::BAR_P_HALF + t),
+                                       bar(L::BAR_P_FULL + t), j, q_base, r, m, l, wctx)))
+          break;
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16 and the bf16 residual, stored from registers
+      if (!(ok = mbar_wait(bar(L::BAR_O_FULL + t), uc & 1, wctx))) break;
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t u0[32], u1[32];
+        tmem_ld32(tO + 64 * c, u0);
+        tmem_ld32(tO + 64 * c + 32, u1);
+        tmem_wait_ld();
+        if (c == D / 64 - 1) {  // O_t fully read: the next unit may overwrite it
+          tc_fence_before();
+          mbar_arrive(bar(L::BAR_O_FREE + t));
+        }
+        uint4 oa[8], ra[8];
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          uint32_t pk[4], rk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * q4 + e;  // packed pair index 0..31 within the chunk
+            const uint32_t* uu = i < 16 ? u0 : u1;
+            const int k = 2 * (i & 15);
+            const float a = __uint_as_float(uu[k]) * inv_l, b = __uint_as_float(uu[k + 1]) * inv_l;
+            pk[e] = pack_bf16(a, b);
+            const float2 ab = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
+            rk[e] = pack_bf16(a - ab.x, b - ab.y);
+          }
+          oa[q4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          ra[q4] = make_uint4(rk[0], rk[1], rk[2], rk[3]);
+        }
+        warp_store_rows_128b(oa, reinterpret_cast<uint8_t*>(p.o + (size_t)x.bh * p.N * D + 64 * c), D * 2,
+                             q_base + wq * 32, p.N);
+        if (p.o_resid != nullptr)
+          warp_store_rows_128b(ra, reinterpret_cast<uint8_t*>(p.o_resid + (size_t)x.bh * p.N * D + 64 * c), D * 2,
+                               q_base + wq * 32, p.N);
+      }
+      if (p.lse != nullptr && r < p.N) p.lse[(size_t)x.bh * p.N + r] = (m + __log2f(l)) * 0.69314718055994531f;
+      G += n_t;
+      u = next_unit(uc + 1, ok);
+      mbar_arrive(bar(L::BAR_UNIT_EMPTY + ((uc + 1) & 1)));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+}  // namespace
+
+namespace {
+template <int D>
 cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                          const FwdParams& p, cudaStream_t s) {
   using L = FwdLayout<D>;
   const dim3 grid((unsigned)(p.n_pairs * p.BH));
-  cudaError_t e = cudaFuncSetAttribute(fa_fwd_sm100_kernel<D, kVf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(fa_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        L::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  fa_fwd_sm100_kernel<D, kVf16><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, to, p);
+  fa_fwd_sm100_kernel<D><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 
 // V (bf16) -> fp16 copy, 8 elements per 16-byte access (exact for |v| in [2^-14, 65504]).
 __global__ void __launch_bounds__(256) fa_fwd_v16_kernel(const uint4* __restrict__ v, uint4* __restrict__ v16,
-                                                         long long n8) {
+                                                         long long n8, unsigned* counter) {
+  if (blockIdx.x == 0 && threadIdx.x == 0 && counter != nullptr) *counter = 0u;  // persistent kernel's work counter
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n8; e += (long long)gridDim.x * blockDim.x) {
     uint4 u = v[e];
     uint32_t* w = reinterpret_cast<uint32_t*>(&u);
@@ -497,17 +833,36 @@ __global__ void __launch_bounds__(256) fa_fwd_v16_kernel(const uint4* __restrict
 }  // namespace
 
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& to, const FwdParams& p, int d, bool v_is_f16, cudaStream_t s) {
-  if (d == 128)
-    return v_is_f16 ? launch_fwd_t<128, true>(tq, tk, tv, to, p, s) : launch_fwd_t<128, false>(tq, tk, tv, to, p, s);
-  return v_is_f16 ? launch_fwd_t<64, true>(tq, tk, tv, to, p, s) : launch_fwd_t<64, false>(tq, tk, tv, to, p, s);
+                             const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t s) {
+  return d == 128 ? launch_fwd_t<128>(tq, tk, tv, to, p, s) : launch_fwd_t<64>(tq, tk, tv, to, p, s);
 }
 
-cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, cudaStream_t s) {
+cudaError_t launch_fwd_persist_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                     const FwdParams& p, int d, cudaStream_t s) {
+  const long long units = (long long)p.n_pairs * p.BH;
+  const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
+  if (d == 128) {
+    using L = FwdPLayout<128>;
+    cudaError_t e = cudaFuncSetAttribute(fa_fwd_persist_sm100_kernel<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    fa_fwd_persist_sm100_kernel<128><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, p);
+  } else {
+    using L = FwdPLayout<64>;
+    cudaError_t e = cudaFuncSetAttribute(fa_fwd_persist_sm100_kernel<64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    fa_fwd_persist_sm100_kernel<64><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, cudaStream_t s) {
   const long long n8 = elems / 8;  // d is a multiple of 8
   long long blocks = (n8 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  fa_fwd_v16_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8);
+  fa_fwd_v16_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8,
+                                                     counter);
   return cudaGetLastError();
 }
 

@@ -105,10 +105,15 @@ FA_API fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o
  * plain multi-head attention) with a caller workspace, used to run the V operand's
  * bf16 -> fp16 conversion as one streaming pass before the attention kernel instead of
  * inside it (fa_fwd / fa_fwd_gqa convert each V tile on chip, on two warps that share
- * SM sub-partitions with half of the softmax warps).  Results are identical to fa_fwd_gqa.
+ * SM sub-partitions with half of the softmax warps).  Results are identical to fa_fwd_gqa
+ * (every unit computes the same values in the same order).
  *   workspace       : device buffer of at least fa_fwd_workspace_size(B, H_kv, N, d)
- *                     bytes (an fp16 copy of V), 256-byte aligned, caller-owned; contents
- *                     on entry do not matter, unspecified on return.  NULL is an error.
+ *                     bytes (an fp16 copy of V and a work counter), 256-byte aligned,
+ *                     caller-owned; contents on entry do not matter, unspecified on
+ *                     return.  NULL is an error.
+ * With a workspace the attention kernel is persistent (one CTA per SM taking work units
+ * from the counter, so one unit's epilogue overlaps the next unit's loads and first
+ * products); calls that overlap on the GPU need separate workspaces.
  *   workspace_bytes : its size.
  * fa_fwd_workspace_size returns 0 for an empty or invalid problem.  Everything else as
  * fa_fwd_gqa.

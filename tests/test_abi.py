@@ -88,8 +88,8 @@ def test_gqa_head_counts_are_checked(lib):
 
 def test_forward_workspace(lib):
     a = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    assert api.fa_fwd_workspace_size(2, 8, 8192, 128) == a(2 * 8 * 8192 * 128 * 2)
-    assert api.fa_fwd_workspace_size(1, 1, 300, 64) == a(300 * 64 * 2)
+    assert api.fa_fwd_workspace_size(2, 8, 8192, 128) == a(2 * 8 * 8192 * 128 * 2) + 256
+    assert api.fa_fwd_workspace_size(1, 1, 300, 64) == a(300 * 64 * 2) + 256
     assert api.fa_fwd_workspace_size(0, 8, 100, 64) == 0
     assert api.fa_fwd_workspace_size(1, 1, 100, 96) == 0
     ws = lambda ptr=A, n=1 << 40, H=4, Hkv=2: lib.fa_fwd_ws(A, A, A, A, A, None, 1, H, Hkv, 16, 64, 0.125, 0,  # noqa: E731
