@@ -107,12 +107,6 @@ __device__ __forceinline__ void warp_store_rows_f32(const float (&v)[NC], float*
   }
 }
 
-template <int N>
-__device__ __forceinline__ float (&acc_lo_view(float (&a)[N]))[64] {
-  static_assert(N >= 64, "needs 64 entries");
-  return *reinterpret_cast<float(*)[64]>(&a[0]);
-}
-
 // Load 64 fp32 columns of this thread's TMEM lane (two 32-column loads, one wait).
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   uint32_t u[32];
@@ -136,7 +130,7 @@ struct DkdvLayout {
   static constexpr int OFF_DO = 4 * TILE;       // two dO buffers
   static constexpr int OFF_LD = 6 * TILE;       // two (lse2[128], delta[128]) pairs, 1 KB each
   static constexpr int OFF_BAR = OFF_LD + 2048;
-  static constexpr int BAR_KV = 0;
+  static constexpr int BAR_KV = 0;        // a unit's K, V landed
   static constexpr int BAR_Q_FULL = 1;    // [2]
   static constexpr int BAR_Q_EMPTY = 3;   // [2]
   static constexpr int BAR_DO_FULL = 5;   // [2]
@@ -145,17 +139,30 @@ struct DkdvLayout {
   static constexpr int BAR_DP = 10;
   static constexpr int BAR_P_READY = 11;
   static constexpr int BAR_DS_READY = 12;
-  static constexpr int BAR_ACC = 13;
+  static constexpr int BAR_ACC = 13;      // a unit's dV, dK complete in TMEM
   static constexpr int BAR_DONE = 14;
   static constexpr int BAR_P_HALF = 15;   // first 32 of each warpgroup's 64 P^T columns written
-  static constexpr int NBAR = 16;
-  static constexpr int OFF_TMEM_SLOT = OFF_BAR + NBAR * 8;
+  static constexpr int BAR_KV_EMPTY = 16; // the MMAs reading a unit's K and V have completed
+  static constexpr int BAR_ACC_FREE = 17; // the epilogue has read a unit's dV, dK out of TMEM
+  static constexpr int BAR_UNIT_FULL = 18;   // [2]
+  static constexpr int BAR_UNIT_EMPTY = 20;  // [2]
+  static constexpr int NBAR = 22;
+  static constexpr int OFF_UNIT = OFF_BAR + NBAR * 8;  // int[2]
+  static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
   static constexpr int SMEM_ALLOC = OFF_ABORT + 8 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
 };
 
+// Persistent dK/dV kernel: one CTA per SM takes work units (key/value head, 128-key tile,
+// share of the group's query heads) one after another from a work counter in the workspace
+// (zeroed by the preprocess), in the order of unit_order; the producer warp takes each
+// index and publishes it to the other roles through a two-slot ring in shared memory (an
+// index >= the unit count means "no more work").  The next unit's K/V loads and first
+// S^T, dP^T products overlap the previous unit's last steps and epilogue.  Ring positions
+// (Q, dO, row statistics) and the per-step barriers count steps across units; the
+// per-unit barriers (KV, KV_EMPTY, ACC, ACC_FREE) count units.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -174,24 +181,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   // heaviest first within groups of heads (see unit_order): under the causal mask the
   // first key tiles of a head meet the most query tiles
   const int n_kt = (p.N + 127) / 128;
-  int bh, rank;  // key/value head, rank of (key tile, split) within the head
-  unit_order((int)blockIdx.x, n_kt * p.kv_split, p.BH / p.H * p.H_kv, p.head_group_kv, bh, rank);
-  const int j = rank / p.kv_split;         // key tile
-  const int sp = rank % p.kv_split;        // which share of the group's query heads
-  const int g_per = p.H / p.H_kv / p.kv_split;  // query heads handled by this CTA
-  const int i_start = p.causal ? j : 0;
-  const int n_q = n_kt - i_start;          // 128-query tiles per query head, >= 1
-  const int n_it = g_per * n_q;            // steps: every query tile of each of this CTA's query heads
-  // step it: query head q_head_of(bh, sp * g_per + it / n_q), query tile i_start + it % n_q
+  const int BH_kv = p.BH / p.H * p.H_kv;
+  const int n_units = n_kt * BH_kv * p.kv_split;
+  const int g_per = p.H / p.H_kv / p.kv_split;  // query heads per unit
+  struct Unit {
+    int bh, j, sp, i_start, n_q, n_it;
+  };
+  auto unit_of = [&](int u) -> Unit {
+    Unit x;
+    int rank;  // rank of (key tile, split) within the key/value head
+    unit_order(u, n_kt * p.kv_split, BH_kv, p.head_group_kv, x.bh, rank);
+    x.j = rank / p.kv_split;   // key tile
+    x.sp = rank % p.kv_split;  // which share of the group's query heads
+    x.i_start = p.causal ? x.j : 0;
+    x.n_q = n_kt - x.i_start;  // 128-query tiles per query head, >= 1
+    x.n_it = g_per * x.n_q;    // steps: query head q_head_of(bh, sp * g_per + it / n_q), tile i_start + it % n_q
+    return x;
+  };
+  int* unit_ring = reinterpret_cast<int*>(gbase + L::OFF_UNIT);
+  auto next_unit = [&](int k, bool& ok) -> int {  // index of this CTA's k-th unit
+    const int slot = k & 1;
+    ok = mbar_wait(bar(L::BAR_UNIT_FULL + slot), (k >> 1) & 1, wctx);
+    return ok ? *reinterpret_cast<volatile int*>(unit_ring + slot) : n_units;
+  };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(bar(L::BAR_KV), 1);
+    mbar_init(bar(L::BAR_KV_EMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(L::BAR_Q_FULL + s), 1);
       mbar_init(bar(L::BAR_Q_EMPTY + s), 1);
       mbar_init(bar(L::BAR_DO_FULL + s), 1);
       mbar_init(bar(L::BAR_DO_EMPTY + s), 1);
+      mbar_init(bar(L::BAR_UNIT_FULL + s), 1);
+      mbar_init(bar(L::BAR_UNIT_EMPTY + s), 1 + 256);
     }
     mbar_init(bar(L::BAR_S), 1);
     mbar_init(bar(L::BAR_DP), 1);
@@ -199,6 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(L::BAR_P_HALF), 256);
     mbar_init(bar(L::BAR_DS_READY), 256);
     mbar_init(bar(L::BAR_ACC), 1);
+    mbar_init(bar(L::BAR_ACC_FREE), 256);
     mbar_init(bar(L::BAR_DONE), 1);
     fence_barrier_init();
   }
@@ -212,43 +237,66 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_TMEM_SLOT);
 
   if (warp == 0) {
-    // ===================================================== TMA producer
+    // ===================================================== TMA producer + work distribution
     regs_dec<kRegsLow>();
     const uint32_t leader = elect_one();
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_do);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
-    mbar_arrive_expect_tx(bar(L::BAR_KV), 2 * L::TILE, leader);
-    for (int c = 0; c < L::KCH; ++c) {
-      tma_load_3d(base + L::OFF_K + c * kBox, &tm_k, c * 64, j * 128, bh, bar(L::BAR_KV), leader);
-      tma_load_3d(base + L::OFF_V + c * kBox, &tm_v, c * 64, j * 128, bh, bar(L::BAR_KV), leader);
+    int T = 0;         // Q / dO tiles issued (ring position, across units)
+    int kv_issued = 0;
+    bool ok = true;
+    for (int uc = 0;; ++uc) {
+      // the ring slot is free once every consumer has read unit uc - 2
+      if (uc >= 2 && !(ok = mbar_wait(bar(L::BAR_UNIT_EMPTY + (uc & 1)), ((uc - 2) >> 1) & 1, wctx))) break;
+      int u = 0;
+      if (lane == 0) u = (int)atomicAdd(p.dkdv_counter, 1u);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (lane == 0) {
+        unit_ring[uc & 1] = u < n_units ? u : n_units;
+        mbar_arrive(bar(L::BAR_UNIT_FULL + (uc & 1)));
+      }
+      __syncwarp();
+      if (u >= n_units) break;
+      const Unit x = unit_of(u);
+      // K, V of this unit replace the previous unit's once its last S^T, dP^T completed
+      if (uc > 0 && !(ok = mbar_wait(bar(L::BAR_KV_EMPTY), (uc - 1) & 1, wctx))) break;
+      mbar_arrive_expect_tx(bar(L::BAR_KV), 2 * L::TILE, leader);
+      for (int c = 0; c < L::KCH; ++c) {
+        tma_load_3d(base + L::OFF_K + c * kBox, &tm_k, c * 64, x.j * 128, x.bh, bar(L::BAR_KV), leader);
+        tma_load_3d(base + L::OFF_V + c * kBox, &tm_v, c * 64, x.j * 128, x.bh, bar(L::BAR_KV), leader);
+      }
+      ++kv_issued;
+      for (int it = 0; it < x.n_it; ++it, ++T) {
+        const int s = T & 1;
+        const uint32_t ph = ((T >> 1) & 1) ^ 1u;
+        const int i = x.i_start + it % x.n_q;
+        const int bhq = q_head_of(x.bh, x.sp * g_per + it / x.n_q, p.H, p.H_kv);
+        if (!(ok = mbar_wait(bar(L::BAR_Q_EMPTY + s), ph, wctx))) break;
+        const uint32_t fq = bar(L::BAR_Q_FULL + s);
+        mbar_arrive_expect_tx(fq, L::TILE + 1024, leader);
+        for (int c = 0; c < L::KCH; ++c)
+          tma_load_3d(base + L::OFF_Q + s * L::TILE + c * kBox, &tm_q, c * 64, i * 128, bhq, fq, leader);
+        const size_t roff = (size_t)bhq * p.Np + (size_t)i * 128;
+        bulk_load(base + L::OFF_LD + s * 1024, p.lse2 + roff, 512, fq, leader);
+        bulk_load(base + L::OFF_LD + s * 1024 + 512, p.delta + roff, 512, fq, leader);
+        if (!(ok = mbar_wait(bar(L::BAR_DO_EMPTY + s), ph, wctx))) {
+          ++T;  // this step's Q tile was issued
+          break;
+        }
+        const uint32_t fd = bar(L::BAR_DO_FULL + s);
+        mbar_arrive_expect_tx(fd, L::TILE, leader);
+        for (int c = 0; c < L::KCH; ++c)
+          tma_load_3d(base + L::OFF_DO + s * L::TILE + c * kBox, &tm_do, c * 64, i * 128, bhq, fd, leader);
+      }
+      if (!ok) break;
     }
-    int issued = 0;
-    for (int it = 0; it < n_it; ++it) {
-      const int s = it & 1;
-      const uint32_t ph = ((it >> 1) & 1) ^ 1u;
-      const int i = i_start + it % n_q;
-      const int bhq = q_head_of(bh, sp * g_per + it / n_q, p.H, p.H_kv);
-      if (!mbar_wait(bar(L::BAR_Q_EMPTY + s), ph, wctx)) break;
-      const uint32_t fq = bar(L::BAR_Q_FULL + s);
-      mbar_arrive_expect_tx(fq, L::TILE + 1024, leader);
-      for (int c = 0; c < L::KCH; ++c)
-        tma_load_3d(base + L::OFF_Q + s * L::TILE + c * kBox, &tm_q, c * 64, i * 128, bhq, fq, leader);
-      const size_t roff = (size_t)bhq * p.Np + (size_t)i * 128;
-      bulk_load(base + L::OFF_LD + s * 1024, p.lse2 + roff, 512, fq, leader);
-      bulk_load(base + L::OFF_LD + s * 1024 + 512, p.delta + roff, 512, fq, leader);
-      if (!mbar_wait(bar(L::BAR_DO_EMPTY + s), ph, wctx)) break;
-      const uint32_t fd = bar(L::BAR_DO_FULL + s);
-      mbar_arrive_expect_tx(fd, L::TILE, leader);
-      for (int c = 0; c < L::KCH; ++c)
-        tma_load_3d(base + L::OFF_DO + s * L::TILE + c * kBox, &tm_do, c * 64, i * 128, bhq, fd, leader);
-      ++issued;
-    }
-    drain_wait(bar(L::BAR_KV), 0);
-    for (int it = (issued > 2 ? issued - 2 : 0); it < issued; ++it) {
-      drain_wait(bar(L::BAR_Q_FULL + (it & 1)), (it >> 1) & 1);
-      drain_wait(bar(L::BAR_DO_FULL + (it & 1)), (it >> 1) & 1);
+    // drain: every issued copy has landed before the CTA may exit
+    if (kv_issued > 0) drain_wait(bar(L::BAR_KV), (kv_issued - 1) & 1);
+    for (int t = (T > 2 ? T - 2 : 0); t < T; ++t) {
+      drain_wait(bar(L::BAR_Q_FULL + (t & 1)), (t >> 1) & 1);
+      drain_wait(bar(L::BAR_DO_FULL + (t & 1)), (t >> 1) & 1);
     }
   } else if (warp == 1) {
     // ===================================================== MMA issuer
@@ -262,50 +310,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dDOk = make_sdesc_sw128(base + L::OFF_DO, 16, 1024);    // dO as K-major B
     const uint64_t dQmn = make_sdesc_sw128(base + L::OFF_Q, kBox, 1024);   // Q as MN-major B
     const uint64_t dDOmn = make_sdesc_sw128(base + L::OFF_DO, kBox, 1024); // dO as MN-major B
-    bool ok = mbar_wait(bar(L::BAR_KV), 0, wctx);
-    if (ok) ok = mbar_wait(bar(L::BAR_Q_FULL + 0), 0, wctx);
-    if (ok) {
+    // S^T(t) = K Q_t^T and dP^T(t) = V dO_t^T for global step t
+    auto issue_s = [&](int t) -> bool {
+      if (!mbar_wait(bar(L::BAR_Q_FULL + (t & 1)), (t >> 1) & 1, wctx)) return false;
       tc_fence_after();
-      issue_ss<D>(tmem + L::T_S, dK, dQk, idesc_s, leader);  // S^T(0) = K Q_0^T
+      issue_ss<D>(tmem + L::T_S, dK, sdesc_add(dQk, (t & 1) * L::TILE), idesc_s, leader);
       mma_commit(bar(L::BAR_S), leader);
-      ok = mbar_wait(bar(L::BAR_DO_FULL + 0), 0, wctx);
-    }
-    if (ok) {
+      return true;
+    };
+    auto issue_dp = [&](int t) -> bool {
+      if (!mbar_wait(bar(L::BAR_DO_FULL + (t & 1)), (t >> 1) & 1, wctx)) return false;
       tc_fence_after();
-      issue_ss<D>(tmem + L::T_DP, dV, dDOk, idesc_s, leader);  // dP^T(0) = V dO_0^T
+      issue_ss<D>(tmem + L::T_DP, dV, sdesc_add(dDOk, (t & 1) * L::TILE), idesc_s, leader);
       mma_commit(bar(L::BAR_DP), leader);
-    }
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int s = it & 1;
-      const uint32_t so = s * L::TILE;
-      // dV += P^T dO in two halves: the first starts while the second half of P^T is computed
-      if (!(ok = mbar_wait(bar(L::BAR_P_HALF), it & 1, wctx))) break;
+      return true;
+    };
+    int T0 = 0;  // global step index of the current unit's step 0
+    bool ok = true;
+    for (int uc = 0; ok; ++uc) {
+      const int u = next_unit(uc, ok);
+      if (lane == 0) mbar_arrive(bar(L::BAR_UNIT_EMPTY + (uc & 1)));
+      if (!ok || u >= n_units) break;
+      const int n = unit_of(u).n_it;
+      if (!(ok = mbar_wait(bar(L::BAR_KV), uc & 1, wctx))) break;
       tc_fence_after();
-      issue_ts_split_part(tmem + L::T_DV, tmem + L::T_S, sdesc_add(dDOmn, so), idesc_g, it == 0, 0, leader);
-      if (!(ok = mbar_wait(bar(L::BAR_P_READY), it & 1, wctx))) break;
-      tc_fence_after();
-      issue_ts_split_part(tmem + L::T_DV, tmem + L::T_S, sdesc_add(dDOmn, so), idesc_g, false, 1, leader);
-      mma_commit(bar(L::BAR_DO_EMPTY + s), leader);
-      if (it + 1 < n_it) {
-        const int s1 = (it + 1) & 1;
-        if (!(ok = mbar_wait(bar(L::BAR_Q_FULL + s1), ((it + 1) >> 1) & 1, wctx))) break;
+      if (!(ok = issue_s(T0))) break;
+      if (!(ok = issue_dp(T0))) break;
+      if (n == 1) mma_commit(bar(L::BAR_KV_EMPTY), leader);  // last S^T, dP^T of the unit issued
+      for (int it = 0; it < n && ok; ++it) {
+        const int t = T0 + it;
+        const int s = t & 1;
+        const uint32_t so = s * L::TILE;
+        // dV += P^T dO in two halves: the first starts while the second half of P^T is computed;
+        // the unit's first product overwrites the accumulators, which the previous unit's
+        // epilogue must have read out of TMEM
+        if (!(ok = mbar_wait(bar(L::BAR_P_HALF), t & 1, wctx))) break;
         tc_fence_after();
-        issue_ss<D>(tmem + L::T_S, dK, sdesc_add(dQk, s1 * L::TILE), idesc_s, leader);  // S^T(it+1)
-        mma_commit(bar(L::BAR_S), leader);
-      }
-      if (!(ok = mbar_wait(bar(L::BAR_DS_READY), it & 1, wctx))) break;
-      tc_fence_after();
-      issue_ts_split(tmem + L::T_DK, tmem + L::T_DP, sdesc_add(dQmn, so), idesc_g, it > 0, leader);  // dK += dS^T Q
-      mma_commit(bar(L::BAR_Q_EMPTY + s), leader);
-      if (it + 1 < n_it) {
-        const int s1 = (it + 1) & 1;
-        if (!(ok = mbar_wait(bar(L::BAR_DO_FULL + s1), ((it + 1) >> 1) & 1, wctx))) break;
+        if (it == 0 && uc > 0) {
+          if (!(ok = mbar_wait(bar(L::BAR_ACC_FREE), (uc - 1) & 1, wctx))) break;
+          tc_fence_after();
+        }
+        issue_ts_split_part(tmem + L::T_DV, tmem + L::T_S, sdesc_add(dDOmn, so), idesc_g, it == 0, 0, leader);
+        if (!(ok = mbar_wait(bar(L::BAR_P_READY), t & 1, wctx))) break;
         tc_fence_after();
-        issue_ss<D>(tmem + L::T_DP, dV, sdesc_add(dDOk, s1 * L::TILE), idesc_s, leader);  // dP^T(it+1)
-        mma_commit(bar(L::BAR_DP), leader);
+        issue_ts_split_part(tmem + L::T_DV, tmem + L::T_S, sdesc_add(dDOmn, so), idesc_g, false, 1, leader);
+        mma_commit(bar(L::BAR_DO_EMPTY + s), leader);
+        if (it + 1 < n && !(ok = issue_s(t + 1))) break;
+        if (!(ok = mbar_wait(bar(L::BAR_DS_READY), t & 1, wctx))) break;
+        tc_fence_after();
+        issue_ts_split(tmem + L::T_DK, tmem + L::T_DP, sdesc_add(dQmn, so), idesc_g, it > 0, leader);  // dK += dS^T Q
+        mma_commit(bar(L::BAR_Q_EMPTY + s), leader);
+        if (it + 1 < n) {
+          if (!(ok = issue_dp(t + 1))) break;
+          if (it + 2 == n) mma_commit(bar(L::BAR_KV_EMPTY), leader);  // last S^T, dP^T of the unit issued
+        }
       }
+      if (!ok) break;
+      mma_commit(bar(L::BAR_ACC), leader);
+      T0 += n;
     }
-    if (ok) mma_commit(bar(L::BAR_ACC), leader);
     mma_commit(bar(L::BAR_DONE), leader);
     drain_wait(bar(L::BAR_DONE), 0);
   } else if (warp < 4) {
@@ -316,111 +379,128 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int w = (warp - 4) >> 2;   // query columns [64 w, 64 w + 64) of every step
     const int wq = (warp - 4) & 3;
     const int row = wq * 32 + lane;  // key row inside the tile
-    const int key = j * 128 + row;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + L::T_S + 64 * w;
     const uint32_t tDP = tmem + lane_off + L::T_DP + 64 * w;
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2pack(sl2, sl2);
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int i = i_start + it % n_q;  // query tile of this step
-      const float* lse2 = reinterpret_cast<const float*>(gbase + L::OFF_LD + (it & 1) * 1024) + 64 * w;
-      const float* delta = lse2 + 128;
-      const int q0 = i * 128 + 64 * w;  // first query of this warpgroup's columns
-      const bool need_mask = p.causal && (q0 < j * 128 + 127);
-      // ---- P^T = 2^(S^T * scale * log2(e) - lse2), written back over S^T as fp16
-      if (!(ok = mbar_wait(bar(L::BAR_S), it & 1, wctx))) break;
-      tc_fence_after();
-      float pr[64];
-      tmem_ld64(tS, pr);
-#pragma unroll
-      for (int g = 0; g < 64; g += 16) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int c = g; c < g + 16; c += 4) {
-          const float4 L4 = *reinterpret_cast<const float4*>(lse2 + c);
-          float t0, t1, t2, t3;
-          f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, f2pack(-L4.x, -L4.y)), t0, t1);
-          f2unpack(ffma2(f2pack(pr[c + 2], pr[c + 3]), sl2x2, f2pack(-L4.z, -L4.w)), t2, t3);
-          if ((c - g) < kDkdvExpFmaPer16) {
-            // both warpgroups run this phase at once, so the MUFU unit is the limit: part of
-            // the exponentials go to the FMA pipe
-            exp2_fma_pipe(t0, t1);
-            exp2_fma_pipe(t2, t3);
-            pr[c] = t0;
-            pr[c + 1] = t1;
-            pr[c + 2] = t2;
-            pr[c + 3] = t3;
-          } else {
-            pr[c] = ex2_approx(t0);
-            pr[c + 1] = ex2_approx(t1);
-            pr[c + 2] = ex2_approx(t2);
-            pr[c + 3] = ex2_approx(t3);
-          }
-          if (need_mask) {
-            if (q0 + c < key) pr[c] = 0.f;
-            if (q0 + c + 1 < key) pr[c + 1] = 0.f;
-            if (q0 + c + 2 < key) pr[c + 2] = 0.f;
-            if (q0 + c + 3 < key) pr[c + 3] = 0.f;
-          }
-          pk[(c - g) / 2] = pack_f16(pr[c], pr[c + 1]);
-          pk[(c - g) / 2 + 1] = pack_f16(pr[c + 2], pr[c + 3]);
-        }
-        tmem_st8(tS + g / 2, pk);
-        if (g == 16) {  // columns 0..31 of this warpgroup done: the first half of dV may start
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(bar(L::BAR_P_HALF));
-        }
+    int T0 = 0;
+    int u = next_unit(0, ok);
+    mbar_arrive(bar(L::BAR_UNIT_EMPTY + 0));
+    for (int uc = 0; ok && u < n_units; ++uc) {
+      int j, i_start, n_q, n_it;
+      {
+        const Unit x = unit_of(u);
+        j = x.j;
+        i_start = x.i_start;
+        n_q = x.n_q;
+        n_it = x.n_it;
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(L::BAR_P_READY));
-      // ---- dS^T = P^T * (dP^T - D), written back over dP^T as fp16
-      if (!(ok = mbar_wait(bar(L::BAR_DP), it & 1, wctx))) break;
-      tc_fence_after();
-      float dp[64];
-      tmem_ld64(tDP, dp);
+      const int key = j * 128 + row;
+      for (int it = 0; it < n_it; ++it) {
+        const int T = T0 + it;
+        const int i = i_start + it % n_q;  // query tile of this step
+        const float* lse2 = reinterpret_cast<const float*>(gbase + L::OFF_LD + (T & 1) * 1024) + 64 * w;
+        const float* delta = lse2 + 128;
+        const int q0 = i * 128 + 64 * w;  // first query of this warpgroup's columns
+        const bool need_mask = p.causal && (q0 < j * 128 + 127);
+        // ---- P^T = 2^(S^T * scale * log2(e) - lse2), written back over S^T as fp16
+        if (!(ok = mbar_wait(bar(L::BAR_S), T & 1, wctx))) break;
+        tc_fence_after();
+        float pr[64];
+        tmem_ld64(tS, pr);
 #pragma unroll
-      for (int g = 0; g < 64; g += 16) {
-        uint32_t pk[8];
+        for (int g = 0; g < 64; g += 16) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int c = g; c < g + 16; c += 4) {
-          const float4 D4 = *reinterpret_cast<const float4*>(delta + c);
-          float d0, d1, d2, d3;
-          f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(f2pack(dp[c], dp[c + 1]), f2pack(D4.x, D4.y))), d0, d1);
-          f2unpack(fmul2(f2pack(pr[c + 2], pr[c + 3]), fsub2(f2pack(dp[c + 2], dp[c + 3]), f2pack(D4.z, D4.w))), d2,
-                   d3);
-          pk[(c - g) / 2] = pack_f16(d0, d1);
-          pk[(c - g) / 2 + 1] = pack_f16(d2, d3);
+          for (int c = g; c < g + 16; c += 4) {
+            const float4 L4 = *reinterpret_cast<const float4*>(lse2 + c);
+            float t0, t1, t2, t3;
+            f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, f2pack(-L4.x, -L4.y)), t0, t1);
+            f2unpack(ffma2(f2pack(pr[c + 2], pr[c + 3]), sl2x2, f2pack(-L4.z, -L4.w)), t2, t3);
+            if ((c - g) < kDkdvExpFmaPer16) {
+              // both warpgroups run this phase at once, so the MUFU unit is the limit: part of
+              // the exponentials go to the FMA pipe
+              exp2_fma_pipe(t0, t1);
+              exp2_fma_pipe(t2, t3);
+              pr[c] = t0;
+              pr[c + 1] = t1;
+              pr[c + 2] = t2;
+              pr[c + 3] = t3;
+            } else {
+              pr[c] = ex2_approx(t0);
+              pr[c + 1] = ex2_approx(t1);
+              pr[c + 2] = ex2_approx(t2);
+              pr[c + 3] = ex2_approx(t3);
+            }
+            if (need_mask) {
+              if (q0 + c < key) pr[c] = 0.f;
+              if (q0 + c + 1 < key) pr[c + 1] = 0.f;
+              if (q0 + c + 2 < key) pr[c + 2] = 0.f;
+              if (q0 + c + 3 < key) pr[c + 3] = 0.f;
+            }
+            pk[(c - g) / 2] = pack_f16(pr[c], pr[c + 1]);
+            pk[(c - g) / 2 + 1] = pack_f16(pr[c + 2], pr[c + 3]);
+          }
+          tmem_st8(tS + g / 2, pk);
+          if (g == 16) {  // columns 0..31 of this warpgroup done: the first half of dV may start
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(L::BAR_P_HALF));
+          }
         }
-        tmem_st8(tDP + g / 2, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::BAR_P_READY));
+        // ---- dS^T = P^T * (dP^T - D), written back over dP^T as fp16
+        if (!(ok = mbar_wait(bar(L::BAR_DP), T & 1, wctx))) break;
+        tc_fence_after();
+        float dp[64];
+        tmem_ld64(tDP, dp);
+#pragma unroll
+        for (int g = 0; g < 64; g += 16) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int c = g; c < g + 16; c += 4) {
+            const float4 D4 = *reinterpret_cast<const float4*>(delta + c);
+            float d0, d1, d2, d3;
+            f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(f2pack(dp[c], dp[c + 1]), f2pack(D4.x, D4.y))), d0, d1);
+            f2unpack(fmul2(f2pack(pr[c + 2], pr[c + 3]), fsub2(f2pack(dp[c + 2], dp[c + 3]), f2pack(D4.z, D4.w))), d2,
+                     d3);
+            pk[(c - g) / 2] = pack_f16(d0, d1);
+            pk[(c - g) / 2 + 1] = pack_f16(d2, d3);
+          }
+          tmem_st8(tDP + g / 2, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::BAR_DS_READY));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(L::BAR_DS_READY));
-    }
-    if (ok) ok = mbar_wait(bar(L::BAR_ACC), 0, wctx);
-    if (ok) {
+      if (!ok) break;
+      if (!(ok = mbar_wait(bar(L::BAR_ACC), uc & 1, wctx))) break;
       tc_fence_after();
       // with the group split over several CTAs each writes its partial sums for the reduction
-      const size_t head_off = p.kv_split == 1 ? (size_t)bh * p.N * D
-                                              : ((size_t)sp * (p.BH / p.H * p.H_kv) + bh) * p.N * D;
+      const Unit x = unit_of(u);
+      const size_t head_off = p.kv_split == 1 ? (size_t)x.bh * p.N * D
+                                              : ((size_t)x.sp * BH_kv + x.bh) * p.N * D;
       float* out = (p.kv_split == 1 ? (w == 0 ? p.dv : p.dk) : (w == 0 ? p.dv_part : p.dk_part)) + head_off;
-      float acc[D];
+      // warpgroup 0 writes dV, warpgroup 1 writes scale * dK (rows past N are padding), 64
+      // columns at a time; once the last columns are loaded the next unit may overwrite them
       const uint32_t t_acc = tmem + lane_off + (w == 0 ? L::T_DV : L::T_DK);
-      if constexpr (D == 128) {
-        float hi[64];
-        tmem_ld64(t_acc, acc_lo_view(acc));
-        tmem_ld64(t_acc + 64, hi);
-#pragma unroll
-        for (int c = 0; c < 64; ++c) acc[64 + c] = hi[c];
-      } else {
-        tmem_ld64(t_acc, acc_lo_view(acc));
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
+        float acc[64];
+        tmem_ld64(t_acc + 64 * c, acc);
+        if (c == D / 64 - 1) {
+          tc_fence_before();
+          mbar_arrive(bar(L::BAR_ACC_FREE));
+        }
+        warp_store_rows_f32<64>(acc, out + 64 * c, D, j * 128 + wq * 32, p.N, w == 0 ? 1.0f : p.scale);
       }
-      // warpgroup 0 writes dV, warpgroup 1 writes scale * dK (rows past N are padding)
-      warp_store_rows_f32<D>(acc, out, D, j * 128 + wq * 32, p.N, w == 0 ? 1.0f : p.scale);
+      T0 += n_it;
+      u = next_unit(uc + 1, ok);
+      mbar_arrive(bar(L::BAR_UNIT_EMPTY + ((uc + 1) & 1)));
     }
   }
 
@@ -788,8 +868,9 @@ cudaError_t launch_one(Kern kern, dim3 grid, const CUtensorMap& a, const CUtenso
 
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                                   const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s) {
-  // key tiles x key/value heads x group splits
-  const dim3 grid((unsigned)(((p.N + 127) / 128) * (p.BH / p.H * p.H_kv) * p.kv_split));
+  // persistent: one CTA per SM (at most one per unit: key tile x key/value head x group split)
+  const long long units = (long long)((p.N + 127) / 128) * (p.BH / p.H * p.H_kv) * p.kv_split;
+  const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
   if (d == 128)
     return launch_one<DkdvLayout<128>>(fa_bwd_dkdv_sm100_kernel<128>, grid, tq, tdo, tk, tv, p, s);
   return launch_one<DkdvLayout<64>>(fa_bwd_dkdv_sm100_kernel<64>, grid, tq, tdo, tk, tv, p, s);

@@ -354,6 +354,7 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
   bp.kv_split = w.kv_split;
   bp.num_sms = g_num_sms[dev];
   bp.dq_counter = pp.counters;
+  bp.dkdv_counter = pp.counters + 1;
   bp.dk_part = w.kv_split > 1 ? reinterpret_cast<float*>(ws + w.off_dk_part) : nullptr;
   bp.dv_part = w.kv_split > 1 ? reinterpret_cast<float*>(ws + w.off_dv_part) : nullptr;
   bp.scale = scale;

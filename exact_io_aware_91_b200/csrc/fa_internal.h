@@ -24,7 +24,7 @@ struct FwdParams {
   int* err;          // device error word
 };
 
-constexpr int kNumCounters = 2;  // [0] dQ kernel, [1] reserved
+constexpr int kNumCounters = 2;  // work counters: [0] dQ kernel, [1] dK/dV kernel
 
 struct BwdPreParams {
   const void* q;     // bf16 (BH, N, d)
@@ -60,6 +60,7 @@ struct BwdParams {
   float* dv_part;      //   summed into dk / dv by launch_bwd_kv_reduce; unused when kv_split == 1
   int num_sms;         // multiprocessors of the device (grid of the persistent kernels)
   unsigned* dq_counter;  // work units handed out so far by the persistent dQ kernel (zeroed by the preprocess)
+  unsigned* dkdv_counter;  // the same for the persistent dK/dV kernel
   float scale;         // softmax scale (applied to dQ and dK)
   float scale_log2;    // scale * log2(e)
   int causal;
