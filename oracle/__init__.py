@@ -21,4 +21,5 @@ from .attention import (  # noqa: F401
     kv_head_of,
     attention_forward_gqa,
     attention_backward_gqa,
+    apply_window,
 )

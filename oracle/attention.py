@@ -40,6 +40,12 @@ consecutive query heads form a group -- and each head's attention is the
 definition above.  The gradients of a shared K or V are the sums of the
 per-query-head gradients over its group (the chain rule through the sharing).
 
+Sliding-window (local) attention ("Flash Attention uitgelegd: een uitgebreide
+gids", section on open problems, names sliding window attention for very long
+contexts without defining it).  Reading taken: a window (left, right) hides key j
+from query i unless i - left <= j <= i + right, a bound of -1 being unbounded; it
+combines with the causal mask, and every row keeps at least its own key.
+
 Parity pins: every function here is pinned by ``tests/test_oracle.py``
 (closed forms, invariants, finite differences, a hand-computed worked example,
 a library special case and a brute-force loop restatement).
@@ -62,6 +68,7 @@ __all__ = [
     "kv_head_of",
     "attention_forward_gqa",
     "attention_backward_gqa",
+    "apply_window",
 ]
 
 
@@ -87,6 +94,22 @@ def _scores(q2: np.ndarray, k2: np.ndarray, scale: float, causal: bool) -> np.nd
         j = np.arange(n_k)[None, :]
         s = np.where(j > i, -np.inf, s)
     return s
+
+
+def apply_window(s: np.ndarray, window=(-1, -1)) -> np.ndarray:
+    """S_ij = -inf outside the sliding window: query i sees key j only if
+    i - left <= j <= i + right (a bound of -1 is unbounded)."""
+    left, right = window
+    if left < 0 and right < 0:
+        return s
+    i = np.arange(s.shape[-2])[:, None]
+    j = np.arange(s.shape[-1])[None, :]
+    hide = np.zeros(s.shape[-2:], dtype=bool)
+    if left >= 0:
+        hide |= j < i - left
+    if right >= 0:
+        hide |= j > i + right
+    return np.where(hide, -np.inf, s)
 
 
 def _lse_rows(s: np.ndarray) -> np.ndarray:
@@ -115,10 +138,11 @@ def attention_probs(q, k, scale: float, causal: bool):
     return P.reshape(lead + P.shape[1:]), L.reshape(lead + (n,))
 
 
-def attention_forward(q, k, v, scale: float, causal: bool):
+def attention_forward(q, k, v, scale: float, causal: bool, window=(-1, -1)):
     """O = P V and LSE, one head at a time (the N x N matrix is materialised per head).
 
-    Inputs (..., N, d); returns O (..., N, d) and LSE (..., N) in float64.
+    Inputs (..., N, d); returns O (..., N, d) and LSE (..., N) in float64.  ``window``:
+    optional sliding window (left, right), see ``apply_window``.
     """
     q = _as_f64(q)
     k = _as_f64(k)
@@ -129,7 +153,7 @@ def attention_forward(q, k, v, scale: float, causal: bool):
     O = np.empty_like(q3, shape=q3.shape[:2] + (v3.shape[2],))
     L = np.empty(q3.shape[:2])
     for h in range(q3.shape[0]):
-        s = _scores(q3[h], k3[h], scale, causal)
+        s = apply_window(_scores(q3[h], k3[h], scale, causal), window)
         lse = _lse_rows(s)
         p = np.exp(s - lse[:, None])
         O[h] = p @ v3[h]
@@ -157,7 +181,7 @@ def attention_forward_rows(q, k, v, scale: float, causal: bool, rows):
     return p @ v, lse
 
 
-def attention_backward(q, k, v, do, scale: float, causal: bool, return_delta: bool = False):
+def attention_backward(q, k, v, do, scale: float, causal: bool, return_delta: bool = False, window=(-1, -1)):
     """Gradients of L = sum(O * dO) with respect to Q, K and V, from the definition.
 
     P is recomputed from Q and K (the backward never reuses a stored P).
@@ -177,7 +201,7 @@ def attention_backward(q, k, v, do, scale: float, causal: bool, return_delta: bo
     dv = np.empty_like(v3)
     D = np.empty(q3.shape[:2])
     for h in range(q3.shape[0]):
-        s = _scores(q3[h], k3[h], scale, causal)
+        s = apply_window(_scores(q3[h], k3[h], scale, causal), window)
         p = np.exp(s - _lse_rows(s)[:, None])
         dv[h] = p.T @ do3[h]
         dp = do3[h] @ v3[h].T
@@ -315,7 +339,7 @@ def _check_gqa_shapes(q, k, v):
         raise ValueError("K and V need (B, H_kv, N, .) with H a multiple of H_kv")
 
 
-def attention_forward_gqa(q, k, v, scale: float, causal: bool):
+def attention_forward_gqa(q, k, v, scale: float, causal: bool, window=(-1, -1)):
     """O and LSE of grouped-query attention, one query head at a time.
 
     q: (B, H, N, d); k, v: (B, H_kv, N, d).  Returns O (B, H, N, d_v), LSE (B, H, N).
@@ -329,14 +353,14 @@ def attention_forward_gqa(q, k, v, scale: float, causal: bool):
     for b in range(B):
         for h in range(H):
             g = kv_head_of(h, H, Hkv)
-            s = _scores(q[b, h], k[b, g], scale, causal)
+            s = apply_window(_scores(q[b, h], k[b, g], scale, causal), window)
             lse = _lse_rows(s)
             O[b, h] = np.exp(s - lse[:, None]) @ v[b, g]
             L[b, h] = lse
     return O, L
 
 
-def attention_backward_gqa(q, k, v, do, scale: float, causal: bool):
+def attention_backward_gqa(q, k, v, do, scale: float, causal: bool, window=(-1, -1)):
     """dQ (B, H, N, d), dK and dV (B, H_kv, N, d) of L = sum(O * dO) for grouped-query attention.
 
     Per query head the gradients are those of the plain definition (see
@@ -353,7 +377,7 @@ def attention_backward_gqa(q, k, v, do, scale: float, causal: bool):
     for b in range(B):
         for h in range(H):
             g = kv_head_of(h, H, Hkv)
-            s = _scores(q[b, h], k[b, g], scale, causal)
+            s = apply_window(_scores(q[b, h], k[b, g], scale, causal), window)
             p = np.exp(s - _lse_rows(s)[:, None])
             dp = do[b, h] @ v[b, g].T
             ds = p * (dp - np.sum(p * dp, axis=-1)[:, None])

@@ -379,3 +379,91 @@ def test_gqa_pin_catches_a_wrong_group_mapping(monkeypatch):
     monkeypatch.setattr(oa, "kv_head_of", lambda h, n_heads, n_kv_heads: h % n_kv_heads)
     with pytest.raises(AssertionError):
         test_gqa_zero_queries_average_their_group_values(True, 4, 2)
+
+
+# ---------------------------------------------------------------- sliding window
+@pytest.mark.parametrize("causal", [False, True])
+def test_window_covering_everything_is_no_window(causal):
+    q, k, v = randn((2, 23, 6), 80), randn((2, 23, 6), 81), randn((2, 23, 6), 82)
+    O1, L1 = attention_forward(q, k, v, 0.4, causal)
+    O2, L2 = attention_forward(q, k, v, 0.4, causal, window=(23, 23))
+    np.testing.assert_allclose(O2, O1, atol=1e-14)
+    np.testing.assert_allclose(L2, L1, atol=1e-14)
+
+
+@pytest.mark.parametrize("causal,window", [(True, (0, -1)), (False, (0, 0)), (True, (0, 5))])
+def test_window_of_one_key_returns_its_own_value(causal, window):
+    # each query sees only its own key: O_i = V_i, LSE_i = scale * q_i . k_i
+    q, k, v = randn((19, 7), 83), randn((19, 7), 84), randn((19, 7), 85)
+    O, L = attention_forward(q, k, v, 0.3, causal, window=window)
+    np.testing.assert_allclose(O, v, atol=1e-13)
+    np.testing.assert_allclose(L, 0.3 * np.sum(q * k, axis=-1), atol=1e-13)
+
+
+@pytest.mark.parametrize("left", [1, 3, 7])
+def test_zero_queries_average_the_window(left):
+    # Q = 0, causal, window (left, -1): query i averages V rows max(0, i - left) .. i
+    n, d = 17, 4
+    v = randn((n, d), 86)
+    O, L = attention_forward(np.zeros((n, d)), randn((n, d), 87), v, 1.0, True, window=(left, -1))
+    for i in range(n):
+        lo = max(0, i - left)
+        np.testing.assert_allclose(O[i], v[lo:i + 1].mean(0), atol=1e-13)
+        np.testing.assert_allclose(L[i], math.log(i - lo + 1), atol=1e-13)
+
+
+@pytest.mark.parametrize("causal,window", [(True, (4, -1)), (False, (3, 2)), (False, (-1, 1))])
+def test_window_agrees_with_torch_sdpa_explicit_mask_fp64(causal, window):
+    torch = pytest.importorskip("torch")
+    import torch.nn.functional as F
+
+    n = 29
+    q, k, v, do = (randn((2, 3, n, 8), s) for s in (88, 89, 90, 91))
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    allow = np.ones((n, n), dtype=bool)
+    if causal:
+        allow &= j <= i
+    if window[0] >= 0:
+        allow &= j >= i - window[0]
+    if window[1] >= 0:
+        allow &= j <= i + window[1]
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    out = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.tensor(allow), scale=0.35)
+    out.backward(torch.tensor(do))
+    O, _ = attention_forward(q, k, v, 0.35, causal, window=window)
+    np.testing.assert_allclose(O, out.detach().numpy(), atol=1e-10)
+    dq, dk, dv = attention_backward(q, k, v, do, 0.35, causal, window=window)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-10)
+
+
+@pytest.mark.parametrize("causal,window", [(True, (2, -1)), (False, (1, 2))])
+def test_window_backward_matches_central_finite_differences(causal, window):
+    q, k, v, do = (randn((6, 3), s) for s in (92, 93, 94, 95))
+    grads = attention_backward(q, k, v, do, 0.9, causal, window=window)
+    loss = lambda a, b, c: float(np.sum(attention_forward(a, b, c, 0.9, causal, window=window)[0] * do))  # noqa: E731
+    h = 1e-6
+    for which, g in zip(range(3), grads):
+        args = [q, k, v]
+        num = np.zeros_like(args[which])
+        for idx in np.ndindex(args[which].shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            num[idx] = (loss(*plus) - loss(*minus)) / (2 * h)
+        assert np.max(np.abs(num - g)) / max(1.0, np.max(np.abs(g))) <= 1e-6
+
+
+def test_window_pin_catches_an_off_by_one(monkeypatch):
+    def wider(s, window=(-1, -1)):  # one key too many on the left
+        left, right = window
+        return _orig_window(s, (left + 1 if left >= 0 else left, right))
+    monkeypatch.setattr(oa, "apply_window", wider)
+    with pytest.raises(AssertionError):
+        test_zero_queries_average_the_window(3)
+
+
+_orig_window = oa.apply_window
