@@ -24,10 +24,18 @@ FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
 
 EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_workspace_size", "fa_fwd_ws", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_gqa_workspace_size",
-           "fa_bwd_gqa", "fa_bwd_noalloc", "fa_device_status", "fa_bwd_set_phase_events", "fa_status_str")
+           "fa_bwd_gqa", "fa_attn_fwd_workspace_size", "fa_attn_fwd", "fa_attn_bwd_workspace_size", "fa_attn_bwd",
+           "fa_bwd_noalloc", "fa_device_status", "fa_bwd_set_phase_events", "fa_status_str")
 
 # Size of the scratch array fa_bwd_noalloc uses instead of a caller workspace.
 FA_BWD_NOALLOC_MAX_WORKSPACE = 64 << 20
+
+
+class FaAttnProblem(ctypes.Structure):
+    """``fa_attn_problem`` of ``include/fa.h``."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int), ("N", ctypes.c_int),
+                ("d", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int),
+                ("window_left", ctypes.c_int), ("window_right", ctypes.c_int)]
 
 
 class FAError(RuntimeError):
@@ -70,6 +78,15 @@ def library() -> ctypes.CDLL:
     lib.fa_bwd_gqa_workspace_size.restype = sz
     lib.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_bwd_gqa.restype = i
+    pp = ctypes.POINTER(FaAttnProblem)
+    lib.fa_attn_fwd_workspace_size.argtypes = [pp]
+    lib.fa_attn_fwd_workspace_size.restype = sz
+    lib.fa_attn_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.fa_attn_fwd.restype = i
+    lib.fa_attn_bwd_workspace_size.argtypes = [pp]
+    lib.fa_attn_bwd_workspace_size.restype = sz
+    lib.fa_attn_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.fa_attn_bwd.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_bwd_noalloc.restype = i
     lib.fa_device_status.argtypes = [vp]
@@ -282,6 +299,75 @@ def fa_bwd_gqa(q, k, v, o, do, lse, causal: bool = False, scale: float | None = 
                               dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N, d, _scale(scale, d),
                               int(bool(causal)), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
     _check("fa_bwd_gqa", st)
+    return dq, dk, dv
+
+
+def _problem(q, k, causal, scale, window) -> FaAttnProblem:
+    B, H, N, d = _shape(q)
+    H_kv = _gqa_heads(q, k)
+    wl, wr = window
+    return FaAttnProblem(B, H, H_kv, N, d, _scale(scale, d), int(bool(causal)), int(wl), int(wr))
+
+
+def fa_attn_fwd_workspace_size(problem: FaAttnProblem) -> int:
+    return int(library().fa_attn_fwd_workspace_size(ctypes.byref(problem)))
+
+
+def fa_attn_bwd_workspace_size(problem: FaAttnProblem) -> int:
+    return int(library().fa_attn_bwd_workspace_size(ctypes.byref(problem)))
+
+
+def fa_attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, window=(-1, -1), o=None, lse=None,
+                o_resid=None, save_residual: bool = False, workspace=None, stream=None):
+    """Forward with every option: grouped K/V heads (k, v (B, H_kv, N, d)) and a sliding
+    window (left, right) (-1 = unbounded).  Returns like ``fa_fwd``."""
+    pr = _problem(q, k, causal, scale, window)
+    B, H, N, d = _shape(q)
+    _same(q, dtype=torch.bfloat16, shape=(B, H, N, d))
+    _same(k, v, dtype=torch.bfloat16, shape=(B, pr.H_kv, N, d))
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if o_resid is None and save_residual:
+        o_resid = torch.empty_like(q)
+    _same(o, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if o_resid is not None:
+        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if workspace is None:
+        workspace = torch.empty(max(fa_attn_fwd_workspace_size(pr), 1), dtype=torch.uint8, device=q.device)
+    st = library().fa_attn_fwd(ctypes.byref(pr), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                               lse.data_ptr(), None if o_resid is None else o_resid.data_ptr(), workspace.data_ptr(),
+                               workspace.numel(), _stream_handle(stream))
+    _check("fa_attn_fwd", st)
+    return (o, lse) if o_resid is None else (o, lse, o_resid)
+
+
+def fa_attn_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, window=(-1, -1),
+                workspace=None, dq=None, dk=None, dv=None, o_resid=None, stream=None):
+    """Backward with every option (the same problem as the forward).  Returns (dq, dk, dv)."""
+    pr = _problem(q, k, causal, scale, window)
+    B, H, N, d = _shape(q)
+    _same(q, o, do, dtype=torch.bfloat16, shape=(B, H, N, d))
+    _same(k, v, dtype=torch.bfloat16, shape=(B, pr.H_kv, N, d))
+    _same(lse, dtype=torch.float32, shape=(B, H, N))
+    if o_resid is not None:
+        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if dq is None:
+        dq = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    if dk is None:
+        dk = torch.empty((B, pr.H_kv, N, d), dtype=torch.float32, device=q.device)
+    if dv is None:
+        dv = torch.empty_like(dk)
+    _same(dq, dtype=torch.float32, shape=(B, H, N, d))
+    _same(dk, dv, dtype=torch.float32, shape=(B, pr.H_kv, N, d))
+    if workspace is None:
+        workspace = torch.empty(max(fa_attn_bwd_workspace_size(pr), 1), dtype=torch.uint8, device=q.device)
+    st = library().fa_attn_bwd(ctypes.byref(pr), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                               None if o_resid is None else o_resid.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                               dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                               _stream_handle(stream))
+    _check("fa_attn_bwd", st)
     return dq, dk, dv
 
 

@@ -193,8 +193,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     unit_order(u, n_kt * p.kv_split, BH_kv, p.head_group_kv, x.bh, rank);
     x.j = rank / p.kv_split;   // key tile
     x.sp = rank % p.kv_split;  // which share of the group's query heads
-    x.i_start = p.causal ? x.j : 0;
-    x.n_q = n_kt - x.i_start;  // 128-query tiles per query head, >= 1
+    // query tiles that see some key of this tile (causal mask, sliding window)
+    x.i_start = query_lo(x.j * 128, p.causal, p.win_right) / 128;
+    x.n_q = query_hi(min(x.j * 128 + 127, p.N - 1), p.N, p.win_left) / 128 - x.i_start + 1;  // >= 1
     x.n_it = g_per * x.n_q;    // steps: query head q_head_of(bh, sp * g_per + it / n_q), tile i_start + it % n_q
     return x;
   };
@@ -398,13 +399,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         n_it = x.n_it;
       }
       const int key = j * 128 + row;
+      const int q_vis_lo = query_lo(key, p.causal, p.win_right);
+      const int q_vis_hi = query_hi(key, p.N, p.win_left);
       for (int it = 0; it < n_it; ++it) {
         const int T = T0 + it;
         const int i = i_start + it % n_q;  // query tile of this step
         const float* lse2 = reinterpret_cast<const float*>(gbase + L::OFF_LD + (T & 1) * 1024) + 64 * w;
         const float* delta = lse2 + 128;
         const int q0 = i * 128 + 64 * w;  // first query of this warpgroup's columns
-        const bool need_mask = p.causal && (q0 < j * 128 + 127);
+        // this key's visible queries (causal mask, sliding window); padded queries have P = 0
+        const bool need_mask = q0 < q_vis_lo || q0 + 63 > q_vis_hi;
         // ---- P^T = 2^(S^T * scale * log2(e) - lse2), written back over S^T as fp16
         if (!(ok = mbar_wait(bar(L::BAR_S), T & 1, wctx))) break;
         tc_fence_after();
@@ -435,10 +439,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               pr[c + 3] = ex2_approx(t3);
             }
             if (need_mask) {
-              if (q0 + c < key) pr[c] = 0.f;
-              if (q0 + c + 1 < key) pr[c + 1] = 0.f;
-              if (q0 + c + 2 < key) pr[c + 2] = 0.f;
-              if (q0 + c + 3 < key) pr[c + 3] = 0.f;
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (q0 + c + e < q_vis_lo || q0 + c + e > q_vis_hi) pr[c + e] = 0.f;
             }
             pk[(c - g) / 2] = pack_f16(pr[c], pr[c + 1]);
             pk[(c - g) / 2 + 1] = pack_f16(pr[c + 2], pr[c + 3]);
@@ -573,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nq = (p.N + 127) / 128;
   const int n_units = nq * p.BH;
   struct Unit {
-    int bh, bh_kv, qt, n_it;
+    int bh, bh_kv, qt, jlo, n_it;
   };
   auto unit_of = [&](int u) -> Unit {
     Unit x;
@@ -581,7 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     unit_order(u, nq, p.BH, p.head_group, x.bh, rank);
     x.bh_kv = kv_head_of(x.bh, p.H, p.H_kv);  // the key/value head this query head reads
     x.qt = p.causal ? (nq - 1 - rank) : rank;
-    x.n_it = p.causal ? x.qt + 1 : nq;        // 128-key steps
+    // key tiles this query tile sees (causal mask, sliding window): 128-key steps
+    x.jlo = key_lo(x.qt * 128, p.N, p.win_left) / 128;
+    x.n_it = key_hi(x.qt * 128 + 127, p.N, p.causal, p.win_right) / 128 - x.jlo + 1;
     return x;
   };
 
@@ -665,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(bar(L::BAR_K_EMPTY + sk), ((T / 3) & 1) ^ 1u, wctx))) break;
         mbar_arrive_expect_tx(bar(L::BAR_K_FULL + sk), L::TILE, leader);
         for (int c = 0; c < L::KCH; ++c)
-          tma_load_3d(base + L::OFF_K + sk * L::TILE + c * kBox, &tm_k, c * 64, it * 128, x.bh_kv,
+          tma_load_3d(base + L::OFF_K + sk * L::TILE + c * kBox, &tm_k, c * 64, (x.jlo + it) * 128, x.bh_kv,
                       bar(L::BAR_K_FULL + sk), leader);
         if (!(ok = mbar_wait(bar(L::BAR_V_EMPTY + sv), ((T >> 1) & 1) ^ 1u, wctx))) {
           ++T;  // the K tile of this step was issued
@@ -673,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(bar(L::BAR_V_FULL + sv), L::TILE, leader);
         for (int c = 0; c < L::KCH; ++c)
-          tma_load_3d(base + L::OFF_V + sv * L::TILE + c * kBox, &tm_v, c * 64, it * 128, x.bh_kv,
+          tma_load_3d(base + L::OFF_V + sv * L::TILE + c * kBox, &tm_v, c * 64, (x.jlo + it) * 128, x.bh_kv,
                       bar(L::BAR_V_FULL + sv), leader);
       }
     }
@@ -772,14 +777,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int uc = 0; ok && u < n_units; ++uc) {
       const Unit x = unit_of(u);
       const int r = x.qt * 128 + row;  // query index
-      const int lim = p.causal ? min(r, p.N - 1) : (p.N - 1);  // last visible key
+      const int k_vis_lo = key_lo(r, p.N, p.win_left);  // visible keys of this row
+      const int k_vis_hi = key_hi(r, p.N, p.causal, p.win_right);
       const uint64_t nl2 = f2pack(-lse2, -lse2), dd = f2pack(delta, delta);
       for (int it = 0; it < x.n_it; ++it) {
         const int t = T0 + it;
         const int b = t & 1;
         const uint32_t tS = tmem + lane_off + L::T_S + 128 * b + 64 * w;
-        const int k0 = it * 128 + 64 * w;  // first key of this warpgroup's columns
-        const bool need_mask = (p.causal && k0 + 63 > x.qt * 128) || (k0 + 64 > p.N);
+        const int k0 = (x.jlo + it) * 128 + 64 * w;  // first key of this warpgroup's columns
+        const bool need_mask = k0 < k_vis_lo || k0 + 63 > k_vis_hi;
         if (!(ok = mbar_wait(bar(L::BAR_S + b), (t >> 1) & 1, wctx))) break;
         tc_fence_after();
         float pr[64];
@@ -791,8 +797,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           pr[c] = ex2_approx(t0);
           pr[c + 1] = ex2_approx(t1);
           if (need_mask) {
-            if (k0 + c > lim) pr[c] = 0.f;
-            if (k0 + c + 1 > lim) pr[c + 1] = 0.f;
+            if (k0 + c < k_vis_lo || k0 + c > k_vis_hi) pr[c] = 0.f;
+            if (k0 + c + 1 < k_vis_lo || k0 + c + 1 > k_vis_hi) pr[c + 1] = 0.f;
           }
         }
         if (!(ok = mbar_wait(bar(L::BAR_DP), t & 1, wctx))) break;

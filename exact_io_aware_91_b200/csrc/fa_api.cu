@@ -86,6 +86,8 @@ fa_status check_problem(int B, int H, int H_kv, int N, int d, float scale, int c
   return FA_OK;
 }
 
+bool window_ok(int wl, int wr) { return wl >= -1 && wr >= -1; }
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct BwdLayout {
@@ -181,9 +183,10 @@ namespace {
 // Shared body of fa_fwd_gqa (V converted on chip) and fa_fwd_ws (V converted to fp16 into
 // the workspace by a streaming pass first).
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
-                   int H_kv, int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
-                   fa_stream_t stream) {
+                   int H_kv, int N, int d, float scale, int causal, int wl, int wr, void* workspace,
+                   size_t workspace_bytes, fa_stream_t stream) {
   bool empty = false;
+  if (!window_ok(wl, wr)) return FA_ERR_INVALID_ARG;
   fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
   if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
@@ -224,6 +227,8 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   p.head_group = head_group_size(BH, 4ull * N * d / (H / H_kv), kFwdGroupBytes);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal;
+  p.win_left = wl;
+  p.win_right = wr;
   p.err = g_err_ptr[dev];
   // with a workspace: the persistent kernel (work counter in the workspace); without: one CTA
   // per unit, V converted on chip
@@ -234,7 +239,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
 
 fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
                      int H_kv, int N, int d, float scale, int causal, fa_stream_t stream) {
-  return fwd_impl(q, k, v, o, lse, o_resid, B, H, H_kv, N, d, scale, causal, nullptr, 0, stream);
+  return fwd_impl(q, k, v, o, lse, o_resid, B, H, H_kv, N, d, scale, causal, -1, -1, nullptr, 0, stream);
 }
 
 size_t fa_fwd_workspace_size(int B, int H_kv, int N, int d) {
@@ -251,7 +256,8 @@ fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float*
     const fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty);
     return (st != FA_OK || empty) ? st : FA_ERR_INVALID_ARG;
   }
-  return fwd_impl(q, k, v, o, lse, o_resid, B, H, H_kv, N, d, scale, causal, workspace, workspace_bytes, stream);
+  return fwd_impl(q, k, v, o, lse, o_resid, B, H, H_kv, N, d, scale, causal, -1, -1, workspace, workspace_bytes,
+                  stream);
 }
 
 fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N,
@@ -285,11 +291,28 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                     workspace_bytes, stream);
 }
 
+namespace {
+fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                   const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int H_kv, int N,
+                   int d, float scale, int causal, int wl, int wr, void* workspace, size_t workspace_bytes,
+                   fa_stream_t stream);
+}  // namespace
+
 fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
                      const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int H_kv,
                      int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
                      fa_stream_t stream) {
+  return bwd_impl(q, k, v, o, o_resid, dout, lse, dq, dk, dv, B, H, H_kv, N, d, scale, causal, -1, -1, workspace,
+                  workspace_bytes, stream);
+}
+
+namespace {
+fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                   const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int H_kv, int N,
+                   int d, float scale, int causal, int wl, int wr, void* workspace, size_t workspace_bytes,
+                   fa_stream_t stream) {
   bool empty = false;
+  if (!window_ok(wl, wr)) return FA_ERR_INVALID_ARG;
   fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty);
   if (st != FA_OK || empty) return st;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
@@ -360,6 +383,8 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
   bp.scale = scale;
   bp.scale_log2 = scale * 1.4426950408889634f;
   bp.causal = causal;
+  bp.win_left = wl;
+  bp.win_right = wr;
   bp.err = g_err_ptr[dev];
   if (launch_bwd_dkdv_sm100(t_q, t_do, t_k, t_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
   if (w.kv_split > 1 &&
@@ -370,6 +395,39 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
     return FA_ERR_CUDA;
   if (launch_bwd_dq_sm100(t_q, t_do, t_k, t_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
+}
+
+}  // namespace
+
+// ---- descriptor-based entry points (every option: grouped heads, sliding window)
+size_t fa_attn_fwd_workspace_size(const fa_attn_problem* pr) {
+  if (pr == nullptr || !window_ok(pr->window_left, pr->window_right)) return 0;
+  return fa_fwd_workspace_size(pr->B, pr->H_kv, pr->N, pr->d);
+}
+
+fa_status fa_attn_fwd(const fa_attn_problem* pr, const void* q, const void* k, const void* v, void* o, float* lse,
+                      void* o_resid, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  if (pr == nullptr) return FA_ERR_INVALID_ARG;
+  if (workspace == nullptr) {
+    bool empty = false;
+    const fa_status st = check_problem(pr->B, pr->H, pr->H_kv, pr->N, pr->d, pr->scale, pr->causal, &empty);
+    return (st != FA_OK || empty) ? st : FA_ERR_INVALID_ARG;
+  }
+  return fwd_impl(q, k, v, o, lse, o_resid, pr->B, pr->H, pr->H_kv, pr->N, pr->d, pr->scale, pr->causal,
+                  pr->window_left, pr->window_right, workspace, workspace_bytes, stream);
+}
+
+size_t fa_attn_bwd_workspace_size(const fa_attn_problem* pr) {
+  if (pr == nullptr || !window_ok(pr->window_left, pr->window_right)) return 0;
+  return fa_bwd_gqa_workspace_size(pr->B, pr->H, pr->H_kv, pr->N, pr->d);
+}
+
+fa_status fa_attn_bwd(const fa_attn_problem* pr, const void* q, const void* k, const void* v, const void* o,
+                      const void* o_resid, const void* dout, const float* lse, float* dq, float* dk, float* dv,
+                      void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  if (pr == nullptr) return FA_ERR_INVALID_ARG;
+  return bwd_impl(q, k, v, o, o_resid, dout, lse, dq, dk, dv, pr->B, pr->H, pr->H_kv, pr->N, pr->d, pr->scale,
+                  pr->causal, pr->window_left, pr->window_right, workspace, workspace_bytes, stream);
 }
 
 void fa_bwd_set_phase_events(void* const* events) { t_phase_events = events; }

@@ -21,8 +21,29 @@ struct FwdParams {
   int head_group;    // heads per group in the CTA order (unit_order)
   float scale_log2;  // softmax scale * log2(e)
   int causal;
+  int win_left, win_right;  // sliding window: query i sees keys i - left .. i + right (-1 unbounded)
   int* err;          // device error word
 };
+
+// Visible keys of query row i under the causal mask and the sliding window (inclusive
+// bounds; rows past N behave like row N - 1, so every row keeps at least one key).
+__host__ __device__ __forceinline__ int key_lo(int i, int N, int wl) {
+  const int r = i < N ? i : N - 1;
+  return (wl >= 0 && r - wl > 0) ? r - wl : 0;
+}
+__host__ __device__ __forceinline__ int key_hi(int i, int N, int causal, int wr) {
+  const int r = i < N ? i : N - 1;
+  if (causal) return r;
+  return (wr >= 0 && r + wr < N - 1) ? r + wr : N - 1;
+}
+// Queries that see key k (the inverse of the row ranges above; N = query count).
+__host__ __device__ __forceinline__ int query_lo(int k, int causal, int wr) {
+  if (causal) return k;
+  return (wr >= 0 && k - wr > 0) ? k - wr : 0;
+}
+__host__ __device__ __forceinline__ int query_hi(int k, int N, int wl) {
+  return (wl >= 0 && k + wl < N - 1) ? k + wl : N - 1;
+}
 
 constexpr int kNumCounters = 2;  // work counters: [0] dQ kernel, [1] dK/dV kernel
 
@@ -64,6 +85,7 @@ struct BwdParams {
   float scale;         // softmax scale (applied to dQ and dK)
   float scale_log2;    // scale * log2(e)
   int causal;
+  int win_left, win_right;  // sliding window (see FwdParams)
   int* err;
 };
 

@@ -102,98 +102,99 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 template <int D>
 __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS, uint32_t tO, uint32_t bar_s_full,
                                                  uint32_t s_parity, uint32_t bar_p_half, uint32_t bar_p_full, int j,
-                                                 int q_base, int r, float& m, float& l, const WaitCtx& wctx) {
+                                                 bool first, int r, float& m, float& l, const WaitCtx& wctx) {
   const float sl2 = p.scale_log2;
   if (!mbar_wait(bar_s_full, s_parity, wctx)) return false;
-    tc_fence_after();
-    float x[128];
-    {
-      uint32_t u[4][32];
+  tc_fence_after();
+  float x[128];
+  {
+    uint32_t u[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, u[c]);
+    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, u[c]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(u[c][i]);
+  }
+  // keys kb .. kb + 127 against this row's visible range (causal mask, sliding window, N);
+  // with a window a row can have no visible key in a tile of its warpgroup's range
+  const int kb = j * 128;
+  const int lo = key_lo(r, p.N, p.win_left), hi = key_hi(r, p.N, p.causal, p.win_right);
+  if (kb < lo || kb + 127 > hi) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      if (kb + c < lo || kb + c > hi) x[c] = -INFINITY;
+  }
+  // row max: four independent 3-input max chains
+  float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
+#pragma unroll
+  for (int c = 4; c < 124; c += 8) {
+    a0 = max3f(a0, x[c], x[c + 1]);
+    a1 = max3f(a1, x[c + 2], x[c + 3]);
+    a2 = max3f(a2, x[c + 4], x[c + 5]);
+    a3 = max3f(a3, x[c + 6], x[c + 7]);
+  }
+  a0 = max3f(a0, x[124], x[125]);
+  a1 = max3f(a1, x[126], x[127]);
+  const float mx = max3f(fmaxf(a0, a1), a2, a3);
+  const float m_new = fmaxf(m, mx * sl2);
+  // keep a stale maximum while it is within 2^8 of the true one: exact in the end
+  // because O / l and the LSE use the same maximum
+  const float m_use = (m_new - m > 8.0f) ? m_new : m;
+  const float alpha = (m_use == m) ? 1.0f : ex2_approx(m - m_use);  // 0 on the first tile
+  const float neg_m = m_use == -INFINITY ? 0.0f : -m_use;  // no visible key yet: every P is 0
+  if (!first && __any_sync(0xffffffffu, alpha != 1.0f)) {
+    // rescale O before this tile's P V starts; the previous O += P V of this tile
+    // completed before S_j did (same issuing thread, in-order tensor pipe)
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t u[32];
+      tmem_ld32(tO + 32 * c, u);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(u[c][i]);
+      for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+      tmem_st32(tO + 32 * c, u);
     }
-    const int kb = j * 128;
-    const bool need_mask = (p.causal && kb + 127 > q_base) || (kb + 128 > p.N);
-    if (need_mask) {
-      const int lim = p.causal ? min(r, p.N - 1) : (p.N - 1);  // last visible key
+  }
+  uint64_t sa = 0, sb = 0;  // packed fp32 partial row sums (0.0f, 0.0f)
 #pragma unroll
-      for (int c = 0; c < 128; ++c)
-        if (kb + c > lim) x[c] = -INFINITY;
-    }
-    // row max: four independent 3-input max chains
-    float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
+  for (int h = 0; h < 2; ++h) {
+    uint32_t pk[32];
 #pragma unroll
-    for (int c = 4; c < 124; c += 8) {
-      a0 = max3f(a0, x[c], x[c + 1]);
-      a1 = max3f(a1, x[c + 2], x[c + 3]);
-      a2 = max3f(a2, x[c + 4], x[c + 5]);
-      a3 = max3f(a3, x[c + 6], x[c + 7]);
-    }
-    a0 = max3f(a0, x[124], x[125]);
-    a1 = max3f(a1, x[126], x[127]);
-    const float mx = max3f(fmaxf(a0, a1), a2, a3);
-    const float m_new = fmaxf(m, mx * sl2);
-    // keep a stale maximum while it is within 2^8 of the true one: exact in the end
-    // because O / l and the LSE use the same maximum
-    const float m_use = (m_new - m > 8.0f) ? m_new : m;
-    const float alpha = (m_use == m) ? 1.0f : ex2_approx(m - m_use);  // 0 on the first tile
-    const float neg_m = -m_use;
-    if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-      // rescale O before this tile's P V starts; the previous O += P V of this tile
-      // completed before S_j did (same issuing thread, in-order tensor pipe)
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(tO + 32 * c, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-        tmem_st32(tO + 32 * c, u);
+    for (int i = 0; i < 32; i += 2) {
+      float* e = &x[64 * h + 2 * i];
+      fma2(e[0], e[1], sl2, neg_m);
+      fma2(e[2], e[3], sl2, neg_m);
+      // kExpFmaPer8 of every 8 element pairs take 2^x on the FMA pipe, the rest on MUFU
+      if ((i & 7) < 2 * (kExpFmaPer8 / 2)) {
+        exp2_fma_pipe(e[0], e[1]);
+        exp2_fma_pipe(e[2], e[3]);
+        pk[i] = pack_f16(e[0], e[1]);
+        pk[i + 1] = pack_f16(e[2], e[3]);
+      } else {
+        e[0] = ex2_approx(e[0]);
+        e[1] = ex2_approx(e[1]);
+        e[2] = ex2_approx(e[2]);
+        e[3] = ex2_approx(e[3]);
+        pk[i] = pack_f16(e[0], e[1]);
+        pk[i + 1] = pack_f16(e[2], e[3]);
       }
+      asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sa) : "l"(f2pack(e[0], e[1])));
+      asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sb) : "l"(f2pack(e[2], e[3])));
     }
-    uint64_t sa = 0, sb = 0;  // packed fp32 partial row sums (0.0f, 0.0f)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t pk[32];
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float* e = &x[64 * h + 2 * i];
-        fma2(e[0], e[1], sl2, neg_m);
-        fma2(e[2], e[3], sl2, neg_m);
-        // kExpFmaPer8 of every 8 element pairs take 2^x on the FMA pipe, the rest on MUFU
-        if ((i & 7) < 2 * (kExpFmaPer8 / 2)) {
-          exp2_fma_pipe(e[0], e[1]);
-          exp2_fma_pipe(e[2], e[3]);
-          pk[i] = pack_f16(e[0], e[1]);
-          pk[i + 1] = pack_f16(e[2], e[3]);
-        } else {
-          e[0] = ex2_approx(e[0]);
-          e[1] = ex2_approx(e[1]);
-          e[2] = ex2_approx(e[2]);
-          e[3] = ex2_approx(e[3]);
-          pk[i] = pack_f16(e[0], e[1]);
-          pk[i + 1] = pack_f16(e[2], e[3]);
-        }
-        asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sa) : "l"(f2pack(e[0], e[1])));
-        asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sb) : "l"(f2pack(e[2], e[3])));
-      }
-      tmem_st32(tS + 32 * h, pk);
-      // first half of P (and any rescale of O) visible to the tensor core: its half of P V
-      // can start while the second half is computed
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(h == 0 ? bar_p_half : bar_p_full);
-    }
-    float s0, s1, s2, s3;
-    f2unpack(sa, s0, s1);
-    f2unpack(sb, s2, s3);
-    l = fmaf(l, alpha, (s0 + s1) + (s2 + s3));
-    m = m_use;
+    tmem_st32(tS + 32 * h, pk);
+    // first half of P (and any rescale of O) visible to the tensor core: its half of P V
+    // can start while the second half is computed
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(h == 0 ? bar_p_half : bar_p_full);
+  }
+  float s0, s1, s2, s3;
+  f2unpack(sa, s0, s1);
+  f2unpack(sb, s2, s3);
+  l = fmaf(l, alpha, (s0 + s1) + (s2 + s3));
+  m = m_use;
   return true;
 }
 
@@ -412,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < n_t; ++j) {
       if (!(ok = fwd_softmax_step<D>(p, tS, tO, bar(L::BAR_S_FULL + t), j & 1, bar(L::BAR_P_HALF + t),
-                                     bar(L::BAR_P_FULL + t), j, q_base, r, m, l, wctx)))
+                                     bar(L::BAR_P_FULL + t), j, j == 0, r, m, l, wctx)))
         break;
     }
     // ---- epilogue: O / l -> bf16 -> swizzled staging (the Q tile's buffer) -> TMA store
@@ -533,9 +534,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   const int n_units = p.n_pairs * p.BH;
-  const int n_kv = (p.N + 127) / 128;
+  // a unit's key tiles: tile t (rows q_base0 + 128 t .. + 127) needs key tiles jlo_t .. jhi_t
+  // (causal mask and sliding window); jlo0 <= jlo1 <= jhi0 + 1 and jhi0 <= jhi1, so the
+  // unit streams jlo0 .. jhi1 once for both tiles
   struct Unit {
-    int bh, bh_kv, q_base0, n0, n1;
+    int bh, bh_kv, q_base0, jlo0, jhi0, jlo1, jhi1;
   };
   auto unit_of = [&](int u) -> Unit {
     Unit x;
@@ -544,8 +547,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pair = p.causal ? (p.n_pairs - 1 - rank) : rank;
     x.bh_kv = kv_head_of(x.bh, p.H, p.H_kv);
     x.q_base0 = pair * 256;
-    x.n0 = p.causal ? min(n_kv, x.q_base0 / 128 + 1) : n_kv;
-    x.n1 = p.causal ? min(n_kv, x.q_base0 / 128 + 2) : n_kv;  // n1 >= n0
+    x.jlo0 = key_lo(x.q_base0, p.N, p.win_left) / 128;
+    x.jhi0 = key_hi(x.q_base0 + 127, p.N, p.causal, p.win_right) / 128;
+    x.jlo1 = key_lo(x.q_base0 + 128, p.N, p.win_left) / 128;
+    x.jhi1 = key_hi(x.q_base0 + 255, p.N, p.causal, p.win_right) / 128;
     return x;
   };
   int* unit_ring = reinterpret_cast<int*>(gbase + L::OFF_UNIT);
@@ -615,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     leader);
       }
       ++q_issued;
-      for (int j = 0; j < x.n1 && ok; ++j) {
+      for (int j = x.jlo0; j <= x.jhi1 && ok; ++j) {
         for (int which = 0; which < 2; ++which) {
           const int st = issued % L::STAGES;
           if (!(ok = mbar_wait(bar(L::BAR_KV_EMPTY + st), ((issued / L::STAGES) & 1) ^ 1u, wctx))) break;
@@ -685,39 +690,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit x = unit_of(u);
       if (!(ok = mbar_wait(bar(L::BAR_Q_FULL), uc & 1, wctx))) break;
       tc_fence_after();
-      int prev_v_stage = 0;
-      for (int j = 0; j < x.n1 && ok; ++j) {
-        const int iK = L0 + 2 * j, iV = iK + 1;
+      // per key tile j of the unit's stream: S0_j, O1 += P1 V_(tile 1's previous step), S1_j,
+      // O0 += P0 V_j -- each only where tile 0 / tile 1 has j in its range
+      int pend1 = -1;        // K/V stage of the V tile of tile 1's pending P V
+      int jt0 = 0, jt1 = 0;  // steps of tile 0 / tile 1 so far in this unit
+      for (int j = x.jlo0; j <= x.jhi1 && ok; ++j) {
+        const int li = j - x.jlo0;
+        const int iK = L0 + 2 * li, iV = iK + 1;
         const int stK = iK % L::STAGES, stV = iV % L::STAGES;
+        const bool in0 = j <= x.jhi0, in1 = j >= x.jlo1;
         if (!(ok = mbar_wait(bar(L::BAR_KV_FULL + stK), (iK / L::STAGES) & 1, wctx))) break;
         tc_fence_after();
-        if (j < x.n0) {
+        if (in0) {
           issue_qk(tS[0], dQ[0], stK);
           mma_commit(bar(L::BAR_S_FULL + 0), leader);
         }
-        if (j > 0) {  // O1 += P1 V_{j-1}
-          if (!(ok = issue_pv(1, j - 1, prev_v_stage, uc))) break;
-          mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage), leader);
+        if (in1 && pend1 >= 0) {  // O1 += P1 V of tile 1's previous step
+          if (!(ok = issue_pv(1, jt1 - 1, pend1, uc))) break;
+          mma_commit(bar(L::BAR_KV_EMPTY + pend1), leader);
         }
-        issue_qk(tS[1], dQ[1], stK);
-        mma_commit(bar(L::BAR_S_FULL + 1), leader);
+        if (in1) {
+          issue_qk(tS[1], dQ[1], stK);
+          mma_commit(bar(L::BAR_S_FULL + 1), leader);
+        }
         mma_commit(bar(L::BAR_KV_EMPTY + stK), leader);
-        if (j == x.n1 - 1) mma_commit(bar(L::BAR_Q_EMPTY), leader);  // the unit's last Q K^T
+        if (j == x.jhi1) mma_commit(bar(L::BAR_Q_EMPTY), leader);  // the unit's last Q K^T
         if (!(ok = mbar_wait(bar(L::BAR_KV_FULL + stV), (iV / L::STAGES) & 1, wctx))) break;
         tc_fence_after();
-        if (j < x.n0) {  // O0 += P0 V_j
-          if (!(ok = issue_pv(0, j, stV, uc))) break;
-          if (j == x.n0 - 1) mma_commit(bar(L::BAR_O_FULL + 0), leader);
+        if (in0) {  // O0 += P0 V_j
+          if (!(ok = issue_pv(0, jt0, stV, uc))) break;
+          if (j == x.jhi0) mma_commit(bar(L::BAR_O_FULL + 0), leader);
+          if (!in1) mma_commit(bar(L::BAR_KV_EMPTY + stV), leader);  // tile 1 does not use V_j
+          ++jt0;
         }
-        prev_v_stage = stV;
+        if (in1) {
+          pend1 = stV;
+          ++jt1;
+        }
       }
       if (!ok) break;
-      if (!(ok = issue_pv(1, x.n1 - 1, prev_v_stage, uc))) break;  // O1 += P1 V_{n1-1}
-      mma_commit(bar(L::BAR_KV_EMPTY + prev_v_stage), leader);
+      if (!(ok = issue_pv(1, jt1 - 1, pend1, uc))) break;  // tile 1's last P V
+      mma_commit(bar(L::BAR_KV_EMPTY + pend1), leader);
       mma_commit(bar(L::BAR_O_FULL + 1), leader);
-      L0 += 2 * x.n1;
-      G0 += x.n0;
-      G1 += x.n1;
+      L0 += 2 * (x.jhi1 - x.jlo0 + 1);
+      G0 += jt0;
+      G1 += jt1;
     }
     // every MMA issued so far has finished before TMEM is released
     mma_commit(bar(L::BAR_MMA_DONE), leader);
@@ -741,13 +758,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit x = unit_of(u);
       const int q_base = x.q_base0 + 128 * t;
       const int r = q_base + row;  // query index
-      const int n_t = t ? x.n1 : x.n0;
+      const int jlo = t ? x.jlo1 : x.jlo0;
+      const int n_t = (t ? x.jhi1 : x.jhi0) - jlo + 1;
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < n_t; ++j) {
-        if (!(ok = fwd_softmax_step<D>(p, tS, tO, bar(L::BAR_S_FULL + t), (G + j) & 1, bar(L::BAR_P_HALF + t),
-                                       bar(L::BAR_P_FULL + t), j, q_base, r, m, l, wctx)))
+      for (int jj = 0; jj < n_t; ++jj) {
+        if (!(ok = fwd_softmax_step<D>(p, tS, tO, bar(L::BAR_S_FULL + t), (G + jj) & 1, bar(L::BAR_P_HALF + t),
+                                       bar(L::BAR_P_FULL + t), jlo + jj, jj == 0, r, m, l, wctx)))
           break;
       }
+      G += n_t;
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 and the bf16 residual, stored from registers
       if (!(ok = mbar_wait(bar(L::BAR_O_FULL + t), uc & 1, wctx))) break;
@@ -787,7 +806,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                q_base + wq * 32, p.N);
       }
       if (p.lse != nullptr && r < p.N) p.lse[(size_t)x.bh * p.N + r] = (m + __log2f(l)) * 0.69314718055994531f;
-      G += n_t;
       u = next_unit(uc + 1, ok);
       mbar_arrive(bar(L::BAR_UNIT_EMPTY + ((uc + 1) & 1)));
     }

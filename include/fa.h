@@ -188,6 +188,41 @@ FA_API fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const v
                             size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * Descriptor-based entry points: every option of the library in one problem
+ * description, so that later options do not need new signatures.
+ *   B, H, H_kv, N, d, scale, causal : as in fa_fwd_gqa / fa_bwd_gqa (H_kv = H for plain
+ *                                     multi-head attention).
+ *   window_left, window_right        : sliding-window (local) attention: query i sees key
+ *                                     j only if i - window_left <= j <= i + window_right;
+ *                                     -1 = unbounded on that side (both -1: no window).
+ *                                     Combined with the causal mask (which already
+ *                                     bounds the right side).  Every row keeps at least
+ *                                     its own key.  ("Flash Attention uitgelegd: een
+ *                                     uitgebreide gids" names sliding window attention for
+ *                                     long contexts; the (left, right) convention is the
+ *                                     reading taken.)  Values < -1 are FA_ERR_INVALID_ARG.
+ * fa_attn_fwd needs a workspace (fa_attn_fwd_workspace_size bytes; the forward of
+ * fa_fwd_ws); fa_attn_bwd as fa_bwd_gqa with fa_attn_bwd_workspace_size bytes.  The
+ * backward must be given the same problem (window included) as the forward whose O, LSE
+ * and residual it receives.  The workspace-size functions return 0 for an empty or
+ * invalid problem (or a NULL descriptor).
+ */
+typedef struct fa_attn_problem {
+  int B, H, H_kv, N, d;
+  float scale;
+  int causal;
+  int window_left, window_right;
+} fa_attn_problem;
+FA_API size_t fa_attn_fwd_workspace_size(const fa_attn_problem* problem);
+FA_API fa_status fa_attn_fwd(const fa_attn_problem* problem, const void* q, const void* k, const void* v, void* o,
+                             float* lse, void* o_resid, void* workspace, size_t workspace_bytes,
+                             fa_stream_t stream);
+FA_API size_t fa_attn_bwd_workspace_size(const fa_attn_problem* problem);
+FA_API fa_status fa_attn_bwd(const fa_attn_problem* problem, const void* q, const void* k, const void* v,
+                             const void* o, const void* o_resid, const void* dout, const float* lse, float* dq,
+                             float* dk, float* dv, void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fa_bwd_noalloc -- the backward pass of fa_bwd for callers that cannot allocate
  * device memory.  (The pages describe no such entry point; it is a service of this
  * library.)  Some callers have no way to obtain a workspace at the moment they run

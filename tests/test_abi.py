@@ -101,6 +101,24 @@ def test_forward_workspace(lib):
     assert lib.fa_fwd_ws(None, None, None, None, None, None, 1, 4, 2, 0, 64, 0.125, 0, None, 0, None) == api.FA_OK
 
 
+def test_descriptor_entry_points_check_their_arguments(lib):
+    import ctypes
+
+    pr = api.FaAttnProblem(1, 4, 2, 300, 64, 0.125, 1, 16, -1)
+    assert api.fa_attn_fwd_workspace_size(pr) == api.fa_fwd_workspace_size(1, 2, 300, 64)
+    assert api.fa_attn_bwd_workspace_size(pr) == api.fa_bwd_gqa_workspace_size(1, 4, 2, 300, 64)
+    assert lib.fa_attn_fwd_workspace_size(None) == 0 and lib.fa_attn_bwd_workspace_size(None) == 0
+    bad = api.FaAttnProblem(1, 4, 2, 300, 64, 0.125, 1, -2, -1)
+    assert api.fa_attn_fwd_workspace_size(bad) == 0
+    fwd = lambda p, ws=A: lib.fa_attn_fwd(ctypes.byref(p), A, A, A, A, A, None, ws, 1 << 40, None)  # noqa: E731
+    bwd = lambda p: lib.fa_attn_bwd(ctypes.byref(p), A, A, A, A, A, A, A, A, A, A, A, 1 << 40, None)  # noqa: E731
+    assert fwd(bad) == api.FA_ERR_INVALID_ARG
+    assert bwd(bad) == api.FA_ERR_INVALID_ARG
+    assert fwd(pr, ws=None) == api.FA_ERR_INVALID_ARG  # the forward needs its workspace
+    assert lib.fa_attn_fwd(None, A, A, A, A, A, None, A, 1 << 40, None) == api.FA_ERR_INVALID_ARG
+    assert fwd(api.FaAttnProblem(1, 6, 4, 300, 64, 0.125, 1, -1, -1)) == api.FA_ERR_INVALID_ARG
+
+
 def test_workspace_size_of_empty_or_bad_problem_is_zero(lib):
     assert api.fa_bwd_workspace_size(0, 1, 10, 64) == 0
     assert api.fa_bwd_workspace_size(1, 1, 0, 64) == 0

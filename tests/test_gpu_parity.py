@@ -128,6 +128,38 @@ def test_forward_with_workspace_matches_on_chip_conversion(B, H, Hkv, N, d, caus
     assert_fwd(o2, l2, O, L, f"fa_fwd_ws B={B} H={H} Hkv={Hkv} N={N} d={d} causal={causal}")
 
 
+WINDOWS = [(True, (0, -1)), (True, (127, -1)), (True, (128, -1)), (True, (300, -1)), (True, (5, 7)),
+           (False, (64, 64)), (False, (0, 0)), (False, (-1, 200)), (False, (333, -1))]
+
+
+@pytest.mark.parametrize("causal,window", WINDOWS)
+@pytest.mark.parametrize("N,d,H,Hkv", [(1000, 128, 2, 2), (577, 64, 4, 2)])
+def test_sliding_window_fwd_bwd(causal, window, N, d, H, Hkv):
+    inp = inputs.make_qkv(1, H, N, d, seed=N + window[0] + 3 * window[1] + causal, kv_heads=Hkv, device="cuda")
+    q, k, v, do = (inp[n] for n in ("q", "k", "v", "do"))
+    scale = 1.0 / np.sqrt(d)
+    o, lse, res = api.fa_attn_fwd(q, k, v, causal=causal, scale=scale, window=window, save_residual=True)
+    grads = api.fa_attn_bwd(q, k, v, o, do, lse, causal=causal, scale=scale, window=window, o_resid=res)
+    torch.cuda.synchronize()
+    tag = f"window={window} causal={causal} N={N} d={d} H={H} Hkv={Hkv}"
+    O, L = oracle.attention_forward_gqa(q, k, v, scale, causal, window=window)
+    assert_fwd(o, lse, O, L, tag)
+    assert_grads(grads, oracle.attention_backward_gqa(q, k, v, do, scale, causal, window=window), tag)
+
+
+def test_unbounded_window_is_the_plain_path():
+    inp = inputs.make_qkv(1, 2, 700, 128, seed=9, device="cuda")
+    q, k, v, do = (inp[n] for n in ("q", "k", "v", "do"))
+    o1, l1, r1 = api.fa_attn_fwd(q, k, v, causal=True, window=(-1, -1), save_residual=True)
+    o2, l2, r2 = api.fa_fwd_ws(q, k, v, causal=True, save_residual=True)
+    g1 = api.fa_attn_bwd(q, k, v, o1, do, l1, causal=True, window=(-1, -1), o_resid=r1)
+    g2 = api.fa_bwd(q, k, v, o2, do, l2, causal=True, o_resid=r2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
+
+
 def test_gqa_long_spiky_matches_oracle_rows():
     # a long grouped problem with peaked softmax rows: all of dK/dV of one key/value head
     # against the oracle, which materialises N x N per query head
