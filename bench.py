@@ -239,6 +239,21 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     if Hkv < 1 or H % Hkv:
         raise SystemExit(f"--kv-heads must divide H = {H}")
     name = w.name if Hkv == H else f"{w.name}_gqa_h{H}_hkv{Hkv}"
+    window = (-1, -1) if args.window is None else (args.window, -1)
+    if args.window is not None:
+        name += f"_window{args.window}"
+    # metric flops: 4 d per visible (query, key) pair and head forward, 2.5x that backward
+    # (w.fwd_flops is the same count for the plain causal / full masks)
+    if args.window is None:
+        fwd_flops = w.fwd_flops
+    else:
+        pairs = 0
+        for i in range(N):
+            lo = max(0, i - args.window)
+            hi = i if w.causal else N - 1
+            pairs += hi - lo + 1
+        fwd_flops = 4.0 * B * H * d * pairs
+    bwd_flops = 2.5 * fwd_flops
     inp_cpu = inputs.make_qkv(B, H, N, d, dtype=w.dtype, dist=w.dist, spiky_frac=w.spiky_frac, backward=True,
                               seed=w.seed, kv_heads=None if Hkv == H else Hkv)
     q, k, v, do = (inp_cpu[n].to(dev) for n in ("q", "k", "v", "do"))
@@ -252,10 +267,17 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     stream = torch.cuda.current_stream()
     # forward with a workspace: V converted to fp16 in one streaming pass, then the kernel
     fws = torch.empty(api.fa_fwd_workspace_size(B, Hkv, N, d), dtype=torch.uint8, device=dev)
-    bwd_call = api.fa_bwd if Hkv == H else api.fa_bwd_gqa
+    if args.window is None:
+        bwd_call = api.fa_bwd if Hkv == H else api.fa_bwd_gqa
 
-    def fwd_call(q, k, v, **kw):
-        return api.fa_fwd_ws(q, k, v, workspace=fws, **kw)
+        def fwd_call(q, k, v, **kw):
+            return api.fa_fwd_ws(q, k, v, workspace=fws, **kw)
+    else:  # sliding window: the descriptor-based entry points
+        def fwd_call(q, k, v, **kw):
+            return api.fa_attn_fwd(q, k, v, window=window, workspace=fws, **kw)
+
+        def bwd_call(*a, **kw):
+            return api.fa_attn_bwd(*a, window=window, **kw)
 
     def step():
         fwd_call(q, k, v, causal=w.causal, scale=w.scale, o=o, lse=lse, o_resid=res)
@@ -304,15 +326,15 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         phase["bwd_dq"].append(e[3].elapsed_time(e[4]))
     mean = {kk: statistics.mean(vv) for kk, vv in phase.items()}
 
-    flops_step = w.fwd_flops + w.bwd_flops
+    flops_step = fwd_flops + bwd_flops
     ms_step = total_ms_max / args.steps
     value = flops_step * world / (ms_step * 1e-3) / 1e12
     peaks = load_peaks()
 
     # dominant kernel (largest mean time) and its algorithmic flops per launch
-    algo = {"fwd": w.fwd_flops,                  # QK^T and PV
-            "bwd_dkdv": 2.0 * w.fwd_flops,        # K Q^T, V dO^T, P^T dO, dS^T Q
-            "bwd_dq": 1.5 * w.fwd_flops}          # Q K^T, dO V^T, dS K
+    algo = {"fwd": fwd_flops,                  # QK^T and PV
+            "bwd_dkdv": 2.0 * fwd_flops,        # K Q^T, V dO^T, P^T dO, dS^T Q
+            "bwd_dq": 1.5 * fwd_flops}          # Q K^T, dO V^T, dS K
     dom = max(("fwd", "bwd_dkdv", "bwd_dq"), key=lambda kk: mean[kk])
     achieved = algo[dom] / (mean[dom] * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
@@ -358,8 +380,8 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, inp_cpu)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.window is None:
+        cpu = cpu_baseline(w, inp_cpu)  # (the oracle timing covers the unwindowed problem)
 
     if rank == 0:
         line = {
@@ -367,11 +389,12 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": name, "B": B, "H": H, "H_kv": Hkv, "N": N, "d": d, "causal": w.causal,
+                       "window": list(window),
                        "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
                        "l2": ("inputs larger than L2 (Q, K, V, dO, O 134 MB each > 126 MB)" if w.N * w.B * w.H >= 2 ** 19
                    else "small workload: inputs may stay in L2")},
-            "fwd_tflops": w.fwd_flops / (mean["fwd"] * 1e-3) / 1e12,
-            "bwd_tflops": w.bwd_flops / ((mean["bwd_pre"] + mean["bwd_dkdv"] + mean["bwd_dq"]) * 1e-3) / 1e12,
+            "fwd_tflops": fwd_flops / (mean["fwd"] * 1e-3) / 1e12,
+            "bwd_tflops": bwd_flops / ((mean["bwd_pre"] + mean["bwd_dkdv"] + mean["bwd_dq"]) * 1e-3) / 1e12,
             "kernel_ms": mean,
             "frac_of_peak": {"measured_burst": value / world / peaks["bf16_tflops"],
                              "measured_sustained": value / world / peaks["bf16_tflops_sustained"],
@@ -397,6 +420,9 @@ def main() -> None:
                     help="workload index (3 = the metric's; others for profiling runs)")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped-query run: K/V with this many heads (fa_fwd_gqa / fa_bwd_gqa); default H")
+    ap.add_argument("--window", type=int, default=None,
+                    help="sliding-window run: each query sees the previous WINDOW keys and itself "
+                         "(fa_attn_fwd / fa_attn_bwd); default no window")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the dominant kernel from an ncu capture (reported as-is)")
     args = ap.parse_args()
