@@ -25,7 +25,8 @@ FA_ERR_TIMEOUT = 5
 
 EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_workspace_size", "fa_fwd_ws", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_gqa_workspace_size",
            "fa_bwd_gqa", "fa_attn_fwd_workspace_size", "fa_attn_fwd", "fa_attn_bwd_workspace_size", "fa_attn_bwd",
-           "fa_bwd_noalloc", "fa_device_status", "fa_bwd_set_phase_events", "fa_status_str")
+           "fa_bwd_noalloc", "fa_device_status", "fa_bwd_set_phase_events", "fa_selftest_wait_timeout",
+           "fa_status_str")
 
 # Size of the scratch array fa_bwd_noalloc uses instead of a caller workspace.
 FA_BWD_NOALLOC_MAX_WORKSPACE = 64 << 20
@@ -89,6 +90,8 @@ def library() -> ctypes.CDLL:
     lib.fa_attn_bwd.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_bwd_noalloc.restype = i
+    lib.fa_selftest_wait_timeout.argtypes = [vp]
+    lib.fa_selftest_wait_timeout.restype = i
     lib.fa_device_status.argtypes = [vp]
     lib.fa_device_status.restype = i
     lib.fa_bwd_set_phase_events.argtypes = [vp]
@@ -389,6 +392,12 @@ def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal: bool = False, scale:
                                   int(bool(causal)), _stream_handle(stream))
     _check("fa_bwd_noalloc", st)
     return dq, dk, dv
+
+
+def fa_selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the bounded-wait self-test (a wait that must give up after ~2 s and report
+    FA_ERR_TIMEOUT through ``fa_device_status``)."""
+    _check("fa_selftest_wait_timeout", library().fa_selftest_wait_timeout(_stream_handle(stream)))
 
 
 def fa_device_status(stream=None) -> int:

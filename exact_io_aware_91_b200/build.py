@@ -22,7 +22,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_NAME = "libfa_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
 
-SOURCES = ["fa_api.cu", "fwd_sm100.cu", "fwd_f32.cu", "bwd_pre.cu", "bwd_sm100.cu", "fa_bwd_noalloc.cu"]
+SOURCES = ["fa_api.cu", "fwd_sm100.cu", "fwd_f32.cu", "bwd_pre.cu", "bwd_sm100.cu", "fa_bwd_noalloc.cu", "selftest.cu"]
 HEADERS = ["sm100.cuh", "fa_internal.h"]
 
 NVCC_FLAGS = [

@@ -432,6 +432,14 @@ fa_status fa_attn_bwd(const fa_attn_problem* pr, const void* q, const void* k, c
 
 void fa_bwd_set_phase_events(void* const* events) { t_phase_events = events; }
 
+fa_status fa_selftest_wait_timeout(fa_stream_t stream) {
+  int dev = 0;
+  const fa_status st = device_setup(&dev);
+  if (st != FA_OK) return st;
+  return launch_selftest_wait(g_err_ptr[dev], reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK
+                                                                                                      : FA_ERR_CUDA;
+}
+
 fa_status fa_device_status(fa_stream_t stream) {
   int dev = 0;
   fa_status st = device_setup(&dev);

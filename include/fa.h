@@ -269,6 +269,16 @@ FA_API fa_status fa_device_status(fa_stream_t stream);
  */
 FA_API void fa_bwd_set_phase_events(void* const* events);
 
+/*
+ * fa_selftest_wait_timeout -- self-test of the failure path: enqueues a one-CTA kernel in
+ * which one thread waits, through the library's bounded-wait helper, on a barrier that
+ * nothing ever completes.  The wait gives up after its wall-time limit (2 s) and records a
+ * timeout, so a following fa_device_status(stream) returns FA_ERR_TIMEOUT (and clears it);
+ * the CUDA context stays usable.  Nothing faults, traps or hangs.  Returns FA_OK once
+ * enqueued.
+ */
+FA_API fa_status fa_selftest_wait_timeout(fa_stream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FA_API const char* fa_status_str(fa_status status);
 
