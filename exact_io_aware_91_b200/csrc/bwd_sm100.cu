@@ -25,6 +25,8 @@
 //     dQ(j) += dS(j) K_j, dP(j+1), S(j+2).
 // All products run in fp16 (exact copies of the bf16 inputs made by the
 // preprocess) with fp32 accumulation; gradients are written in fp32.
+#include <type_traits>
+
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -401,58 +403,69 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int key = j * 128 + row;
       const int q_vis_lo = query_lo(key, p.causal, p.win_right);
       const int q_vis_hi = query_hi(key, p.N, p.win_left);
+      // queries that every key of the tile sees: both bounds grow with the key
+      const int all_lo = query_lo(min(j * 128 + 127, p.N - 1), p.causal, p.win_right);
+      const int all_hi = query_hi(j * 128, p.N, p.win_left);
       for (int it = 0; it < n_it; ++it) {
         const int T = T0 + it;
         const int i = i_start + it % n_q;  // query tile of this step
         const float* lse2 = reinterpret_cast<const float*>(gbase + L::OFF_LD + (T & 1) * 1024) + 64 * w;
         const float* delta = lse2 + 128;
         const int q0 = i * 128 + 64 * w;  // first query of this warpgroup's columns
-        // this key's visible queries (causal mask, sliding window); padded queries have P = 0
-        const bool need_mask = q0 < q_vis_lo || q0 + 63 > q_vis_hi;
         // ---- P^T = 2^(S^T * scale * log2(e) - lse2), written back over S^T as fp16
         if (!(ok = mbar_wait(bar(L::BAR_S), T & 1, wctx))) break;
         tc_fence_after();
         float pr[64];
         tmem_ld64(tS, pr);
+        // the same for every thread of the CTA: tiles inside every key's visible query range
+        // take the loop without compares; the others mask column c unless c_lo <= c <= c_hi
+        // (this key's visible queries; padded queries have P = 0)
+        auto probs = [&](auto masked) {
+          const int c_lo = q_vis_lo - q0, c_hi = q_vis_hi - q0;
 #pragma unroll
-        for (int g = 0; g < 64; g += 16) {
-          uint32_t pk[8];
+          for (int g = 0; g < 64; g += 16) {
+            uint32_t pk[8];
 #pragma unroll
-          for (int c = g; c < g + 16; c += 4) {
-            const float4 L4 = *reinterpret_cast<const float4*>(lse2 + c);
-            float t0, t1, t2, t3;
-            f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, f2pack(-L4.x, -L4.y)), t0, t1);
-            f2unpack(ffma2(f2pack(pr[c + 2], pr[c + 3]), sl2x2, f2pack(-L4.z, -L4.w)), t2, t3);
-            if ((c - g) < kDkdvExpFmaPer16) {
-              // both warpgroups run this phase at once, so the MUFU unit is the limit: part of
-              // the exponentials go to the FMA pipe
-              exp2_fma_pipe(t0, t1);
-              exp2_fma_pipe(t2, t3);
-              pr[c] = t0;
-              pr[c + 1] = t1;
-              pr[c + 2] = t2;
-              pr[c + 3] = t3;
-            } else {
-              pr[c] = ex2_approx(t0);
-              pr[c + 1] = ex2_approx(t1);
-              pr[c + 2] = ex2_approx(t2);
-              pr[c + 3] = ex2_approx(t3);
+            for (int c = g; c < g + 16; c += 4) {
+              const float4 L4 = *reinterpret_cast<const float4*>(lse2 + c);
+              float t0, t1, t2, t3;
+              f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, f2pack(-L4.x, -L4.y)), t0, t1);
+              f2unpack(ffma2(f2pack(pr[c + 2], pr[c + 3]), sl2x2, f2pack(-L4.z, -L4.w)), t2, t3);
+              if ((c - g) < kDkdvExpFmaPer16) {
+                // both warpgroups run this phase at once, so the MUFU unit is the limit: part of
+                // the exponentials go to the FMA pipe
+                exp2_fma_pipe(t0, t1);
+                exp2_fma_pipe(t2, t3);
+                pr[c] = t0;
+                pr[c + 1] = t1;
+                pr[c + 2] = t2;
+                pr[c + 3] = t3;
+              } else {
+                pr[c] = ex2_approx(t0);
+                pr[c + 1] = ex2_approx(t1);
+                pr[c + 2] = ex2_approx(t2);
+                pr[c + 3] = ex2_approx(t3);
+              }
+              if constexpr (decltype(masked)::value) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (c + e < c_lo || c + e > c_hi) pr[c + e] = 0.f;
+              }
+              pk[(c - g) / 2] = pack_f16(pr[c], pr[c + 1]);
+              pk[(c - g) / 2 + 1] = pack_f16(pr[c + 2], pr[c + 3]);
             }
-            if (need_mask) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (q0 + c + e < q_vis_lo || q0 + c + e > q_vis_hi) pr[c + e] = 0.f;
+            tmem_st8(tS + g / 2, pk);
+            if (g == 16) {  // columns 0..31 of this warpgroup done: the first half of dV may start
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(bar(L::BAR_P_HALF));
             }
-            pk[(c - g) / 2] = pack_f16(pr[c], pr[c + 1]);
-            pk[(c - g) / 2 + 1] = pack_f16(pr[c + 2], pr[c + 3]);
           }
-          tmem_st8(tS + g / 2, pk);
-          if (g == 16) {  // columns 0..31 of this warpgroup done: the first half of dV may start
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(L::BAR_P_HALF));
-          }
-        }
+        };
+        if (q0 < all_lo || q0 + 63 > all_hi)
+          probs(std::true_type{});
+        else
+          probs(std::false_type{});
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(L::BAR_P_READY));
@@ -779,28 +792,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = x.qt * 128 + row;  // query index
       const int k_vis_lo = key_lo(r, p.N, p.win_left);  // visible keys of this row
       const int k_vis_hi = key_hi(r, p.N, p.causal, p.win_right);
+      // keys that every row of the tile sees: both bounds grow with the row
+      const int all_lo = key_lo(min(x.qt * 128 + 127, p.N - 1), p.N, p.win_left);
+      const int all_hi = key_hi(x.qt * 128, p.N, p.causal, p.win_right);
       const uint64_t nl2 = f2pack(-lse2, -lse2), dd = f2pack(delta, delta);
       for (int it = 0; it < x.n_it; ++it) {
         const int t = T0 + it;
         const int b = t & 1;
         const uint32_t tS = tmem + lane_off + L::T_S + 128 * b + 64 * w;
         const int k0 = (x.jlo + it) * 128 + 64 * w;  // first key of this warpgroup's columns
-        const bool need_mask = k0 < k_vis_lo || k0 + 63 > k_vis_hi;
         if (!(ok = mbar_wait(bar(L::BAR_S + b), (t >> 1) & 1, wctx))) break;
         tc_fence_after();
         float pr[64];
         tmem_ld64(tS, pr);
+        // the same for every thread of the CTA: tiles inside every row's visible range take
+        // the loop without compares; the others mask column c unless c_lo <= c <= c_hi
+        auto probs = [&](auto masked) {
+          const int c_lo = k_vis_lo - k0, c_hi = k_vis_hi - k0;
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float t0, t1;
-          f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, nl2), t0, t1);
-          pr[c] = ex2_approx(t0);
-          pr[c + 1] = ex2_approx(t1);
-          if (need_mask) {
-            if (k0 + c < k_vis_lo || k0 + c > k_vis_hi) pr[c] = 0.f;
-            if (k0 + c + 1 < k_vis_lo || k0 + c + 1 > k_vis_hi) pr[c + 1] = 0.f;
+          for (int c = 0; c < 64; c += 2) {
+            float t0, t1;
+            f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, nl2), t0, t1);
+            pr[c] = ex2_approx(t0);
+            pr[c + 1] = ex2_approx(t1);
+            if constexpr (decltype(masked)::value) {
+              if (c < c_lo || c > c_hi) pr[c] = 0.f;
+              if (c + 1 < c_lo || c + 1 > c_hi) pr[c + 1] = 0.f;
+            }
           }
-        }
+        };
+        if (k0 < all_lo || k0 + 63 > all_hi)
+          probs(std::true_type{});
+        else
+          probs(std::false_type{});
         if (!(ok = mbar_wait(bar(L::BAR_DP), t & 1, wctx))) break;
         tc_fence_after();
         float dp[64];

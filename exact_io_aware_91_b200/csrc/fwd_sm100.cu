@@ -72,8 +72,11 @@ constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 2-3 V to fp16, w
 constexpr uint32_t kRegsLaunch = 168, kRegsLow = 64, kRegsHigh = 216;
 static_assert(kRegsLow + 2 * kRegsHigh <= 3 * kRegsLaunch, "register split exceeds the launch budget");
 constexpr int kConvThreads = 64;
+// A quarter of the softmax exponentials run on the FMA pipe (degree-3 polynomial, see
+// exp2_fma_pipe): measured on B200 with the fp16-V forward, 2 of 8 gives -6 % at N = 8192
+// (4 of 8 is slower again: the single softmax warp per sub-partition becomes issue-bound).
 #ifndef FA_EXP_FMA_PER8
-#define FA_EXP_FMA_PER8 0
+#define FA_EXP_FMA_PER8 2
 #endif
 // element pairs out of every 8 whose exponentials run on the FMA pipe (even, 0..8)
 constexpr int kExpFmaPer8 = FA_EXP_FMA_PER8;
@@ -102,7 +105,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 template <int D>
 __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS, uint32_t tO, uint32_t bar_s_full,
                                                  uint32_t s_parity, uint32_t bar_p_half, uint32_t bar_p_full, int j,
-                                                 bool first, int r, float& m, float& l, const WaitCtx& wctx) {
+                                                 bool first, int q_base, int r, float& m, float& l,
+                                                 const WaitCtx& wctx) {
   const float sl2 = p.scale_log2;
   if (!mbar_wait(bar_s_full, s_parity, wctx)) return false;
   tc_fence_after();
@@ -118,10 +122,14 @@ __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS
       for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(u[c][i]);
   }
   // keys kb .. kb + 127 against this row's visible range (causal mask, sliding window, N);
-  // with a window a row can have no visible key in a tile of its warpgroup's range
+  // with a window a row can have no visible key in a tile of its warpgroup's range.  The
+  // test is on the range every row of the tile sees (both bounds grow with the row), the
+  // same for the whole warpgroup, so tiles inside it skip the per-element compares.
   const int kb = j * 128;
-  const int lo = key_lo(r, p.N, p.win_left), hi = key_hi(r, p.N, p.causal, p.win_right);
-  if (kb < lo || kb + 127 > hi) {
+  const int all_lo = key_lo(min(q_base + 127, p.N - 1), p.N, p.win_left);
+  const int all_hi = key_hi(q_base, p.N, p.causal, p.win_right);
+  if (kb < all_lo || kb + 127 > all_hi) {
+    const int lo = key_lo(r, p.N, p.win_left), hi = key_hi(r, p.N, p.causal, p.win_right);
 #pragma unroll
     for (int c = 0; c < 128; ++c)
       if (kb + c < lo || kb + c > hi) x[c] = -INFINITY;
@@ -413,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < n_t; ++j) {
       if (!(ok = fwd_softmax_step<D>(p, tS, tO, bar(L::BAR_S_FULL + t), j & 1, bar(L::BAR_P_HALF + t),
-                                     bar(L::BAR_P_FULL + t), j, j == 0, r, m, l, wctx)))
+                                     bar(L::BAR_P_FULL + t), j, j == 0, q_base, r, m, l, wctx)))
         break;
     }
     // ---- epilogue: O / l -> bf16 -> swizzled staging (the Q tile's buffer) -> TMA store
@@ -763,7 +771,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY, l = 0.f;
       for (int jj = 0; jj < n_t; ++jj) {
         if (!(ok = fwd_softmax_step<D>(p, tS, tO, bar(L::BAR_S_FULL + t), (G + jj) & 1, bar(L::BAR_P_HALF + t),
-                                       bar(L::BAR_P_FULL + t), jlo + jj, jj == 0, r, m, l, wctx)))
+                                       bar(L::BAR_P_FULL + t), jlo + jj, jj == 0, q_base, r, m,
+                                       l, wctx)))
           break;
       }
       G += n_t;
