@@ -43,3 +43,5 @@ def test_bounded_wait_reports_timeout_and_the_context_stays_usable():
     assert api.fa_device_status() == api.FA_OK
     O, _ = oracle.attention_forward(q, k, v, 1 / np.sqrt(64), True)
     assert np.abs(o.float().cpu().numpy() - O).max() < 2e-2
+    for got, ref in zip((dq, dk, dv), oracle.attention_backward(q, k, v, do, 1 / np.sqrt(64), True)):
+        assert np.abs(got.cpu().numpy() - ref).max() < 5e-2
