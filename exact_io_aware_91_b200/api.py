@@ -25,7 +25,7 @@ FA_ERR_TIMEOUT = 5
 
 EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_workspace_size", "fa_fwd_ws", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_gqa_workspace_size",
            "fa_bwd_gqa", "fa_attn_fwd_workspace_size", "fa_attn_fwd", "fa_attn_bwd_workspace_size", "fa_attn_bwd",
-           "fa_bwd_noalloc", "fa_device_status", "fa_bwd_set_phase_events", "fa_selftest_wait_timeout",
+           "fa_attn_fwd_fp8_workspace_size", "fa_attn_fwd_fp8", "fa_bwd_noalloc", "fa_device_status", "fa_bwd_set_phase_events", "fa_selftest_wait_timeout",
            "fa_status_str")
 
 # Size of the scratch array fa_bwd_noalloc uses instead of a caller workspace.
@@ -88,6 +88,10 @@ def library() -> ctypes.CDLL:
     lib.fa_attn_bwd_workspace_size.restype = sz
     lib.fa_attn_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.fa_attn_bwd.restype = i
+    lib.fa_attn_fwd_fp8_workspace_size.argtypes = [pp]
+    lib.fa_attn_fwd_fp8_workspace_size.restype = sz
+    lib.fa_attn_fwd_fp8.argtypes = [pp, vp, vp, vp, f, f, f, vp, vp, vp, sz, vp]
+    lib.fa_attn_fwd_fp8.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_bwd_noalloc.restype = i
     lib.fa_selftest_wait_timeout.argtypes = [vp]
@@ -344,6 +348,34 @@ def fa_attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, windo
                                workspace.numel(), _stream_handle(stream))
     _check("fa_attn_fwd", st)
     return (o, lse) if o_resid is None else (o, lse, o_resid)
+
+
+def fa_attn_fwd_fp8_workspace_size(problem: FaAttnProblem) -> int:
+    return int(library().fa_attn_fwd_fp8_workspace_size(ctypes.byref(problem)))
+
+
+def fa_attn_fwd_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float, causal: bool = False,
+                    scale: float | None = None, window=(-1, -1), o=None, lse=None, workspace=None, stream=None):
+    """8-bit forward: q (B, H, N, d), k and v (B, H_kv, N, d) ``torch.float8_e4m3fn`` CUDA
+    tensors holding Q / q_descale etc. (per-tensor descales, d = 128).  Computes the
+    attention of the dequantized inputs; returns (o bf16, lse fp32)."""
+    pr = _problem(q, k, causal, scale, window)
+    B, H, N, d = _shape(q)
+    _same(q, dtype=torch.float8_e4m3fn, shape=(B, H, N, d))
+    _same(k, v, dtype=torch.float8_e4m3fn, shape=(B, pr.H_kv, N, d))
+    if o is None:
+        o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _same(o, dtype=torch.bfloat16, shape=(B, H, N, d))
+    _same(lse, dtype=torch.float32, shape=(B, H, N))
+    if workspace is None:
+        workspace = torch.empty(max(fa_attn_fwd_fp8_workspace_size(pr), 1), dtype=torch.uint8, device=q.device)
+    st = library().fa_attn_fwd_fp8(ctypes.byref(pr), q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_descale),
+                                   float(k_descale), float(v_descale), o.data_ptr(), lse.data_ptr(),
+                                   workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    _check("fa_attn_fwd_fp8", st)
+    return o, lse
 
 
 def fa_attn_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, window=(-1, -1),

@@ -226,6 +226,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   // K and V bytes per query head: a group of H / H_kv query heads shares them
   p.head_group = head_group_size(BH, 4ull * N * d / (H / H_kv), kFwdGroupBytes);
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.out_scale = 1.0f;
   p.causal = causal;
   p.win_left = wl;
   p.win_right = wr;
@@ -428,6 +429,62 @@ fa_status fa_attn_bwd(const fa_attn_problem* pr, const void* q, const void* k, c
   if (pr == nullptr) return FA_ERR_INVALID_ARG;
   return bwd_impl(q, k, v, o, o_resid, dout, lse, dq, dk, dv, pr->B, pr->H, pr->H_kv, pr->N, pr->d, pr->scale,
                   pr->causal, pr->window_left, pr->window_right, workspace, workspace_bytes, stream);
+}
+
+// ---- 8-bit forward: E4M3 inputs with per-tensor descales (d = 128)
+size_t fa_attn_fwd_fp8_workspace_size(const fa_attn_problem* pr) {
+  if (pr == nullptr || !window_ok(pr->window_left, pr->window_right)) return 0;
+  return 256;  // the persistent kernel's work counter
+}
+
+fa_status fa_attn_fwd_fp8(const fa_attn_problem* pr, const void* q, const void* k, const void* v, float q_descale,
+                          float k_descale, float v_descale, void* o, float* lse, void* workspace,
+                          size_t workspace_bytes, fa_stream_t stream) {
+  if (pr == nullptr || !window_ok(pr->window_left, pr->window_right)) return FA_ERR_INVALID_ARG;
+  const int B = pr->B, H = pr->H, H_kv = pr->H_kv, N = pr->N, d = pr->d;
+  bool empty = false;
+  fa_status st = check_problem(B, H, H_kv, N, d, pr->scale, pr->causal, &empty);
+  if (st != FA_OK) return st;
+  for (const float ds : {q_descale, k_descale, v_descale})
+    if (!(std::isfinite(ds) && ds > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;  // one 128-byte swizzle row per Q / K / V row
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !workspace || workspace_bytes < 256) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(workspace, 256))
+    return FA_ERR_MISALIGNED;
+  int dev = 0;
+  if ((st = device_setup(&dev)) != FA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H, BH_kv = B * H_kv;
+  unsigned* counter = static_cast<unsigned*>(workspace);
+  if (cudaMemsetAsync(counter, 0, sizeof(unsigned), s) != cudaSuccess) return FA_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if (!make_tmap_3d(&tq, q, u8, 1, d, N, BH, 128, 128, true) ||
+      !make_tmap_3d(&tk, k, u8, 1, d, N, BH_kv, 128, 128, true) ||
+      !make_tmap_3d(&tv, v, u8, 1, d, N, BH_kv, 128, 128, true))
+    return FA_ERR_CUDA;
+  FwdParams p{};
+  p.lse = lse;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_resid = nullptr;
+  p.counter = counter;
+  p.num_sms = g_num_sms[dev];
+  p.N = N;
+  p.BH = BH;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.n_pairs = (N + 255) / 256;
+  p.head_group = head_group_size(BH, 2ull * N * d / (H / H_kv), kFwdGroupBytes);  // 8-bit K and V
+  // S = q_descale * k_descale * (Q8 K8^T): both descales fold into the exponent's scale
+  p.scale_log2 = (float)((double)pr->scale * q_descale * k_descale * 1.4426950408889634);
+  p.out_scale = v_descale;
+  p.causal = pr->causal;
+  p.win_left = pr->window_left;
+  p.win_right = pr->window_right;
+  p.err = g_err_ptr[dev];
+  return launch_fwd_persist_fp8_sm100(tq, tk, tv, p, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 void fa_bwd_set_phase_events(void* const* events) { t_phase_events = events; }

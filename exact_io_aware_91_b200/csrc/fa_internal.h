@@ -19,7 +19,8 @@ struct FwdParams {
   int H, H_kv;       // query heads and key/value heads per batch entry (H a multiple of H_kv)
   int n_pairs;       // ceil(N / 256): work units per head (two 128-row query tiles each)
   int head_group;    // heads per group in the CTA order (unit_order)
-  float scale_log2;  // softmax scale * log2(e)
+  float scale_log2;  // softmax scale * log2(e) (times the Q and K descales for 8-bit inputs)
+  float out_scale;   // factor on O / l: 1, or the V descale for 8-bit inputs
   int causal;
   int win_left, win_right;  // sliding window: query i sees keys i - left .. i + right (-1 unbounded)
   int* err;          // device error word
@@ -111,6 +112,8 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
 cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, cudaStream_t s);
 cudaError_t launch_fwd_persist_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                      const FwdParams& p, int d, cudaStream_t s);
+cudaError_t launch_fwd_persist_fp8_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                         const FwdParams& p, cudaStream_t s);  // d = 128, E4M3 inputs
 cudaError_t launch_selftest_wait(int* err, cudaStream_t s);
 cudaError_t launch_bwd_kv_reduce(const float* dk_part, const float* dv_part, float* dk, float* dv,
                                  long long elems, int splits, cudaStream_t s);

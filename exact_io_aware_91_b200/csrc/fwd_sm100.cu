@@ -101,8 +101,10 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // running maximum (kept while within 2^8 of the true one), O rescaled in TMEM when the
 // maximum moves, P = 2^(scale*log2(e)*S - m) written back over S as fp16 in two halves
 // (the tensor core starts on the first half's P V while the second half is computed).
+// With F8, P is written as E4M3 (four per TMEM column, 16 columns per half) for the 8-bit
+// P V product; the row sum uses the fp32 values before rounding.
 // Returns false if a bounded wait gave up.
-template <int D>
+template <int D, bool F8 = false>
 __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS, uint32_t tO, uint32_t bar_s_full,
                                                  uint32_t s_parity, uint32_t bar_p_half, uint32_t bar_p_full, int j,
                                                  bool first, int q_base, int r, float& m, float& l,
@@ -178,20 +180,25 @@ __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS
       if ((i & 7) < 2 * (kExpFmaPer8 / 2)) {
         exp2_fma_pipe(e[0], e[1]);
         exp2_fma_pipe(e[2], e[3]);
-        pk[i] = pack_f16(e[0], e[1]);
-        pk[i + 1] = pack_f16(e[2], e[3]);
       } else {
         e[0] = ex2_approx(e[0]);
         e[1] = ex2_approx(e[1]);
         e[2] = ex2_approx(e[2]);
         e[3] = ex2_approx(e[3]);
+      }
+      if constexpr (F8) {
+        pk[i / 2] = pack_e4m3x4(e[0], e[1], e[2], e[3]);
+      } else {
         pk[i] = pack_f16(e[0], e[1]);
         pk[i + 1] = pack_f16(e[2], e[3]);
       }
       asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sa) : "l"(f2pack(e[0], e[1])));
       asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sb) : "l"(f2pack(e[2], e[3])));
     }
-    tmem_st32(tS + 32 * h, pk);
+    if constexpr (F8)
+      tmem_st16(tS + 16 * h, pk);
+    else
+      tmem_st32(tS + 32 * h, pk);
     // first half of P (and any rescale of O) visible to the tensor core: its half of P V
     // can start while the second half is computed
     tmem_wait_st();
@@ -495,12 +502,23 @@ namespace {
 // O_FULL, O_FREE) count units.  O and the residual are stored straight from registers
 // (coalesced by warp_store_rows_128b): the Q buffers are reloaded for the next unit and
 // cannot serve as the output staging tile.
-template <int D>
+//
+// F8 (8-bit inputs, d = 128): Q, K and V are E4M3, so a row of d elements is one 128-byte
+// swizzle row and every tile is 16 KB; S = Q K^T and O += P V run as kind::f8f6f4 products
+// (K = 32 per instruction), V read MN-major straight from its (N, d) layout, P written to TMEM
+// as E4M3; the per-tensor descales enter through scale_log2 (Q, K) and out_scale (V).
+template <int D, bool F8 = false>
 struct FwdPLayout {
-  static constexpr int KCH = D / 64;
+  static constexpr int ROW_BYTES = F8 ? D : 2 * D;  // bytes of one row of Q, K or V
+  static constexpr int CH_ELEMS = F8 ? 128 : 64;     // elements of one 128-byte column chunk
+  static constexpr int KCH = ROW_BYTES / 128;
   static constexpr int BOX = 128 * 128;
   static constexpr int TILE = KCH * BOX;
-  static constexpr int STAGES = (D == 128) ? 4 : 8;
+  static constexpr int STAGES = (TILE == 2 * BOX) ? 4 : 8;
+  static constexpr int K_STEP = F8 ? 32 : 16;          // K of one tensor-core instruction
+  static constexpr int QK_STEPS = ROW_BYTES / 32;      // instructions per Q K^T (32 bytes of K each)
+  static constexpr int PV_STEPS_HALF = 64 / K_STEP;    // instructions per half of P V (64 keys)
+  static constexpr int PV_B_STEP = K_STEP * 128;       // bytes between the V rows of consecutive steps
   static constexpr int OFF_Q0 = 0;
   static constexpr int OFF_Q1 = TILE;
   static constexpr int OFF_KV = 2 * TILE;
@@ -526,11 +544,11 @@ struct FwdPLayout {
   static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
 };
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_persist_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                                 const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = FwdPLayout<D>;
+  using L = FwdPLayout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -623,9 +641,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (uc > 0 && !(ok = mbar_wait(bar(L::BAR_Q_EMPTY), (uc - 1) & 1, wctx))) break;
       mbar_arrive_expect_tx(bar(L::BAR_Q_FULL), 2 * L::TILE, leader);
       for (int c = 0; c < L::KCH; ++c) {
-        tma_load_3d(base + L::OFF_Q0 + c * L::BOX, &tm_q, c * 64, x.q_base0, x.bh, bar(L::BAR_Q_FULL), leader);
-        tma_load_3d(base + L::OFF_Q1 + c * L::BOX, &tm_q, c * 64, x.q_base0 + 128, x.bh, bar(L::BAR_Q_FULL),
+        tma_load_3d(base + L::OFF_Q0 + c * L::BOX, &tm_q, c * L::CH_ELEMS, x.q_base0, x.bh, bar(L::BAR_Q_FULL),
                     leader);
+        tma_load_3d(base + L::OFF_Q1 + c * L::BOX, &tm_q, c * L::CH_ELEMS, x.q_base0 + 128, x.bh,
+                    bar(L::BAR_Q_FULL), leader);
       }
       ++q_issued;
       for (int j = x.jlo0; j <= x.jhi1 && ok; ++j) {
@@ -635,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar(L::BAR_KV_FULL + st), L::TILE, leader);
           const CUtensorMap* m = which ? &tm_v : &tm_k;
           for (int c = 0; c < L::KCH; ++c)
-            tma_load_3d(base + L::OFF_KV + st * L::TILE + c * L::BOX, m, c * 64, j * 128, x.bh_kv,
+            tma_load_3d(base + L::OFF_KV + st * L::TILE + c * L::BOX, m, c * L::CH_ELEMS, j * 128, x.bh_kv,
                         bar(L::BAR_KV_FULL + st), leader);
           ++issued;
         }
@@ -650,8 +669,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ===================================================== MMA issuer
     regs_dec<kRegsLow>();
     const uint32_t leader = elect_one();
-    constexpr uint32_t idesc_qk = make_idesc(128, 128, true, false, false);
-    constexpr uint32_t idesc_pv = make_idesc(128, D, false, false, true);  // fp16 P (TMEM) x fp16 V
+    // bf16 Q, K (format 1), or E4M3 (format 0 of kind::f8f6f4; 1 there would mean E5M2)
+    constexpr uint32_t idesc_qk = make_idesc(128, 128, !F8, false, false);
+    // fp16 P (TMEM) x fp16 V, or E4M3 x E4M3 (format code 0 in both kinds); V MN-major
+    constexpr uint32_t idesc_pv = make_idesc(128, D, false, false, true);
     const uint32_t tS[2] = {tmem + L::T_S0, tmem + L::T_S1};
     const uint32_t tO[2] = {tmem + L::T_O0, tmem + L::T_O1};
     const uint64_t dQ[2] = {make_sdesc_sw128(base + L::OFF_Q0, 16, 1024), make_sdesc_sw128(base + L::OFF_Q1, 16, 1024)};
@@ -660,17 +681,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_qk = [&](uint32_t d_tmem, uint64_t q_desc, int stage) {
       const uint64_t k_desc = sdesc_add(dKV0, stage * L::TILE);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
+      for (int k = 0; k < L::QK_STEPS; ++k) {
         const uint32_t off = (k >> 2) * L::BOX + (k & 3) * 32;
-        mma_ss(d_tmem, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, k > 0 ? 1u : 0u, leader);
+        if constexpr (F8)
+          mma_ss_f8(d_tmem, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, k > 0 ? 1u : 0u, leader);
+        else
+          mma_ss(d_tmem, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, k > 0 ? 1u : 0u, leader);
       }
     };
+    // P for keys [K_STEP k, K_STEP (k + 1)) sits in TMEM columns [8 k, 8 k + 8) in both forms
     auto issue_pv_half = [&](uint32_t d_tmem, uint32_t p_tmem, int stage, bool acc, int part) {
       const uint64_t v_desc = sdesc_add(dV0, stage * L::TILE);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const int k = part * 4 + kk;
-        mma_ts(d_tmem, p_tmem + k * 8, sdesc_add(v_desc, k * 2048), idesc_pv, (acc || k > 0) ? 1u : 0u, leader);
+      for (int kk = 0; kk < L::PV_STEPS_HALF; ++kk) {
+        const int k = part * L::PV_STEPS_HALF + kk;
+        if constexpr (F8)
+          mma_ts_f8(d_tmem, p_tmem + k * 8, sdesc_add(v_desc, k * L::PV_B_STEP), idesc_pv, (acc || k > 0) ? 1u : 0u,
+                    leader);
+        else
+          mma_ts(d_tmem, p_tmem + k * 8, sdesc_add(v_desc, k * L::PV_B_STEP), idesc_pv, (acc || k > 0) ? 1u : 0u,
+                 leader);
       }
     };
     int L0 = 0, G0 = 0, G1 = 0;  // K/V loads and tile steps of the previous units
@@ -770,7 +800,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_t = (t ? x.jhi1 : x.jhi0) - jlo + 1;
       float m = -INFINITY, l = 0.f;
       for (int jj = 0; jj < n_t; ++jj) {
-        if (!(ok = fwd_softmax_step<D>(p, tS, tO, bar(L::BAR_S_FULL + t), (G + jj) & 1, bar(L::BAR_P_HALF + t),
+        if (!(ok = fwd_softmax_step<D, F8>(p, tS, tO, bar(L::BAR_S_FULL + t), (G + jj) & 1, bar(L::BAR_P_HALF + t),
                                        bar(L::BAR_P_FULL + t), jlo + jj, jj == 0, q_base, r, m,
                                        l, wctx)))
           break;
@@ -780,7 +810,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue: O / l -> bf16 and the bf16 residual, stored from registers
       if (!(ok = mbar_wait(bar(L::BAR_O_FULL + t), uc & 1, wctx))) break;
       tc_fence_after();
-      const float inv_l = 1.0f / l;
+      const float inv_l = p.out_scale / l;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t u0[32], u1[32];
@@ -842,6 +872,17 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   return cudaGetLastError();
 }
 
+template <int D, bool F8>
+cudaError_t launch_persist_t(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const FwdParams& p, cudaStream_t s) {
+  using L = FwdPLayout<D, F8>;
+  cudaError_t e = cudaFuncSetAttribute(fa_fwd_persist_sm100_kernel<D, F8>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  fa_fwd_persist_sm100_kernel<D, F8><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
 // V (bf16) -> fp16 copy, 8 elements per 16-byte access (exact for |v| in [2^-14, 65504]).
 __global__ void __launch_bounds__(256) fa_fwd_v16_kernel(const uint4* __restrict__ v, uint4* __restrict__ v16,
                                                          long long n8, unsigned* counter) {
@@ -868,20 +909,15 @@ cudaError_t launch_fwd_persist_sm100(const CUtensorMap& tq, const CUtensorMap& t
                                      const FwdParams& p, int d, cudaStream_t s) {
   const long long units = (long long)p.n_pairs * p.BH;
   const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
-  if (d == 128) {
-    using L = FwdPLayout<128>;
-    cudaError_t e = cudaFuncSetAttribute(fa_fwd_persist_sm100_kernel<128>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    fa_fwd_persist_sm100_kernel<128><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, p);
-  } else {
-    using L = FwdPLayout<64>;
-    cudaError_t e = cudaFuncSetAttribute(fa_fwd_persist_sm100_kernel<64>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    fa_fwd_persist_sm100_kernel<64><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, p);
-  }
-  return cudaGetLastError();
+  return d == 128 ? launch_persist_t<128, false>(grid, tq, tk, tv, p, s)
+                  : launch_persist_t<64, false>(grid, tq, tk, tv, p, s);
+}
+
+cudaError_t launch_fwd_persist_fp8_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                         const FwdParams& p, cudaStream_t s) {
+  const long long units = (long long)p.n_pairs * p.BH;
+  const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
+  return launch_persist_t<128, true>(grid, tq, tk, tv, p, s);
 }
 
 cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, cudaStream_t s) {

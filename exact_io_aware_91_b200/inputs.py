@@ -17,7 +17,7 @@ import math
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "workload", "make_inputs", "make_qkv"]
+__all__ = ["Workload", "WORKLOADS", "workload", "make_inputs", "make_qkv", "make_qkv_fp8"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -106,3 +106,27 @@ def make_inputs(idx_or_workload, device: str | torch.device = "cpu") -> dict:
     w = idx_or_workload if isinstance(idx_or_workload, Workload) else WORKLOADS[idx_or_workload]
     return make_qkv(w.B, w.H, w.N, w.d, dtype=w.dtype, dist=w.dist, spiky_frac=w.spiky_frac,
                     backward=w.backward, seed=w.seed, device=device)
+
+
+E4M3_MAX = 448.0  # largest finite E4M3 value
+
+
+def make_qkv_fp8(B: int, H: int, N: int, d: int, *, dist: str = "normal", spiky_frac: float = 0.0,
+                 seed: int = 0, device: str | torch.device = "cpu", kv_heads: int | None = None) -> dict:
+    """8-bit inputs: the fp32 draws of ``make_qkv`` (same seed, same spiky keys), each tensor
+    divided by its own descale amax / 448 and rounded to E4M3 (torch's round to nearest even).
+
+    Returns {"q", "k", "v": torch.float8_e4m3fn tensors, "q_descale", "k_descale",
+    "v_descale": floats}; the real-valued inputs are descale * tensor."""
+    f = make_qkv(B, H, N, d, dtype=torch.float32, dist=dist, spiky_frac=spiky_frac, backward=False, seed=seed,
+                 kv_heads=kv_heads)
+    out = {}
+    for name in ("q", "k", "v"):
+        x = f[name]
+        amax = float(x.abs().max()) if x.numel() else 1.0
+        # a float32 value, as the C interface receives it
+        descale = float(torch.tensor(amax / E4M3_MAX if amax > 0 else 1.0, dtype=torch.float32))
+        out[name] = (x / descale).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn).to(device)
+        out[name + "_descale"] = descale
+    return out
+

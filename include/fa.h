@@ -223,6 +223,40 @@ FA_API fa_status fa_attn_bwd(const fa_attn_problem* problem, const void* q, cons
                              float* dk, float* dv, void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * fa_attn_fwd_fp8_workspace_size / fa_attn_fwd_fp8 -- forward pass on 8-bit inputs.
+ * ("Flash Attention uitgelegd: een uitgebreide gids", section "Native FP8-precisie";
+ * "FlashAttention (EL)", section "FlashAttention-3 (2024)": FlashAttention-3 runs the
+ * attention products in FP8 on the tensor cores.  The pages give no format or scaling
+ * scheme; the reading taken is E4M3 operands with one descale factor per tensor.)
+ *   problem          : as for fa_attn_fwd (grouped heads, causal mask, sliding window);
+ *                      d must be 128 (FA_ERR_UNSUPPORTED otherwise).
+ *   q                : const E4M3 (B, H, N, d), 16-byte aligned; k, v: const E4M3
+ *                      (B, H_kv, N, d), 16-byte aligned.  One byte per element in the
+ *                      OCP FP8 E4M3 encoding (bias 7, no infinities, 0x7F / 0xFF NaN).
+ *   q_descale, k_descale, v_descale : positive finite floats; the attention is computed
+ *                      for the real-valued inputs q_descale * Q, k_descale * K and
+ *                      v_descale * V (FA_ERR_INVALID_ARG otherwise).
+ *   o                : bf16 (B, H, N, d), 16-byte aligned, written.
+ *   lse              : fp32 (B, H, N) or NULL, natural-log LSE of the scaled scores.
+ *   workspace        : device buffer of fa_attn_fwd_fp8_workspace_size(problem) bytes
+ *                      (256), 256-byte aligned, caller-owned; contents on entry do not
+ *                      matter; one call at a time per workspace.
+ * Both products run on the tensor cores in 8 bits with fp32 accumulation (the E4M3
+ * products themselves are exact in fp32), and P V takes the probabilities P
+ * rounded to E4M3 (round to nearest even; P <= 2^8 because the running maximum is
+ * allowed to lag the true one by less than 8 in base-2 exponent).  The row sum that
+ * divides O uses P before that rounding, so an output row differs from the exact
+ * attention of the dequantized inputs by at most about 2^-4 times the P-weighted mean
+ * of |V| (plus an absolute 2^-10 per key whose P falls below E4M3's normal range); LSE
+ * is as accurate as the bf16 forward's.  No residual is produced (the backward takes
+ * bf16 inputs).  Asynchronous on `stream`.
+ */
+FA_API size_t fa_attn_fwd_fp8_workspace_size(const fa_attn_problem* problem);
+FA_API fa_status fa_attn_fwd_fp8(const fa_attn_problem* problem, const void* q, const void* k, const void* v,
+                                 float q_descale, float k_descale, float v_descale, void* o, float* lse,
+                                 void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fa_bwd_noalloc -- the backward pass of fa_bwd for callers that cannot allocate
  * device memory.  (The pages describe no such entry point; it is a service of this
  * library.)  Some callers have no way to obtain a workspace at the moment they run

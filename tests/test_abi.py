@@ -187,3 +187,32 @@ def test_f32_forward_argument_errors(lib):
 def test_valid_call_without_a_gpu_fails_loudly(lib):
     # all arguments valid: the call reaches the CUDA runtime, which has no device here
     assert fwd(lib) == api.FA_ERR_CUDA
+
+
+def test_fp8_forward_checks_its_arguments(lib):
+    import ctypes
+
+    pr = api.FaAttnProblem(1, 4, 2, 300, 128, 0.125, 1, -1, -1)
+    assert api.fa_attn_fwd_fp8_workspace_size(pr) == 256
+    assert lib.fa_attn_fwd_fp8_workspace_size(None) == 0
+    assert api.fa_attn_fwd_fp8_workspace_size(api.FaAttnProblem(1, 4, 2, 300, 128, 0.125, 1, -3, -1)) == 0
+
+    def call(p=pr, q=A, o=A, lse=A, ws=A, ws_bytes=256, ds=(1.0, 1.0, 1.0)):
+        return lib.fa_attn_fwd_fp8(None if p is None else ctypes.byref(p), q, A, A, *ds, o, lse, ws, ws_bytes, None)
+
+    assert call(p=None) == api.FA_ERR_INVALID_ARG
+    assert call(ds=(0.0, 1.0, 1.0)) == api.FA_ERR_INVALID_ARG
+    assert call(ds=(1.0, -1.0, 1.0)) == api.FA_ERR_INVALID_ARG
+    assert call(ds=(1.0, 1.0, float("inf"))) == api.FA_ERR_INVALID_ARG
+    assert call(ds=(1.0, float("nan"), 1.0)) == api.FA_ERR_INVALID_ARG
+    assert call(p=api.FaAttnProblem(1, 4, 2, 300, 64, 0.125, 1, -1, -1)) == api.FA_ERR_UNSUPPORTED  # d = 128 only
+    assert call(p=api.FaAttnProblem(1, 6, 4, 300, 128, 0.125, 1, -1, -1)) == api.FA_ERR_INVALID_ARG
+    assert call(q=None) == api.FA_ERR_INVALID_ARG
+    assert call(ws=None) == api.FA_ERR_INVALID_ARG
+    assert call(ws_bytes=255) == api.FA_ERR_INVALID_ARG
+    assert call(q=MIS) == api.FA_ERR_MISALIGNED
+    assert call(lse=A + 2) == api.FA_ERR_MISALIGNED
+    assert call(ws=A + 16) == api.FA_ERR_MISALIGNED
+    empty = api.FaAttnProblem(1, 4, 2, 0, 128, 0.125, 1, -1, -1)
+    assert lib.fa_attn_fwd_fp8(ctypes.byref(empty), None, None, None, 1.0, 1.0, 1.0, None, None, None, 0,
+                               None) == api.FA_OK
