@@ -42,7 +42,8 @@ def recorded_traffic(kernel: str, workload_name: str):
     """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
     import hashlib
 
-    short = {"causal_b2_h32_n8192_d128_spiky": "causal_b2_h32_n8192_d128"}.get(workload_name)
+    short = {"causal_b2_h32_n8192_d128_spiky": "causal_b2_h32_n8192_d128",
+             "causal_b2_h32_n8192_d128_spiky_fp8": "causal_b2_h32_n8192_d128_fp8"}.get(workload_name)
     if short is None:
         return None
     path = os.path.join(ROOT, "profiles", f"traffic_{short}.json")
@@ -471,6 +472,132 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- 8-bit forward
+METRIC_FP8 = "attention fwd TFLOPS (FP8 E4M3 inputs, causal, N=8k, d=128) & % of B200 fp8 tensor peak"
+
+
+def oracle_fp8_head(inp8: dict, codes: dict, w: inputs.Workload, b: int, h: int) -> None:
+    import oracle
+
+    oracle.attention_forward_fp8(codes["q"][b:b + 1, h:h + 1], codes["k"][b:b + 1, h:h + 1],
+                                 codes["v"][b:b + 1, h:h + 1], inp8["q_descale"], inp8["k_descale"],
+                                 inp8["v_descale"], w.scale, w.causal)
+
+
+def run_fp8(args, rank: int, world: int) -> None:
+    """--fp8: the 8-bit forward (fa_attn_fwd_fp8) on the workload's shape, forward only."""
+    from exact_io_aware_91_b200 import api
+
+    w = inputs.workload(args.workload)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    inp8 = inputs.make_qkv_fp8(B, H, N, d, spiky_frac=w.spiky_frac, seed=w.seed + rank)
+    q, k, v = (inp8[n].cuda() for n in ("q", "k", "v"))
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    pr = api.FaAttnProblem(B, H, H, N, d, w.scale, int(w.causal), -1, -1)
+    ws = torch.empty(api.fa_attn_fwd_fp8_workspace_size(pr), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > the 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        api.fa_attn_fwd_fp8(q, k, v, inp8["q_descale"], inp8["k_descale"], inp8["v_descale"], causal=w.causal,
+                            scale=w.scale, o=o, lse=lse, workspace=ws)
+
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    for e0, e1 in ev:
+        flush.zero_()  # L2 flushed between timed forwards (outside the events)
+        e0.record(stream)
+        fwd()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    if api.fa_device_status() != api.FA_OK:
+        raise RuntimeError("device status not OK after the timed region")
+    ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(ms), world)
+    ms_step = total_ms / args.steps
+    value = w.fwd_flops * world / (ms_step * 1e-3) / 1e12
+    peaks = load_peaks()
+    bf16_peak, kind = tensor_peak(peaks, clk)
+    peak = 2.0 * bf16_peak  # dense fp8 = 2x dense bf16 (4.5 vs 2.25 PFLOP/s nominal)
+    achieved = w.fwd_flops / (statistics.mean(ms) * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "fwd_fp8", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak,
+                "traffic": args.traffic if args.traffic is not None else recorded_traffic("fwd_fp8", w.name + "_fp8"),
+                "peak_kind": kind.replace("bf16 dense matmul", "bf16 dense matmul x 2 (fp8 / bf16 nominal ratio)")}
+
+    e2e = None
+    if not args.no_e2e:
+        h_in = {n: inp8[n].view(torch.uint8).pin_memory() for n in ("q", "k", "v")}
+        h_out = {"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
+                 "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory()}
+        dev_in = {"q": q.view(torch.uint8), "k": k.view(torch.uint8), "v": v.view(torch.uint8)}
+        n_e2e = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            for n, t in h_in.items():
+                dev_in[n].copy_(t, non_blocking=True)
+            fwd()
+            h_out["o"].copy_(o, non_blocking=True)
+            h_out["lse"].copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, world)
+        e2e = {"value": w.fwd_flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+               "h2d_bytes_per_step": sum(t.numel() for t in h_in.values()),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_out.values()),
+               "ms_per_step": e2e_ms, "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        codes = {n: inp8[n].view(torch.uint8).numpy() for n in ("q", "k", "v")}
+        per_head = w.fwd_flops / (B * H)
+        heads, t0 = 0, time.perf_counter()
+        while True:
+            oracle_fp8_head(inp8, codes, w, heads // H % B, heads % H)
+            heads += 1
+            if time.perf_counter() - t0 > 12.0 or heads >= B * H:
+                break
+        dt = time.perf_counter() - t0
+        cpu = {"value": per_head * heads / dt / 1e12, "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{heads} of {B * H} heads (forward of the dequantized E4M3 inputs, fp64 numpy), {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC_FP8, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": w.name + "_fp8", "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+                       "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
+                       "step": "forward only", "l2": "flushed between timed forwards (256 MB write)"},
+            "frac_of_peak": {"measured_burst_x2": value / world / (2.0 * peaks["bf16_tflops"]),
+                             "measured_sustained_x2": value / world / (2.0 * peaks["bf16_tflops_sustained"]),
+                             "datasheet_4500": value / world / 4500.0},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps,  # the persistent forward (its work counter is reset by a memset)
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -486,6 +613,8 @@ def main() -> None:
     ap.add_argument("--window", type=int, default=None,
                     help="sliding-window run: each query sees the previous WINDOW keys and itself "
                          "(fa_attn_fwd / fa_attn_bwd); default no window")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the 8-bit forward (E4M3 inputs, fa_attn_fwd_fp8) on the workload's shape")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the dominant kernel from an ncu capture (reported as-is)")
     args = ap.parse_args()
@@ -495,6 +624,8 @@ def main() -> None:
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.fp8:
+            run_fp8(args, rank, world)
         else:
             run_ours(args, rank, world, local)
     finally:

@@ -78,9 +78,16 @@ constexpr int kConvThreads = 64;
 #ifndef FA_EXP_FMA_PER8
 #define FA_EXP_FMA_PER8 2
 #endif
+// The 8-bit forward's products take half the tensor-core time, so the exponentials (16 per
+// clock per SM on the MUFU) are its bound: it moves a larger share to the FMA pipe.
+#ifndef FA_EXP_FMA_PER8_F8
+#define FA_EXP_FMA_PER8_F8 2
+#endif
 // element pairs out of every 8 whose exponentials run on the FMA pipe (even, 0..8)
 constexpr int kExpFmaPer8 = FA_EXP_FMA_PER8;
+constexpr int kExpFmaPer8F8 = FA_EXP_FMA_PER8_F8;
 static_assert(kExpFmaPer8 % 2 == 0 && kExpFmaPer8 >= 0 && kExpFmaPer8 <= 8, "pairs are taken two at a time");
+static_assert(kExpFmaPer8F8 % 2 == 0 && kExpFmaPer8F8 >= 0 && kExpFmaPer8F8 <= 8, "pairs are taken two at a time");
 static_assert(FwdLayout<128>::STAGES % 2 == 0 && FwdLayout<64>::STAGES % 2 == 0,
               "K and V tiles must alternate over fixed ring stages");
 
@@ -176,8 +183,10 @@ __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS
       float* e = &x[64 * h + 2 * i];
       fma2(e[0], e[1], sl2, neg_m);
       fma2(e[2], e[3], sl2, neg_m);
-      // kExpFmaPer8 of every 8 element pairs take 2^x on the FMA pipe, the rest on MUFU
-      if ((i & 7) < 2 * (kExpFmaPer8 / 2)) {
+      // kExpFmaPer8 (kExpFmaPer8F8) of every 8 element pairs take 2^x on the FMA pipe, the
+      // rest on MUFU
+      constexpr int fma_per8 = F8 ? kExpFmaPer8F8 : kExpFmaPer8;
+      if ((i & 7) < 2 * (fma_per8 / 2)) {
         exp2_fma_pipe(e[0], e[1]);
         exp2_fma_pipe(e[2], e[3]);
       } else {
