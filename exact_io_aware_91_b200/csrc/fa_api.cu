@@ -70,12 +70,14 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // Shared validation of sizes/scalars.  Returns FA_OK and sets *empty when there is nothing to do.
 // H_kv: key/value heads (H for plain multi-head attention); H must be a multiple of it.
-fa_status check_problem(int B, int H, int H_kv, int N, int d, float scale, int causal, bool* empty) {
+// allow_d256: the forward with a workspace also takes d = 256 (its own persistent kernel)
+fa_status check_problem(int B, int H, int H_kv, int N, int d, float scale, int causal, bool* empty,
+                        bool allow_d256 = false) {
   if (B < 0 || H < 0 || N < 0 || H_kv < 0) return FA_ERR_INVALID_ARG;
   if (H > 0 && (H_kv < 1 || H % H_kv != 0)) return FA_ERR_INVALID_ARG;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && !(allow_d256 && d == 256)) return FA_ERR_UNSUPPORTED;
   *empty = (B == 0 || H == 0 || N == 0);
   if (*empty) return FA_OK;
   const long long BH = (long long)B * H;
@@ -187,7 +189,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
                    size_t workspace_bytes, fa_stream_t stream) {
   bool empty = false;
   if (!window_ok(wl, wr)) return FA_ERR_INVALID_ARG;
-  fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty);
+  fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty, workspace != nullptr);
   if (st != FA_OK || empty) return st;
   if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
@@ -206,10 +208,15 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   CUtensorMap tq, tk, tv, to;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const bool v16 = workspace != nullptr;
+  if (d == 256) {  // V (fp16, in the workspace) in 64-key x 64-column boxes for the d = 256 kernel
+    if (!make_tmap_3d(&tv, workspace, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, BH_kv, 64, 64, true))
+      return FA_ERR_CUDA;
+  } else if (!make_tmap_3d(&tv, v16 ? workspace : v, v16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : bf, 2, d, N, BH_kv,
+                           64, 128, true)) {
+    return FA_ERR_CUDA;
+  }
   if (!make_tmap_3d(&tq, q, bf, 2, d, N, BH, 64, 128, true) ||
       !make_tmap_3d(&tk, k, bf, 2, d, N, BH_kv, 64, 128, true) ||
-      !make_tmap_3d(&tv, v16 ? workspace : v, v16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : bf, 2, d, N, BH_kv, 64, 128,
-                    true) ||
       !make_tmap_3d(&to, o, bf, 2, d, N, BH, 64, 128, true))
     return FA_ERR_CUDA;
   FwdParams p{};
@@ -233,7 +240,9 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   p.err = g_err_ptr[dev];
   // with a workspace: the persistent kernel (work counter in the workspace); without: one CTA
   // per unit, V converted on chip
-  const cudaError_t e = v16 ? launch_fwd_persist_sm100(tq, tk, tv, p, d, s) : launch_fwd_sm100(tq, tk, tv, to, p, d, s);
+  const cudaError_t e = d == 256 ? launch_fwd_d256_sm100(tq, tk, tv, p, s)
+                        : v16    ? launch_fwd_persist_sm100(tq, tk, tv, p, d, s)
+                                 : launch_fwd_sm100(tq, tk, tv, to, p, d, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 }  // namespace
@@ -245,7 +254,7 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float
 
 size_t fa_fwd_workspace_size(int B, int H_kv, int N, int d) {
   bool empty = false;
-  if (check_problem(B, H_kv, H_kv, N, d, 1.0f, 0, &empty) != FA_OK || empty) return 0;
+  if (check_problem(B, H_kv, H_kv, N, d, 1.0f, 0, &empty, true) != FA_OK || empty) return 0;
   return align256((size_t)B * H_kv * N * d * 2) + 256;  // fp16 V, then the work counter
 }
 
@@ -254,7 +263,7 @@ fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float*
                     fa_stream_t stream) {
   if (workspace == nullptr) {
     bool empty = false;
-    const fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty);
+    const fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty, true);
     return (st != FA_OK || empty) ? st : FA_ERR_INVALID_ARG;
   }
   return fwd_impl(q, k, v, o, lse, o_resid, B, H, H_kv, N, d, scale, causal, -1, -1, workspace, workspace_bytes,
@@ -411,7 +420,7 @@ fa_status fa_attn_fwd(const fa_attn_problem* pr, const void* q, const void* k, c
   if (pr == nullptr) return FA_ERR_INVALID_ARG;
   if (workspace == nullptr) {
     bool empty = false;
-    const fa_status st = check_problem(pr->B, pr->H, pr->H_kv, pr->N, pr->d, pr->scale, pr->causal, &empty);
+    const fa_status st = check_problem(pr->B, pr->H, pr->H_kv, pr->N, pr->d, pr->scale, pr->causal, &empty, true);
     return (st != FA_OK || empty) ? st : FA_ERR_INVALID_ARG;
   }
   return fwd_impl(q, k, v, o, lse, o_resid, pr->B, pr->H, pr->H_kv, pr->N, pr->d, pr->scale, pr->causal,

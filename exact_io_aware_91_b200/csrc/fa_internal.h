@@ -112,6 +112,8 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
 cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, cudaStream_t s);
 cudaError_t launch_fwd_persist_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                      const FwdParams& p, int d, cudaStream_t s);
+cudaError_t launch_fwd_d256_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                  const FwdParams& p, cudaStream_t s);  // d = 256, fp16 V in 64 x 64 boxes
 cudaError_t launch_fwd_persist_fp8_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                          const FwdParams& p, cudaStream_t s);  // d = 128, E4M3 inputs
 cudaError_t launch_selftest_wait(int* err, cudaStream_t s);

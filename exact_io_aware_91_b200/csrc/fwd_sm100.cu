@@ -109,13 +109,16 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // maximum moves, P = 2^(scale*log2(e)*S - m) written back over S as fp16 in two halves
 // (the tensor core starts on the first half's P V while the second half is computed).
 // With F8, P is written as E4M3 (four per TMEM column, 16 columns per half) for the 8-bit
-// P V product; the row sum uses the fp32 values before rounding.
+// P V product; the row sum uses the fp32 values before rounding.  bar_o_ready (non-zero)
+// is waited on, with parity o_ready_parity, before a rescale of O: for a kernel whose
+// previous P V into O may still be running when this step starts.
 // Returns false if a bounded wait gave up.
 template <int D, bool F8 = false>
 __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS, uint32_t tO, uint32_t bar_s_full,
                                                  uint32_t s_parity, uint32_t bar_p_half, uint32_t bar_p_full, int j,
                                                  bool first, int q_base, int r, float& m, float& l,
-                                                 const WaitCtx& wctx) {
+                                                 const WaitCtx& wctx, uint32_t bar_o_ready = 0,
+                                                 uint32_t o_ready_parity = 0) {
   const float sl2 = p.scale_log2;
   if (!mbar_wait(bar_s_full, s_parity, wctx)) return false;
   tc_fence_after();
@@ -162,8 +165,11 @@ __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS
   const float alpha = (m_use == m) ? 1.0f : ex2_approx(m - m_use);  // 0 on the first tile
   const float neg_m = m_use == -INFINITY ? 0.0f : -m_use;  // no visible key yet: every P is 0
   if (!first && __any_sync(0xffffffffu, alpha != 1.0f)) {
-    // rescale O before this tile's P V starts; the previous O += P V of this tile
-    // completed before S_j did (same issuing thread, in-order tensor pipe)
+    // rescale O before this tile's P V starts; either the previous O += P V of this tile
+    // completed before S_j did (issued before it by the same thread, in-order tensor pipe),
+    // or the caller names the barrier its completion arrives on
+    if (bar_o_ready != 0 && !mbar_wait(bar_o_ready, o_ready_parity, wctx)) return false;
+    tc_fence_after();
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       uint32_t u[32];
@@ -866,6 +872,341 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
 }
+
+// ============================================================================ head dim 256
+// Persistent forward for d = 256 (fa_fwd_ws / fa_attn_fwd with d = 256).  A 128-row tile
+// needs S (128 TMEM columns) and O (256), so two tiles do not fit in the 512 columns: a unit
+// is ONE 128-row query tile, S is double-buffered (S_A, S_B) and the tensor core runs
+// S_{j+1} = Q K_{j+1}^T while the softmax warpgroup turns S_j into P_j; the issue order is
+// S_0, S_1, PV_0, S_2, PV_1, ..., so the softmax of step j has the time of S_{j+1} and PV_{j-1}
+// (~2100 cycles) to finish.  PV_{j-1} is issued after S_j, so a rescale of O in the softmax
+// of step j first waits for PV_{j-1} to complete (BAR_PV_DONE; rescales are rare: the running
+// maximum may lag by < 2^8).
+// Shared memory: Q (4 boxes of 128 x 64 bf16, 64 KB) and a FIFO of 32 KB slots filled in the
+// order the tensor core consumes them -- K_0, K_1, V_0, K_2, V_1, ..., V_{n-1} -- so one running
+// index serves producer and issuer.  A K slot holds one d-half of K_j (two 128 x 64 boxes,
+// K-major); a V slot holds one key-half of V_j (four 64-key x 64-column fp16 boxes, read
+// MN-major by the N = 256 P V products).
+struct FwdWLayout {
+  static constexpr int D = 256;
+  static constexpr int BOX = 128 * 128;  // 128 rows x 64 bf16 columns (Q, K boxes)
+  static constexpr int VBOX = 64 * 128;  // 64 rows x 64 fp16 columns (V boxes)
+  static constexpr int SLOT = 32768;
+  static constexpr int SLOTS = 5;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = 4 * BOX;
+  static constexpr int OFF_BAR = OFF_RING + SLOTS * SLOT;
+  static constexpr int BAR_Q_FULL = 0;
+  static constexpr int BAR_Q_EMPTY = 1;
+  static constexpr int BAR_SLOT_FULL = 2;                    // [SLOTS]
+  static constexpr int BAR_SLOT_EMPTY = 2 + SLOTS;           // [SLOTS]
+  static constexpr int BAR_S_FULL = 2 + 2 * SLOTS;           // [2]
+  static constexpr int BAR_P_HALF = BAR_S_FULL + 2;          // [2]
+  static constexpr int BAR_P_FULL = BAR_P_HALF + 2;          // [2]
+  static constexpr int BAR_PV_DONE = BAR_P_FULL + 2;         // one phase per P V product
+  static constexpr int BAR_O_FULL = BAR_PV_DONE + 1;         // a unit's last P V completed
+  static constexpr int BAR_O_FREE = BAR_O_FULL + 1;          // the epilogue has read O out of TMEM
+  static constexpr int BAR_UNIT_FULL = BAR_O_FREE + 1;       // [2]
+  static constexpr int BAR_UNIT_EMPTY = BAR_UNIT_FULL + 2;   // [2]
+  static constexpr int BAR_MMA_DONE = BAR_UNIT_EMPTY + 2;
+  static constexpr int NBAR = BAR_MMA_DONE + 1;
+  static constexpr int OFF_UNIT = OFF_BAR + NBAR * 8;  // int[2]
+  static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
+  static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
+  static constexpr int SMEM_ALLOC = OFF_ABORT + 8 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O = 256;
+};
+static_assert(FwdWLayout::SMEM_ALLOC <= 232448, "d = 256 forward exceeds the shared memory of a CTA");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_d256_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdWLayout;
+  constexpr int D = L::D;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + L::OFF_BAR + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_ABORT);
+  const WaitCtx wctx{abort_flag, p.err};
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int n_qt = (p.N + 127) / 128;
+  const int n_units = n_qt * p.BH;
+  struct Unit {
+    int bh, bh_kv, q_base, jlo, n;  // key tiles jlo .. jlo + n - 1
+  };
+  auto unit_of = [&](int u) -> Unit {
+    Unit x;
+    int rank;
+    unit_order(u, n_qt, p.BH, p.head_group, x.bh, rank);
+    const int qt = p.causal ? (n_qt - 1 - rank) : rank;
+    x.bh_kv = kv_head_of(x.bh, p.H, p.H_kv);
+    x.q_base = qt * 128;
+    x.jlo = key_lo(x.q_base, p.N, p.win_left) / 128;
+    x.n = key_hi(x.q_base + 127, p.N, p.causal, p.win_right) / 128 - x.jlo + 1;  // >= 1
+    return x;
+  };
+  int* unit_ring = reinterpret_cast<int*>(gbase + L::OFF_UNIT);
+  auto next_unit = [&](int k, bool& ok) -> int {
+    const int slot = k & 1;
+    ok = mbar_wait(bar(L::BAR_UNIT_FULL + slot), (k >> 1) & 1, wctx);
+    return ok ? *reinterpret_cast<volatile int*>(unit_ring + slot) : n_units;
+  };
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(L::BAR_Q_FULL), 1);
+    mbar_init(bar(L::BAR_Q_EMPTY), 1);
+    for (int s = 0; s < L::SLOTS; ++s) {
+      mbar_init(bar(L::BAR_SLOT_FULL + s), 1);
+      mbar_init(bar(L::BAR_SLOT_EMPTY + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::BAR_S_FULL + t), 1);
+      mbar_init(bar(L::BAR_P_HALF + t), 128);
+      mbar_init(bar(L::BAR_P_FULL + t), 128);
+      mbar_init(bar(L::BAR_UNIT_FULL + t), 1);
+      mbar_init(bar(L::BAR_UNIT_EMPTY + t), 1 + 128);
+    }
+    mbar_init(bar(L::BAR_PV_DONE), 1);
+    mbar_init(bar(L::BAR_O_FULL), 1);
+    mbar_init(bar(L::BAR_O_FREE), 128);
+    mbar_init(bar(L::BAR_MMA_DONE), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(base + L::OFF_TMEM_SLOT, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_TMEM_SLOT);
+
+  if (warp == 0) {
+    // ===================================================== TMA producer + work distribution
+    regs_dec<kRegsLow>();
+    const uint32_t leader = elect_one();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    int issued = 0, q_issued = 0;  // FIFO slot loads and Q loads so far
+    bool ok = true;
+    // one FIFO entry: the K d-half (kind 0) or V key-half (kind 1) `half` of key tile j
+    auto load_slot = [&](int kind, int j, int half, int bh_kv) -> bool {
+      const int st = issued % L::SLOTS;
+      if (!mbar_wait(bar(L::BAR_SLOT_EMPTY + st), ((issued / L::SLOTS) & 1) ^ 1u, wctx)) return false;
+      const uint32_t dst = base + L::OFF_RING + st * L::SLOT;
+      mbar_arrive_expect_tx(bar(L::BAR_SLOT_FULL + st), L::SLOT, leader);
+      if (kind == 0) {
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(dst + c * L::BOX, &tm_k, (2 * half + c) * 64, j * 128, bh_kv, bar(L::BAR_SLOT_FULL + st),
+                      leader);
+      } else {
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d(dst + c * L::VBOX, &tm_v, c * 64, j * 128 + 64 * half, bh_kv, bar(L::BAR_SLOT_FULL + st),
+                      leader);
+      }
+      ++issued;
+      return true;
+    };
+    for (int uc = 0;; ++uc) {
+      if (uc >= 2 && !(ok = mbar_wait(bar(L::BAR_UNIT_EMPTY + (uc & 1)), ((uc - 2) >> 1) & 1, wctx))) break;
+      int u = 0;
+      if (lane == 0) u = (int)atomicAdd(p.counter, 1u);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (lane == 0) {
+        unit_ring[uc & 1] = u < n_units ? u : n_units;
+        mbar_arrive(bar(L::BAR_UNIT_FULL + (uc & 1)));
+      }
+      __syncwarp();
+      if (u >= n_units) break;
+      const Unit x = unit_of(u);
+      if (uc > 0 && !(ok = mbar_wait(bar(L::BAR_Q_EMPTY), (uc - 1) & 1, wctx))) break;
+      mbar_arrive_expect_tx(bar(L::BAR_Q_FULL), 4 * L::BOX, leader);
+      for (int c = 0; c < 4; ++c)
+        tma_load_3d(base + L::OFF_Q + c * L::BOX, &tm_q, c * 64, x.q_base, x.bh, bar(L::BAR_Q_FULL), leader);
+      ++q_issued;
+      // consumption order: K_0, then K_{t+1}, V_t for t = 0 .. n - 2, then V_{n-1}
+      for (int h = 0; h < 2 && ok; ++h) ok = load_slot(0, x.jlo, h, x.bh_kv);
+      for (int t = 0; t < x.n && ok; ++t) {
+        if (t + 1 < x.n)
+          for (int h = 0; h < 2 && ok; ++h) ok = load_slot(0, x.jlo + t + 1, h, x.bh_kv);
+        for (int h = 0; h < 2 && ok; ++h) ok = load_slot(1, x.jlo + t, h, x.bh_kv);
+      }
+      if (!ok) break;
+    }
+    if (q_issued > 0) drain_wait(bar(L::BAR_Q_FULL), (q_issued - 1) & 1);
+    for (int i = (issued > L::SLOTS ? issued - L::SLOTS : 0); i < issued; ++i)
+      drain_wait(bar(L::BAR_SLOT_FULL + (i % L::SLOTS)), (i / L::SLOTS) & 1);
+  } else if (warp == 1) {
+    // ===================================================== MMA issuer
+    regs_dec<kRegsLow>();
+    const uint32_t leader = elect_one();
+    constexpr uint32_t idesc_qk = make_idesc(128, 128, true, false, false);  // bf16 Q, K; K-major
+    constexpr uint32_t idesc_pv = make_idesc(128, D, false, false, true);    // fp16 P (TMEM) x fp16 V, MN-major
+    const uint32_t tS[2] = {tmem + L::T_S0, tmem + L::T_S1};
+    const uint32_t tO = tmem + L::T_O;
+    const uint64_t dQ = make_sdesc_sw128(base + L::OFF_Q, 16, 1024);
+    const uint64_t dRingK = make_sdesc_sw128(base + L::OFF_RING, 16, 1024);       // K slots, K-major
+    const uint64_t dRingV = make_sdesc_sw128(base + L::OFF_RING, L::VBOX, 1024);  // V slots, MN-major
+    int consumed = 0;  // FIFO entries consumed so far
+    int T = 0;         // S / P buffer steps so far (all units)
+    bool ok = true;
+    auto take = [&]() -> int {  // wait for the next FIFO entry, return its slot
+      const int st = consumed % L::SLOTS;
+      ok = mbar_wait(bar(L::BAR_SLOT_FULL + st), (consumed / L::SLOTS) & 1, wctx);
+      ++consumed;
+      return st;
+    };
+    // S_T = Q K_j^T: 16 products over d, the two d-halves from two FIFO entries
+    auto issue_qk = [&](int b) -> bool {
+      for (int h = 0; h < 2; ++h) {
+        const int st = take();
+        if (!ok) return false;
+        tc_fence_after();
+        const uint64_t k_desc = sdesc_add(dRingK, st * L::SLOT);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t qoff = (2 * h + (k >> 2)) * L::BOX + (k & 3) * 32;
+          const uint32_t koff = (k >> 2) * L::BOX + (k & 3) * 32;
+          mma_ss(tS[b], sdesc_add(dQ, qoff), sdesc_add(k_desc, koff), idesc_qk, (h | k) > 0 ? 1u : 0u, leader);
+        }
+        mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
+      }
+      mma_commit(bar(L::BAR_S_FULL + b), leader);
+      return true;
+    };
+    // O += P_t V_t (t: step of this unit, Tt: global step): the two key-halves from two FIFO
+    // entries, each after its half of P is in TMEM
+    auto issue_pv = [&](int t, int Tt, int uc) -> bool {
+      const int b = Tt & 1;
+      const uint32_t ph = (Tt >> 1) & 1;
+      if (t == 0 && uc > 0) {  // the previous unit's epilogue has read O
+        if (!mbar_wait(bar(L::BAR_O_FREE), (uc - 1) & 1, wctx)) return false;
+        tc_fence_after();
+      }
+      for (int h = 0; h < 2; ++h) {
+        const int st = take();
+        if (!ok) return false;
+        if (!mbar_wait(bar(h == 0 ? L::BAR_P_HALF + b : L::BAR_P_FULL + b), ph, wctx)) return false;
+        tc_fence_after();
+        const uint64_t v_desc = sdesc_add(dRingV, st * L::SLOT);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const int k = 4 * h + kk;  // 16-key step
+          mma_ts(tO, tS[b] + k * 8, sdesc_add(v_desc, kk * 2048), idesc_pv, (t > 0 || k > 0) ? 1u : 0u, leader);
+        }
+        mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
+      }
+      mma_commit(bar(L::BAR_PV_DONE), leader);
+      return true;
+    };
+    for (int uc = 0; ok; ++uc) {
+      const int u = next_unit(uc, ok);
+      if (lane == 0) mbar_arrive(bar(L::BAR_UNIT_EMPTY + (uc & 1)));
+      if (!ok || u >= n_units) break;
+      const Unit x = unit_of(u);
+      if (!(ok = mbar_wait(bar(L::BAR_Q_FULL), uc & 1, wctx))) break;
+      tc_fence_after();
+      const int T0 = T;
+      if (!(ok = issue_qk(T & 1))) break;  // S_0
+      ++T;
+      for (int t = 1; t < x.n && ok; ++t) {
+        ok = issue_qk(T & 1);  // S_t
+        if (!ok) break;
+        if (t == x.n - 1) mma_commit(bar(L::BAR_Q_EMPTY), leader);  // the unit's last Q K^T
+        ++T;
+        ok = issue_pv(t - 1, T0 + t - 1, uc);
+      }
+      if (!ok) break;
+      if (x.n == 1) mma_commit(bar(L::BAR_Q_EMPTY), leader);
+      if (!(ok = issue_pv(x.n - 1, T0 + x.n - 1, uc))) break;
+      mma_commit(bar(L::BAR_O_FULL), leader);
+    }
+    mma_commit(bar(L::BAR_MMA_DONE), leader);
+    drain_wait(bar(L::BAR_MMA_DONE), 0);
+  } else if (warp < 4 || warp >= 8) {
+    regs_dec<kRegsLow>();  // warps 2-3 and 8-11: idle
+  } else {
+    // ===================================================== softmax + epilogue warpgroup
+    regs_inc<kRegsHigh>();
+    const int wq = warp - 4;         // TMEM lane quarter
+    const int row = wq * 32 + lane;  // row inside the tile
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tO = tmem + lane_off + L::T_O;
+    bool ok = true;
+    int T = 0;
+    int u = next_unit(0, ok);
+    mbar_arrive(bar(L::BAR_UNIT_EMPTY + 0));
+    for (int uc = 0; ok && u < n_units; ++uc) {
+      const Unit x = unit_of(u);
+      const int r = x.q_base + row;
+      float m = -INFINITY, l = 0.f;
+      for (int t = 0; t < x.n; ++t, ++T) {
+        const int b = T & 1;
+        const uint32_t tS = tmem + lane_off + (b ? L::T_S1 : L::T_S0);
+        // a rescale of O waits for the previous step's P V (global product T - 1)
+        if (!(ok = fwd_softmax_step<D>(p, tS, tO, bar(L::BAR_S_FULL + b), (T >> 1) & 1, bar(L::BAR_P_HALF + b),
+                                       bar(L::BAR_P_FULL + b), x.jlo + t, t == 0, x.q_base, r, m, l, wctx,
+                                       bar(L::BAR_PV_DONE), (uint32_t)((T - 1) & 1))))
+          break;
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16 and the bf16 residual, stored from registers
+      if (!(ok = mbar_wait(bar(L::BAR_O_FULL), uc & 1, wctx))) break;
+      tc_fence_after();
+      const float inv_l = p.out_scale / l;
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t u0[32], u1[32];
+        tmem_ld32(tO + 64 * c, u0);
+        tmem_ld32(tO + 64 * c + 32, u1);
+        tmem_wait_ld();
+        if (c == D / 64 - 1) {  // O fully read: the next unit may accumulate into it
+          tc_fence_before();
+          mbar_arrive(bar(L::BAR_O_FREE));
+        }
+        uint4 oa[8], ra[8];
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          uint32_t pk[4], rk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * q4 + e;
+            const uint32_t* uu = i < 16 ? u0 : u1;
+            const int k = 2 * (i & 15);
+            const float a = __uint_as_float(uu[k]) * inv_l, bb = __uint_as_float(uu[k + 1]) * inv_l;
+            pk[e] = pack_bf16(a, bb);
+            const float2 ab = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
+            rk[e] = pack_bf16(a - ab.x, bb - ab.y);
+          }
+          oa[q4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          ra[q4] = make_uint4(rk[0], rk[1], rk[2], rk[3]);
+        }
+        warp_store_rows_128b(oa, reinterpret_cast<uint8_t*>(p.o + (size_t)x.bh * p.N * D + 64 * c), D * 2,
+                             x.q_base + wq * 32, p.N);
+        if (p.o_resid != nullptr)
+          warp_store_rows_128b(ra, reinterpret_cast<uint8_t*>(p.o_resid + (size_t)x.bh * p.N * D + 64 * c), D * 2,
+                               x.q_base + wq * 32, p.N);
+      }
+      if (p.lse != nullptr && r < p.N) p.lse[(size_t)x.bh * p.N + r] = (m + __log2f(l)) * 0.69314718055994531f;
+      u = next_unit(uc + 1, ok);
+      mbar_arrive(bar(L::BAR_UNIT_EMPTY + ((uc + 1) & 1)));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
 }  // namespace
 
 namespace {
@@ -935,6 +1276,17 @@ cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* 
   if (blocks > 148 * 16) blocks = 148 * 16;
   fa_fwd_v16_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8,
                                                      counter);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_d256_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                  const FwdParams& p, cudaStream_t s) {
+  const long long units = (long long)((p.N + 127) / 128) * p.BH;
+  const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
+  cudaError_t e = cudaFuncSetAttribute(fa_fwd_d256_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       FwdWLayout::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  fa_fwd_d256_sm100_kernel<<<grid, kThreads, FwdWLayout::SMEM_ALLOC, s>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 

@@ -216,3 +216,21 @@ def test_fp8_forward_checks_its_arguments(lib):
     empty = api.FaAttnProblem(1, 4, 2, 0, 128, 0.125, 1, -1, -1)
     assert lib.fa_attn_fwd_fp8(ctypes.byref(empty), None, None, None, 1.0, 1.0, 1.0, None, None, None, 0,
                                None) == api.FA_OK
+
+
+def test_head_dim_256_is_a_forward_with_workspace(lib):
+    assert api.fa_fwd_workspace_size(1, 2, 300, 256) == _align256(1 * 2 * 300 * 256 * 2) + 256
+    pr = api.FaAttnProblem(1, 4, 2, 300, 256, 0.0625, 1, -1, -1)
+    assert api.fa_attn_fwd_workspace_size(pr) == api.fa_fwd_workspace_size(1, 2, 300, 256)
+    assert api.fa_bwd_workspace_size(1, 2, 300, 256) == 0
+    assert api.fa_bwd_gqa_workspace_size(1, 4, 2, 300, 256) == 0
+    assert fwd(lib, d=256) == api.FA_ERR_UNSUPPORTED  # fa_fwd: no workspace, no d = 256 kernel
+    # fa_fwd_ws without its workspace: the problem is valid, the missing workspace is the error
+    assert lib.fa_fwd_ws(A, A, A, A, A, None, 1, 4, 2, 300, 256, 0.0625, 1, None, 0, None) == api.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_ws(A, A, A, A, A, None, 1, 4, 2, 300, 512, 0.0625, 1, A, 1 << 40, None) == \
+        api.FA_ERR_UNSUPPORTED
+    assert bwd(lib, d=256) == api.FA_ERR_UNSUPPORTED
+
+
+def _align256(x):
+    return (x + 255) // 256 * 256
