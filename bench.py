@@ -43,7 +43,8 @@ def recorded_traffic(kernel: str, workload_name: str):
     import hashlib
 
     short = {"causal_b2_h32_n8192_d128_spiky": "causal_b2_h32_n8192_d128",
-             "causal_b2_h32_n8192_d128_spiky_fp8": "causal_b2_h32_n8192_d128_fp8"}.get(workload_name)
+             "causal_b2_h32_n8192_d128_spiky_fp8": "causal_b2_h32_n8192_d128_fp8",
+             "causal_b2_h16_n8192_d256_spiky": "causal_b2_h16_n8192_d256"}.get(workload_name)
     if short is None:
         return None
     path = os.path.join(ROOT, "profiles", f"traffic_{short}.json")
@@ -514,39 +515,49 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
         print(json.dumps(line), flush=True)
 
 
-# ----------------------------------------------------------------------------- 8-bit forward
+# ----------------------------------------------------------------------------- forward-only runs
 METRIC_FP8 = "attention fwd TFLOPS (FP8 E4M3 inputs, causal, N=8k, d=128) & % of B200 fp8 tensor peak"
+METRIC_D256 = "attention fwd TFLOPS (BF16, causal, N=8k, d=256) & % of B200 tensor peak"
 
 
-def oracle_fp8_head(inp8: dict, codes: dict, w: inputs.Workload, b: int, h: int) -> None:
-    import oracle
-
-    oracle.attention_forward_fp8(codes["q"][b:b + 1, h:h + 1], codes["k"][b:b + 1, h:h + 1],
-                                 codes["v"][b:b + 1, h:h + 1], inp8["q_descale"], inp8["k_descale"],
-                                 inp8["v_descale"], w.scale, w.causal)
-
-
-def run_fp8(args, rank: int, world: int) -> None:
-    """--fp8: the 8-bit forward (fa_attn_fwd_fp8) on the workload's shape, forward only."""
+def run_fwd_only(args, rank: int, world: int, kind: str) -> None:
+    """--fp8: the 8-bit forward (fa_attn_fwd_fp8) on workload 3's shape.  --head-dim 256: the
+    bf16 forward with d = 256 (fa_fwd_ws) on B = 2, H = 16, N = 8192 (workload 3's B * H * d).
+    Forward only; L2 flushed between the timed forwards."""
     from exact_io_aware_91_b200 import api
 
     w = inputs.workload(args.workload)
-    B, H, N, d = w.B, w.H, w.N, w.d
-    inp8 = inputs.make_qkv_fp8(B, H, N, d, spiky_frac=w.spiky_frac, seed=w.seed + rank)
-    q, k, v = (inp8[n].cuda() for n in ("q", "k", "v"))
+    fp8 = kind == "fp8"
+    B, H, N, d = (w.B, w.H, w.N, w.d) if fp8 else (w.B, w.H * w.d // 256, w.N, 256)
+    fwd_flops = 4.0 * B * H * N * N * d / (2 if w.causal else 1)
+    if fp8:
+        x = inputs.make_qkv_fp8(B, H, N, d, spiky_frac=w.spiky_frac, seed=w.seed + rank)
+        host_in = {n: x[n].view(torch.uint8) for n in ("q", "k", "v")}
+    else:
+        x = inputs.make_qkv(B, H, N, d, dtype=torch.bfloat16, spiky_frac=w.spiky_frac, backward=False,
+                            seed=w.seed + rank)
+        host_in = {n: x[n] for n in ("q", "k", "v")}
+    dev_in = {n: t.cuda() for n, t in host_in.items()}
     o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
-    pr = api.FaAttnProblem(B, H, H, N, d, w.scale, int(w.causal), -1, -1)
-    ws = torch.empty(api.fa_attn_fwd_fp8_workspace_size(pr), dtype=torch.uint8, device="cuda")
+    pr = api.FaAttnProblem(B, H, H, N, d, w.scale if fp8 else 1.0 / 16.0, int(w.causal), -1, -1)
+    ws_bytes = api.fa_attn_fwd_fp8_workspace_size(pr) if fp8 else api.fa_attn_fwd_workspace_size(pr)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > the 126 MB L2
     stream = torch.cuda.current_stream()
 
-    def fwd():
-        api.fa_attn_fwd_fp8(q, k, v, inp8["q_descale"], inp8["k_descale"], inp8["v_descale"], causal=w.causal,
-                            scale=w.scale, o=o, lse=lse, workspace=ws)
+    def compute(din, dout):
+        if fp8:
+            api.fa_attn_fwd_fp8(din["q"].view(torch.float8_e4m3fn), din["k"].view(torch.float8_e4m3fn),
+                                din["v"].view(torch.float8_e4m3fn), x["q_descale"], x["k_descale"], x["v_descale"],
+                                causal=w.causal, scale=pr.scale, o=dout["o"], lse=dout["lse"], workspace=ws)
+        else:
+            api.fa_fwd_ws(din["q"], din["k"], din["v"], causal=w.causal, scale=pr.scale, o=dout["o"],
+                          lse=dout["lse"], workspace=ws)
 
+    dev_out = {"o": o, "lse": lse}
     for _ in range(args.warmup):
-        fwd()
+        compute(dev_in, dev_out)
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks = ClockSampler(torch.cuda.current_device())
@@ -556,7 +567,7 @@ def run_fp8(args, rank: int, world: int) -> None:
     for e0, e1 in ev:
         flush.zero_()  # L2 flushed between timed forwards (outside the events)
         e0.record(stream)
-        fwd()
+        compute(dev_in, dev_out)
         e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -564,21 +575,24 @@ def run_fp8(args, rank: int, world: int) -> None:
     if api.fa_device_status() != api.FA_OK:
         raise RuntimeError("device status not OK after the timed region")
     ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(sum(ms), world)
-    ms_step = total_ms / args.steps
-    value = w.fwd_flops * world / (ms_step * 1e-3) / 1e12
+    ms_step = max_over_ranks(sum(ms), world) / args.steps
+    value = fwd_flops * world / (ms_step * 1e-3) / 1e12
     peaks = load_peaks()
-    bf16_peak, kind = tensor_peak(peaks, clk)
-    peak = 2.0 * bf16_peak  # dense fp8 = 2x dense bf16 (4.5 vs 2.25 PFLOP/s nominal)
-    achieved = w.fwd_flops / (statistics.mean(ms) * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "fwd_fp8", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak,
-                "traffic": args.traffic if args.traffic is not None else recorded_traffic("fwd_fp8", w.name + "_fp8"),
-                "peak_kind": kind.replace("bf16 dense matmul", "bf16 dense matmul x 2 (fp8 / bf16 nominal ratio)")}
+    bf16_peak, peak_kind = tensor_peak(peaks, clk)
+    ratio = 2.0 if fp8 else 1.0  # dense fp8 = 2x dense bf16 (4.5 vs 2.25 PFLOP/s nominal)
+    achieved = fwd_flops / (statistics.mean(ms) * 1e-3) / 1e12
+    name = w.name + "_fp8" if fp8 else f"causal_b{B}_h{H}_n{N}_d256_spiky"
+    dom = "fwd_fp8" if fp8 else "fwd_d256"
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": ratio * bf16_peak,
+                "unit": "TFLOP/s", "frac": achieved / (ratio * bf16_peak),
+                "traffic": args.traffic if args.traffic is not None else recorded_traffic(dom, name),
+                "peak_kind": peak_kind.replace("bf16 dense matmul",
+                                               "bf16 dense matmul x 2 (fp8 / bf16 nominal ratio)" if fp8
+                                               else "bf16 dense matmul")}
 
     e2e = None
     if not args.no_e2e:
-        h_in = {n: inp8[n].view(torch.uint8).pin_memory() for n in ("q", "k", "v")}
+        h_in = {n: t.pin_memory() for n, t in host_in.items()}
         h_out = {"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
                  "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory()}
 
@@ -586,44 +600,49 @@ def run_fp8(args, rank: int, world: int) -> None:
             return ({n: torch.empty_like(t, device="cuda") for n, t in h_in.items()},
                     {n: torch.empty_like(t, device="cuda") for n, t in h_out.items()})
 
-        def compute(din, dout):
-            api.fa_attn_fwd_fp8(din["q"].view(torch.float8_e4m3fn), din["k"].view(torch.float8_e4m3fn),
-                                din["v"].view(torch.float8_e4m3fn), inp8["q_descale"], inp8["k_descale"],
-                                inp8["v_descale"], causal=w.causal, scale=w.scale, o=dout["o"], lse=dout["lse"],
-                                workspace=ws)
-
         e2e = pipelined_e2e(h_in, h_out, make_set, compute, max(4, min(args.steps, 8)), world)
-        e2e = {"value": w.fwd_flops * world / (e2e["ms_per_step"] * 1e-3) / 1e12, "unit": "TFLOPS", **e2e}
+        e2e = {"value": fwd_flops * world / (e2e["ms_per_step"] * 1e-3) / 1e12, "unit": "TFLOPS", **e2e}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        codes = {n: inp8[n].view(torch.uint8).numpy() for n in ("q", "k", "v")}
-        per_head = w.fwd_flops / (B * H)
+        import oracle
+
+        per_head = fwd_flops / (B * H)
         heads, t0 = 0, time.perf_counter()
+        codes = {n: t.numpy() for n, t in host_in.items()} if fp8 else None
         while True:
-            oracle_fp8_head(inp8, codes, w, heads // H % B, heads % H)
+            b, h = heads // H % B, heads % H
+            if fp8:
+                oracle.attention_forward_fp8(codes["q"][b:b + 1, h:h + 1], codes["k"][b:b + 1, h:h + 1],
+                                             codes["v"][b:b + 1, h:h + 1], x["q_descale"], x["k_descale"],
+                                             x["v_descale"], pr.scale, w.causal)
+            else:
+                oracle.attention_forward(x["q"][b, h], x["k"][b, h], x["v"][b, h], pr.scale, w.causal)
             heads += 1
             if time.perf_counter() - t0 > 12.0 or heads >= B * H:
                 break
         dt = time.perf_counter() - t0
+        what = "forward of the dequantized E4M3 inputs" if fp8 else "forward, d = 256"
         cpu = {"value": per_head * heads / dt / 1e12, "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{heads} of {B * H} heads (forward of the dequantized E4M3 inputs, fp64 numpy), {dt:.1f} s"}
+               "sample": f"{heads} of {B * H} heads ({what}, fp64 numpy), {dt:.1f} s"}
 
     if rank == 0:
         line = {
-            "metric": METRIC_FP8, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
-            "config": {"workload": w.name + "_fp8", "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+            "metric": METRIC_FP8 if fp8 else METRIC_D256, "value": value, "unit": "TFLOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
+            "config": {"workload": name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
                        "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
                        "step": "forward only", "l2": "flushed between timed forwards (256 MB write)"},
-            "frac_of_peak": {"measured_burst_x2": value / world / (2.0 * peaks["bf16_tflops"]),
-                             "measured_sustained_x2": value / world / (2.0 * peaks["bf16_tflops_sustained"]),
-                             "datasheet_4500": value / world / 4500.0},
+            "frac_of_peak": {"measured_burst": value / world / (ratio * peaks["bf16_tflops"]),
+                             "measured_sustained": value / world / (ratio * peaks["bf16_tflops_sustained"]),
+                             "datasheet": value / world / (ratio * 2250.0)},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps,  # the persistent forward (its work counter is reset by a memset)
+            # the persistent forward per step (the 8-bit one's work counter is reset by a memset;
+            # the d = 256 one's by the V conversion pass, a second kernel)
+            "gpu_launches": args.steps * (1 if fp8 else 2),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
@@ -644,6 +663,8 @@ def main() -> None:
     ap.add_argument("--window", type=int, default=None,
                     help="sliding-window run: each query sees the previous WINDOW keys and itself "
                          "(fa_attn_fwd / fa_attn_bwd); default no window")
+    ap.add_argument("--head-dim", type=int, default=None, choices=[256],
+                    help="time the bf16 forward with d = 256 (fa_fwd_ws) on B=2, H=16, N=8192")
     ap.add_argument("--fp8", action="store_true",
                     help="time the 8-bit forward (E4M3 inputs, fa_attn_fwd_fp8) on the workload's shape")
     ap.add_argument("--traffic", type=float, default=None,
@@ -656,7 +677,9 @@ def main() -> None:
         if args.impl == "reference":
             run_reference(args, rank, world)
         elif args.fp8:
-            run_fp8(args, rank, world)
+            run_fwd_only(args, rank, world, "fp8")
+        elif args.head_dim == 256:
+            run_fwd_only(args, rank, world, "d256")
         else:
             run_ours(args, rank, world, local)
     finally:

@@ -31,7 +31,8 @@
  *    not synchronise.  Argument errors are detected on the host before anything
  *    is launched; nothing is written then.
  *  - B, H or N equal to 0 is an empty problem: FA_OK, nothing launched.
- *  - Supported: d in {64, 128}; a B200-class GPU (compute capability 10.0).
+ *  - Supported: d in {64, 128}; also d = 256 for the forward with a workspace
+ *    (fa_fwd_ws, fa_attn_fwd); a B200-class GPU (compute capability 10.0).
  *
  * Thread safety: calls may be issued from several host threads; calls whose
  * work overlaps on the GPU must not share output buffers or a workspace.
@@ -58,7 +59,7 @@ typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad scale/causal, H not a multiple of
                              H_kv, workspace too small */
-  FA_ERR_UNSUPPORTED = 2, /* head dim not in {64,128}, sizes beyond limits, not a CC 10.0 device */
+  FA_ERR_UNSUPPORTED = 2, /* head dim not supported by the call, sizes beyond limits, not a CC 10.0 device */
   FA_ERR_MISALIGNED = 3,  /* a tensor base address is not 16-byte aligned (TMA requirement) */
   FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
   FA_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (reported by fa_device_status) */
@@ -116,7 +117,10 @@ FA_API fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o
  * products); calls that overlap on the GPU need separate workspaces.
  *   workspace_bytes : its size.
  * fa_fwd_workspace_size returns 0 for an empty or invalid problem.  Everything else as
- * fa_fwd_gqa.
+ * fa_fwd_gqa, except that d may also be 256 (the head dimension FlashAttention-2 added:
+ * "FlashAttention (EL)", section "FlashAttention-2 (2023)"): a kernel of its own with one
+ * 128-row query tile per work unit, because S and a 256-column O of two tiles do not fit in
+ * tensor memory.  The backward takes d in {64, 128} only.
  */
 FA_API size_t fa_fwd_workspace_size(int B, int H_kv, int N, int d);
 FA_API fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B,
