@@ -42,8 +42,9 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
   constexpr int LPR = D / 8;          // lanes per row
   constexpr int RPW = 32 / LPR;       // rows per warp
   const int lane = threadIdx.x & 31;
-  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const long long row_global = (long long)warp_global * RPW + lane / LPR;  // over BH * Np
+  // 64-bit: B * H * Np rows reach 2^31 at the largest problems (2^24 heads)
+  const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long row_global = warp_global * RPW + lane / LPR;  // over BH * Np
   const int sub = lane % LPR;
   const long long total = (long long)p.BH * p.Np;
   const bool valid_slot = row_global < total;

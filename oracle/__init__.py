@@ -14,6 +14,7 @@ from .attention import (  # noqa: F401
     attention_probs,
     attention_forward,
     attention_forward_rows,
+    attention_backward_dq_rows,
     attention_backward,
     online_softmax_forward,
     loop_attention_forward,

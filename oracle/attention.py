@@ -181,6 +181,26 @@ def attention_forward_rows(q, k, v, scale: float, causal: bool, rows):
     return p @ v, lse
 
 
+def attention_backward_dq_rows(q, k, v, do, scale: float, causal: bool, rows):
+    """dQ of the given query rows of one head, from the definition row by row.
+
+    q, k, v, do: (N, d) for a single head.  A row's dQ depends only on its own probabilities:
+    with P_i = softmax of the row's scaled, masked scores, dP_ij = dO_i . V_j,
+    D_i = sum_j P_ij dP_ij and dS_ij = P_ij (dP_ij - D_i), dQ_i = scale * sum_j dS_ij K_j.
+    Used where the full N x N matrices would not fit in host memory.
+    """
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    rows = np.asarray(rows, dtype=np.int64)
+    s = scale * (q[rows] @ k.T)
+    if causal:
+        j = np.arange(k.shape[0])[None, :]
+        s = np.where(j > rows[:, None], -np.inf, s)
+    p = np.exp(s - _lse_rows(s)[:, None])
+    dp = do[rows] @ v.T
+    delta = (p * dp).sum(axis=1, keepdims=True)
+    return scale * ((p * (dp - delta)) @ k)
+
+
 def attention_backward(q, k, v, do, scale: float, causal: bool, return_delta: bool = False, window=(-1, -1)):
     """Gradients of L = sum(O * dO) with respect to Q, K and V, from the definition.
 

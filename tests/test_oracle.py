@@ -166,6 +166,26 @@ def test_row_sampler_matches_full_forward():
         np.testing.assert_allclose(Lr, L[rows], atol=1e-14)
 
 
+def test_row_dq_matches_full_backward_and_finite_differences():
+    # against the full backward (itself pinned by finite differences below) and, for one row,
+    # directly against central finite differences of sum(O * dO) in that row's query
+    q, k, v, do = randn((40, 8), 31), randn((40, 8), 32), randn((40, 8), 33), randn((40, 8), 34)
+    rows = [0, 1, 13, 38, 39]
+    for causal in (False, True):
+        dq, _, _ = attention_backward(q, k, v, do, 0.4, causal)
+        np.testing.assert_allclose(oracle.attention_backward_dq_rows(q, k, v, do, 0.4, causal, rows), dq[rows],
+                                   atol=1e-13)
+        i, h = 13, 1e-6
+        g = oracle.attention_backward_dq_rows(q, k, v, do, 0.4, causal, [i])[0]
+        num = np.empty(8)
+        for c in range(8):
+            qp, qm = q.copy(), q.copy()
+            qp[i, c] += h
+            qm[i, c] -= h
+            num[c] = (_loss(qp, k, v, do, 0.4, causal) - _loss(qm, k, v, do, 0.4, causal)) / (2 * h)
+        assert np.max(np.abs(num - g)) <= 1e-6 * max(1.0, np.max(np.abs(g)))
+
+
 # ---------------------------------------------------------------- backward
 def _loss(q, k, v, do, scale, causal):
     O, _ = attention_forward(q, k, v, scale, causal)
