@@ -38,10 +38,48 @@ METRIC = "attention fwd/bwd TFLOPS (BF16, causal, N=8k, d=128) & % of B200 tenso
 WORKLOAD = 3  # the metric's workload; --workload picks another one for profiling only
 
 
-def recorded_traffic(kernel: str, workload_name: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
-    import hashlib
+KERNEL_OF = {"fwd": "fa_fwd_persist_sm100_kernel", "fwd_fp8": "fa_fwd_persist_sm100_kernel",
+             "fwd_d256": "fa_fwd_d256_sm100_kernel", "bwd_dkdv": "fa_bwd_dkdv_sm100_kernel",
+             "bwd_dq": "fa_bwd_dq_sm100_kernel"}
+SHARED_HEADERS = ("sm100.cuh", "fa_internal.h")
 
+
+def kernel_source_digest(source: str, kernel_fn: str, text: str | None = None) -> str:
+    """sha256 of what a kernel's code can depend on: its source file with the bodies of the
+    file's OTHER __global__ kernels removed, followed by the shared headers.  A recorded ncu
+    figure stays valid exactly while this digest is unchanged."""
+    import hashlib
+    import re
+
+    csrc = os.path.join(ROOT, "exact_io_aware_91_b200", "csrc")
+    if text is None:
+        with open(os.path.join(csrc, source)) as f:
+            text = f.read()
+    spans = []
+    for mt in re.finditer(r"__global__\s+void\s+(?:__launch_bounds__\([^)]*\)\s*)?(\w+)\s*\(", text):
+        if mt.group(1) == kernel_fn:
+            continue
+        i = text.index("{", mt.end())
+        depth = 0
+        for j in range(i, len(text)):
+            depth += {"{": 1, "}": -1}.get(text[j], 0)
+            if depth == 0:
+                spans.append((i, j + 1))
+                break
+    kept, pos = [], 0
+    for i, j in spans:
+        kept.append(text[pos:i])
+        pos = j
+    kept.append(text[pos:])
+    h = hashlib.sha256("".join(kept).encode())
+    for name in SHARED_HEADERS:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, workload_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's code is unchanged."""
     short = {"causal_b2_h32_n8192_d128_spiky": "causal_b2_h32_n8192_d128",
              "causal_b2_h32_n8192_d128_spiky_fp8": "causal_b2_h32_n8192_d128_fp8",
              "causal_b2_h16_n8192_d256_spiky": "causal_b2_h16_n8192_d256"}.get(workload_name)
@@ -52,12 +90,10 @@ def recorded_traffic(kernel: str, workload_name: str):
         return None
     with open(path) as f:
         rec = json.load(f).get(kernel)
-    if not rec:
+    if not rec or "kernel_sha256" not in rec:
         return None
-    src = os.path.join(ROOT, "exact_io_aware_91_b200", "csrc", rec["source"])
-    with open(src, "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-            return None  # the kernel changed since the counters were taken
+    if kernel_source_digest(rec["source"], KERNEL_OF[kernel]) != rec["kernel_sha256"]:
+        return None  # the kernel (or code it depends on) changed since the counters were taken
     return rec["bytes"]
 
 

@@ -55,3 +55,25 @@ def test_single_rank_needs_no_process_group():
 
     assert bench.max_over_ranks(3.5, 1) == 3.5
     bench.barrier(1)
+
+
+def test_kernel_source_digest_follows_only_its_kernel():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    # a recorded ncu figure is keyed to the code a kernel can depend on: its file without the
+    # other kernels' bodies, plus the shared headers
+    text = ("#include <x>\nconstexpr int k = 1;\n"
+            "template <int D>\n__global__ void __launch_bounds__(384, 1)\n    ka(int a) {\n  if (a) { a = 2; }\n}\n"
+            "__global__ void __launch_bounds__(256) kb(int b) { b = 3; }\n")
+    base_a = bench.kernel_source_digest("bwd_sm100.cu", "ka", text)
+    base_b = bench.kernel_source_digest("bwd_sm100.cu", "kb", text)
+    t_a = text.replace("a = 2", "a = 5")    # change inside ka
+    t_b = text.replace("b = 3", "b = 7")    # change inside kb
+    t_top = text.replace("k = 1", "k = 2")  # change outside both kernels
+    assert bench.kernel_source_digest("bwd_sm100.cu", "ka", t_a) != base_a
+    assert bench.kernel_source_digest("bwd_sm100.cu", "kb", t_a) == base_b
+    assert bench.kernel_source_digest("bwd_sm100.cu", "ka", t_b) == base_a
+    assert bench.kernel_source_digest("bwd_sm100.cu", "kb", t_b) != base_b
+    assert bench.kernel_source_digest("bwd_sm100.cu", "ka", t_top) != base_a
+    assert bench.kernel_source_digest("bwd_sm100.cu", "kb", t_top) != base_b
