@@ -77,3 +77,16 @@ def test_kernel_source_digest_follows_only_its_kernel():
     assert bench.kernel_source_digest("bwd_sm100.cu", "kb", t_b) != base_b
     assert bench.kernel_source_digest("bwd_sm100.cu", "ka", t_top) != base_a
     assert bench.kernel_source_digest("bwd_sm100.cu", "kb", t_top) != base_b
+
+
+def test_roofline_peak_follows_the_sampled_clock():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    peaks = {"bf16_tflops": 1617.9, "bf16_tflops_sustained": 1374.1, "source": "measured"}
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}  # flag, clock not lowered
+    low = {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    none = {"sm_mhz": None, "sm_max_mhz": None, "reasons": []}
+    assert bench.tensor_peak(peaks, full)[0] == 1617.9
+    assert bench.tensor_peak(peaks, low)[0] == 1374.1
+    assert bench.tensor_peak(peaks, none)[0] == 1617.9
