@@ -44,10 +44,20 @@ KERNEL_OF = {"fwd": "fa_fwd_persist_sm100_kernel", "fwd_fp8": "fa_fwd_persist_sm
 SHARED_HEADERS = ("sm100.cuh", "fa_internal.h")
 
 
+def _strip_comments(text: str) -> str:
+    """C++ source without its comments and blank lines (the kernel sources hold no comment
+    markers inside string literals)."""
+    import re
+
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_digest(source: str, kernel_fn: str, text: str | None = None) -> str:
-    """sha256 of what a kernel's code can depend on: its source file with the bodies of the
-    file's OTHER __global__ kernels removed, followed by the shared headers.  A recorded ncu
-    figure stays valid exactly while this digest is unchanged."""
+    """sha256 of the code a kernel can depend on: its source file with the bodies of the
+    file's OTHER __global__ kernels removed, followed by the shared headers, all without
+    comments.  A recorded ncu figure stays valid exactly while this digest is unchanged."""
     import hashlib
     import re
 
@@ -55,6 +65,7 @@ def kernel_source_digest(source: str, kernel_fn: str, text: str | None = None) -
     if text is None:
         with open(os.path.join(csrc, source)) as f:
             text = f.read()
+    text = _strip_comments(text)
     spans = []
     for mt in re.finditer(r"__global__\s+void\s+(?:__launch_bounds__\([^)]*\)\s*)?(\w+)\s*\(", text):
         if mt.group(1) == kernel_fn:
@@ -73,8 +84,8 @@ def kernel_source_digest(source: str, kernel_fn: str, text: str | None = None) -
     kept.append(text[pos:])
     h = hashlib.sha256("".join(kept).encode())
     for name in SHARED_HEADERS:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name)) as f:
+            h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

@@ -8,9 +8,11 @@
 //   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  dQ = scale * dS K,
 //   dK = scale * dS^T Q,  with D_i = rowsum(dO * O)_i from the preprocess.
 //
-// Two kernels, one CTA per 128-row tile, every tensor-core product an
-// M=128, N=128 (or N=d) tcgen05.mma (smaller N runs the tensor core well below
-// its peak on sm_100a).  Warp 0 streams tiles with TMA, warp 1 issues the MMAs
+// Two persistent kernels (one CTA per SM taking 128-row work units from a work counter,
+// heaviest first within groups of heads), every tensor-core product an M=128, N=128 (or
+// N=d) tcgen05.mma (smaller N runs the tensor core well below its peak on sm_100a).
+// Grouped-query heads and the sliding window only change which units and steps exist and
+// which entries are masked.  Warp 0 streams tiles with TMA, warp 1 issues the MMAs
 // (warp-convergent, one elected lane), warps 4-7 and 8-11 are two compute
 // warpgroups that split every step's 128 columns in halves (one thread per TMEM
 // lane = tile row, 64 columns each).

@@ -27,6 +27,13 @@
 //   * the epilogue divides by the row sum, converts to bf16 and TMA-stores O, and
 //     optionally writes the bf16 residual O_fp32 - O_bf16 so that the backward
 //     pass can form rowsum(dO * O) from an fp32-accurate O.
+//
+// Kernels in this file:
+//   fa_fwd_sm100_kernel<d>            one CTA per unit, V converted on chip (fa_fwd, fa_fwd_gqa)
+//   fa_fwd_persist_sm100_kernel<d,F8> persistent, V already fp16 (fa_fwd_ws, fa_attn_fwd); with
+//                                     F8 the E4M3 forward (fa_attn_fwd_fp8)
+//   fa_fwd_d256_sm100_kernel          persistent, head dim 256, one query tile per unit
+//   fa_fwd_v16_kernel                 V bf16 -> fp16 into the workspace (and the work counter reset)
 #include "fa_internal.h"
 #include "sm100.cuh"
 

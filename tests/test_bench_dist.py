@@ -77,6 +77,8 @@ def test_kernel_source_digest_follows_only_its_kernel():
     assert bench.kernel_source_digest("bwd_sm100.cu", "kb", t_b) != base_b
     assert bench.kernel_source_digest("bwd_sm100.cu", "ka", t_top) != base_a
     assert bench.kernel_source_digest("bwd_sm100.cu", "kb", t_top) != base_b
+    t_comment = text.replace("constexpr int k = 1;", "// a comment\nconstexpr int k = 1;  /* another */")
+    assert bench.kernel_source_digest("bwd_sm100.cu", "ka", t_comment) == base_a  # comments do not count
 
 
 def test_roofline_peak_follows_the_sampled_clock():
