@@ -403,8 +403,8 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     from exact_io_aware_91_b200 import api
 
     w = inputs.workload(args.workload)
-    if not w.backward:
-        raise SystemExit("bench.py times forward + backward: pick a workload with a backward pass")
+    if not w.backward:  # a forward-only workload (4): timed by the forward-only runner
+        return run_fwd_only(args, rank, world, "plain")
     dev = torch.device("cuda", torch.cuda.current_device())
     B, H, N, d = w.B, w.H, w.N, w.d
     Hkv = H if args.kv_heads is None else args.kv_heads
@@ -557,6 +557,10 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
                    else "small workload: inputs may stay in L2")},
             "fwd_tflops": fwd_flops / (mean["fwd"] * 1e-3) / 1e12,
             "bwd_tflops": bwd_flops / ((mean["bwd_pre"] + mean["bwd_dkdv"] + mean["bwd_dq"]) * 1e-3) / 1e12,
+            # the products the separate dK/dV and dQ kernels execute: 3.5x the forward's flops
+            # (S and dP are formed in both), against the metric's 2.5x
+            "bwd_executed_tflops": 3.5 * fwd_flops / ((mean["bwd_pre"] + mean["bwd_dkdv"] + mean["bwd_dq"]) * 1e-3)
+                                   / 1e12,
             "kernel_ms": mean,
             "frac_of_peak": {"measured_burst": value / world / peaks["bf16_tflops"],
                              "measured_sustained": value / world / peaks["bf16_tflops_sustained"],
@@ -578,24 +582,32 @@ METRIC_D256 = "attention fwd TFLOPS (BF16, causal, N=8k, d=256) & % of B200 tens
 def run_fwd_only(args, rank: int, world: int, kind: str) -> None:
     """--fp8: the 8-bit forward (fa_attn_fwd_fp8) on workload 3's shape.  --head-dim 256: the
     bf16 forward with d = 256 (fa_fwd_ws) on B = 2, H = 16, N = 8192 (workload 3's B * H * d).
-    Forward only; L2 flushed between the timed forwards."""
+    kind "plain": a forward-only workload (4) on its own shape, whose roofline is the larger
+    of its HBM time and its tensor-core time.  Forward only; L2 flushed between the timed
+    forwards."""
     from exact_io_aware_91_b200 import api
 
     w = inputs.workload(args.workload)
-    fp8 = kind == "fp8"
-    B, H, N, d = (w.B, w.H, w.N, w.d) if fp8 else (w.B, w.H * w.d // 256, w.N, 256)
+    fp8, plain = kind == "fp8", kind == "plain"
+    if fp8 or plain:
+        B, H, N, d = w.B, w.H, w.N, w.d
+    else:
+        B, H, N, d = w.B, w.H * w.d // 256, w.N, 256
+    scale = 1.0 / 16.0 if kind == "d256" else w.scale
     fwd_flops = 4.0 * B * H * N * N * d / (2 if w.causal else 1)
+    # algorithmic bytes: Q, K, V read and O written in bf16 (8-bit inputs: one byte each), LSE
+    fwd_bytes = (3 * (1 if fp8 else 2) + 2) * B * H * N * d + 4 * B * H * N
     if fp8:
         x = inputs.make_qkv_fp8(B, H, N, d, spiky_frac=w.spiky_frac, seed=w.seed + rank)
         host_in = {n: x[n].view(torch.uint8) for n in ("q", "k", "v")}
     else:
-        x = inputs.make_qkv(B, H, N, d, dtype=torch.bfloat16, spiky_frac=w.spiky_frac, backward=False,
-                            seed=w.seed + rank)
+        x = inputs.make_qkv(B, H, N, d, dtype=torch.bfloat16, dist=w.dist, spiky_frac=w.spiky_frac,
+                            backward=False, seed=w.seed + rank)
         host_in = {n: x[n] for n in ("q", "k", "v")}
     dev_in = {n: t.cuda() for n, t in host_in.items()}
     o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
-    pr = api.FaAttnProblem(B, H, H, N, d, w.scale if fp8 else 1.0 / 16.0, int(w.causal), -1, -1)
+    pr = api.FaAttnProblem(B, H, H, N, d, scale, int(w.causal), -1, -1)
     ws_bytes = api.fa_attn_fwd_fp8_workspace_size(pr) if fp8 else api.fa_attn_fwd_workspace_size(pr)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > the 126 MB L2
@@ -636,15 +648,25 @@ def run_fwd_only(args, rank: int, world: int, kind: str) -> None:
     peaks = load_peaks()
     bf16_peak, peak_kind = tensor_peak(peaks, clk)
     ratio = 2.0 if fp8 else 1.0  # dense fp8 = 2x dense bf16 (4.5 vs 2.25 PFLOP/s nominal)
-    achieved = fwd_flops / (statistics.mean(ms) * 1e-3) / 1e12
-    name = w.name + "_fp8" if fp8 else f"causal_b{B}_h{H}_n{N}_d256_spiky"
-    dom = "fwd_fp8" if fp8 else "fwd_d256"
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": ratio * bf16_peak,
-                "unit": "TFLOP/s", "frac": achieved / (ratio * bf16_peak),
-                "traffic": args.traffic if args.traffic is not None else recorded_traffic(dom, name),
-                "peak_kind": peak_kind.replace("bf16 dense matmul",
-                                               "bf16 dense matmul x 2 (fp8 / bf16 nominal ratio)" if fp8
-                                               else "bf16 dense matmul")}
+    mean_s = statistics.mean(ms) * 1e-3
+    achieved = fwd_flops / mean_s / 1e12
+    achieved_gbs = fwd_bytes / mean_s / 1e9
+    name = (w.name + "_fp8" if fp8 else w.name if plain else f"causal_b{B}_h{H}_n{N}_d256_spiky")
+    dom = "fwd_fp8" if fp8 else "fwd" if plain else "fwd_d256"
+    traffic = args.traffic if args.traffic is not None else recorded_traffic(dom, name)
+    # the bound: HBM when moving the algorithmic bytes at the measured copy bandwidth takes longer
+    # than the products at the tensor peak
+    hbm_bound = fwd_bytes / (peaks["hbm_gbs"] * 1e9) > fwd_flops / (ratio * bf16_peak * 1e12)
+    if hbm_bound:
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                    "peak_kind": f"{peaks['source']} copy bandwidth"}
+    else:
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": ratio * bf16_peak,
+                    "unit": "TFLOP/s", "frac": achieved / (ratio * bf16_peak), "traffic": traffic,
+                    "peak_kind": peak_kind.replace("bf16 dense matmul",
+                                                   "bf16 dense matmul x 2 (fp8 / bf16 nominal ratio)" if fp8
+                                                   else "bf16 dense matmul")}
 
     e2e = None
     if not args.no_e2e:
@@ -671,20 +693,22 @@ def run_fwd_only(args, rank: int, world: int, kind: str) -> None:
             if fp8:
                 oracle.attention_forward_fp8(codes["q"][b:b + 1, h:h + 1], codes["k"][b:b + 1, h:h + 1],
                                              codes["v"][b:b + 1, h:h + 1], x["q_descale"], x["k_descale"],
-                                             x["v_descale"], pr.scale, w.causal)
+                                             x["v_descale"], scale, w.causal)
             else:
-                oracle.attention_forward(x["q"][b, h], x["k"][b, h], x["v"][b, h], pr.scale, w.causal)
+                oracle.attention_forward(x["q"][b, h], x["k"][b, h], x["v"][b, h], scale, w.causal)
             heads += 1
             if time.perf_counter() - t0 > 12.0 or heads >= B * H:
                 break
         dt = time.perf_counter() - t0
-        what = "forward of the dequantized E4M3 inputs" if fp8 else "forward, d = 256"
+        what = "forward of the dequantized E4M3 inputs" if fp8 else f"forward, d = {d}"
         cpu = {"value": per_head * heads / dt / 1e12, "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
                "sample": f"{heads} of {B * H} heads ({what}, fp64 numpy), {dt:.1f} s"}
 
     if rank == 0:
         line = {
-            "metric": METRIC_FP8 if fp8 else METRIC_D256, "value": value, "unit": "TFLOPS", "n_gpus": world,
+            "metric": (METRIC_FP8 if fp8 else METRIC_D256 if not plain else
+                       f"attention fwd TFLOPS (BF16, {'causal' if w.causal else 'non-causal'}, N={N}, d={d})"),
+            "value": value, "unit": "TFLOPS", "n_gpus": world, "achieved_gbs": achieved_gbs,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
             "config": {"workload": name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
@@ -712,7 +736,7 @@ def main() -> None:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[2, 3, 5],
+    ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[2, 3, 4, 5],
                     help="workload index (3 = the metric's; others for profiling runs)")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped-query run: K/V with this many heads (fa_fwd_gqa / fa_bwd_gqa); default H")
