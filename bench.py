@@ -568,7 +568,9 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 5 * args.steps,  # V conversion + forward, preprocess, dK/dV, dQ
+            # V conversion + forward, preprocess, dK/dV, dQ; plus the partial-sum reduce when the
+            # library splits a group's query heads (fewer than 4 x 148 dK/dV units, group > 1)
+            "gpu_launches": args.steps * (5 + (1 if H // Hkv > 1 and B * Hkv * ((N + 127) // 128) < 592 else 0)),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
