@@ -275,10 +275,14 @@ def tensor_peak(peaks: dict, clk: dict) -> tuple[float, str]:
     return peaks["bf16_tflops"], f"{peaks['source']} bf16 dense matmul, burst ({why})"
 
 
-def wait_event(ev) -> None:
+def wait_event(ev, limit_s: float = 600.0) -> None:
     """Wait for a recorded CUDA event by polling with short sleeps, which release the GIL, so
-    that the clock-sampling thread keeps running while the GPU works."""
+    that the clock-sampling thread keeps running while the GPU works; give up with an error
+    after limit_s seconds (the timed regions take well under a second)."""
+    t0 = time.monotonic()
     while not ev.query():
+        if time.monotonic() - t0 > limit_s:
+            raise RuntimeError(f"timed region did not complete within {limit_s:.0f} s")
         time.sleep(0.0005)
 
 

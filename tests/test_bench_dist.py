@@ -92,3 +92,26 @@ def test_roofline_peak_follows_the_sampled_clock():
     assert bench.tensor_peak(peaks, full)[0] == 1617.9
     assert bench.tensor_peak(peaks, low)[0] == 1374.1
     assert bench.tensor_peak(peaks, none)[0] == 1617.9
+
+
+def test_wait_event_polls_until_done_and_gives_up():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Ev:  # stands in for a CUDA event: completes on the third query
+        n = 0
+
+        def query(self):
+            self.n += 1
+            return self.n >= 3
+
+    ev = Ev()
+    bench.wait_event(ev)
+    assert ev.n == 3
+
+    class Never:
+        def query(self):
+            return False
+
+    with pytest.raises(RuntimeError):
+        bench.wait_event(Never(), limit_s=0.01)
