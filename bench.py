@@ -361,17 +361,30 @@ def blas_threads() -> int:
 
 
 def cpu_baseline(w: inputs.Workload, inp_cpu: dict, budget_s: float = 12.0) -> dict:
-    """The oracle, as it stands, on whole heads of the workload until ~budget_s of CPU work."""
-    per_head = (w.fwd_flops + w.bwd_flops) / (w.B * w.H)
+    """The oracle, as it stands, on whole heads of the workload until ~budget_s of CPU work.
+    Sequences too long for the oracle's N x N matrices (N > 16384) are sampled the way their
+    parity test checks them: the 4096-token causal prefix problem of a head, forward and
+    backward."""
+    import oracle
+
+    P = 4096 if w.N > 16384 else w.N
+    per_head = (w.fwd_flops + w.bwd_flops) / (w.B * w.H) * (P / w.N) ** 2
     heads, t0 = 0, time.perf_counter()
     while True:
-        oracle_head_step(inp_cpu, w, heads // w.H % w.B, heads % w.H)
+        b, h = heads // w.H % w.B, heads % w.H
+        if P == w.N:
+            oracle_head_step(inp_cpu, w, b, h)
+        else:
+            q, k, v, do = (inp_cpu[n][b, h, :P] for n in ("q", "k", "v", "do"))
+            oracle.attention_forward(q, k, v, w.scale, w.causal)
+            oracle.attention_backward(q, k, v, do, w.scale, w.causal)
         heads += 1
         if time.perf_counter() - t0 > budget_s or heads >= w.B * w.H:
             break
     dt = time.perf_counter() - t0
+    what = "heads" if P == w.N else f"heads' {P}-token prefix problems"
     return {"value": per_head * heads / dt / 1e12, "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{heads} of {w.B * w.H} heads (fwd+bwd, fp64 numpy, S and P materialised), {dt:.1f} s"}
+            "sample": f"{heads} of {w.B * w.H} {what} (fwd+bwd, fp64 numpy, S and P materialised), {dt:.1f} s"}
 
 
 def run_reference(args, rank: int, world: int) -> None:
@@ -444,7 +457,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     # forward with a workspace: V converted to fp16 in one streaming pass, then the kernel
     fws = torch.empty(api.fa_fwd_workspace_size(B, Hkv, N, d), dtype=torch.uint8, device=dev)
     if args.window is None:
-        bwd_call = api.fa_bwd if Hkv == H else api.fa_bwd_gqa
+        bwd_call = api.fa_bwd_gqa  # the backward that takes the forward's residual
 
         def fwd_call(q, k, v, **kw):
             return api.fa_fwd_ws(q, k, v, workspace=fws, **kw)
@@ -463,7 +476,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    if api.fa_device_status() != api.FA_OK:
+    if api.fa_last_device_status() != api.FA_OK:
         raise RuntimeError("device status not OK after warm-up")
 
     # ---- timed region: K steps, per-kernel events on the launching stream
@@ -492,7 +505,7 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     clk = clocks.stop()
     total_ms = start.elapsed_time(end)
     total_ms_max = max_over_ranks(total_ms, world)
-    if api.fa_device_status() != api.FA_OK:
+    if api.fa_last_device_status() != api.FA_OK:
         raise RuntimeError("device status not OK after the timed region")
 
     phase = {"fwd": [], "bwd_pre": [], "bwd_dkdv": [], "bwd_dq": []}
@@ -572,9 +585,9 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            # V conversion + forward, preprocess, dK/dV, dQ; plus the partial-sum reduce when the
-            # library splits a group's query heads (fewer than 4 x 148 dK/dV units, group > 1)
-            "gpu_launches": args.steps * (5 + (1 if H // Hkv > 1 and B * Hkv * ((N + 127) // 128) < 592 else 0)),
+            # V pass + its fix-up + forward, preprocess + its fix-up, dK/dV, dQ; plus the partial-sum
+            # reduce when the library splits a group's query heads (fewer than 4 x 148 dK/dV units)
+            "gpu_launches": args.steps * (7 + (1 if H // Hkv > 1 and B * Hkv * ((N + 127) // 128) < 592 else 0)),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
@@ -646,7 +659,7 @@ def run_fwd_only(args, rank: int, world: int, kind: str) -> None:
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
-    if api.fa_device_status() != api.FA_OK:
+    if api.fa_last_device_status() != api.FA_OK:
         raise RuntimeError("device status not OK after the timed region")
     ms = [a.elapsed_time(b) for a, b in ev]
     ms_step = max_over_ranks(sum(ms), world) / args.steps
@@ -727,8 +740,8 @@ def run_fwd_only(args, rank: int, world: int, kind: str) -> None:
             "cpu_baseline": cpu,
             "e2e": e2e,
             # the persistent forward per step (the 8-bit one's work counter is reset by a memset;
-            # the d = 256 one's by the V conversion pass, a second kernel)
-            "gpu_launches": args.steps * (1 if fp8 else 2),
+            # the bf16 ones follow the V pass and its fix-up)
+            "gpu_launches": args.steps * (1 if fp8 else 3),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)

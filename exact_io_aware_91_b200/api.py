@@ -22,10 +22,12 @@ FA_ERR_UNSUPPORTED = 2
 FA_ERR_MISALIGNED = 3
 FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
+FA_ERR_RANGE = 6
 
 EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_workspace_size", "fa_fwd_ws", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_gqa_workspace_size",
            "fa_bwd_gqa", "fa_attn_fwd_workspace_size", "fa_attn_fwd", "fa_attn_bwd_workspace_size", "fa_attn_bwd",
-           "fa_attn_fwd_fp8_workspace_size", "fa_attn_fwd_fp8", "fa_bwd_noalloc", "fa_device_status", "fa_bwd_set_phase_events", "fa_selftest_wait_timeout",
+           "fa_attn_fwd_fp8_workspace_size", "fa_attn_fwd_fp8", "fa_bwd_noalloc", "fa_last_device_status",
+           "fa_device_status", "fa_bwd_set_phase_events", "fa_selftest_wait_timeout", "fa_selftest_exp2",
            "fa_status_str")
 
 # Size of the scratch array fa_bwd_noalloc uses instead of a caller workspace.
@@ -61,7 +63,7 @@ def library() -> ctypes.CDLL:
         )
     lib = ctypes.CDLL(path)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_fwd.restype = i
     lib.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     lib.fa_fwd_gqa.restype = i
@@ -73,7 +75,7 @@ def library() -> ctypes.CDLL:
     lib.fa_fwd_f32.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd_workspace_size.restype = sz
-    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp]
     lib.fa_bwd.restype = i
     lib.fa_bwd_gqa_workspace_size.argtypes = [i, i, i, i, i]
     lib.fa_bwd_gqa_workspace_size.restype = sz
@@ -96,6 +98,10 @@ def library() -> ctypes.CDLL:
     lib.fa_bwd_noalloc.restype = i
     lib.fa_selftest_wait_timeout.argtypes = [vp]
     lib.fa_selftest_wait_timeout.restype = i
+    lib.fa_selftest_exp2.argtypes = [vp, vp, i, vp]
+    lib.fa_selftest_exp2.restype = i
+    lib.fa_last_device_status.argtypes = [vp]
+    lib.fa_last_device_status.restype = i
     lib.fa_device_status.argtypes = [vp]
     lib.fa_device_status.restype = i
     lib.fa_bwd_set_phase_events.argtypes = [vp]
@@ -141,29 +147,23 @@ def _scale(scale, d: int) -> float:
 
 
 def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, scale: float | None = None,
-           o: torch.Tensor | None = None, lse: torch.Tensor | None = None, o_resid: torch.Tensor | None = None,
-           save_residual: bool = False, stream=None):
-    """Attention forward on bf16 (B, H, N, d) CUDA tensors.
+           o: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """Attention forward on bf16 (B, H, N, d) CUDA tensors (C ``fa_fwd``).  Returns (o, lse).
 
-    Returns (o, lse), or (o, lse, o_resid) when ``save_residual`` (or ``o_resid``) is
-    given: the bf16 residual of O's final rounding, to be passed to ``fa_bwd``.
-    """
+    The residual a training forward can hand to the backward is written by ``fa_fwd_gqa``,
+    ``fa_fwd_ws`` and ``fa_attn_fwd`` (``save_residual=True``)."""
     B, H, N, d = _shape(q)
     _same(q, k, v, dtype=torch.bfloat16, shape=(B, H, N, d))
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if o_resid is None and save_residual:
-        o_resid = torch.empty_like(q)
     _same(o, dtype=torch.bfloat16, shape=(B, H, N, d))
-    if o_resid is not None:
-        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
-    st = library().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                          None if o_resid is None else o_resid.data_ptr(), B, H, N, d, _scale(scale, d),
-                          int(bool(causal)), _stream_handle(stream))
+    _same(lse, dtype=torch.float32, shape=(B, H, N))
+    st = library().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N, d,
+                          _scale(scale, d), int(bool(causal)), _stream_handle(stream))
     _check("fa_fwd", st)
-    return (o, lse) if o_resid is None else (o, lse, o_resid)
+    return o, lse
 
 
 def _gqa_heads(q: torch.Tensor, k: torch.Tensor) -> int:
@@ -250,28 +250,27 @@ def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 
 
 def fa_bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,
-           dq=None, dk=None, dv=None, o_resid=None, stream=None):
-    """dQ, dK, dV (fp32) of sum(O * dO). ``o_resid``: the forward's residual (recommended).
-
-    Returns (dq, dk, dv)."""
+           dq=None, dk=None, dv=None, stream=None):
+    """dQ, dK, dV (fp32) of sum(O * dO) (C ``fa_bwd``; rowsum(dO * O) from the bf16 O --
+    ``fa_bwd_gqa`` / ``fa_attn_bwd`` take the forward's residual).  Returns (dq, dk, dv)."""
     B, H, N, d = _shape(q)
     _same(q, k, v, o, do, dtype=torch.bfloat16, shape=(B, H, N, d))
     _same(lse, dtype=torch.float32, shape=(B, H, N))
-    if o_resid is not None:
-        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
     if dq is None:
         dq = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
     if dk is None:
         dk = torch.empty_like(dq)
     if dv is None:
         dv = torch.empty_like(dq)
+    _same(dq, dk, dv, dtype=torch.float32, shape=(B, H, N, d))
     ws_bytes = fa_bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
-    st = library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                          None if o_resid is None else o_resid.data_ptr(), do.data_ptr(), lse.data_ptr(),
+    if workspace.numel() < ws_bytes:  # the C call trusts the size (its signature carries none)
+        raise ValueError(f"workspace of {workspace.numel()} bytes, fa_bwd needs {ws_bytes}")
+    st = library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, _scale(scale, d),
-                          int(bool(causal)), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+                          int(bool(causal)), workspace.data_ptr(), _stream_handle(stream))
     _check("fa_bwd", st)
     return dq, dk, dv
 
@@ -432,8 +431,24 @@ def fa_selftest_wait_timeout(stream=None) -> None:
     _check("fa_selftest_wait_timeout", library().fa_selftest_wait_timeout(_stream_handle(stream)))
 
 
+def fa_selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The FMA-pipe exponential of the softmax kernels applied to a 1-D fp32 CUDA tensor."""
+    if x.dtype != torch.float32 or x.dim() != 1 or not x.is_contiguous() or not x.is_cuda:
+        raise ValueError("expected a contiguous 1-D fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    _check("fa_selftest_exp2", library().fa_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(),
+                                                          _stream_handle(stream)))
+    return y
+
+
+def fa_last_device_status(stream=None) -> int:
+    """Synchronise and return (and clear) the device status code: FA_OK, FA_ERR_TIMEOUT,
+    FA_ERR_RANGE or FA_ERR_CUDA."""
+    return int(library().fa_last_device_status(_stream_handle(stream)))
+
+
 def fa_device_status(stream=None) -> int:
-    """Synchronise and return the device status code (FA_OK, FA_ERR_TIMEOUT or FA_ERR_CUDA)."""
+    """``fa_last_device_status`` under its earlier name."""
     return int(library().fa_device_status(_stream_handle(stream)))
 
 

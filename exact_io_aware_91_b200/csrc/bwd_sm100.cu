@@ -25,8 +25,10 @@
 //   * dQ kernel (128 queries per CTA, Q and dO resident; 128-key steps, three K
 //     buffers and two V buffers): S double-buffered in TMEM; order per step j:
 //     dQ(j) += dS(j) K_j, dP(j+1), S(j+2).
-// All products run in fp16 (exact copies of the bf16 inputs made by the
-// preprocess) with fp32 accumulation; gradients are written in fp32.
+// All products run in fp16 with fp32 accumulation on copies of the bf16 inputs made by the
+// preprocess, each exactly the input times a power of two 2^e chosen per tensor (e = 0 in
+// the common case; see bwd_pre.cu); the kernels read the exponents, fold those of Q and K
+// into the softmax scale and undo the others in the epilogues.  Gradients are fp32.
 #include <type_traits>
 
 #include "fa_internal.h"
@@ -94,19 +96,34 @@ __device__ __forceinline__ void issue_ts_split_part(uint32_t d_tmem, uint32_t a_
   }
 }
 
+// 2^E as a product of two floats, each a power of two within the normal range, so that
+// x * mult * f.a * f.b scales x by mult * 2^E exactly (up to the final rounding) for the
+// exponent sums of the copies (|E| <= 252); both are 1 in the common case E = 0.
+struct Pow2 {
+  float a, b;
+};
+__device__ __forceinline__ Pow2 pow2_factors(int E) {
+  const int e1 = E < -126 ? -126 : (E > 126 ? 126 : E);
+  int e2 = E - e1;
+  e2 = e2 < -126 ? -126 : (e2 > 126 ? 126 : e2);
+  return Pow2{__int_as_float((e1 + 127) << 23), __int_as_float((e2 + 127) << 23)};
+}
+
 // Coalesced store of a warp's rows: lane l holds NC fp32 values of row `row0 + l` (times
-// `mult`) to be written at dst_base + (row0 + l) * ld (in floats); see warp_store_rows_128b.
+// `mult` and the factors f) to be written at dst_base + (row0 + l) * ld (in floats); see
+// warp_store_rows_128b.
 template <int NC>
 __device__ __forceinline__ void warp_store_rows_f32(const float (&v)[NC], float* dst_base, size_t ld, int row0,
-                                                    int n_rows, float mult) {
+                                                    int n_rows, float mult, Pow2 f) {
   static_assert(NC % 32 == 0, "32-column chunks");
+  auto sc = [&](float x) { return __float_as_uint(x * mult * f.a * f.b); };
 #pragma unroll
   for (int ch = 0; ch < NC / 32; ++ch) {
     uint4 a[8];
 #pragma unroll
     for (int m = 0; m < 8; ++m)
-      a[m] = make_uint4(__float_as_uint(v[32 * ch + 4 * m] * mult), __float_as_uint(v[32 * ch + 4 * m + 1] * mult),
-                        __float_as_uint(v[32 * ch + 4 * m + 2] * mult), __float_as_uint(v[32 * ch + 4 * m + 3] * mult));
+      a[m] = make_uint4(sc(v[32 * ch + 4 * m]), sc(v[32 * ch + 4 * m + 1]), sc(v[32 * ch + 4 * m + 2]),
+                        sc(v[32 * ch + 4 * m + 3]));
     warp_store_rows_128b(a, reinterpret_cast<uint8_t*>(dst_base + 32 * ch), ld * sizeof(float), row0, n_rows);
   }
 }
@@ -387,7 +404,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + L::T_S + 64 * w;
     const uint32_t tDP = tmem + lane_off + L::T_DP + 64 * w;
-    const float sl2 = p.scale_log2;
+    // the copies are Q 2^eq, K 2^ek, V 2^ev, dO 2^edo: S^T carries 2^(eq+ek), dP^T and D (and so
+    // the fp16 dS^T) 2^(ev+edo), dV's accumulator 2^edo, dK's 2^(ev+edo+eq)
+    const float sl2 = ldexpf(p.scale_log2, -(p.exps[kExpQ] + p.exps[kExpK]));
     const uint64_t sl2x2 = f2pack(sl2, sl2);
     bool ok = true;
     int T0 = 0;
@@ -506,6 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // warpgroup 0 writes dV, warpgroup 1 writes scale * dK (rows past N are padding), 64
       // columns at a time; once the last columns are loaded the next unit may overwrite them
       const uint32_t t_acc = tmem + lane_off + (w == 0 ? L::T_DV : L::T_DK);
+      const Pow2 out_f = pow2_factors(w == 0 ? -p.exps[kExpDO] : -(p.exps[kExpV] + p.exps[kExpDO] + p.exps[kExpQ]));
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         float acc[64];
@@ -514,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(bar(L::BAR_ACC_FREE));
         }
-        warp_store_rows_f32<64>(acc, out + 64 * c, D, j * 128 + wq * 32, p.N, w == 0 ? 1.0f : p.scale);
+        warp_store_rows_f32<64>(acc, out + 64 * c, D, j * 128 + wq * 32, p.N, w == 0 ? 1.0f : p.scale, out_f);
       }
       T0 += n_it;
       u = next_unit(uc + 1, ok);
@@ -782,7 +802,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = (warp - 4) & 3;
     const int row = wq * 32 + lane;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const float sl2 = p.scale_log2;
+    // copies Q 2^eq, K 2^ek, V 2^ev, dO 2^edo: S carries 2^(eq+ek), dP and D (and the fp16 dS)
+    // 2^(ev+edo), dQ's accumulator 2^(ev+edo+ek)
+    const float sl2 = ldexpf(p.scale_log2, -(p.exps[kExpQ] + p.exps[kExpK]));
     const uint64_t sl2x2 = f2pack(sl2, sl2);
     bool ok = true;
     int T0 = 0;
@@ -885,8 +907,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         delta = p.delta[prow];
       }
       // this warp's 32 query rows, columns [w D/2, (w + 1) D/2) of scale * dQ
+      const Pow2 out_f = pow2_factors(-(p.exps[kExpV] + p.exps[kExpDO] + p.exps[kExpK]));
       warp_store_rows_f32<D / 2>(acc, p.dq + (size_t)x.bh * p.N * D + w * (D / 2), D, x.qt * 128 + wq * 32, p.N,
-                                 p.scale);
+                                 p.scale, out_f);
       T0 += x.n_it;
       u = u_next;
     }

@@ -92,11 +92,28 @@ bool window_ok(int wl, int wr) { return wl >= -1 && wr >= -1; }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Forward workspace: the fp16 copy of V, then a 256-byte control block (the persistent
+// kernel's work counter at 0, the copy's exponent at 4), then the V pass's per-block maxima.
+struct FwdLayout {
+  size_t off_ctrl, off_amax, total;
+};
+FwdLayout fwd_layout(int B, int H_kv, int N, int d) {
+  FwdLayout w{};
+  w.off_ctrl = align256((size_t)B * H_kv * N * d * 2);
+  w.off_amax = w.off_ctrl + 256;
+  w.total = w.off_amax + align256(sizeof(uint32_t) * kVPassBlocks);
+  return w;
+}
+
 struct BwdLayout {
-  size_t off_q16, off_k16, off_v16, off_do16, off_delta, off_lse2, off_dk_part, off_dv_part, off_counters, total;
+  size_t off_q16, off_k16, off_v16, off_do16, off_delta, off_lse2, off_dk_part, off_dv_part, off_ctrl, off_amax,
+      total;
   int Np;
   int kv_split;
 };
+// The 256-byte control block of the backward workspace: the persistent kernels' work
+// counters, then the exponents of the Q, K, V, dO copies.
+constexpr size_t kCtrlCounters = 0, kCtrlExps = 16;
 
 // Grouped-query attention with few key/value heads leaves the dK/dV kernel (one CTA per
 // key/value head and key tile) with too few, very unequal CTAs: then each group's query
@@ -113,8 +130,9 @@ int kv_split_for(int B, int H, int H_kv, int N) {
 
 // Workspace: fp16 copies of Q and dO (B*H heads) and of K and V (B*H_kv heads), then
 // D and LSE*log2(e) per query row padded to a multiple of 128 rows, then (only when the
-// group is split, see kv_split_for) fp32 partial dK and dV per split, then 256 bytes for the
-// work counters of the persistent kernels.
+// group is split, see kv_split_for) fp32 partial dK and dV per split, then a 256-byte control
+// block (work counters of the persistent kernels, exponents of the copies), then the
+// preprocess's per-block maxima of |Q|, |K|, |V|, |dO|.
 BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d) {
   BwdLayout w{};
   w.kv_split = kv_split_for(B, H, H_kv, N);
@@ -131,8 +149,9 @@ BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d) {
   w.off_dk_part = w.off_lse2 + rows;
   const size_t part = w.kv_split > 1 ? align256((size_t)w.kv_split * B * H_kv * N * d * 4) : 0;
   w.off_dv_part = w.off_dk_part + part;
-  w.off_counters = w.off_dv_part + part;
-  w.total = w.off_counters + 256;
+  w.off_ctrl = w.off_dv_part + part;
+  w.off_amax = w.off_ctrl + 256;
+  w.total = w.off_amax + align256(4 * sizeof(uint32_t) * kPreBlocks);
   return w;
 }
 
@@ -172,13 +191,14 @@ const char* fa_status_str(fa_status s) {
     case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_RANGE: return "FA_ERR_RANGE";
   }
   return "FA_ERR_UNKNOWN";
 }
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
-                 int N, int d, float scale, int causal, fa_stream_t stream) {
-  return fa_fwd_gqa(q, k, v, o, lse, o_resid, B, H, H, N, d, scale, causal, stream);
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, fa_stream_t stream) {
+  return fa_fwd_gqa(q, k, v, o, lse, nullptr, B, H, H, N, d, scale, causal, stream);
 }
 
 namespace {
@@ -195,15 +215,18 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
       !aligned(o_resid, 16) || !aligned(workspace, 256))
     return FA_ERR_MISALIGNED;
-  const size_t v16_bytes = align256((size_t)B * H_kv * N * d * 2);
-  if (workspace != nullptr && workspace_bytes < v16_bytes + 256) return FA_ERR_INVALID_ARG;
+  const FwdLayout fl = fwd_layout(B, H_kv, N, d);
+  if (workspace != nullptr && workspace_bytes < fl.total) return FA_ERR_INVALID_ARG;
   int dev = 0;
   if ((st = device_setup(&dev)) != FA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int BH = B * H, BH_kv = B * H_kv;
-  unsigned* counter = workspace != nullptr ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + v16_bytes)
-                                           : nullptr;
-  if (workspace != nullptr && launch_fwd_v16(v, workspace, (long long)BH_kv * N * d, counter, s) != cudaSuccess)
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  unsigned* counter = workspace != nullptr ? reinterpret_cast<unsigned*>(wsb + fl.off_ctrl) : nullptr;
+  int* v_exp = workspace != nullptr ? reinterpret_cast<int*>(wsb + fl.off_ctrl + 4) : nullptr;
+  if (workspace != nullptr &&
+      launch_fwd_v16(v, workspace, (long long)BH_kv * N * d, counter, reinterpret_cast<uint32_t*>(wsb + fl.off_amax),
+                     v_exp, g_err_ptr[dev], s) != cudaSuccess)
     return FA_ERR_CUDA;
   CUtensorMap tq, tk, tv, to;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -234,6 +257,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   p.head_group = head_group_size(BH, 4ull * N * d / (H / H_kv), kFwdGroupBytes);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out_scale = 1.0f;
+  p.v_exp = v_exp;  // the V copy's exponent (persistent kernels); the on-chip kernel scales per tile
   p.causal = causal;
   p.win_left = wl;
   p.win_right = wr;
@@ -255,7 +279,7 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float
 size_t fa_fwd_workspace_size(int B, int H_kv, int N, int d) {
   bool empty = false;
   if (check_problem(B, H_kv, H_kv, N, d, 1.0f, 0, &empty, true) != FA_OK || empty) return 0;
-  return align256((size_t)B * H_kv * N * d * 2) + 256;  // fp16 V, then the work counter
+  return fwd_layout(B, H_kv, N, d).total;  // fp16 V, control block, per-block maxima
 }
 
 fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B, int H,
@@ -294,11 +318,12 @@ size_t fa_bwd_gqa_workspace_size(int B, int H, int H_kv, int N, int d) {
   return bwd_layout(B, H, H_kv, N, d).total;
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* o_resid, const void* dout,
-                 const float* lse, float* dq, float* dk, float* dv, int B, int H, int N, int d, float scale,
-                 int causal, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  return fa_bwd_gqa(q, k, v, o, o_resid, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, workspace,
-                    workspace_bytes, stream);
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 float* dq, float* dk, float* dv, int B, int H, int N, int d, float scale, int causal,
+                 void* workspace, fa_stream_t stream) {
+  // the caller provides at least fa_bwd_workspace_size(B, H, N, d) bytes (the signature carries no size)
+  return fa_bwd_gqa(q, k, v, o, nullptr, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, workspace,
+                    fa_bwd_workspace_size(B, H, N, d), stream);
 }
 
 namespace {
@@ -355,7 +380,10 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   pp.Np = w.Np;
   pp.BH = BH;
   pp.BH_kv = BH_kv;
-  pp.counters = reinterpret_cast<unsigned*>(ws + w.off_counters);
+  pp.counters = reinterpret_cast<unsigned*>(ws + w.off_ctrl + kCtrlCounters);
+  pp.amax_part = reinterpret_cast<uint32_t*>(ws + w.off_amax);
+  pp.exps = reinterpret_cast<int*>(ws + w.off_ctrl + kCtrlExps);
+  pp.err = g_err_ptr[dev];
   pp.d = d;
   if (launch_bwd_pre(pp, s) != cudaSuccess) return FA_ERR_CUDA;
   if (t_phase_events != nullptr && t_phase_events[0] != nullptr &&
@@ -372,6 +400,7 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   BwdParams bp{};
   bp.delta = pp.delta;
   bp.lse2 = pp.lse2;
+  bp.exps = pp.exps;
   bp.dq = dq;
   bp.dk = dk;
   bp.dv = dv;
@@ -506,7 +535,18 @@ fa_status fa_selftest_wait_timeout(fa_stream_t stream) {
                                                                                                       : FA_ERR_CUDA;
 }
 
-fa_status fa_device_status(fa_stream_t stream) {
+fa_status fa_selftest_exp2(const float* x, float* y, int n, fa_stream_t stream) {
+  if (n < 0) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (x == nullptr || y == nullptr) return FA_ERR_INVALID_ARG;
+  if (!aligned(x, 4) || !aligned(y, 4)) return FA_ERR_MISALIGNED;
+  int dev = 0;
+  const fa_status st = device_setup(&dev);
+  if (st != FA_OK) return st;
+  return launch_selftest_exp2(x, y, n, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_last_device_status(fa_stream_t stream) {
   int dev = 0;
   fa_status st = device_setup(&dev);
   if (st != FA_OK) return st;
@@ -516,9 +556,11 @@ fa_status fa_device_status(fa_stream_t stream) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_fa_err_word, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
-    return FA_ERR_TIMEOUT;
+    return v == FA_ERR_RANGE ? FA_ERR_RANGE : FA_ERR_TIMEOUT;
   }
   return FA_OK;
 }
+
+fa_status fa_device_status(fa_stream_t stream) { return fa_last_device_status(stream); }
 
 }  // extern "C"

@@ -21,6 +21,7 @@ struct FwdParams {
   int head_group;    // heads per group in the CTA order (unit_order)
   float scale_log2;  // softmax scale * log2(e) (times the Q and K descales for 8-bit inputs)
   float out_scale;   // factor on O / l: 1, or the V descale for 8-bit inputs
+  const int* v_exp;  // persistent kernels: exponent e of the fp16 V copy (V16 = V * 2^e), or null (0)
   int causal;
   int win_left, win_right;  // sliding window: query i sees keys i - left .. i + right (-1 unbounded)
   int* err;          // device error word
@@ -48,6 +49,21 @@ __host__ __device__ __forceinline__ int query_hi(int k, int N, int wl) {
 
 constexpr int kNumCounters = 2;  // work counters: [0] dQ kernel, [1] dK/dV kernel
 
+// Streaming passes that make fp16 copies (the forward's V pass, the backward preprocess)
+// run on a fixed grid and leave one partial maximum |x| per block and tensor (float bits);
+// the fix-up kernel that follows reduces them and picks each copy's exponent.
+constexpr int kVPassBlocks = 148 * 16;  // forward V pass
+constexpr int kPreBlocks = 148 * 8;     // backward preprocess
+constexpr int kFixupBlocks = 148 * 4;   // fix-up kernels (re-conversion only when a copy needs 2^e != 1)
+// Copy exponents (see copy_exponent): a copy keeps e = 0 while its tensor's largest
+// magnitude lies in [2^kCopyLoLog2, 2^kCopyHiLog2].
+constexpr int kCopyLoLog2 = -4;
+constexpr int kCopyHiLog2 = 15;
+// The backward's dS = P * (dP - D) is packed to fp16 unscaled in the units of the dO and V
+// copies: |dS| <= 2 d max|dO| max|V| must stay <= 2^15 there.
+constexpr float kDsBound = 32768.0f;
+enum { kExpQ = 0, kExpK = 1, kExpV = 2, kExpDO = 3 };  // slots of the backward's exponent table
+
 struct BwdPreParams {
   const void* q;     // bf16 (BH, N, d)
   const void* k;
@@ -60,16 +76,20 @@ struct BwdPreParams {
   void* k16;
   void* v16;
   void* do16;
-  float* delta;      // (BH, Np): rowsum(dO * O); 0 on padded rows
+  float* delta;      // (BH, Np): rowsum(dO * O) (times 2^(e_V + e_dO) after the fix-up); 0 on padded rows
   float* lse2;       // (BH, Np): LSE * log2(e); +inf on padded rows
   int N, Np, BH, d;
   int BH_kv;         // B * H_kv: rows of k / v / k16 / v16 (<= BH)
   unsigned* counters;  // work counters of the persistent kernels, zeroed here (kNumCounters)
+  uint32_t* amax_part; // [4][kPreBlocks] partial max |x| (float bits) of Q, K, V, dO per block
+  int* exps;         // [4] exponents of the Q, K, V, dO copies (written by the fix-up)
+  int* err;          // device error word
 };
 
 struct BwdParams {
-  const float* delta;  // (BH, Np)
+  const float* delta;  // (BH, Np), in the units of the dO and V copies
   const float* lse2;   // (BH, Np)
+  const int* exps;     // [4] exponents of the Q, K, V, dO copies (kExpQ ...)
   float* dq;           // fp32 (BH, N, d)
   float* dk;
   float* dv;
@@ -109,7 +129,10 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int 
 
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t s);
-cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, cudaStream_t s);
+// V pass of the workspace forward: V -> fp16 copy (exponent 0) with per-block maxima, then the
+// fix-up that picks the copy's exponent (v_exp) and re-converts V if it is not 0.
+cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, uint32_t* amax_part,
+                           int* v_exp, int* err, cudaStream_t s);
 cudaError_t launch_fwd_persist_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                      const FwdParams& p, int d, cudaStream_t s);
 cudaError_t launch_fwd_d256_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -117,10 +140,13 @@ cudaError_t launch_fwd_d256_sm100(const CUtensorMap& tq, const CUtensorMap& tk, 
 cudaError_t launch_fwd_persist_fp8_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                          const FwdParams& p, cudaStream_t s);  // d = 128, E4M3 inputs
 cudaError_t launch_selftest_wait(int* err, cudaStream_t s);
+cudaError_t launch_selftest_exp2(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_bwd_kv_reduce(const float* dk_part, const float* dv_part, float* dk, float* dv,
                                  long long elems, int splits, cudaStream_t s);
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int BH, int N,
                            int d, float scale, int causal, cudaStream_t s);
+// Backward preprocess (D, LSE * log2(e), fp16 copies with exponent 0, per-block maxima), then
+// the fix-up that picks the copies' exponents, re-converts where they are not 0 and scales D.
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t s);
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                                   const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s);

@@ -34,6 +34,7 @@
 //                                     F8 the E4M3 forward (fa_attn_fwd_fp8)
 //   fa_fwd_d256_sm100_kernel          persistent, head dim 256, one query tile per unit
 //   fa_fwd_v16_kernel                 V bf16 -> fp16 into the workspace (and the work counter reset)
+//   fa_fwd_v16_fixup_kernel           the V copy's exponent (re-conversion when it is not 0)
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -53,7 +54,7 @@ struct FwdLayout {
   static constexpr int OFF_KV = 2 * TILE;
   static constexpr int OFF_BAR = OFF_KV + STAGES * TILE;
   // barriers: q_full, kv_full[STAGES], kv_empty[STAGES], v_conv[STAGES], s_full[2], p_half[2],
-  // p_full[2], o_full[2], mma_done
+  // p_full[2], o_full[2], mma_done, v_exp[STAGES]
   static constexpr int BAR_Q = 0;
   static constexpr int BAR_KV_FULL = 1;
   static constexpr int BAR_KV_EMPTY = 1 + STAGES;
@@ -64,10 +65,14 @@ struct FwdLayout {
   static_assert(BAR_P_FULL == BAR_P_HALF + 2, "the softmax arrives on BAR_P_HALF + t + 2 * half");
   static constexpr int BAR_O_FULL = BAR_P_FULL + 2;
   static constexpr int BAR_MMA_DONE = BAR_O_FULL + 2;
-  static constexpr int NBAR = BAR_MMA_DONE + 1;
+  static constexpr int BAR_V_EXP = BAR_MMA_DONE + 1;  // [STAGES] the V tile's copy exponent is published
+  static constexpr int BAR_V_AMAX = BAR_V_EXP + STAGES;  // [2] both converter warps' tile maxima written
+  static constexpr int NBAR = BAR_V_AMAX + 2;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NBAR * 8;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
-  static constexpr int BYTES = OFF_ABORT + 8;
+  static constexpr int OFF_VEXP = OFF_ABORT + 8;       // int[STAGES]: exponent of the V tile in each stage
+  static constexpr int OFF_VAMAX = OFF_VEXP + 4 * STAGES;  // uint32[2][2]: the two converter warps' maxima
+  static constexpr int BYTES = OFF_VAMAX + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;  // slack to align the base to 1024 bytes
   static constexpr uint32_t TMEM_COLS = 512;       // S0, S1 (128 each), O0, O1 (D each)
   static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
@@ -119,13 +124,20 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // P V product; the row sum uses the fp32 values before rounding.  bar_o_ready (non-zero)
 // is waited on, with parity o_ready_parity, before a rescale of O: for a kernel whose
 // previous P V into O may still be running when this step starts.
+// TILE_EXP: the V tile of this step is an fp16 copy V_j 2^v (v <= 0, published in *vexp_slot
+// once bar_vexp completes with parity vexp_parity); the step then writes P' = P 2^-v, so that
+// P' V_j 2^v = P V_j, and adds 2^v sum(P') to the row sum.  P' must stay within fp16 (P'
+// <= 2^15): the running maximum may then lag the true one by at most min(8, 15 + v).
+// A tile whose P sum exceeds what valid scores allow (a non-finite input, or a score beyond
+// the fp32 range) is recorded as kDevRange in the error word.
 // Returns false if a bounded wait gave up.
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, bool TILE_EXP = false>
 __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS, uint32_t tO, uint32_t bar_s_full,
                                                  uint32_t s_parity, uint32_t bar_p_half, uint32_t bar_p_full, int j,
                                                  bool first, int q_base, int r, float& m, float& l,
                                                  const WaitCtx& wctx, uint32_t bar_o_ready = 0,
-                                                 uint32_t o_ready_parity = 0) {
+                                                 uint32_t o_ready_parity = 0, uint32_t bar_vexp = 0,
+                                                 uint32_t vexp_parity = 0, const int* vexp_slot = nullptr) {
   const float sl2 = p.scale_log2;
   if (!mbar_wait(bar_s_full, s_parity, wctx)) return false;
   tc_fence_after();
@@ -166,11 +178,18 @@ __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS
   a1 = max3f(a1, x[126], x[127]);
   const float mx = max3f(fmaxf(a0, a1), a2, a3);
   const float m_new = fmaxf(m, mx * sl2);
+  int v = 0;  // exponent of this step's V tile copy (TILE_EXP)
+  if constexpr (TILE_EXP) {
+    if (!mbar_wait(bar_vexp, vexp_parity, wctx)) return false;
+    v = *reinterpret_cast<const volatile int*>(vexp_slot);
+  }
   // keep a stale maximum while it is within 2^8 of the true one: exact in the end
   // because O / l and the LSE use the same maximum
-  const float m_use = (m_new - m > 8.0f) ? m_new : m;
+  const float lag = TILE_EXP ? (float)min(8, 15 + v) : 8.0f;
+  const float m_use = (m_new - m > lag) ? m_new : m;
   const float alpha = (m_use == m) ? 1.0f : ex2_approx(m - m_use);  // 0 on the first tile
-  const float neg_m = m_use == -INFINITY ? 0.0f : -m_use;  // no visible key yet: every P is 0
+  float neg_m = m_use == -INFINITY ? 0.0f : -m_use;  // no visible key yet: every P is 0
+  if constexpr (TILE_EXP) neg_m -= (float)v;         // P' = P 2^-v
   if (!first && __any_sync(0xffffffffu, alpha != 1.0f)) {
     // rescale O before this tile's P V starts; either the previous O += P V of this tile
     // completed before S_j did (issued before it by the same thread, in-order tensor pipe),
@@ -230,7 +249,15 @@ __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS
   float s0, s1, s2, s3;
   f2unpack(sa, s0, s1);
   f2unpack(sb, s2, s3);
-  l = fmaf(l, alpha, (s0 + s1) + (s2 + s3));
+  const float tile_sum = (s0 + s1) + (s2 + s3);
+  // a valid row's P (P') are each <= 2^15 (<= 2^8 unless TILE_EXP), so the tile's sum is <= 2^22:
+  // a larger, infinite or NaN sum means a non-finite score (a non-finite input or a score beyond
+  // the fp32 range: the row maximum is then +inf or ignores NaN elements)
+  if (!(tile_sum <= 8388608.0f)) atomicExch(p.err, kDevRange);
+  if constexpr (TILE_EXP)
+    l = fmaf(l, alpha, tile_sum * __int_as_float((127 + v) << 23));  // 2^v sum(P')
+  else
+    l = fmaf(l, alpha, tile_sum);
   m = m_use;
   return true;
 }
@@ -272,6 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(L::BAR_KV_FULL + s), 1);
       mbar_init(bar(L::BAR_KV_EMPTY + s), 1);
       mbar_init(bar(L::BAR_V_CONV + s), kConvThreads);
+      mbar_init(bar(L::BAR_V_EXP + s), kConvThreads);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::BAR_S_FULL + t), 1);
@@ -280,6 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(L::BAR_O_FULL + t), 1);
     }
     mbar_init(bar(L::BAR_MMA_DONE), 1);
+    mbar_init(bar(L::BAR_V_AMAX + 0), kConvThreads);
+    mbar_init(bar(L::BAR_V_AMAX + 1), kConvThreads);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -410,14 +440,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2 || warp == 3) {
     // ===================================================== V tiles: bf16 -> fp16 in place
+    // Each tile is converted as V_j 2^v with v = 0 unless its largest |v| exceeds 2^15 (fp16
+    // ends at 65504); then v in [-15, -1] brings that maximum into [2^14, 2^15).  The
+    // exponent is published (BAR_V_EXP) after a first pass that finds the maximum, and the
+    // softmax writes P 2^-v for this tile.  A tile beyond 2^15 even at v = -15 (|v| >= about
+    // 2^31), or with a non-finite element, is recorded as kDevRange.
     regs_dec<kRegsLow>();
     const int ct = threadIdx.x - 64;  // 0..63
+    volatile uint32_t* vamax = reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_VAMAX);
+    volatile int* vexp = reinterpret_cast<volatile int*>(gbase + L::OFF_VEXP);
     bool ok = true;
     for (int j = 0; j < n1 && ok; ++j) {
       const int iV = 2 * j + 1;
       const int st = iV % L::STAGES;
       if (!(ok = mbar_wait(bar(L::BAR_KV_FULL + st), (iV / L::STAGES) & 1, wctx))) break;
       uint4* tile = reinterpret_cast<uint4*>(gbase + L::OFF_KV + st * L::TILE);
+      uint32_t am = 0u;  // largest |v| of the tile, as fp32 bits
+#pragma unroll 4
+      for (int i = ct; i < L::TILE / 16; i += kConvThreads) {
+        const uint4 u = tile[i];
+        am = abs_bits_max_bf16x2(abs_bits_max_bf16x2(am, u.x), u.y);
+        am = abs_bits_max_bf16x2(abs_bits_max_bf16x2(am, u.z), u.w);
+      }
+      am = __reduce_max_sync(0xffffffffu, am);
+      // the two warps' maxima, in a slot pair and barrier that alternate with the tile (a warp
+      // writes pair j & 1 again only after the other one arrived for tile j + 1, i.e. after it
+      // read pair j & 1); the wait is bounded like every other
+      if (lane == 0) vamax[2 * (j & 1) + (warp - 2)] = am;
+      mbar_arrive(bar(L::BAR_V_AMAX + (j & 1)));
+      if (!(ok = mbar_wait(bar(L::BAR_V_AMAX + (j & 1)), (j >> 1) & 1, wctx))) break;
+      am = max(vamax[2 * (j & 1)], vamax[2 * (j & 1) + 1]);
+      int v = 0;
+      if (am >= kBitsInf) {
+        if (ct == 0) atomicExch(p.err, kDevRange);
+      } else if (am > 0x47000000u) {  // > 2^15
+        v = max(14 - floor_log2_bits(am), -15);
+        if (ct == 0 && ldexpf(__uint_as_float(am), v) >= 65520.0f) atomicExch(p.err, kDevRange);
+      }
+      if (ct == 0) vexp[st] = v;
+      mbar_arrive(bar(L::BAR_V_EXP + st));
+      const float mult = __int_as_float((127 + v) << 23);  // 2^v
 #pragma unroll 4
       for (int i = ct; i < L::TILE / 16; i += kConvThreads) {
         uint4 u = tile[i];
@@ -425,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-          w[e] = pack_f16(f.x, f.y);
+          w[e] = v == 0 ? pack_f16(f.x, f.y) : pack_f16(f.x * mult, f.y * mult);
         }
         tile[i] = u;
       }
@@ -448,9 +510,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY;  // running max of scale*log2(e)*S (possibly stale by < 8)
     float l = 0.f;        // running sum of 2^(scale*log2(e)*S - m)
     bool ok = true;
+    const int* vexp = reinterpret_cast<const int*>(gbase + L::OFF_VEXP);
     for (int j = 0; j < n_t; ++j) {
-      if (!(ok = fwd_softmax_step<D>(p, tS, tO, bar(L::BAR_S_FULL + t), j & 1, bar(L::BAR_P_HALF + t),
-                                     bar(L::BAR_P_FULL + t), j, j == 0, q_base, r, m, l, wctx)))
+      const int iV = 2 * j + 1, stV = iV % L::STAGES;  // the stage holding V_j
+      if (!(ok = fwd_softmax_step<D, false, true>(p, tS, tO, bar(L::BAR_S_FULL + t), j & 1, bar(L::BAR_P_HALF + t),
+                                                  bar(L::BAR_P_FULL + t), j, j == 0, q_base, r, m, l, wctx, 0, 0,
+                                                  bar(L::BAR_V_EXP + stV), (iV / L::STAGES) & 1, vexp + stV)))
         break;
     }
     // ---- epilogue: O / l -> bf16 -> swizzled staging (the Q tile's buffer) -> TMA store
@@ -810,6 +875,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + (t ? L::T_S1 : L::T_S0);
     const uint32_t tO = tmem + lane_off + (t ? L::T_O1 : L::T_O0);
+    // the V copy is V 2^e (one exponent for the tensor): O / l is divided by 2^e
+    const float out_scale = p.v_exp != nullptr ? ldexpf(p.out_scale, -*p.v_exp) : p.out_scale;
     bool ok = true;
     int G = 0;  // this tile's steps in the previous units
     int u = next_unit(0, ok);
@@ -832,7 +899,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue: O / l -> bf16 and the bf16 residual, stored from registers
       if (!(ok = mbar_wait(bar(L::BAR_O_FULL + t), uc & 1, wctx))) break;
       tc_fence_after();
-      const float inv_l = p.out_scale / l;
+      const float inv_l = out_scale / l;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t u0[32], u1[32];
@@ -1146,6 +1213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = wq * 32 + lane;  // row inside the tile
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tO = tmem + lane_off + L::T_O;
+    const float out_scale = p.v_exp != nullptr ? ldexpf(p.out_scale, -*p.v_exp) : p.out_scale;  // V copy: V 2^e
     bool ok = true;
     int T = 0;
     int u = next_unit(0, ok);
@@ -1167,7 +1235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue: O / l -> bf16 and the bf16 residual, stored from registers
       if (!(ok = mbar_wait(bar(L::BAR_O_FULL), uc & 1, wctx))) break;
       tc_fence_after();
-      const float inv_l = p.out_scale / l;
+      const float inv_l = out_scale / l;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t u0[32], u1[32];
@@ -1240,19 +1308,69 @@ cudaError_t launch_persist_t(dim3 grid, const CUtensorMap& tq, const CUtensorMap
   return cudaGetLastError();
 }
 
-// V (bf16) -> fp16 copy, 8 elements per 16-byte access (exact for |v| in [2^-14, 65504]).
+// V (bf16) -> fp16 copy with exponent 0, 8 elements per 16-byte access, on a fixed grid whose
+// blocks leave their largest |v| (fp32 bits) in amax_part[block]; the fix-up below picks the
+// copy's exponent.  Also zeroes the persistent kernel's work counter.
 __global__ void __launch_bounds__(256) fa_fwd_v16_kernel(const uint4* __restrict__ v, uint4* __restrict__ v16,
-                                                         long long n8, unsigned* counter) {
+                                                         long long n8, unsigned* counter, uint32_t* amax_part) {
   if (blockIdx.x == 0 && threadIdx.x == 0 && counter != nullptr) *counter = 0u;  // persistent kernel's work counter
+  uint32_t am2 = 0u;  // packed bf16 maxima of |v|
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n8; e += (long long)gridDim.x * blockDim.x) {
     uint4 u = v[e];
     uint32_t* w = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
+      am2 = amax_bf16x2_step(am2, w[i]);
       const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
       w[i] = pack_f16(f.x, f.y);
     }
     v16[e] = u;
+  }
+  __shared__ uint32_t red[8];
+  uint32_t am = __reduce_max_sync(0xffffffffu, amax_bf16x2_bits(am2));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) am = max(am, red[w]);
+    amax_part[blockIdx.x] = am;
+  }
+}
+
+// Fix-up of the V copy: every block reduces the n_part block maxima to V's largest |v| and
+// derives the copy's exponent e (copy_exponent: 0 while it lies in [2^-4, 2^15], else the
+// exponent that brings it into [4, 8)); block 0 records e in *v_exp (the attention kernel
+// divides O by 2^e) and a non-finite V as kDevRange.  With e != 0 the blocks re-convert V as
+// V 2^e.
+__global__ void __launch_bounds__(256) fa_fwd_v16_fixup_kernel(const uint4* __restrict__ v, uint4* __restrict__ v16,
+                                                               long long n8, const uint32_t* amax_part, int n_part,
+                                                               int* v_exp, int* err) {
+  __shared__ uint32_t red[8];
+  __shared__ int e_s;
+  uint32_t am = 0u;
+  for (int i = threadIdx.x; i < n_part; i += blockDim.x) am = max(am, amax_part[i]);
+  am = __reduce_max_sync(0xffffffffu, am);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) am = max(am, red[w]);
+    e_s = copy_exponent(am, kCopyLoLog2, kCopyHiLog2);
+    if (blockIdx.x == 0) {
+      *v_exp = e_s;
+      if (am >= kBitsInf) atomicExch(err, kDevRange);
+    }
+  }
+  __syncthreads();
+  const int e = e_s;
+  if (e == 0) return;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    uint4 u = v[i];
+    uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+      w[k] = pack_f16(ldexpf(f.x, e), ldexpf(f.y, e));
+    }
+    v16[i] = u;
   }
 }
 }  // namespace
@@ -1277,12 +1395,17 @@ cudaError_t launch_fwd_persist_fp8_sm100(const CUtensorMap& tq, const CUtensorMa
   return launch_persist_t<128, true>(grid, tq, tk, tv, p, s);
 }
 
-cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, cudaStream_t s) {
+cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, uint32_t* amax_part,
+                           int* v_exp, int* err, cudaStream_t s) {
   const long long n8 = elems / 8;  // d is a multiple of 8
   long long blocks = (n8 + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks > kVPassBlocks) blocks = kVPassBlocks;
   fa_fwd_v16_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8,
-                                                     counter);
+                                                     counter, amax_part);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  fa_fwd_v16_fixup_kernel<<<kFixupBlocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8,
+                                                       amax_part, (int)blocks, v_exp, err);
   return cudaGetLastError();
 }
 

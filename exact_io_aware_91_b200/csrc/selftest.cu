@@ -23,7 +23,21 @@ __global__ void __launch_bounds__(32) fa_selftest_wait_kernel(int* err) {
     (void)mbar_wait(bar, 0, w);  // bounded: returns false and sets the error word
   }
 }
+// y[i] = exp2_fma_pipe(x[i]): the FMA-pipe exponential the softmax kernels use for part of
+// their exponentials, evaluated element by element for a check against 2^x.
+__global__ void __launch_bounds__(256) fa_selftest_exp2_kernel(const float* x, float* y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float a = x[i], b = x[i];
+  exp2_fma_pipe(a, b);
+  y[i] = a;
+}
 }  // namespace
+
+cudaError_t launch_selftest_exp2(const float* x, float* y, int n, cudaStream_t s) {
+  fa_selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_selftest_wait(int* err, cudaStream_t s) {
   fa_selftest_wait_kernel<<<1, 32, 0, s>>>(err);

@@ -13,9 +13,11 @@
 namespace fa {
 
 // ----------------------------------------------------------------- error word
-// Device-side failures (a bounded wait that ran out) are recorded here; the host
-// reads and clears it with fa_device_status().
-enum : int { kDevOk = 0, kDevTimeout = 5 };
+// Device-side failures are recorded here (the host reads and clears it with
+// fa_last_device_status()): a bounded wait that ran out (kDevTimeout), or a value outside
+// what the arithmetic can represent -- a non-finite input, a score Q K^T beyond the fp32
+// range, a V element too large for the scaled fp16 copy (kDevRange).
+enum : int { kDevOk = 0, kDevTimeout = 5, kDevRange = 6 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -378,6 +380,62 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+// max(a, b) that is NaN if either operand is NaN (fmaxf returns the other operand).
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+// ----------------------------------------------------------------- power-of-two range scaling
+// The tensor-core products of the kernels take fp16 copies of bf16 tensors (fp16 keeps 11
+// significant bits where bf16 keeps 8, but covers only |x| < 65504 and rounds |x| < 2^-14
+// to its subnormal grid).  A copy is therefore made as x * 2^e with one exponent e per
+// tensor, and every product that reads it undoes 2^e exactly (a power of two) in a scalar
+// that it applies anyway: the softmax's scale, the output's 1/l, a gradient's scale.
+// amax (the tensor's largest |x|) is handled as its float bits, which order like the values
+// for non-negative floats (and put NaN above +inf).
+constexpr uint32_t kBitsInf = 0x7F800000u;
+__device__ __forceinline__ uint32_t abs_bits(float x) { return __float_as_uint(x) & 0x7FFFFFFFu; }
+__device__ __forceinline__ uint32_t abs_bits_max_bf16x2(uint32_t acc, uint32_t two_bf16) {
+  // |x| of both bf16 halves widened exactly to fp32 bit patterns
+  const uint32_t lo = (two_bf16 << 16) & 0x7FFF0000u, hi = two_bf16 & 0x7FFF0000u;
+  return max(acc, max(lo, hi));
+}
+// Streaming form for the passes that read whole tensors: a running pair of bf16 maxima of |x|
+// (one packed NaN-propagating max per 32-bit word), folded to fp32 bits once at the end.
+__device__ __forceinline__ uint32_t amax_bf16x2_step(uint32_t acc2, uint32_t two_bf16) {
+  __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&acc2);
+  const uint32_t m = two_bf16 & 0x7FFF7FFFu;
+  a = __hmax2_nan(a, *reinterpret_cast<const __nv_bfloat162*>(&m));
+  return *reinterpret_cast<const uint32_t*>(&a);
+}
+__device__ __forceinline__ uint32_t amax_bf16x2_bits(uint32_t acc2) {  // fp32 bits of max(|lo|, |hi|)
+  return max(acc2 << 16, acc2 & 0xFFFF0000u);
+}
+// floor(log2(x)) of a positive finite float given as its bits (subnormals included).
+__host__ __device__ __forceinline__ int floor_log2_bits(uint32_t bits) {
+  if (bits >= 0x00800000u) return (int)(bits >> 23) - 127;
+  int E = -150;  // subnormal: the position of the leading mantissa bit
+  for (uint32_t m = bits; m != 0u; m >>= 1) ++E;
+  return E;
+}
+// Exponent that brings a largest magnitude (bits) into [4, 8): e = 2 - floor(log2(amax)),
+// capped at 64 (magnitudes below 2^-62 gain nothing further); 0 for zero and non-finite.
+__host__ __device__ __forceinline__ int target_exponent(uint32_t amax_bits) {
+  if (amax_bits == 0u || amax_bits >= kBitsInf) return 0;
+  const int e = 2 - floor_log2_bits(amax_bits);
+  return e > 64 ? 64 : e;
+}
+// Exponent of the copy of a tensor whose largest magnitude has bits `amax_bits`: 0 while
+// amax lies in [2^lo_log2, 2^hi_log2] (the common case: the copy is the plain conversion),
+// else target_exponent.
+__host__ __device__ __forceinline__ int copy_exponent(uint32_t amax_bits, int lo_log2, int hi_log2) {
+  if (amax_bits == 0u || amax_bits >= kBitsInf) return 0;
+  const int E = floor_log2_bits(amax_bits);
+  if (E >= lo_log2 && (E < hi_log2 || (E == hi_log2 && (amax_bits & 0x007FFFFFu) == 0u))) return 0;
+  return target_exponent(amax_bits);
+}
 // (x0, x1) * (s, s) + (t, t) with one packed instruction.
 __device__ __forceinline__ void fma2(float& x0, float& x1, float s, float t) {
   uint64_t a, b, c;
@@ -425,19 +483,23 @@ __device__ __forceinline__ void add_f16x2_to_f32(float& s0, float& s1, uint32_t 
 // per clock per SM, the softmax's throughput limit on sm_100a).  Method: round-to-
 // nearest range reduction x = j + f, j integer, f in [-1/2, 1/2] (adding 1.5 * 2^23
 // leaves round(x) in the low mantissa bits), 2^f by a degree-3 polynomial fitted for
-// minimum relative error on [-1/2, 1/2] (max relative error 7.5e-5 in fp32 Horner form,
-// below the 2^-11 rounding that P gets next when it is packed to fp16), and 2^j
+// minimum relative error on [-1/2, 1/2] (max relative error 7.5e-5 in fp32 Horner form on
+// [-125.99, 8], below the 2^-11 rounding that P gets next when it is packed to fp16; within
+// 1e-4 of -126 the result is an fp32 denormal, relative error up to 1.5e-4), and 2^j
 // applied by adding j to the exponent field.  Inputs are clamped to >= -126 so the
 // scaled result stays a normal float (2^-126 becomes 0 once rounded to fp16); the
-// largest input the softmax produces is 8 (a stale running maximum).
+// largest input the softmax produces is 8 (a stale running maximum).  A NaN argument passes
+// the clamp and comes out as a huge value (about 3.4e38) rather than NaN: NaN scores come only
+// from non-finite inputs or fp32 overflow, which the kernels report as a range error (input
+// maxima, the forward's tile sums of P).
 constexpr float kExp2Shifter = 12582912.0f;  // 1.5 * 2^23
 constexpr float kExp2C0 = 0.9999280571937561f;
 constexpr float kExp2C1 = 0.6932609677314758f;
 constexpr float kExp2C2 = 0.2426111400127411f;
 constexpr float kExp2C3 = 0.0551716685295105f;
 __device__ __forceinline__ void exp2_fma_pipe(float& a, float& b) {
-  a = fmaxf(a, -126.0f);
-  b = fmaxf(b, -126.0f);
+  a = max_nan(a, -126.0f);
+  b = max_nan(b, -126.0f);
   uint64_t x, t, f, p;
   asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a), "f"(b));
   const uint64_t shifter = ((uint64_t)__float_as_uint(kExp2Shifter) << 32) | __float_as_uint(kExp2Shifter);

@@ -26,7 +26,19 @@
  *    scaled, masked scores), fp32.
  *  - Every pointer is CALLER-OWNED DEVICE memory on the current CUDA device.  The
  *    library allocates no memory and keeps no state between calls except one
- *    device-resident error word per device (see fa_device_status).
+ *    device-resident error word per device (see fa_last_device_status).
+ *  - Value range.  The tensor-core products that need more than bf16's 8 significant
+ *    bits (P V in the forward; all products of the backward) read fp16 copies of the bf16
+ *    inputs.  fp16 ends at 65504, so every copy is the input times a power of two 2^e
+ *    chosen from the tensor's largest magnitude (one e per tensor; per 128-key tile of V
+ *    in the forward without a workspace), and the kernels undo 2^e exactly; e = 0, i.e.
+ *    the plain conversion, whenever the magnitudes lie in [2^-4, 2^15].  Every finite
+ *    bf16 input is therefore handled, with these limits, reported as FA_ERR_RANGE by
+ *    fa_last_device_status (the outputs of the rows concerned are then unspecified):
+ *    a non-finite input; a score Q K^T or a D = rowsum(dO * O) beyond the fp32 range
+ *    (about max|Q| max|K| d >= 2^128); in fa_fwd / fa_fwd_gqa (no workspace), a V element of
+ *    magnitude 2^31 or more.  In fa_fwd / fa_fwd_gqa V tiles are only scaled down, so V
+ *    elements below 2^-14 keep fp16's subnormal grid (absolute error <= 2^-25 each).
  *  - Calls are asynchronous on `stream` (NULL = the legacy default stream) and do
  *    not synchronise.  Argument errors are detected on the host before anything
  *    is launched; nothing is written then.
@@ -62,7 +74,8 @@ typedef enum {
   FA_ERR_UNSUPPORTED = 2, /* head dim not supported by the call, sizes beyond limits, not a CC 10.0 device */
   FA_ERR_MISALIGNED = 3,  /* a tensor base address is not 16-byte aligned (TMA requirement) */
   FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
-  FA_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (reported by fa_device_status) */
+  FA_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait (reported by fa_last_device_status) */
+  FA_ERR_RANGE = 6        /* an input beyond the value range above (reported by fa_last_device_status) */
 } fa_status;
 
 /*
@@ -70,30 +83,35 @@ typedef enum {
  *   q, k, v : const bf16 (B, H, N, d), 16-byte aligned.
  *   o       : bf16 (B, H, N, d) output, 16-byte aligned; must not alias q, k, v.
  *   lse     : fp32 (B, H, N) output (natural-log LSE, see above), or NULL to skip.
- *   o_resid : bf16 (B, H, N, d) output or NULL: the residual O_fp32 - O_bf16 of
- *             the final rounding of O.  A training forward passes it and hands it
- *             to fa_bwd, which then forms rowsum(dO * O) from an fp32-accurate O
- *             (the bf16 rounding of O alone costs the gradients up to ~0.2 of
- *             absolute accuracy on sharply peaked softmax rows).
  *   B, H, N : batch, heads, sequence length (>= 0).  d: head dim, 64 or 128.
  *   scale   : finite, > 0.   causal: 0 or 1.   stream: CUDA stream.
  * Q K^T is a bf16 product with fp32 accumulation; the probabilities are rounded
- * to fp16 (round to nearest even) for the P V product, whose V operand is an
- * exact fp16 copy of the bf16 V made on chip (|V| must stay below 65504); the row
- * sums are fp32; O is rounded to bf16 once at the end.
+ * to fp16 (round to nearest even) for the P V product, whose V operand is an fp16
+ * copy of the bf16 V made on chip (each 128-key tile scaled by a power of two when its
+ * magnitudes exceed 2^15, see "Value range"); the row sums are fp32; O is rounded to
+ * bf16 once at the end.  The attention formula is "FlashAttention (EL)", section
+ * "Problem of standard attention"; the tiled computation with an online softmax is its
+ * sections "Tiling" and "Online computation of Softmax".
+ * A training forward that feeds fa_bwd_gqa / fa_attn_bwd can also write the bf16
+ * residual O_fp32 - O_bf16 (fa_fwd_gqa with H_kv = H, fa_fwd_ws, fa_attn_fwd): the
+ * backward then forms rowsum(dO * O) from an fp32-accurate O.  Without it (fa_fwd ->
+ * fa_bwd) D carries O's bf16 rounding, which costs the gradients up to ~0.2 of absolute
+ * accuracy on sharply peaked softmax rows (a few keys ~8x larger than the rest).
  * Returns FA_OK once the kernel is enqueued.
  */
-FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B,
-                        int H, int N, int d, float scale, int causal, fa_stream_t stream);
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                        float scale, int causal, fa_stream_t stream);
 
 /*
  * fa_fwd_gqa -- fa_fwd for grouped-query / multi-query attention ("Flash
  * Attention: Ako transformery ...", section 5, and "FlashAttention (EL)", the list
  * of extensions, name GQA/MQA support; the grouping below is the reading taken).
- *   q, o, o_resid : (B, H, N, d) as in fa_fwd;  lse: (B, H, N).
- *   k, v          : const bf16 (B, H_kv, N, d), 16-byte aligned.
- *   H_kv          : key/value heads, >= 1, H a multiple of H_kv (H_kv = 1: MQA,
- *                   H_kv = H: plain multi-head attention, identical to fa_fwd).
+ *   q, o    : (B, H, N, d) as in fa_fwd;  lse: (B, H, N).
+ *   o_resid : bf16 (B, H, N, d) output or NULL: the residual O_fp32 - O_bf16 of the
+ *             final rounding of O, for fa_bwd_gqa / fa_attn_bwd.
+ *   k, v    : const bf16 (B, H_kv, N, d), 16-byte aligned.
+ *   H_kv    : key/value heads, >= 1, H a multiple of H_kv (H_kv = 1: MQA, H_kv = H: plain
+ *             multi-head attention; with o_resid = NULL identical to fa_fwd).
  * Query head h of batch entry b attends with key/value head h / (H / H_kv) of the
  * same batch entry (consecutive groups of H / H_kv query heads share one K/V head).
  * Everything else (precision, alignment, errors, asynchrony) as fa_fwd.
@@ -107,9 +125,12 @@ FA_API fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o
  * bf16 -> fp16 conversion as one streaming pass before the attention kernel instead of
  * inside it (fa_fwd / fa_fwd_gqa convert each V tile on chip, on two warps that share
  * SM sub-partitions with half of the softmax warps).  Results are identical to fa_fwd_gqa
- * (every unit computes the same values in the same order).
+ * (every unit computes the same values in the same order) whenever V's magnitudes lie in
+ * [2^-4, 2^15] (both copies unscaled; outside it the workspace copy is scaled per tensor,
+ * the on-chip one per tile).
  *   workspace       : device buffer of at least fa_fwd_workspace_size(B, H_kv, N, d)
- *                     bytes (an fp16 copy of V and a work counter), 256-byte aligned,
+ *                     bytes (an fp16 copy V 2^e of V with one exponent e for the tensor,
+ *                     a work counter and 9.5 KB of per-block maxima), 256-byte aligned,
  *                     caller-owned; contents on entry do not matter, unspecified on
  *                     return.  NULL is an error.
  * With a workspace the attention kernel is persistent (one CTA per SM taking work units
@@ -139,38 +160,38 @@ FA_API fa_status fa_fwd_f32(const float* q, const float* k, const float* v, floa
 /*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for this
  * problem (fp16 copies of Q, K, V, dO, two fp32 (B, H, N rounded up to 128) row
- * vectors and 256 bytes of work counters).  Returns 0 for an empty or invalid
- * problem.
+ * vectors, 256 bytes of work counters and copy exponents, 18.5 KB of per-block
+ * maxima).  Returns 0 for an empty or invalid problem.
  */
 FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
 /*
  * fa_bwd -- backward pass: gradients of sum(O * dO) with respect to Q, K, V.
- *   q, k, v, o, dout : const bf16 (B, H, N, d), 16-byte aligned; o, o_resid and
- *                      lse are the outputs of fa_fwd on the same q, k, v, scale
- *                      and causal.
- *   o_resid          : const bf16 (B, H, N, d) residual from fa_fwd, or NULL
- *                      (then rowsum(dO * O) uses the bf16 O alone: less accurate).
+ *   q, k, v, o, dout : const bf16 (B, H, N, d), 16-byte aligned; o and lse are the
+ *                      outputs of fa_fwd on the same q, k, v, scale and causal.
  *   lse              : const fp32 (B, H, N).
  *   dq, dk, dv       : fp32 (B, H, N, d) outputs, 16-byte aligned, not aliasing
  *                      any input.  Overwritten (not accumulated into).
  *   workspace        : device buffer of at least fa_bwd_workspace_size(B,H,N,d)
- *                      bytes, 256-byte aligned, caller-owned; its contents on
- *                      entry do not matter and on return are unspecified.
- *   workspace_bytes  : its size.
- * The probabilities are recomputed from LSE.  The tensor-core products run in
- * fp16 on exact fp16 copies of the bf16 inputs (exact for |x| in [2^-14, 65504];
- * larger magnitudes overflow), with fp32 accumulation; gradients are fp32.
+ *                      bytes (the call trusts that size: the signature carries none),
+ *                      256-byte aligned, caller-owned; its contents on entry do not
+ *                      matter and on return are unspecified.
+ * The probabilities are recomputed from LSE ("Flash Attention uitgelegd: een
+ * uitgebreide gids", section "Recomputation"); the gradients follow from the softmax
+ * Jacobian.  The tensor-core products run in fp16 on copies x 2^e of the bf16 inputs
+ * (one exponent per tensor, see "Value range"), with fp32 accumulation; gradients are
+ * fp32.  rowsum(dO * O) uses the bf16 O (see fa_fwd for the residual variant).
  */
-FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
-                        const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int N,
-                        int d, float scale, int causal, void* workspace, size_t workspace_bytes,
-                        fa_stream_t stream);
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, float* dq, float* dk, float* dv, int B, int H, int N, int d, float scale,
+                        int causal, void* workspace, fa_stream_t stream);
 
 /*
  * fa_bwd_gqa_workspace_size / fa_bwd_gqa -- fa_bwd for grouped-query attention
  * (grouping as in fa_fwd_gqa).
- *   q, o, o_resid, dout, dq : (B, H, N, d);  lse: (B, H, N).
+ *   q, o, dout, dq          : (B, H, N, d);  lse: (B, H, N).
+ *   o_resid                 : const bf16 (B, H, N, d) residual from the forward, or NULL
+ *                             (then rowsum(dO * O) uses the bf16 O alone: less accurate).
  *   k, v                    : const bf16 (B, H_kv, N, d).
  *   dk, dv                  : fp32 (B, H_kv, N, d) outputs: the gradient of a shared
  *                             key/value head is the sum over the query heads of its
@@ -182,8 +203,9 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
  *                             for the CTAs that split a group's query heads; their
  *                             sum is formed in a fixed order: results are
  *                             deterministic).
- * With H_kv = H both are identical to fa_bwd_workspace_size / fa_bwd.  Everything
- * else as fa_bwd.
+ *   workspace_bytes         : its size.
+ * With H_kv = H and o_resid = NULL both are identical to fa_bwd_workspace_size / fa_bwd.
+ * Everything else as fa_bwd.
  */
 FA_API size_t fa_bwd_gqa_workspace_size(int B, int H, int H_kv, int N, int d);
 FA_API fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
@@ -267,8 +289,8 @@ FA_API fa_status fa_attn_fwd_fp8(const fa_attn_problem* problem, const void* q, 
  * the backward pass: a plugin's enqueue callback inside an engine that owns all
  * device memory and forbids allocation there, or a latency-bound loop in which
  * cudaMalloc (which may synchronise the device) is not acceptable.  This entry
- * point takes the same arguments as fa_bwd minus the workspace and uses instead a
- * scratch array compiled into the library: a file-scope device array of
+ * point takes the arguments of fa_bwd_gqa with H_kv = H, minus the workspace, and uses
+ * instead a scratch array compiled into the library: a file-scope device array of
  * FA_BWD_NOALLOC_MAX_WORKSPACE bytes (64 MiB) that every GPU which loads the
  * library holds until the process exits.  It calls no cudaMalloc, cudaFree or any
  * other allocating routine.
@@ -282,7 +304,7 @@ FA_API fa_status fa_attn_fwd_fp8(const fa_attn_problem* problem, const void* q, 
  *     left in it.  Nothing in it needs to start at zero (each call overwrites every
  *     byte it reads), but calls whose work overlaps on the GPU -- on different
  *     streams, or from different host threads -- race on the array: serialise them.
- * Results are identical to fa_bwd with a workspace of its own.
+ * Results are identical to fa_bwd_gqa (H_kv = H) with a workspace of its own.
  */
 #define FA_BWD_NOALLOC_MAX_WORKSPACE ((size_t)64 << 20)
 FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
@@ -290,11 +312,13 @@ FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, con
                                 int N, int d, float scale, int causal, fa_stream_t stream);
 
 /*
- * fa_device_status -- synchronises `stream`, then reports whether any kernel of
- * this library on the current device gave up a bounded wait since the last call
- * (FA_ERR_TIMEOUT; the word is then cleared) or whether the CUDA context holds an
- * error (FA_ERR_CUDA).  FA_OK otherwise.
+ * fa_last_device_status -- synchronises `stream`, then reports what the kernels of this
+ * library on the current device recorded since the last call: FA_ERR_TIMEOUT (a bounded
+ * wait gave up) or FA_ERR_RANGE (an input beyond the value range above); the word is
+ * then cleared.  FA_ERR_CUDA if the CUDA context holds an error, FA_OK otherwise.
+ * fa_device_status is the same function under its earlier name.
  */
+FA_API fa_status fa_last_device_status(fa_stream_t stream);
 FA_API fa_status fa_device_status(fa_stream_t stream);
 
 /*
@@ -311,11 +335,23 @@ FA_API void fa_bwd_set_phase_events(void* const* events);
  * fa_selftest_wait_timeout -- self-test of the failure path: enqueues a one-CTA kernel in
  * which one thread waits, through the library's bounded-wait helper, on a barrier that
  * nothing ever completes.  The wait gives up after its wall-time limit (2 s) and records a
- * timeout, so a following fa_device_status(stream) returns FA_ERR_TIMEOUT (and clears it);
+ * timeout, so a following fa_last_device_status(stream) returns FA_ERR_TIMEOUT (and clears it);
  * the CUDA context stays usable.  Nothing faults, traps or hangs.  Returns FA_OK once
  * enqueued.
  */
 FA_API fa_status fa_selftest_wait_timeout(fa_stream_t stream);
+
+/*
+ * fa_selftest_exp2 -- self-test of the exponential that the softmax kernels evaluate on the
+ * FMA pipe for part of their probabilities (instead of the special-function unit): y[i] =
+ * that function of x[i] for i < n.  x, y: device fp32 arrays, 4-byte aligned.  The function
+ * is meant for the arguments the kernels produce, x in [-126, 8]: on [-125.99, 8] its
+ * relative error is at most 7.5e-5; closer to -126 the results are fp32 denormals (relative
+ * error up to 1.5e-4), and below -126 it returns about 2^-126 -- values that round to 0 in
+ * fp16.  Asynchronous on `stream`.  (A service of this library for its own tests; the pages
+ * describe no such function.)
+ */
+FA_API fa_status fa_selftest_exp2(const float* x, float* y, int n, fa_stream_t stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 FA_API const char* fa_status_str(fa_status status);

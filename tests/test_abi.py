@@ -35,15 +35,21 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings(lib):
     for code, name in [(0, "FA_OK"), (1, "FA_ERR_INVALID_ARG"), (2, "FA_ERR_UNSUPPORTED"),
-                       (3, "FA_ERR_MISALIGNED"), (4, "FA_ERR_CUDA"), (5, "FA_ERR_TIMEOUT")]:
+                       (3, "FA_ERR_MISALIGNED"), (4, "FA_ERR_CUDA"), (5, "FA_ERR_TIMEOUT"), (6, "FA_ERR_RANGE")]:
         assert api.status_str(code) == name
     assert api.status_str(99) == "FA_ERR_UNKNOWN"
+
+
+# blocks of the streaming passes that leave per-block maxima in the workspaces
+PRE_BLOCKS = 148 * 8     # backward preprocess: 4 tensors x 4 bytes per block
+VPASS_BLOCKS = 148 * 16  # forward V pass: 4 bytes per block
 
 
 def _ws_expected(B, H, N, d):
     a = lambda x: (x + 255) // 256 * 256  # noqa: E731
     Np = (N + 127) // 128 * 128
-    return 4 * a(B * H * N * d * 2) + 2 * a(B * H * Np * 4) + 256  # + work counters
+    # fp16 Q, dO, K, V; D and LSE*log2(e); control block (counters, exponents); maxima
+    return 4 * a(B * H * N * d * 2) + 2 * a(B * H * Np * 4) + 256 + a(16 * PRE_BLOCKS)
 
 
 @pytest.mark.parametrize("shape", [(1, 1, 1, 64), (4, 16, 2048, 128), (2, 32, 8192, 128), (1, 8, 131072, 128),
@@ -59,7 +65,8 @@ def _ws_expected_gqa(B, H, Hkv, N, d):
     group, units = H // Hkv, B * Hkv * ((N + 127) // 128)
     split = next((s for s in range(1, group) if group % s == 0 and units * s >= 4 * 148), group)
     part = 2 * a(split * B * Hkv * N * d * 4) if split > 1 else 0
-    return 2 * a(B * H * N * d * 2) + 2 * a(B * Hkv * N * d * 2) + 2 * a(B * H * Np * 4) + part + 256
+    return (2 * a(B * H * N * d * 2) + 2 * a(B * Hkv * N * d * 2) + 2 * a(B * H * Np * 4) + part + 256 +
+            a(16 * PRE_BLOCKS))
 
 
 @pytest.mark.parametrize("shape", [(1, 4, 1, 1, 64), (2, 32, 8, 8192, 128), (1, 8, 1, 131072, 128),
@@ -88,8 +95,9 @@ def test_gqa_head_counts_are_checked(lib):
 
 def test_forward_workspace(lib):
     a = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    assert api.fa_fwd_workspace_size(2, 8, 8192, 128) == a(2 * 8 * 8192 * 128 * 2) + 256
-    assert api.fa_fwd_workspace_size(1, 1, 300, 64) == a(300 * 64 * 2) + 256
+    # fp16 V, control block (work counter, the copy's exponent), the V pass's maxima
+    assert api.fa_fwd_workspace_size(2, 8, 8192, 128) == a(2 * 8 * 8192 * 128 * 2) + 256 + a(4 * VPASS_BLOCKS)
+    assert api.fa_fwd_workspace_size(1, 1, 300, 64) == a(300 * 64 * 2) + 256 + a(4 * VPASS_BLOCKS)
     assert api.fa_fwd_workspace_size(0, 8, 100, 64) == 0
     assert api.fa_fwd_workspace_size(1, 1, 100, 96) == 0
     ws = lambda ptr=A, n=1 << 40, H=4, Hkv=2: lib.fa_fwd_ws(A, A, A, A, A, None, 1, H, Hkv, 16, 64, 0.125, 0,  # noqa: E731
@@ -132,13 +140,24 @@ A = 0x10000  # 16-byte (and 256-byte) aligned
 MIS = 0x10008
 
 
-def fwd(lib, q=A, k=A, v=A, o=A, lse=A, resid=None, B=1, H=1, N=16, d=64, scale=0.125, causal=0):
-    return lib.fa_fwd(q, k, v, o, lse, resid, B, H, N, d, scale, causal, None)
+# fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream) and
+# fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, stream):
+# the boundary's plain signatures
+def fwd(lib, q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=16, d=64, scale=0.125, causal=0):
+    return lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, None)
 
 
-def bwd(lib, ptr=A, ws=A, ws_bytes=1 << 40, B=1, H=1, N=16, d=64, scale=0.125, causal=0, dq=A, resid=A):
-    return lib.fa_bwd(ptr, ptr, ptr, ptr, resid, ptr, ptr, dq, ptr, ptr, B, H, N, d, scale, causal, ws, ws_bytes,
-                      None)
+def bwd(lib, ptr=A, ws=A, B=1, H=1, N=16, d=64, scale=0.125, causal=0, dq=A):
+    return lib.fa_bwd(ptr, ptr, ptr, ptr, ptr, ptr, dq, ptr, ptr, B, H, N, d, scale, causal, ws, None)
+
+
+# the grouped entry points carry the residual and the workspace size
+def fwd_gqa(lib, resid=None, B=1, H=1, N=16, d=64):
+    return lib.fa_fwd_gqa(A, A, A, A, A, resid, B, H, H, N, d, 0.125, 0, None)
+
+
+def bwd_gqa(lib, ws_bytes=1 << 40, resid=A, B=1, H=1, N=16, d=64):
+    return lib.fa_bwd_gqa(A, A, A, A, resid, A, A, A, A, A, B, H, H, N, d, 0.125, 0, A, ws_bytes, None)
 
 
 def test_forward_argument_errors(lib):
@@ -154,7 +173,7 @@ def test_forward_argument_errors(lib):
     assert fwd(lib, q=MIS) == api.FA_ERR_MISALIGNED
     assert fwd(lib, o=MIS) == api.FA_ERR_MISALIGNED
     assert fwd(lib, lse=A + 2) == api.FA_ERR_MISALIGNED
-    assert fwd(lib, resid=A + 8) == api.FA_ERR_MISALIGNED
+    assert fwd_gqa(lib, resid=A + 8) == api.FA_ERR_MISALIGNED
     assert fwd(lib, B=1 << 25) == api.FA_ERR_UNSUPPORTED
 
 
@@ -162,18 +181,18 @@ def test_empty_problems_are_no_ops(lib):
     # nothing to compute: FA_OK even with null pointers, nothing launched
     assert fwd(lib, q=None, k=None, v=None, o=None, lse=None, N=0) == api.FA_OK
     assert fwd(lib, q=None, k=None, v=None, o=None, lse=None, B=0) == api.FA_OK
-    assert bwd(lib, ptr=None, ws=None, dq=None, resid=None, H=0) == api.FA_OK
+    assert bwd(lib, ptr=None, ws=None, dq=None, H=0) == api.FA_OK
     assert lib.fa_fwd_f32(None, None, None, None, None, 1, 1, 0, 64, 0.125, 0, None) == api.FA_OK
 
 
 def test_backward_argument_errors(lib):
     assert bwd(lib, ptr=None) == api.FA_ERR_INVALID_ARG
     assert bwd(lib, ws=None) == api.FA_ERR_INVALID_ARG
-    assert bwd(lib, ws_bytes=_ws_expected(1, 1, 16, 64) - 1) == api.FA_ERR_INVALID_ARG
+    assert bwd_gqa(lib, ws_bytes=_ws_expected(1, 1, 16, 64) - 1) == api.FA_ERR_INVALID_ARG
     assert bwd(lib, d=32) == api.FA_ERR_UNSUPPORTED
     assert bwd(lib, causal=-1) == api.FA_ERR_INVALID_ARG
     assert bwd(lib, dq=MIS) == api.FA_ERR_MISALIGNED
-    assert bwd(lib, resid=MIS) == api.FA_ERR_MISALIGNED
+    assert bwd_gqa(lib, resid=MIS) == api.FA_ERR_MISALIGNED
     assert bwd(lib, ws=A + 16) == api.FA_ERR_MISALIGNED  # workspace needs 256-byte alignment
 
 
@@ -219,7 +238,8 @@ def test_fp8_forward_checks_its_arguments(lib):
 
 
 def test_head_dim_256_is_a_forward_with_workspace(lib):
-    assert api.fa_fwd_workspace_size(1, 2, 300, 256) == _align256(1 * 2 * 300 * 256 * 2) + 256
+    assert api.fa_fwd_workspace_size(1, 2, 300, 256) == _align256(1 * 2 * 300 * 256 * 2) + 256 + \
+        _align256(4 * VPASS_BLOCKS)
     pr = api.FaAttnProblem(1, 4, 2, 300, 256, 0.0625, 1, -1, -1)
     assert api.fa_attn_fwd_workspace_size(pr) == api.fa_fwd_workspace_size(1, 2, 300, 256)
     assert api.fa_bwd_workspace_size(1, 2, 300, 256) == 0

@@ -23,7 +23,7 @@ def _device():
         pytest.skip("needs a CUDA device")
     torch.cuda.set_device(0)
     yield
-    assert api.fa_device_status() == api.FA_OK
+    assert api.fa_last_device_status() == api.FA_OK
 
 
 def f64(t):

@@ -26,7 +26,7 @@ def _device():
         pytest.skip("needs a CUDA device")
     torch.cuda.set_device(0)
     yield
-    assert api.fa_device_status() == api.FA_OK
+    assert api.fa_last_device_status() == api.FA_OK
 
 
 def test_maximum_head_count_single_token():
@@ -35,8 +35,8 @@ def test_maximum_head_count_single_token():
     q, k, v, do = (torch.randn((B, H, N, d), generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)
                    for _ in range(4))
     scale = 0.125
-    o, lse, res = api.fa_fwd(q, k, v, causal=True, scale=scale, save_residual=True)
-    dq, dk, dv = api.fa_bwd(q, k, v, o, do, lse, causal=True, scale=scale, o_resid=res)
+    o, lse, res = api.fa_fwd_gqa(q, k, v, causal=True, scale=scale, save_residual=True)
+    dq, dk, dv = api.fa_bwd_gqa(q, k, v, o, do, lse, causal=True, scale=scale, o_resid=res)
     torch.cuda.synchronize()
     # one key: P = 1, so O = V up to the fp16 copy of V (values below fp16's normal range)
     # and the output rounding
@@ -58,7 +58,7 @@ def test_million_token_causal_sequence():
     q, k, v, do = inp["q"], inp["k"], inp["v"], inp["do"]
     scale = 1.0 / np.sqrt(d)
     o, lse, res = api.fa_fwd_ws(q, k, v, causal=True, scale=scale, save_residual=True)
-    dq, dk, dv = api.fa_bwd(q, k, v, o, do, lse, causal=True, scale=scale, o_resid=res)
+    dq, dk, dv = api.fa_bwd_gqa(q, k, v, o, do, lse, causal=True, scale=scale, o_resid=res)
     torch.cuda.synchronize()
     rows = sorted({0, 1, 127, 128, 255, 1 << 19, N - 129, N - 128, N - 2, N - 1} |
                   set(np.random.default_rng(5).integers(0, N, 14).tolist()))

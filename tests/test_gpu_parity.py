@@ -45,22 +45,30 @@ def _device():
         pytest.skip("needs a CUDA device")
     torch.cuda.set_device(0)
     yield
-    assert api.fa_device_status() == api.FA_OK
+    assert api.fa_last_device_status() == api.FA_OK
 
 
 def run_fwd_bwd(w: inputs.Workload | None = None, *, B=1, H=2, N=128, d=128, causal=True, seed=0,
-                backward=True, spiky=0.0):
+                backward=True, spiky=0.0, check_on_chip=False):
+    """The path the benchmark times: fa_fwd_ws (V pass + persistent kernel, with the
+    residual) then fa_bwd_gqa with the residual.  check_on_chip: also run the workspace-less
+    forward (fa_fwd_gqa, V converted on chip, one CTA per unit) and require the same bits."""
     if w is not None:
         inp = inputs.make_inputs(w, device="cuda")
         d, causal, backward, scale = w.d, w.causal, w.backward, w.scale
     else:
         inp = inputs.make_qkv(B, H, N, d, seed=seed, spiky_frac=spiky, backward=backward, device="cuda")
         scale = 1.0 / np.sqrt(d)
-    o, lse, res = api.fa_fwd(inp["q"], inp["k"], inp["v"], causal=causal, scale=scale, save_residual=True)
+    o, lse, res = api.fa_fwd_ws(inp["q"], inp["k"], inp["v"], causal=causal, scale=scale, save_residual=True)
     out = {"inp": inp, "o": o, "lse": lse, "res": res, "scale": scale, "causal": causal}
+    if check_on_chip:
+        o2, lse2, res2 = api.fa_fwd_gqa(inp["q"], inp["k"], inp["v"], causal=causal, scale=scale, save_residual=True)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o2) and torch.equal(lse, lse2) and torch.equal(res, res2), "fa_fwd_ws != fa_fwd_gqa"
+        del o2, lse2, res2
     if backward:
-        out["grads"] = api.fa_bwd(inp["q"], inp["k"], inp["v"], o, inp["do"], lse, causal=causal, scale=scale,
-                                  o_resid=res)
+        out["grads"] = api.fa_bwd_gqa(inp["q"], inp["k"], inp["v"], o, inp["do"], lse, causal=causal, scale=scale,
+                                      o_resid=res)
     torch.cuda.synchronize()
     return out
 
@@ -104,12 +112,13 @@ def test_gqa_fwd_bwd(B, H, Hkv, N, d, causal):
     O, L = oracle.attention_forward_gqa(q, k, v, scale, causal)
     assert_fwd(o, lse, O, L, tag)
     assert_grads(grads, oracle.attention_backward_gqa(q, k, v, do, scale, causal), tag)
-    if Hkv == H:  # the grouped entry points with H_kv = H are plain multi-head attention
-        o2, lse2, res2 = api.fa_fwd(q, k, v, causal=causal, scale=scale, save_residual=True)
-        g2 = api.fa_bwd(q, k, v, o2, do, lse2, causal=causal, scale=scale, o_resid=res2)
+    if Hkv == H:  # with H_kv = H and no residual the grouped entry points are fa_fwd / fa_bwd
+        o2, lse2 = api.fa_fwd(q, k, v, causal=causal, scale=scale)
+        g1 = api.fa_bwd_gqa(q, k, v, o2, do, lse2, causal=causal, scale=scale)
+        g2 = api.fa_bwd(q, k, v, o2, do, lse2, causal=causal, scale=scale)
         torch.cuda.synchronize()
         assert torch.equal(o, o2) and torch.equal(lse, lse2)
-        for a, b in zip(grads, g2):
+        for a, b in zip(g1, g2):
             assert torch.equal(a, b)
 
 
@@ -153,7 +162,7 @@ def test_unbounded_window_is_the_plain_path():
     o1, l1, r1 = api.fa_attn_fwd(q, k, v, causal=True, window=(-1, -1), save_residual=True)
     o2, l2, r2 = api.fa_fwd_ws(q, k, v, causal=True, save_residual=True)
     g1 = api.fa_attn_bwd(q, k, v, o1, do, l1, causal=True, window=(-1, -1), o_resid=r1)
-    g2 = api.fa_bwd(q, k, v, o2, do, l2, causal=True, o_resid=r2)
+    g2 = api.fa_bwd_gqa(q, k, v, o2, do, l2, causal=True, o_resid=r2)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     for a, b in zip(g1, g2):
@@ -189,7 +198,7 @@ def test_workload1_fp32_forward():
 
 def test_workload2_full():
     w = inputs.workload(2)
-    r = run_fwd_bwd(w)
+    r = run_fwd_bwd(w, check_on_chip=True)
     q, k, v, do = (r["inp"][n] for n in ("q", "k", "v", "do"))
     O, L = oracle.attention_forward(q, k, v, w.scale, w.causal)
     assert_fwd(r["o"], r["lse"], O, L, "workload 2")
@@ -202,8 +211,10 @@ def test_workload2_full():
 
 
 def test_workload3_sampled_heads_and_rows():
+    # the benchmark's forward at full size: 2048 work units on one CTA per SM, so every CTA
+    # takes many units in turn; bit-equal to the one-CTA-per-unit forward
     w = inputs.workload(3)
-    r = run_fwd_bwd(w)
+    r = run_fwd_bwd(w, check_on_chip=True)
     q, k, v, do = (r["inp"][n] for n in ("q", "k", "v", "do"))
     o, lse = r["o"], r["lse"]
     dq, dk, dv = r["grads"]
@@ -224,7 +235,7 @@ def test_workload3_sampled_heads_and_rows():
 
 def test_workload4_full_forward():
     w = inputs.workload(4)
-    r = run_fwd_bwd(w)
+    r = run_fwd_bwd(w, check_on_chip=True)
     q, k, v = (r["inp"][n] for n in ("q", "k", "v"))
     O, L = oracle.attention_forward(q, k, v, w.scale, w.causal)
     assert_fwd(r["o"], r["lse"], O, L, "workload 4")
@@ -246,8 +257,8 @@ def test_workload5_sampled_rows_and_prefix():
     # backward: the 4096-token prefix problem run on its own ...
     P = 4096
     qp, kp, vp, dop = (t[:, :, :P].contiguous() for t in (q, k, v, do))
-    op, lsep, rp = api.fa_fwd(qp, kp, vp, causal=True, scale=w.scale, save_residual=True)
-    gp = api.fa_bwd(qp, kp, vp, op, dop, lsep, causal=True, scale=w.scale, o_resid=rp)
+    op, lsep, rp = api.fa_fwd_ws(qp, kp, vp, causal=True, scale=w.scale, save_residual=True)
+    gp = api.fa_bwd_gqa(qp, kp, vp, op, dop, lsep, causal=True, scale=w.scale, o_resid=rp)
     torch.cuda.synchronize()
     ref = oracle.attention_backward(qp[0], kp[0], vp[0], dop[0], w.scale, True)
     assert_grads((gp[0][0], gp[1][0], gp[2][0]), ref, "workload 5 prefix")
@@ -259,9 +270,9 @@ def test_workload5_sampled_rows_and_prefix():
 # ------------------------------------------------------------------ properties
 def test_deterministic():
     a = run_fwd_bwd(B=2, H=3, N=777, d=128, causal=True, seed=11)
-    o2, lse2, r2 = api.fa_fwd(a["inp"]["q"], a["inp"]["k"], a["inp"]["v"], causal=True, save_residual=True)
-    g2 = api.fa_bwd(a["inp"]["q"], a["inp"]["k"], a["inp"]["v"], a["o"], a["inp"]["do"], a["lse"], causal=True,
-                    o_resid=a["res"])
+    o2, lse2, r2 = api.fa_fwd_ws(a["inp"]["q"], a["inp"]["k"], a["inp"]["v"], causal=True, save_residual=True)
+    g2 = api.fa_bwd_gqa(a["inp"]["q"], a["inp"]["k"], a["inp"]["v"], a["o"], a["inp"]["do"], a["lse"], causal=True,
+                        o_resid=a["res"])
     torch.cuda.synchronize()
     assert torch.equal(a["o"], o2) and torch.equal(a["lse"], lse2) and torch.equal(a["res"], r2)
     for x, y in zip(a["grads"], g2):
@@ -282,7 +293,7 @@ def test_library_allocates_nothing():
 def test_residual_is_the_rounding_of_o():
     # O + residual is the forward's fp32 O: much closer to the oracle than the bf16 O alone
     inp = inputs.make_qkv(1, 2, 1000, 128, seed=9, device="cuda")
-    o, lse, res = api.fa_fwd(inp["q"], inp["k"], inp["v"], causal=True, save_residual=True)
+    o, lse, res = api.fa_fwd_gqa(inp["q"], inp["k"], inp["v"], causal=True, save_residual=True)
     torch.cuda.synchronize()
     O, _ = oracle.attention_forward(inp["q"], inp["k"], inp["v"], 1 / np.sqrt(128), True)
     full = f64(o) + f64(res)
@@ -298,3 +309,33 @@ def test_backward_without_residual_on_a_plain_workload():
     torch.cuda.synchronize()
     ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["do"], 1 / np.sqrt(64), False)
     assert_grads(g, ref, "no residual")
+
+
+# ------------------------------------------------------------------ the boundary's own signatures
+@pytest.mark.parametrize("N,d,causal", [(1, 64, True), (300, 128, True), (1000, 64, False), (257, 128, False)])
+def test_exact_signatures_small(N, d, causal):
+    # fa_fwd(q,k,v,o,lse,B,H,N,d,scale,causal,stream) and
+    # fa_bwd(q,k,v,o,dout,lse,dq,dk,dv,B,H,N,d,scale,causal,workspace,stream) through ctypes
+    inp = inputs.make_qkv(2, 3, N, d, seed=N + d + 5 * causal, device="cuda")
+    q, k, v, do = (inp[n] for n in ("q", "k", "v", "do"))
+    scale = 1.0 / np.sqrt(d)
+    o, lse = api.fa_fwd(q, k, v, causal=causal, scale=scale)
+    grads = api.fa_bwd(q, k, v, o, do, lse, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    tag = f"fa_fwd/fa_bwd N={N} d={d} causal={causal}"
+    O, L = oracle.attention_forward(q, k, v, scale, causal)
+    assert_fwd(o, lse, O, L, tag)
+    assert_grads(grads, oracle.attention_backward(q, k, v, do, scale, causal), tag)
+
+
+def test_exact_signatures_workload2():
+    # the boundary's plain pair (no residual: D from the bf16 O) on workload 2 in full
+    w = inputs.workload(2)
+    inp = inputs.make_inputs(w, device="cuda")
+    q, k, v, do = (inp[n] for n in ("q", "k", "v", "do"))
+    o, lse = api.fa_fwd(q, k, v, causal=w.causal, scale=w.scale)
+    grads = api.fa_bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    O, L = oracle.attention_forward(q, k, v, w.scale, w.causal)
+    assert_fwd(o, lse, O, L, "fa_fwd workload 2")
+    assert_grads(grads, oracle.attention_backward(q, k, v, do, w.scale, w.causal), "fa_bwd workload 2")
