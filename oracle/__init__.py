@@ -24,4 +24,4 @@ from .attention import (  # noqa: F401
     attention_backward_gqa,
     apply_window,
 )
-from .fp8 import e4m3_decode, attention_forward_fp8  # noqa: F401
+from .fp8 import e4m3_decode, attention_forward_fp8, attention_forward_fp8_rows  # noqa: F401

@@ -161,21 +161,28 @@ def attention_forward(q, k, v, scale: float, causal: bool, window=(-1, -1)):
     return O.reshape(lead + O.shape[1:]), L.reshape(lead + (q3.shape[1],))
 
 
-def attention_forward_rows(q, k, v, scale: float, causal: bool, rows):
+def attention_forward_rows(q, k, v, scale: float, causal: bool, rows, window=(-1, -1)):
     """The same definition evaluated only for the query rows ``rows`` of one head.
 
     q, k, v: (N, d) for a single head.  Returns O[rows] (len(rows), d) and LSE[rows].
-    Row i sees keys 0..i when causal, all keys otherwise.  Used where the full
-    N x N matrix would not fit in host memory.
+    Row i sees keys 0..i when causal, all keys otherwise, and with a sliding window
+    (left, right) only keys i - left .. i + right (as ``apply_window``).  Used where the
+    full N x N matrix would not fit in host memory.
     """
     q = _as_f64(q)
     k = _as_f64(k)
     v = _as_f64(v)
     rows = np.asarray(rows, dtype=np.int64)
     s = scale * (q[rows] @ k.T)
+    j = np.arange(k.shape[0])[None, :]
+    i = rows[:, None]
     if causal:
-        j = np.arange(k.shape[0])[None, :]
-        s = np.where(j > rows[:, None], -np.inf, s)
+        s = np.where(j > i, -np.inf, s)
+    left, right = window
+    if left >= 0:
+        s = np.where(j < i - left, -np.inf, s)
+    if right >= 0:
+        s = np.where(j > i + right, -np.inf, s)
     lse = _lse_rows(s)
     p = np.exp(s - lse[:, None])
     return p @ v, lse

@@ -22,7 +22,7 @@ rounded to E4M3 before the P V product) is a property of the kernels, bounded in
 
 import numpy as np
 
-from .attention import attention_forward_gqa
+from .attention import attention_forward_gqa, attention_forward_rows
 
 
 def e4m3_decode(bits) -> np.ndarray:
@@ -48,3 +48,14 @@ def attention_forward_fp8(q_bits, k_bits, v_bits, q_descale: float, k_descale: f
     k = k_descale * e4m3_decode(k_bits)
     v = v_descale * e4m3_decode(v_bits)
     return attention_forward_gqa(q, k, v, scale, causal, window)
+
+
+def attention_forward_fp8_rows(q_bits, k_bits, v_bits, q_descale: float, k_descale: float, v_descale: float,
+                               scale: float, causal: bool, rows, window=(-1, -1)):
+    """(O[rows], LSE[rows]) of one head of the same attention, for long sequences.
+
+    q_bits, k_bits, v_bits: (N, d) E4M3 codes of one query head and its key/value head."""
+    q = q_descale * e4m3_decode(q_bits)
+    k = k_descale * e4m3_decode(k_bits)
+    v = v_descale * e4m3_decode(v_bits)
+    return attention_forward_rows(q, k, v, scale, causal, rows, window)

@@ -157,13 +157,16 @@ def test_loop_restatement_matches_numpy_oracle(causal, n, d):
 
 
 def test_row_sampler_matches_full_forward():
+    # the full forward with a window is pinned by its own tests (SDPA with the explicit mask,
+    # closed forms); the row sampler must agree with it row by row
     q, k, v = randn((50, 8), 27), randn((50, 8), 28), randn((50, 8), 29)
     rows = [0, 1, 17, 48, 49]
     for causal in (False, True):
-        O, L = attention_forward(q, k, v, 0.35, causal)
-        Or, Lr = attention_forward_rows(q, k, v, 0.35, causal, rows)
-        np.testing.assert_allclose(Or, O[rows], atol=1e-14)
-        np.testing.assert_allclose(Lr, L[rows], atol=1e-14)
+        for window in ((-1, -1), (5, -1), (3, 4), (0, 0), (-1, 2)):
+            O, L = attention_forward(q, k, v, 0.35, causal, window=window)
+            Or, Lr = attention_forward_rows(q, k, v, 0.35, causal, rows, window=window)
+            np.testing.assert_allclose(Or, O[rows], atol=1e-14)
+            np.testing.assert_allclose(Lr, L[rows], atol=1e-14)
 
 
 def test_row_dq_matches_full_backward_and_finite_differences():

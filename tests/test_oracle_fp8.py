@@ -145,3 +145,18 @@ def test_descale_pins_catch_a_descale_on_the_wrong_operand(monkeypatch):
     monkeypatch.setattr(oracle, "attention_forward_fp8", swapped)
     with pytest.raises(AssertionError):
         test_value_descale_scales_the_output_only()
+
+
+@pytest.mark.parametrize("causal,window", [(False, (-1, -1)), (True, (-1, -1)), (True, (7, -1)), (False, (5, 3))])
+def test_row_sampler_matches_the_full_8bit_forward(causal, window):
+    # the per-head row sampler used for long sequences must agree with the pinned full forward
+    x = inputs.make_qkv_fp8(1, 2, 60, 16, seed=9, spiky_frac=0.05)
+    bits = {n: x[n].view(torch.uint8).numpy() for n in ("q", "k", "v")}
+    ds = (x["q_descale"], x["k_descale"], x["v_descale"])
+    O, L = oracle.attention_forward_fp8(bits["q"], bits["k"], bits["v"], *ds, 0.25, causal, window)
+    rows = [0, 1, 29, 58, 59]
+    for h in range(2):
+        Or, Lr = oracle.attention_forward_fp8_rows(bits["q"][0, h], bits["k"][0, h], bits["v"][0, h], *ds, 0.25,
+                                                   causal, rows, window)
+        np.testing.assert_allclose(Or, O[0, h, rows], atol=1e-13)
+        np.testing.assert_allclose(Lr, L[0, h, rows], atol=1e-13)
