@@ -165,18 +165,16 @@ __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS
     for (int c = 0; c < 128; ++c)
       if (kb + c < lo || kb + c > hi) x[c] = -INFINITY;
   }
-  // row max: four independent 3-input max chains
-  float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
+  // row max: a tree of 3-input maxima (depth 4)
+  float a_[43], b_[15];
 #pragma unroll
-  for (int c = 4; c < 124; c += 8) {
-    a0 = max3f(a0, x[c], x[c + 1]);
-    a1 = max3f(a1, x[c + 2], x[c + 3]);
-    a2 = max3f(a2, x[c + 4], x[c + 5]);
-    a3 = max3f(a3, x[c + 6], x[c + 7]);
-  }
-  a0 = max3f(a0, x[124], x[125]);
-  a1 = max3f(a1, x[126], x[127]);
-  const float mx = max3f(fmaxf(a0, a1), a2, a3);
+  for (int i = 0; i < 42; ++i) a_[i] = max3f(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+  a_[42] = fmaxf(x[126], x[127]);
+#pragma unroll
+  for (int i = 0; i < 14; ++i) b_[i] = max3f(a_[3 * i], a_[3 * i + 1], a_[3 * i + 2]);
+  b_[14] = a_[42];
+  const float mx = max3f(max3f(max3f(b_[0], b_[1], b_[2]), max3f(b_[3], b_[4], b_[5]), max3f(b_[6], b_[7], b_[8])),
+                         max3f(b_[9], b_[10], b_[11]), max3f(b_[12], b_[13], b_[14]));
   const float m_new = fmaxf(m, mx * sl2);
   int v = 0;  // exponent of this step's V tile copy (TILE_EXP)
   if constexpr (TILE_EXP) {
