@@ -255,7 +255,9 @@ cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t s) {
   const long long warps = (rows + rpw - 1) / rpw;
   long long blocks = (warps + 7) / 8;
   if (blocks > kPreBlocks) blocks = kPreBlocks;
-  if (p.d == 128)
+  if (p.d == 256)
+    fa_bwd_pre_kernel<256><<<(unsigned)blocks, 256, 0, s>>>(p);
+  else if (p.d == 128)
     fa_bwd_pre_kernel<128><<<(unsigned)blocks, 256, 0, s>>>(p);
   else
     fa_bwd_pre_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(p);

@@ -923,6 +923,794 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ============================================================================ head dim 256
+// At d = 256 the accumulators do not fit next to S^T and dP^T in tensor memory (dV and dK of
+// a 128-key tile take 256 columns each), and the tiles do not fit in shared memory (K, V, Q
+// and dO of 128 rows take 64 KB each).  The two kernels below therefore:
+//   * dK/dV: a work unit is (key/value head, 128-key tile, d-half h, share of the group's
+//     query heads).  It recomputes S^T = K Q^T and dP^T = V dO^T over the full d and
+//     accumulates only dV[:, h] += P^T dO[:, h] and dK[:, h] += dS^T Q[:, h]: TMEM holds S^T,
+//     dP^T, dV_h, dK_h (128 columns each).  K and V stay resident (64 KB each); Q and dO
+//     stream as 128-column halves (32 KB) through a 3-slot FIFO, and the half h of each is
+//     loaded a second time for its gradient product, so the FIFO releases slots in the order
+//     it fills them.
+//   * dQ: Q and dO stay resident; S is single-buffered (S, dP 128 columns, dQ 256); K and V
+//     stream as halves through the same kind of FIFO, K's halves a second time for dQ += dS K.
+// Both are persistent like the d = 128 kernels; every other step (recomputed probabilities,
+// masks, grouped heads, windows, work order, coalesced epilogues) is the same.
+constexpr int kHalf = 2 * kBox;  // 128 rows x 128 fp16 columns (two 64-column boxes), 32 KB
+constexpr int kWSlots = 3;       // FIFO slots of one half each
+constexpr int kSmemMax = 232448;  // dynamic shared memory of one CTA on sm_100
+
+// SS product D (+)= A * B^T over K = 128 (one half of d): `first` marks the first product into D.
+__device__ __forceinline__ void issue_ss_half(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              bool first, uint32_t issue) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
+    mma_ss(d_tmem, sdesc_add(a_desc, off), sdesc_add(b_desc, off), idesc, (first && k == 0) ? 0u : 1u, issue);
+  }
+}
+
+struct DkdvWLayout {
+  static constexpr int OFF_K = 0;                      // K: two halves
+  static constexpr int OFF_V = 2 * kHalf;              // V: two halves
+  static constexpr int OFF_RING = 4 * kHalf;           // kWSlots halves of Q or dO
+  static constexpr int OFF_LD = OFF_RING + kWSlots * kHalf;  // two (lse2[128], delta[128]) pairs, 1 KB each
+  static constexpr int OFF_BAR = OFF_LD + 2048;
+  static constexpr int BAR_KV = 0;          // a unit's K, V landed
+  static constexpr int BAR_KV_EMPTY = 1;    // the MMAs reading a unit's K and V have completed
+  static constexpr int BAR_SLOT_FULL = 2;   // [kWSlots]
+  static constexpr int BAR_SLOT_EMPTY = 5;  // [kWSlots]
+  static constexpr int BAR_LD_EMPTY = 8;    // [2] the step whose LSE / D a buffer holds is finished
+  static constexpr int BAR_S = 10;
+  static constexpr int BAR_DP = 11;
+  static constexpr int BAR_P_READY = 12;
+  static constexpr int BAR_P_HALF = 13;
+  static constexpr int BAR_DS_READY = 14;
+  static constexpr int BAR_ACC = 15;
+  static constexpr int BAR_ACC_FREE = 16;
+  static constexpr int BAR_UNIT_FULL = 17;   // [2]
+  static constexpr int BAR_UNIT_EMPTY = 19;  // [2]
+  static constexpr int BAR_DONE = 21;
+  static constexpr int NBAR = 22;
+  static constexpr int OFF_UNIT = OFF_BAR + NBAR * 8;  // int[2]
+  static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
+  static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
+  static constexpr int BYTES = OFF_ABORT + 8;
+  // the base is rounded up to 1024 bytes inside the allocation; the kernel checks that the
+  // rounding fits (it does for a 1024-aligned start, which the declaration asks for)
+  static constexpr int SMEM_ALLOC = BYTES + 1024 <= kSmemMax ? BYTES + 1024 : kSmemMax;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
+};
+static_assert(DkdvWLayout::BYTES <= kSmemMax, "d = 256 dK/dV kernel exceeds the shared memory of a CTA");
+
+template <typename L>
+__device__ __forceinline__ bool smem_base_fits(uint32_t raw, uint32_t base) {
+  return base - raw + (uint32_t)L::BYTES <= (uint32_t)L::SMEM_ALLOC;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_bwd_dkdv_d256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                            const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                            const BwdParams p) {
+  using L = DkdvWLayout;
+  constexpr int D = 256;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  if (!smem_base_fits<L>(raw, base)) {  // cannot happen with a 1024-aligned start; report, do nothing
+    if (threadIdx.x == 0) atomicExch(p.err, kDevRange);
+    return;
+  }
+  uint8_t* gbase = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + L::OFF_BAR + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_ABORT);
+  const WaitCtx wctx{abort_flag, p.err};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int n_kt = (p.N + 127) / 128;
+  const int BH_kv = p.BH / p.H * p.H_kv;
+  const int per_head = n_kt * 2 * p.kv_split;  // (key tile, d-half, split) per key/value head
+  const int n_units = per_head * BH_kv;
+  const int g_per = p.H / p.H_kv / p.kv_split;
+  struct Unit {
+    int bh, j, h, sp, i_start, n_q, n_it;
+  };
+  auto unit_of = [&](int u) -> Unit {
+    Unit x;
+    int rank;
+    unit_order(u, per_head, BH_kv, p.head_group_kv, x.bh, rank);
+    x.j = rank / (2 * p.kv_split);  // heaviest (first) key tiles first
+    const int rem = rank % (2 * p.kv_split);
+    x.h = rem / p.kv_split;
+    x.sp = rem % p.kv_split;
+    x.i_start = query_lo(x.j * 128, p.causal, p.win_right) / 128;
+    x.n_q = query_hi(min(x.j * 128 + 127, p.N - 1), p.N, p.win_left) / 128 - x.i_start + 1;
+    x.n_it = g_per * x.n_q;
+    return x;
+  };
+  int* unit_ring = reinterpret_cast<int*>(gbase + L::OFF_UNIT);
+  auto next_unit = [&](int k, bool& ok) -> int {
+    const int slot = k & 1;
+    ok = mbar_wait(bar(L::BAR_UNIT_FULL + slot), (k >> 1) & 1, wctx);
+    return ok ? *reinterpret_cast<volatile int*>(unit_ring + slot) : n_units;
+  };
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(L::BAR_KV), 1);
+    mbar_init(bar(L::BAR_KV_EMPTY), 1);
+    for (int s = 0; s < kWSlots; ++s) {
+      mbar_init(bar(L::BAR_SLOT_FULL + s), 1);
+      mbar_init(bar(L::BAR_SLOT_EMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::BAR_LD_EMPTY + s), 1);
+      mbar_init(bar(L::BAR_UNIT_FULL + s), 1);
+      mbar_init(bar(L::BAR_UNIT_EMPTY + s), 1 + 256);
+    }
+    mbar_init(bar(L::BAR_S), 1);
+    mbar_init(bar(L::BAR_DP), 1);
+    mbar_init(bar(L::BAR_P_READY), 256);
+    mbar_init(bar(L::BAR_P_HALF), 256);
+    mbar_init(bar(L::BAR_DS_READY), 256);
+    mbar_init(bar(L::BAR_ACC), 1);
+    mbar_init(bar(L::BAR_ACC_FREE), 256);
+    mbar_init(bar(L::BAR_DONE), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(base + L::OFF_TMEM_SLOT, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_TMEM_SLOT);
+
+  // The FIFO order of a unit with n steps (step t: query tile and head of `it`), which the
+  // producer fills and the MMA warp drains:  Q0(0) Q1(0) dO0(0) dO1(0), then for it = 0..n-1:
+  // dOh(it), [Q0(it+1) Q1(it+1)], Qh(it), [dO0(it+1) dO1(it+1)]  (bracketed parts while
+  // it + 1 < n; Xk = half k of X, h = the unit's half).
+  if (warp == 0) {
+    // ===================================================== TMA producer + work distribution
+    regs_dec<kRegsLow>();
+    const uint32_t leader = elect_one();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    int F = 0;  // halves put in the FIFO so far (all units)
+    int T = 0;  // steps of the previous units
+    int kv_issued = 0;
+    bool ok = true;
+    // half `half` of Q (which = 0) or dO (which = 1) for the unit step `it`; with_ld: also the
+    // step's LSE * log2(e) and D rows (global step t) into their buffer
+    auto load_half = [&](const Unit& x, int which, int half, int it, bool with_ld) -> bool {
+      const int st = F % kWSlots;
+      if (!mbar_wait(bar(L::BAR_SLOT_EMPTY + st), ((F / kWSlots) & 1) ^ 1u, wctx)) return false;
+      const int t = T + it;
+      const int i = x.i_start + it % x.n_q;
+      const int bhq = q_head_of(x.bh, x.sp * g_per + it / x.n_q, p.H, p.H_kv);
+      if (with_ld && t >= 2 && !mbar_wait(bar(L::BAR_LD_EMPTY + (t & 1)), ((t >> 1) - 1) & 1, wctx)) return false;
+      const uint32_t fb = bar(L::BAR_SLOT_FULL + st);
+      mbar_arrive_expect_tx(fb, kHalf + (with_ld ? 1024 : 0), leader);
+      const CUtensorMap* m = which ? &tm_do : &tm_q;
+      const uint32_t dst = base + L::OFF_RING + st * kHalf;
+      for (int b = 0; b < 2; ++b) tma_load_3d(dst + b * kBox, m, half * 128 + b * 64, i * 128, bhq, fb, leader);
+      if (with_ld) {
+        const size_t roff = (size_t)bhq * p.Np + (size_t)i * 128;
+        bulk_load(base + L::OFF_LD + (t & 1) * 1024, p.lse2 + roff, 512, fb, leader);
+        bulk_load(base + L::OFF_LD + (t & 1) * 1024 + 512, p.delta + roff, 512, fb, leader);
+      }
+      ++F;
+      return true;
+    };
+    for (int uc = 0;; ++uc) {
+      if (uc >= 2 && !(ok = mbar_wait(bar(L::BAR_UNIT_EMPTY + (uc & 1)), ((uc - 2) >> 1) & 1, wctx))) break;
+      int u = 0;
+      if (lane == 0) u = (int)atomicAdd(p.dkdv_counter, 1u);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (lane == 0) {
+        unit_ring[uc & 1] = u < n_units ? u : n_units;
+        mbar_arrive(bar(L::BAR_UNIT_FULL + (uc & 1)));
+      }
+      __syncwarp();
+      if (u >= n_units) break;
+      const Unit x = unit_of(u);
+      if (uc > 0 && !(ok = mbar_wait(bar(L::BAR_KV_EMPTY), (uc - 1) & 1, wctx))) break;
+      mbar_arrive_expect_tx(bar(L::BAR_KV), 4 * kHalf, leader);
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t off = (c >> 1) * kHalf + (c & 1) * kBox;
+        tma_load_3d(base + L::OFF_K + off, &tm_k, c * 64, x.j * 128, x.bh, bar(L::BAR_KV), leader);
+        tma_load_3d(base + L::OFF_V + off, &tm_v, c * 64, x.j * 128, x.bh, bar(L::BAR_KV), leader);
+      }
+      ++kv_issued;
+      const int n = x.n_it;
+      ok = load_half(x, 0, 0, 0, true) && load_half(x, 0, 1, 0, false) && load_half(x, 1, 0, 0, false) &&
+           load_half(x, 1, 1, 0, false);
+      for (int it = 0; it < n && ok; ++it) {
+        ok = load_half(x, 1, x.h, it, false);  // dO half h for dV(it)
+        if (ok && it + 1 < n) ok = load_half(x, 0, 0, it + 1, true) && load_half(x, 0, 1, it + 1, false);
+        if (ok) ok = load_half(x, 0, x.h, it, false);  // Q half h for dK(it)
+        if (ok && it + 1 < n) ok = load_half(x, 1, 0, it + 1, false) && load_half(x, 1, 1, it + 1, false);
+      }
+      if (!ok) break;
+      T += n;
+    }
+    // drain: every issued copy has landed before the CTA may exit
+    if (kv_issued > 0) drain_wait(bar(L::BAR_KV), (kv_issued - 1) & 1);
+    for (int f = (F > kWSlots ? F - kWSlots : 0); f < F; ++f)
+      drain_wait(bar(L::BAR_SLOT_FULL + f % kWSlots), (f / kWSlots) & 1);
+  } else if (warp == 1) {
+    // ===================================================== MMA issuer
+    regs_dec<kRegsLow>();
+    const uint32_t leader = elect_one();
+    constexpr uint32_t idesc_s = make_idesc(128, 128, false, false, false);  // M=128 keys, N=128 queries
+    constexpr uint32_t idesc_g = make_idesc(128, 128, false, false, true);   // N=128 (a d-half), B MN-major
+    const uint64_t dKs[2] = {make_sdesc_sw128(base + L::OFF_K, 16, 1024),
+                             make_sdesc_sw128(base + L::OFF_K + kHalf, 16, 1024)};
+    const uint64_t dVs[2] = {make_sdesc_sw128(base + L::OFF_V, 16, 1024),
+                             make_sdesc_sw128(base + L::OFF_V + kHalf, 16, 1024)};
+    const uint64_t dRingK = make_sdesc_sw128(base + L::OFF_RING, 16, 1024);     // a half as K-major B
+    const uint64_t dRingMN = make_sdesc_sw128(base + L::OFF_RING, kBox, 1024);  // a half as MN-major B
+    int C = 0;  // halves taken from the FIFO so far
+    bool ok = true;
+    auto take = [&]() -> int {
+      const int st = C % kWSlots;
+      ok = mbar_wait(bar(L::BAR_SLOT_FULL + st), (C / kWSlots) & 1, wctx);
+      ++C;
+      if (ok) tc_fence_after();
+      return st;
+    };
+    // S^T = K Q^T (or dP^T = V dO^T) over both d-halves, each half taken from the FIFO
+    auto issue_full = [&](uint32_t d_tmem, const uint64_t (&a)[2], uint32_t done_bar) -> bool {
+      for (int hh = 0; hh < 2; ++hh) {
+        const int st = take();
+        if (!ok) return false;
+        issue_ss_half(d_tmem, a[hh], sdesc_add(dRingK, st * kHalf), idesc_s, hh == 0, leader);
+        mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
+      }
+      mma_commit(done_bar, leader);
+      return true;
+    };
+    int T0 = 0;
+    for (int uc = 0; ok; ++uc) {
+      const int u = next_unit(uc, ok);
+      if (lane == 0) mbar_arrive(bar(L::BAR_UNIT_EMPTY + (uc & 1)));
+      if (!ok || u >= n_units) break;
+      const int n = unit_of(u).n_it;
+      if (!(ok = mbar_wait(bar(L::BAR_KV), uc & 1, wctx))) break;
+      tc_fence_after();
+      if (!(ok = issue_full(tmem + L::T_S, dKs, bar(L::BAR_S)))) break;
+      if (!(ok = issue_full(tmem + L::T_DP, dVs, bar(L::BAR_DP)))) break;
+      if (n == 1) mma_commit(bar(L::BAR_KV_EMPTY), leader);
+      for (int it = 0; it < n && ok; ++it) {
+        const int t = T0 + it;
+        // dV_h += P^T dO_h in two halves (the first while the second half of P^T is computed);
+        // the unit's first product overwrites the accumulators, which the previous unit's
+        // epilogue must have read
+        int st = take();
+        if (!ok) break;
+        if (!(ok = mbar_wait(bar(L::BAR_P_HALF), t & 1, wctx))) break;
+        tc_fence_after();
+        if (it == 0 && uc > 0) {
+          if (!(ok = mbar_wait(bar(L::BAR_ACC_FREE), (uc - 1) & 1, wctx))) break;
+          tc_fence_after();
+        }
+        const uint64_t dmn = sdesc_add(dRingMN, st * kHalf);
+        issue_ts_split_part(tmem + L::T_DV, tmem + L::T_S, dmn, idesc_g, it == 0, 0, leader);
+        if (!(ok = mbar_wait(bar(L::BAR_P_READY), t & 1, wctx))) break;
+        tc_fence_after();
+        issue_ts_split_part(tmem + L::T_DV, tmem + L::T_S, dmn, idesc_g, false, 1, leader);
+        mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
+        if (it + 1 < n && !(ok = issue_full(tmem + L::T_S, dKs, bar(L::BAR_S)))) break;  // S^T(it + 1)
+        st = take();
+        if (!ok) break;
+        if (!(ok = mbar_wait(bar(L::BAR_DS_READY), t & 1, wctx))) break;
+        tc_fence_after();
+        issue_ts_split(tmem + L::T_DK, tmem + L::T_DP, sdesc_add(dRingMN, st * kHalf), idesc_g, it > 0,
+                       leader);  // dK_h += dS^T Q_h
+        mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
+        mma_commit(bar(L::BAR_LD_EMPTY + (t & 1)), leader);  // step t's LSE / D buffer is free after this
+        if (it + 1 < n) {
+          if (!(ok = issue_full(tmem + L::T_DP, dVs, bar(L::BAR_DP)))) break;  // dP^T(it + 1)
+          if (it + 2 == n) mma_commit(bar(L::BAR_KV_EMPTY), leader);  // the unit's last S^T, dP^T issued
+        }
+      }
+      if (!ok) break;
+      mma_commit(bar(L::BAR_ACC), leader);
+      T0 += n;
+    }
+    mma_commit(bar(L::BAR_DONE), leader);
+    drain_wait(bar(L::BAR_DONE), 0);
+  } else if (warp < 4) {
+    regs_dec<kRegsLow>();  // warps 2-3: idle
+  } else {
+    // ===================================================== compute warpgroups
+    regs_inc<kRegsHigh>();
+    const int w = (warp - 4) >> 2;   // query columns [64 w, 64 w + 64) of every step
+    const int wq = (warp - 4) & 3;
+    const int row = wq * 32 + lane;  // key row inside the tile
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + L::T_S + 64 * w;
+    const uint32_t tDP = tmem + lane_off + L::T_DP + 64 * w;
+    const float sl2 = ldexpf(p.scale_log2, -(p.exps[kExpQ] + p.exps[kExpK]));
+    const uint64_t sl2x2 = f2pack(sl2, sl2);
+    bool ok = true;
+    int T0 = 0;
+    int u = next_unit(0, ok);
+    mbar_arrive(bar(L::BAR_UNIT_EMPTY + 0));
+    for (int uc = 0; ok && u < n_units; ++uc) {
+      const Unit x = unit_of(u);
+      const int j = x.j, i_start = x.i_start, n_q = x.n_q, n_it = x.n_it;
+      const int key = j * 128 + row;
+      const int q_vis_lo = query_lo(key, p.causal, p.win_right);
+      const int q_vis_hi = query_hi(key, p.N, p.win_left);
+      const int all_lo = query_lo(min(j * 128 + 127, p.N - 1), p.causal, p.win_right);
+      const int all_hi = query_hi(j * 128, p.N, p.win_left);
+      for (int it = 0; it < n_it; ++it) {
+        const int T = T0 + it;
+        const int i = i_start + it % n_q;
+        const float* lse2 = reinterpret_cast<const float*>(gbase + L::OFF_LD + (T & 1) * 1024) + 64 * w;
+        const float* delta = lse2 + 128;
+        const int q0 = i * 128 + 64 * w;
+        if (!(ok = mbar_wait(bar(L::BAR_S), T & 1, wctx))) break;
+        tc_fence_after();
+        float pr[64];
+        tmem_ld64(tS, pr);
+        auto probs = [&](auto masked) {
+          const int c_lo = q_vis_lo - q0, c_hi = q_vis_hi - q0;
+#pragma unroll
+          for (int g = 0; g < 64; g += 16) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int c = g; c < g + 16; c += 4) {
+              const float4 L4 = *reinterpret_cast<const float4*>(lse2 + c);
+              float t0, t1, t2, t3;
+              f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, f2pack(-L4.x, -L4.y)), t0, t1);
+              f2unpack(ffma2(f2pack(pr[c + 2], pr[c + 3]), sl2x2, f2pack(-L4.z, -L4.w)), t2, t3);
+              if ((c - g) < kDkdvExpFmaPer16) {
+                exp2_fma_pipe(t0, t1);
+                exp2_fma_pipe(t2, t3);
+                pr[c] = t0;
+                pr[c + 1] = t1;
+                pr[c + 2] = t2;
+                pr[c + 3] = t3;
+              } else {
+                pr[c] = ex2_approx(t0);
+                pr[c + 1] = ex2_approx(t1);
+                pr[c + 2] = ex2_approx(t2);
+                pr[c + 3] = ex2_approx(t3);
+              }
+              if constexpr (decltype(masked)::value) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (c + e < c_lo || c + e > c_hi) pr[c + e] = 0.f;
+              }
+              pk[(c - g) / 2] = pack_f16(pr[c], pr[c + 1]);
+              pk[(c - g) / 2 + 1] = pack_f16(pr[c + 2], pr[c + 3]);
+            }
+            tmem_st8(tS + g / 2, pk);
+            if (g == 16) {
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(bar(L::BAR_P_HALF));
+            }
+          }
+        };
+        if (q0 < all_lo || q0 + 63 > all_hi)
+          probs(std::true_type{});
+        else
+          probs(std::false_type{});
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::BAR_P_READY));
+        if (!(ok = mbar_wait(bar(L::BAR_DP), T & 1, wctx))) break;
+        tc_fence_after();
+        float dp[64];
+        tmem_ld64(tDP, dp);
+#pragma unroll
+        for (int g = 0; g < 64; g += 16) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int c = g; c < g + 16; c += 4) {
+            const float4 D4 = *reinterpret_cast<const float4*>(delta + c);
+            float d0, d1, d2, d3;
+            f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(f2pack(dp[c], dp[c + 1]), f2pack(D4.x, D4.y))), d0, d1);
+            f2unpack(fmul2(f2pack(pr[c + 2], pr[c + 3]), fsub2(f2pack(dp[c + 2], dp[c + 3]), f2pack(D4.z, D4.w))), d2,
+                     d3);
+            pk[(c - g) / 2] = pack_f16(d0, d1);
+            pk[(c - g) / 2 + 1] = pack_f16(d2, d3);
+          }
+          tmem_st8(tDP + g / 2, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::BAR_DS_READY));
+      }
+      if (!ok) break;
+      if (!(ok = mbar_wait(bar(L::BAR_ACC), uc & 1, wctx))) break;
+      tc_fence_after();
+      // warpgroup 0 writes dV[:, h], warpgroup 1 scale * dK[:, h] (128 columns each)
+      const size_t head_off = p.kv_split == 1 ? (size_t)x.bh * p.N * D : ((size_t)x.sp * BH_kv + x.bh) * p.N * D;
+      float* out = (p.kv_split == 1 ? (w == 0 ? p.dv : p.dk) : (w == 0 ? p.dv_part : p.dk_part)) + head_off +
+                   128 * x.h;
+      const uint32_t t_acc = tmem + lane_off + (w == 0 ? L::T_DV : L::T_DK);
+      const Pow2 out_f = pow2_factors(w == 0 ? -p.exps[kExpDO] : -(p.exps[kExpV] + p.exps[kExpDO] + p.exps[kExpQ]));
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float acc[64];
+        tmem_ld64(t_acc + 64 * c, acc);
+        if (c == 1) {
+          tc_fence_before();
+          mbar_arrive(bar(L::BAR_ACC_FREE));
+        }
+        warp_store_rows_f32<64>(acc, out + 64 * c, D, j * 128 + wq * 32, p.N, w == 0 ? 1.0f : p.scale, out_f);
+      }
+      T0 += n_it;
+      u = next_unit(uc + 1, ok);
+      mbar_arrive(bar(L::BAR_UNIT_EMPTY + ((uc + 1) & 1)));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+struct DqWLayout {
+  static constexpr int OFF_Q = 0;              // Q: two halves (resident for the unit)
+  static constexpr int OFF_DO = 2 * kHalf;     // dO: two halves
+  static constexpr int OFF_RING = 4 * kHalf;   // kWSlots halves of K or V
+  static constexpr int OFF_BAR = OFF_RING + kWSlots * kHalf;
+  static constexpr int BAR_Q = 0;           // a unit's Q and dO landed
+  static constexpr int BAR_Q_EMPTY = 1;     // the MMAs reading a unit's Q and dO have completed
+  static constexpr int BAR_SLOT_FULL = 2;   // [kWSlots]
+  static constexpr int BAR_SLOT_EMPTY = 5;  // [kWSlots]
+  static constexpr int BAR_S = 8;
+  static constexpr int BAR_DP = 9;
+  static constexpr int BAR_DS = 10;         // dS of a step written over S, dP read
+  static constexpr int BAR_ACC = 11;
+  static constexpr int BAR_DQ_FREE = 12;
+  static constexpr int BAR_UNIT_FULL = 13;   // [2]
+  static constexpr int BAR_UNIT_EMPTY = 15;  // [2]
+  static constexpr int BAR_DONE = 17;
+  static constexpr int NBAR = 18;
+  static constexpr int OFF_UNIT = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
+  static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
+  static constexpr int BYTES = OFF_ABORT + 8;
+  static constexpr int SMEM_ALLOC = BYTES + 1024 <= kSmemMax ? BYTES + 1024 : kSmemMax;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
+};
+static_assert(DqWLayout::BYTES <= kSmemMax, "d = 256 dQ kernel exceeds the shared memory of a CTA");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_bwd_dq_d256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const BwdParams p) {
+  using L = DqWLayout;
+  constexpr int D = 256;
+#ifndef FA_DQ_EXP_FMA_PER16
+#define FA_DQ_EXP_FMA_PER16 4
+#endif
+  constexpr int kDqExpFmaPer16 = FA_DQ_EXP_FMA_PER16;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  if (!smem_base_fits<L>(raw, base)) {
+    if (threadIdx.x == 0) atomicExch(p.err, kDevRange);
+    return;
+  }
+  uint8_t* gbase = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + L::OFF_BAR + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_ABORT);
+  const WaitCtx wctx{abort_flag, p.err};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int nq = (p.N + 127) / 128;
+  const int n_units = nq * p.BH;
+  struct Unit {
+    int bh, bh_kv, qt, jlo, n_it;
+  };
+  auto unit_of = [&](int u) -> Unit {
+    Unit x;
+    int rank;
+    unit_order(u, nq, p.BH, p.head_group, x.bh, rank);
+    x.bh_kv = kv_head_of(x.bh, p.H, p.H_kv);
+    x.qt = p.causal ? (nq - 1 - rank) : rank;
+    x.jlo = key_lo(x.qt * 128, p.N, p.win_left) / 128;
+    x.n_it = key_hi(x.qt * 128 + 127, p.N, p.causal, p.win_right) / 128 - x.jlo + 1;
+    return x;
+  };
+  int* unit_ring = reinterpret_cast<int*>(gbase + L::OFF_UNIT);
+  auto next_unit = [&](int k, bool& ok) -> int {
+    const int slot = k & 1;
+    ok = mbar_wait(bar(L::BAR_UNIT_FULL + slot), (k >> 1) & 1, wctx);
+    return ok ? *reinterpret_cast<volatile int*>(unit_ring + slot) : n_units;
+  };
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(L::BAR_Q), 1);
+    mbar_init(bar(L::BAR_Q_EMPTY), 1);
+    for (int s = 0; s < kWSlots; ++s) {
+      mbar_init(bar(L::BAR_SLOT_FULL + s), 1);
+      mbar_init(bar(L::BAR_SLOT_EMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::BAR_UNIT_FULL + s), 1);
+      mbar_init(bar(L::BAR_UNIT_EMPTY + s), 1 + 256);
+    }
+    mbar_init(bar(L::BAR_S), 1);
+    mbar_init(bar(L::BAR_DP), 1);
+    mbar_init(bar(L::BAR_DS), 256);
+    mbar_init(bar(L::BAR_ACC), 1);
+    mbar_init(bar(L::BAR_DQ_FREE), 256);
+    mbar_init(bar(L::BAR_DONE), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(base + L::OFF_TMEM_SLOT, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_TMEM_SLOT);
+
+  // FIFO order of a unit with n key steps: K0(0) K1(0) V0(0) V1(0), then for it = 0..n-1:
+  // K0(it) K1(it) [dQ], [V0(it+1) V1(it+1) K0(it+1) K1(it+1)]  (bracketed part while it + 1 < n).
+  if (warp == 0) {
+    // ===================================================== TMA producer + work distribution
+    regs_dec<kRegsLow>();
+    const uint32_t leader = elect_one();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    int F = 0, q_issued = 0;
+    bool ok = true;
+    auto load_half = [&](const Unit& x, int which, int half, int it) -> bool {  // half of K (0) or V (1)
+      const int st = F % kWSlots;
+      if (!mbar_wait(bar(L::BAR_SLOT_EMPTY + st), ((F / kWSlots) & 1) ^ 1u, wctx)) return false;
+      const uint32_t fb = bar(L::BAR_SLOT_FULL + st);
+      mbar_arrive_expect_tx(fb, kHalf, leader);
+      const CUtensorMap* m = which ? &tm_v : &tm_k;
+      const uint32_t dst = base + L::OFF_RING + st * kHalf;
+      for (int b = 0; b < 2; ++b)
+        tma_load_3d(dst + b * kBox, m, half * 128 + b * 64, (x.jlo + it) * 128, x.bh_kv, fb, leader);
+      ++F;
+      return true;
+    };
+    for (int uc = 0;; ++uc) {
+      if (uc >= 2 && !(ok = mbar_wait(bar(L::BAR_UNIT_EMPTY + (uc & 1)), ((uc - 2) >> 1) & 1, wctx))) break;
+      int u = 0;
+      if (lane == 0) u = (int)atomicAdd(p.dq_counter, 1u);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (lane == 0) {
+        unit_ring[uc & 1] = u < n_units ? u : n_units;
+        mbar_arrive(bar(L::BAR_UNIT_FULL + (uc & 1)));
+      }
+      __syncwarp();
+      if (u >= n_units) break;
+      const Unit x = unit_of(u);
+      if (uc > 0 && !(ok = mbar_wait(bar(L::BAR_Q_EMPTY), (uc - 1) & 1, wctx))) break;
+      mbar_arrive_expect_tx(bar(L::BAR_Q), 4 * kHalf, leader);
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t off = (c >> 1) * kHalf + (c & 1) * kBox;
+        tma_load_3d(base + L::OFF_Q + off, &tm_q, c * 64, x.qt * 128, x.bh, bar(L::BAR_Q), leader);
+        tma_load_3d(base + L::OFF_DO + off, &tm_do, c * 64, x.qt * 128, x.bh, bar(L::BAR_Q), leader);
+      }
+      ++q_issued;
+      const int n = x.n_it;
+      ok = load_half(x, 0, 0, 0) && load_half(x, 0, 1, 0) && load_half(x, 1, 0, 0) && load_half(x, 1, 1, 0);
+      for (int it = 0; it < n && ok; ++it) {
+        ok = load_half(x, 0, 0, it) && load_half(x, 0, 1, it);  // K again, for dQ(it)
+        if (ok && it + 1 < n)
+          ok = load_half(x, 1, 0, it + 1) && load_half(x, 1, 1, it + 1) && load_half(x, 0, 0, it + 1) &&
+               load_half(x, 0, 1, it + 1);
+      }
+      if (!ok) break;
+    }
+    if (q_issued > 0) drain_wait(bar(L::BAR_Q), (q_issued - 1) & 1);
+    for (int f = (F > kWSlots ? F - kWSlots : 0); f < F; ++f)
+      drain_wait(bar(L::BAR_SLOT_FULL + f % kWSlots), (f / kWSlots) & 1);
+  } else if (warp == 1) {
+    // ===================================================== MMA issuer
+    regs_dec<kRegsLow>();
+    const uint32_t leader = elect_one();
+    constexpr uint32_t idesc_s = make_idesc(128, 128, false, false, false);  // M=128 queries, N=128 keys
+    constexpr uint32_t idesc_g = make_idesc(128, 128, false, false, true);   // N=128 (a d-half), B MN-major
+    const uint64_t dQs[2] = {make_sdesc_sw128(base + L::OFF_Q, 16, 1024),
+                             make_sdesc_sw128(base + L::OFF_Q + kHalf, 16, 1024)};
+    const uint64_t dDOs[2] = {make_sdesc_sw128(base + L::OFF_DO, 16, 1024),
+                              make_sdesc_sw128(base + L::OFF_DO + kHalf, 16, 1024)};
+    const uint64_t dRingK = make_sdesc_sw128(base + L::OFF_RING, 16, 1024);
+    const uint64_t dRingMN = make_sdesc_sw128(base + L::OFF_RING, kBox, 1024);
+    int C = 0;
+    bool ok = true;
+    auto take = [&]() -> int {
+      const int st = C % kWSlots;
+      ok = mbar_wait(bar(L::BAR_SLOT_FULL + st), (C / kWSlots) & 1, wctx);
+      ++C;
+      if (ok) tc_fence_after();
+      return st;
+    };
+    // S = Q K^T (dP = dO V^T) over both d-halves, each half of K (V) taken from the FIFO
+    auto issue_full = [&](uint32_t d_tmem, const uint64_t (&a)[2], uint32_t done_bar) -> bool {
+      for (int hh = 0; hh < 2; ++hh) {
+        const int st = take();
+        if (!ok) return false;
+        issue_ss_half(d_tmem, a[hh], sdesc_add(dRingK, st * kHalf), idesc_s, hh == 0, leader);
+        mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
+      }
+      mma_commit(done_bar, leader);
+      return true;
+    };
+    int T0 = 0;
+    for (int uc = 0;; ++uc) {
+      const int u = next_unit(uc, ok);
+      if (lane == 0) mbar_arrive(bar(L::BAR_UNIT_EMPTY + (uc & 1)));
+      if (!ok || u >= n_units) break;
+      const int n = unit_of(u).n_it;
+      if (!(ok = mbar_wait(bar(L::BAR_Q), uc & 1, wctx))) break;
+      tc_fence_after();
+      if (!(ok = issue_full(tmem + L::T_S, dQs, bar(L::BAR_S)))) break;
+      if (!(ok = issue_full(tmem + L::T_DP, dDOs, bar(L::BAR_DP)))) break;
+      if (n == 1) mma_commit(bar(L::BAR_Q_EMPTY), leader);
+      for (int it = 0; it < n && ok; ++it) {
+        const int t = T0 + it;
+        if (!(ok = mbar_wait(bar(L::BAR_DS), t & 1, wctx))) break;
+        tc_fence_after();
+        if (it == 0 && uc > 0) {
+          if (!(ok = mbar_wait(bar(L::BAR_DQ_FREE), (uc - 1) & 1, wctx))) break;
+          tc_fence_after();
+        }
+        for (int hh = 0; hh < 2 && ok; ++hh) {  // dQ[:, 128 hh ..] += dS K_hh
+          const int st = take();
+          if (!ok) break;
+          issue_ts_split(tmem + L::T_DQ + 128 * hh, tmem + L::T_S, sdesc_add(dRingMN, st * kHalf), idesc_g, it > 0,
+                         leader);
+          mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
+        }
+        if (!ok) break;
+        if (it + 1 < n) {
+          if (!(ok = issue_full(tmem + L::T_DP, dDOs, bar(L::BAR_DP)))) break;  // dP(it + 1)
+          if (!(ok = issue_full(tmem + L::T_S, dQs, bar(L::BAR_S)))) break;     // S(it + 1), after dQ(it)
+          if (it + 2 == n) mma_commit(bar(L::BAR_Q_EMPTY), leader);
+        }
+      }
+      if (ok) mma_commit(bar(L::BAR_ACC), leader);
+      T0 += n;
+    }
+    mma_commit(bar(L::BAR_DONE), leader);
+    drain_wait(bar(L::BAR_DONE), 0);
+  } else if (warp < 4) {
+    regs_dec<kRegsLow>();  // warps 2-3: idle
+  } else {
+    // ===================================================== compute warpgroups
+    regs_inc<kRegsHigh>();
+    const int w = (warp - 4) >> 2;   // key columns [64 w, 64 w + 64) of every step
+    const int wq = (warp - 4) & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + L::T_S + 64 * w;
+    const float sl2 = ldexpf(p.scale_log2, -(p.exps[kExpQ] + p.exps[kExpK]));
+    const uint64_t sl2x2 = f2pack(sl2, sl2);
+    bool ok = true;
+    int T0 = 0;
+    float lse2 = 0.f, delta = 0.f;
+    int u = next_unit(0, ok);
+    mbar_arrive(bar(L::BAR_UNIT_EMPTY + 0));
+    if (ok && u < n_units) {
+      const Unit x0 = unit_of(u);
+      const size_t prow = (size_t)x0.bh * p.Np + x0.qt * 128 + row;
+      lse2 = p.lse2[prow];
+      delta = p.delta[prow];
+    }
+    for (int uc = 0; ok && u < n_units; ++uc) {
+      const Unit x = unit_of(u);
+      const int r = x.qt * 128 + row;
+      const int k_vis_lo = key_lo(r, p.N, p.win_left);
+      const int k_vis_hi = key_hi(r, p.N, p.causal, p.win_right);
+      const int all_lo = key_lo(min(x.qt * 128 + 127, p.N - 1), p.N, p.win_left);
+      const int all_hi = key_hi(x.qt * 128, p.N, p.causal, p.win_right);
+      const uint64_t nl2 = f2pack(-lse2, -lse2), dd = f2pack(delta, delta);
+      for (int it = 0; it < x.n_it; ++it) {
+        const int t = T0 + it;
+        const int k0 = (x.jlo + it) * 128 + 64 * w;
+        if (!(ok = mbar_wait(bar(L::BAR_S), t & 1, wctx))) break;
+        tc_fence_after();
+        float pr[64];
+        tmem_ld64(tS, pr);
+        auto probs = [&](auto masked) {
+          const int c_lo = k_vis_lo - k0, c_hi = k_vis_hi - k0;
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            float t0, t1;
+            f2unpack(ffma2(f2pack(pr[c], pr[c + 1]), sl2x2, nl2), t0, t1);
+            if ((c & 15) < kDqExpFmaPer16) {
+              exp2_fma_pipe(t0, t1);
+              pr[c] = t0;
+              pr[c + 1] = t1;
+            } else {
+              pr[c] = ex2_approx(t0);
+              pr[c + 1] = ex2_approx(t1);
+            }
+            if constexpr (decltype(masked)::value) {
+              if (c < c_lo || c > c_hi) pr[c] = 0.f;
+              if (c + 1 < c_lo || c + 1 > c_hi) pr[c + 1] = 0.f;
+            }
+          }
+        };
+        if (k0 < all_lo || k0 + 63 > all_hi)
+          probs(std::true_type{});
+        else
+          probs(std::false_type{});
+        if (!(ok = mbar_wait(bar(L::BAR_DP), t & 1, wctx))) break;
+        tc_fence_after();
+        float dp[64];
+        tmem_ld64(tmem + lane_off + L::T_DP + 64 * w, dp);
+#pragma unroll
+        for (int g = 0; g < 64; g += 16) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int c = g; c < g + 16; c += 2) {
+            float d0, d1;
+            f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(f2pack(dp[c], dp[c + 1]), dd)), d0, d1);
+            pk[(c - g) / 2] = pack_f16(d0, d1);
+          }
+          tmem_st8(tS + g / 2, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::BAR_DS));
+      }
+      if (!ok) break;
+      if (!(ok = mbar_wait(bar(L::BAR_ACC), uc & 1, wctx))) break;
+      tc_fence_after();
+      // each warpgroup writes 128 of the 256 columns of scale * dQ, 64 at a time
+      const Pow2 out_f = pow2_factors(-(p.exps[kExpV] + p.exps[kExpDO] + p.exps[kExpK]));
+      const int u_next = next_unit(uc + 1, ok);
+      mbar_arrive(bar(L::BAR_UNIT_EMPTY + ((uc + 1) & 1)));
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float acc[64];
+        tmem_ld64(tmem + lane_off + L::T_DQ + w * 128 + 64 * c, acc);
+        if (c == 1) {
+          tc_fence_before();
+          mbar_arrive(bar(L::BAR_DQ_FREE));
+        }
+        warp_store_rows_f32<64>(acc, p.dq + (size_t)x.bh * p.N * D + w * 128 + 64 * c, D, x.qt * 128 + wq * 32,
+                                p.N, p.scale, out_f);
+      }
+      if (ok && u_next < n_units) {  // the next unit's row statistics
+        const Unit xn = unit_of(u_next);
+        const size_t prow = (size_t)xn.bh * p.Np + xn.qt * 128 + row;
+        lse2 = p.lse2[prow];
+        delta = p.delta[prow];
+      }
+      T0 += x.n_it;
+      u = u_next;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
 template <typename Layout, typename Kern>
 cudaError_t launch_one(Kern kern, dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                        const CUtensorMap& d, const BwdParams& p, cudaStream_t s) {
@@ -936,9 +1724,12 @@ cudaError_t launch_one(Kern kern, dim3 grid, const CUtensorMap& a, const CUtenso
 
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                                   const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s) {
-  // persistent: one CTA per SM (at most one per unit: key tile x key/value head x group split)
-  const long long units = (long long)((p.N + 127) / 128) * (p.BH / p.H * p.H_kv) * p.kv_split;
+  // persistent: one CTA per SM (at most one per unit: key tile x key/value head x group split,
+  // and x the d-half at d = 256)
+  const long long units =
+      (long long)((p.N + 127) / 128) * (p.BH / p.H * p.H_kv) * p.kv_split * (d == 256 ? 2 : 1);
   const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
+  if (d == 256) return launch_one<DkdvWLayout>(fa_bwd_dkdv_d256_kernel, grid, tq, tdo, tk, tv, p, s);
   if (d == 128)
     return launch_one<DkdvLayout<128>>(fa_bwd_dkdv_sm100_kernel<128>, grid, tq, tdo, tk, tv, p, s);
   return launch_one<DkdvLayout<64>>(fa_bwd_dkdv_sm100_kernel<64>, grid, tq, tdo, tk, tv, p, s);
@@ -949,6 +1740,7 @@ cudaError_t launch_bwd_dq_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, c
   // persistent: one CTA per SM (at most one per work unit)
   const long long units = (long long)((p.N + 127) / 128) * p.BH;
   const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
+  if (d == 256) return launch_one<DqWLayout>(fa_bwd_dq_d256_kernel, grid, tq, tdo, tk, tv, p, s);
   if (d == 128) return launch_one<DqLayout<128>>(fa_bwd_dq_sm100_kernel<128>, grid, tq, tdo, tk, tv, p, s);
   return launch_one<DqLayout<64>>(fa_bwd_dq_sm100_kernel<64>, grid, tq, tdo, tk, tv, p, s);
 }

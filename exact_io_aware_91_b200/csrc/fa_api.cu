@@ -70,7 +70,7 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // Shared validation of sizes/scalars.  Returns FA_OK and sets *empty when there is nothing to do.
 // H_kv: key/value heads (H for plain multi-head attention); H must be a multiple of it.
-// allow_d256: the forward with a workspace also takes d = 256 (its own persistent kernel)
+// allow_d256: the forward with a workspace and the backward also take d = 256 (kernels of their own)
 fa_status check_problem(int B, int H, int H_kv, int N, int d, float scale, int causal, bool* empty,
                         bool allow_d256 = false) {
   if (B < 0 || H < 0 || N < 0 || H_kv < 0) return FA_ERR_INVALID_ARG;
@@ -120,9 +120,10 @@ constexpr size_t kCtrlCounters = 0, kCtrlExps = 16;
 // heads are split over kv_split CTAs -- the smallest divisor of the group size that gives at
 // least four CTAs per SM -- whose partial sums a reduction kernel adds up.
 constexpr long long kDkdvMinUnits = 4 * 148;
-int kv_split_for(int B, int H, int H_kv, int N) {
+int kv_split_for(int B, int H, int H_kv, int N, int d) {
   const int group = H / H_kv;
-  const long long units = (long long)B * H_kv * ((N + 127) / 128);
+  // at d = 256 every key tile is two units (one per d-half of dK, dV)
+  const long long units = (long long)B * H_kv * ((N + 127) / 128) * (d == 256 ? 2 : 1);
   for (int s = 1; s < group; ++s)
     if (group % s == 0 && units * s >= kDkdvMinUnits) return s;
   return group;
@@ -135,7 +136,7 @@ int kv_split_for(int B, int H, int H_kv, int N) {
 // preprocess's per-block maxima of |Q|, |K|, |V|, |dO|.
 BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d) {
   BwdLayout w{};
-  w.kv_split = kv_split_for(B, H, H_kv, N);
+  w.kv_split = kv_split_for(B, H, H_kv, N, d);
   const size_t t16 = align256((size_t)B * H * N * d * 2);
   const size_t t16kv = align256((size_t)B * H_kv * N * d * 2);
   w.Np = ((N + 127) / 128) * 128;
@@ -314,7 +315,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) { return fa_bwd_gqa_wor
 
 size_t fa_bwd_gqa_workspace_size(int B, int H, int H_kv, int N, int d) {
   bool empty = false;
-  if (check_problem(B, H, H_kv, N, d, 1.0f, 0, &empty) != FA_OK || empty) return 0;
+  if (check_problem(B, H, H_kv, N, d, 1.0f, 0, &empty, true) != FA_OK || empty) return 0;
   return bwd_layout(B, H, H_kv, N, d).total;
 }
 
@@ -348,7 +349,7 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
                    fa_stream_t stream) {
   bool empty = false;
   if (!window_ok(wl, wr)) return FA_ERR_INVALID_ARG;
-  fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty);
+  fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty, true);  // d in {64, 128, 256}
   if (st != FA_OK || empty) return st;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
   const BwdLayout w = bwd_layout(B, H, H_kv, N, d);

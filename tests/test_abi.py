@@ -62,7 +62,7 @@ def _ws_expected_gqa(B, H, Hkv, N, d):
     a = lambda x: (x + 255) // 256 * 256  # noqa: E731
     Np = (N + 127) // 128 * 128
     # few key/value tiles: the group's query heads are split over CTAs with fp32 partial dK, dV
-    group, units = H // Hkv, B * Hkv * ((N + 127) // 128)
+    group, units = H // Hkv, B * Hkv * ((N + 127) // 128) * (2 if d == 256 else 1)
     split = next((s for s in range(1, group) if group % s == 0 and units * s >= 4 * 148), group)
     part = 2 * a(split * B * Hkv * N * d * 4) if split > 1 else 0
     return (2 * a(B * H * N * d * 2) + 2 * a(B * Hkv * N * d * 2) + 2 * a(B * H * Np * 4) + part + 256 +
@@ -242,14 +242,17 @@ def test_head_dim_256_is_a_forward_with_workspace(lib):
         _align256(4 * VPASS_BLOCKS)
     pr = api.FaAttnProblem(1, 4, 2, 300, 256, 0.0625, 1, -1, -1)
     assert api.fa_attn_fwd_workspace_size(pr) == api.fa_fwd_workspace_size(1, 2, 300, 256)
-    assert api.fa_bwd_workspace_size(1, 2, 300, 256) == 0
-    assert api.fa_bwd_gqa_workspace_size(1, 4, 2, 300, 256) == 0
+    # the backward takes d = 256 (dK/dV per d-half: twice the key-tile units for the split rule)
+    assert api.fa_bwd_workspace_size(1, 2, 300, 256) == _ws_expected(1, 2, 300, 256)
+    assert api.fa_bwd_gqa_workspace_size(1, 4, 2, 300, 256) == _ws_expected_gqa(1, 4, 2, 300, 256)
     assert fwd(lib, d=256) == api.FA_ERR_UNSUPPORTED  # fa_fwd: no workspace, no d = 256 kernel
     # fa_fwd_ws without its workspace: the problem is valid, the missing workspace is the error
     assert lib.fa_fwd_ws(A, A, A, A, A, None, 1, 4, 2, 300, 256, 0.0625, 1, None, 0, None) == api.FA_ERR_INVALID_ARG
     assert lib.fa_fwd_ws(A, A, A, A, A, None, 1, 4, 2, 300, 512, 0.0625, 1, A, 1 << 40, None) == \
         api.FA_ERR_UNSUPPORTED
-    assert bwd(lib, d=256) == api.FA_ERR_UNSUPPORTED
+    # rejected on the host before any launch: a missing workspace, an unsupported head dimension
+    assert bwd(lib, d=256, ws=None) == api.FA_ERR_INVALID_ARG
+    assert bwd(lib, d=512) == api.FA_ERR_UNSUPPORTED
 
 
 def _align256(x):
