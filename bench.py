@@ -606,7 +606,7 @@ METRIC_D256 = "attention fwd TFLOPS (BF16, causal, N=8k, d=256) & % of B200 tens
 
 
 def run_fwd_only(args, rank: int, world: int, kind: str) -> None:
-    """--fp8: the 8-bit forward (fa_attn_fwd_fp8) on workload 3's shape.  --head-dim 256: the
+    """--fp8: the 8-bit forward (fa_attn_fwd_fp8) on the workload's shape (3 by default; 4 for d = 64).  --head-dim 256: the
     bf16 forward with d = 256 (fa_fwd_ws) on B = 2, H = 16, N = 8192 (workload 3's B * H * d).
     kind "plain": a forward-only workload (4) on its own shape, whose roofline is the larger
     of its HBM time and its tensor-core time.  Forward only; L2 flushed between the timed
@@ -624,7 +624,7 @@ def run_fwd_only(args, rank: int, world: int, kind: str) -> None:
     # algorithmic bytes: Q, K, V read and O written in bf16 (8-bit inputs: one byte each), LSE
     fwd_bytes = (3 * (1 if fp8 else 2) + 2) * B * H * N * d + 4 * B * H * N
     if fp8:
-        x = inputs.make_qkv_fp8(B, H, N, d, spiky_frac=w.spiky_frac, seed=w.seed + rank)
+        x = inputs.make_qkv_fp8(B, H, N, d, dist=w.dist, spiky_frac=w.spiky_frac, seed=w.seed + rank)
         host_in = {n: x[n].view(torch.uint8) for n in ("q", "k", "v")}
     else:
         x = inputs.make_qkv(B, H, N, d, dtype=torch.bfloat16, dist=w.dist, spiky_frac=w.spiky_frac,
@@ -732,7 +732,9 @@ def run_fwd_only(args, rank: int, world: int, kind: str) -> None:
 
     if rank == 0:
         line = {
-            "metric": (METRIC_FP8 if fp8 else METRIC_D256 if not plain else
+            "metric": (METRIC_FP8 if fp8 and args.workload == WORKLOAD else
+                       f"attention fwd TFLOPS (FP8 E4M3 inputs, {'causal' if w.causal else 'non-causal'}, N={N}, "
+                       f"d={d})" if fp8 else METRIC_D256 if not plain else
                        f"attention fwd TFLOPS (BF16, {'causal' if w.causal else 'non-causal'}, N={N}, d={d})"),
             "value": value, "unit": "TFLOPS", "n_gpus": world, "achieved_gbs": achieved_gbs,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,

@@ -165,7 +165,8 @@ int* device_error_word() {
 }
 
 bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
-                  int box_cols, int box_rows, bool swizzle128) {
+                  int box_cols, int box_rows, int swizzle_bytes) {
+  if ((swizzle_bytes != 128 && swizzle_bytes != 64) || box_cols * elem_bytes != swizzle_bytes) return false;
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
@@ -173,7 +174,7 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int 
   const cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -233,15 +234,15 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const bool v16 = workspace != nullptr;
   if (d == 256) {  // V (fp16, in the workspace) in 64-key x 64-column boxes for the d = 256 kernel
-    if (!make_tmap_3d(&tv, workspace, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, BH_kv, 64, 64, true))
+    if (!make_tmap_3d(&tv, workspace, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, BH_kv, 64, 64, 128))
       return FA_ERR_CUDA;
   } else if (!make_tmap_3d(&tv, v16 ? workspace : v, v16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : bf, 2, d, N, BH_kv,
-                           64, 128, true)) {
+                           64, 128, 128)) {
     return FA_ERR_CUDA;
   }
-  if (!make_tmap_3d(&tq, q, bf, 2, d, N, BH, 64, 128, true) ||
-      !make_tmap_3d(&tk, k, bf, 2, d, N, BH_kv, 64, 128, true) ||
-      !make_tmap_3d(&to, o, bf, 2, d, N, BH, 64, 128, true))
+  if (!make_tmap_3d(&tq, q, bf, 2, d, N, BH, 64, 128, 128) ||
+      !make_tmap_3d(&tk, k, bf, 2, d, N, BH_kv, 64, 128, 128) ||
+      !make_tmap_3d(&to, o, bf, 2, d, N, BH, 64, 128, 128))
     return FA_ERR_CUDA;
   FwdParams p{};
   p.lse = lse;
@@ -393,10 +394,10 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
 
   const CUtensorMapDataType h = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap t_q, t_do, t_k, t_v;  // 128-row boxes, shared by the dK/dV and dQ kernels
-  if (!make_tmap_3d(&t_q, pp.q16, h, 2, d, N, BH, 64, 128, true) ||
-      !make_tmap_3d(&t_do, pp.do16, h, 2, d, N, BH, 64, 128, true) ||
-      !make_tmap_3d(&t_k, pp.k16, h, 2, d, N, BH_kv, 64, 128, true) ||
-      !make_tmap_3d(&t_v, pp.v16, h, 2, d, N, BH_kv, 64, 128, true))
+  if (!make_tmap_3d(&t_q, pp.q16, h, 2, d, N, BH, 64, 128, 128) ||
+      !make_tmap_3d(&t_do, pp.do16, h, 2, d, N, BH, 64, 128, 128) ||
+      !make_tmap_3d(&t_k, pp.k16, h, 2, d, N, BH_kv, 64, 128, 128) ||
+      !make_tmap_3d(&t_v, pp.v16, h, 2, d, N, BH_kv, 64, 128, 128))
     return FA_ERR_CUDA;
   BwdParams bp{};
   bp.delta = pp.delta;
@@ -470,7 +471,7 @@ fa_status fa_attn_bwd(const fa_attn_problem* pr, const void* q, const void* k, c
                   pr->causal, pr->window_left, pr->window_right, workspace, workspace_bytes, stream);
 }
 
-// ---- 8-bit forward: E4M3 inputs with per-tensor descales (d = 128)
+// ---- 8-bit forward: E4M3 inputs with per-tensor descales (d = 128 or 64)
 size_t fa_attn_fwd_fp8_workspace_size(const fa_attn_problem* pr) {
   if (pr == nullptr || !window_ok(pr->window_left, pr->window_right)) return 0;
   return 256;  // the persistent kernel's work counter
@@ -486,7 +487,7 @@ fa_status fa_attn_fwd_fp8(const fa_attn_problem* pr, const void* q, const void* 
   if (st != FA_OK) return st;
   for (const float ds : {q_descale, k_descale, v_descale})
     if (!(std::isfinite(ds) && ds > 0.f)) return FA_ERR_INVALID_ARG;
-  if (d != 128) return FA_ERR_UNSUPPORTED;  // one 128-byte swizzle row per Q / K / V row
+  if (d != 128 && d != 64) return FA_ERR_UNSUPPORTED;  // one 128- or 64-byte swizzle row per Q / K / V row
   if (empty) return FA_OK;
   if (!q || !k || !v || !o || !workspace || workspace_bytes < 256) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
@@ -500,9 +501,8 @@ fa_status fa_attn_fwd_fp8(const fa_attn_problem* pr, const void* q, const void* 
   if (cudaMemsetAsync(counter, 0, sizeof(unsigned), s) != cudaSuccess) return FA_ERR_CUDA;
   CUtensorMap tq, tk, tv;
   const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  if (!make_tmap_3d(&tq, q, u8, 1, d, N, BH, 128, 128, true) ||
-      !make_tmap_3d(&tk, k, u8, 1, d, N, BH_kv, 128, 128, true) ||
-      !make_tmap_3d(&tv, v, u8, 1, d, N, BH_kv, 128, 128, true))
+  if (!make_tmap_3d(&tq, q, u8, 1, d, N, BH, d, 128, d) || !make_tmap_3d(&tk, k, u8, 1, d, N, BH_kv, d, 128, d) ||
+      !make_tmap_3d(&tv, v, u8, 1, d, N, BH_kv, d, 128, d))
     return FA_ERR_CUDA;
   FwdParams p{};
   p.lse = lse;
@@ -523,7 +523,7 @@ fa_status fa_attn_fwd_fp8(const fa_attn_problem* pr, const void* q, const void* 
   p.win_left = pr->window_left;
   p.win_right = pr->window_right;
   p.err = g_err_ptr[dev];
-  return launch_fwd_persist_fp8_sm100(tq, tk, tv, p, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return launch_fwd_persist_fp8_sm100(tq, tk, tv, p, d, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 void fa_bwd_set_phase_events(void* const* events) { t_phase_events = events; }

@@ -124,8 +124,10 @@ inline int head_group_size(int BH, unsigned long long per_head, unsigned long lo
   return g > (unsigned long long)BH ? BH : (int)g;
 }
 
+// (d, N, BH) tensor, boxes of box_cols x box_rows, with the 128- or 64-byte swizzle (a box row
+// of box_cols elements must be exactly that many bytes)
 bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
-                  int box_cols, int box_rows, bool swizzle128);
+                  int box_cols, int box_rows, int swizzle_bytes);
 
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t s);
@@ -138,7 +140,7 @@ cudaError_t launch_fwd_persist_sm100(const CUtensorMap& tq, const CUtensorMap& t
 cudaError_t launch_fwd_d256_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                   const FwdParams& p, cudaStream_t s);  // d = 256, fp16 V in 64 x 64 boxes
 cudaError_t launch_fwd_persist_fp8_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                         const FwdParams& p, cudaStream_t s);  // d = 128, E4M3 inputs
+                                         const FwdParams& p, int d, cudaStream_t s);  // d = 128 or 64, E4M3
 cudaError_t launch_selftest_wait(int* err, cudaStream_t s);
 cudaError_t launch_selftest_exp2(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_bwd_kv_reduce(const float* dk_part, const float* dv_part, float* dk, float* dv,

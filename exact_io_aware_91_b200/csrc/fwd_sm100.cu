@@ -588,22 +588,27 @@ namespace {
 // (coalesced by warp_store_rows_128b): the Q buffers are reloaded for the next unit and
 // cannot serve as the output staging tile.
 //
-// F8 (8-bit inputs, d = 128): Q, K and V are E4M3, so a row of d elements is one 128-byte
-// swizzle row and every tile is 16 KB; S = Q K^T and O += P V run as kind::f8f6f4 products
-// (K = 32 per instruction), V read MN-major straight from its (N, d) layout, P written to TMEM
-// as E4M3; the per-tensor descales enter through scale_log2 (Q, K) and out_scale (V).
+// F8 (8-bit inputs, d = 128 or 64): Q, K and V are E4M3, so a row of d elements is one
+// 128-byte swizzle row (d = 128; 16 KB tiles) or one 64-byte swizzle row (d = 64; 8 KB tiles);
+// S = Q K^T and O += P V run as kind::f8f6f4 products (K = 32 per instruction), V read
+// MN-major straight from its (N, d) layout, P written to TMEM as E4M3; the per-tensor
+// descales enter through scale_log2 (Q, K) and out_scale (V).
 template <int D, bool F8 = false>
 struct FwdPLayout {
   static constexpr int ROW_BYTES = F8 ? D : 2 * D;  // bytes of one row of Q, K or V
-  static constexpr int CH_ELEMS = F8 ? 128 : 64;     // elements of one 128-byte column chunk
-  static constexpr int KCH = ROW_BYTES / 128;
-  static constexpr int BOX = 128 * 128;
+  static constexpr int SW = ROW_BYTES < 128 ? 64 : 128;  // swizzle span: bytes of one column chunk row
+  static_assert(ROW_BYTES % SW == 0, "rows are whole swizzle rows");
+  static constexpr int CH_ELEMS = F8 ? SW : SW / 2;  // elements of one column chunk
+  static constexpr int KCH = ROW_BYTES / SW;
+  static constexpr int BOX = 128 * SW;                // one chunk of 128 rows
   static constexpr int TILE = KCH * BOX;
   static constexpr int STAGES = (TILE == 2 * BOX) ? 4 : 8;
   static constexpr int K_STEP = F8 ? 32 : 16;          // K of one tensor-core instruction
   static constexpr int QK_STEPS = ROW_BYTES / 32;      // instructions per Q K^T (32 bytes of K each)
+  static constexpr int QK_STEPS_CH = SW / 32;          // of which inside one column chunk
+  static constexpr int ATOM = 8 * SW;                  // bytes of an 8-row swizzle atom
   static constexpr int PV_STEPS_HALF = 64 / K_STEP;    // instructions per half of P V (64 keys)
-  static constexpr int PV_B_STEP = K_STEP * 128;       // bytes between the V rows of consecutive steps
+  static constexpr int PV_B_STEP = K_STEP * SW;        // bytes between the V rows of consecutive steps
   static constexpr int OFF_Q0 = 0;
   static constexpr int OFF_Q1 = TILE;
   static constexpr int OFF_KV = 2 * TILE;
@@ -760,14 +765,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t idesc_pv = make_idesc(128, D, false, false, true);
     const uint32_t tS[2] = {tmem + L::T_S0, tmem + L::T_S1};
     const uint32_t tO[2] = {tmem + L::T_O0, tmem + L::T_O1};
-    const uint64_t dQ[2] = {make_sdesc_sw128(base + L::OFF_Q0, 16, 1024), make_sdesc_sw128(base + L::OFF_Q1, 16, 1024)};
-    const uint64_t dKV0 = make_sdesc_sw128(base + L::OFF_KV, 16, 1024);     // K-major (K tiles)
-    const uint64_t dV0 = make_sdesc_sw128(base + L::OFF_KV, L::BOX, 1024);  // MN-major (V tiles)
+    auto sdesc = [](uint32_t saddr, uint32_t lbo) -> uint64_t {
+      return L::SW == 128 ? make_sdesc_sw128(saddr, lbo, L::ATOM) : make_sdesc_sw64(saddr, lbo, L::ATOM);
+    };
+    const uint64_t dQ[2] = {sdesc(base + L::OFF_Q0, 16), sdesc(base + L::OFF_Q1, 16)};
+    const uint64_t dKV0 = sdesc(base + L::OFF_KV, 16);     // K-major (K tiles)
+    const uint64_t dV0 = sdesc(base + L::OFF_KV, L::BOX);  // MN-major (V tiles)
     auto issue_qk = [&](uint32_t d_tmem, uint64_t q_desc, int stage) {
       const uint64_t k_desc = sdesc_add(dKV0, stage * L::TILE);
 #pragma unroll
       for (int k = 0; k < L::QK_STEPS; ++k) {
-        const uint32_t off = (k >> 2) * L::BOX + (k & 3) * 32;
+        const uint32_t off = (k / L::QK_STEPS_CH) * L::BOX + (k % L::QK_STEPS_CH) * 32;
         if constexpr (F8)
           mma_ss_f8(d_tmem, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, k > 0 ? 1u : 0u, leader);
         else
@@ -1387,10 +1395,11 @@ cudaError_t launch_fwd_persist_sm100(const CUtensorMap& tq, const CUtensorMap& t
 }
 
 cudaError_t launch_fwd_persist_fp8_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                         const FwdParams& p, cudaStream_t s) {
+                                         const FwdParams& p, int d, cudaStream_t s) {
   const long long units = (long long)p.n_pairs * p.BH;
   const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
-  return launch_persist_t<128, true>(grid, tq, tk, tv, p, s);
+  return d == 128 ? launch_persist_t<128, true>(grid, tq, tk, tv, p, s)
+                  : launch_persist_t<64, true>(grid, tq, tk, tv, p, s);
 }
 
 cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, uint32_t* amax_part,

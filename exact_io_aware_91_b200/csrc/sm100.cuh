@@ -315,6 +315,16 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same descriptor with the 64-byte swizzle (mode 4): rows of 64 bytes, 8-row atoms of
+// 512 bytes.  K-major: `sbo` = 512, start advanced by 32 bytes per instruction step inside
+// a row.  MN-major: 64-byte MN blocks `lbo` apart, 8-row K groups `sbo` = 512 apart.  The
+// 64-byte swizzle of the tensor-memory-access unit writes exactly this layout into a
+// 512-byte-aligned buffer.
+__device__ __forceinline__ uint64_t make_sdesc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
+}
+
 // Advance a descriptor's start address by `bytes` (a multiple of 16; the 14-bit
 // field holds addresses < 256 KB, so the add never carries out of it).
 __device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }

@@ -255,7 +255,7 @@ FA_API fa_status fa_attn_bwd(const fa_attn_problem* problem, const void* q, cons
  * attention products in FP8 on the tensor cores.  The pages give no format or scaling
  * scheme; the reading taken is E4M3 operands with one descale factor per tensor.)
  *   problem          : as for fa_attn_fwd (grouped heads, causal mask, sliding window);
- *                      d must be 128 (FA_ERR_UNSUPPORTED otherwise).
+ *                      d must be 128 or 64 (FA_ERR_UNSUPPORTED otherwise).
  *   q                : const E4M3 (B, H, N, d), 16-byte aligned; k, v: const E4M3
  *                      (B, H_kv, N, d), 16-byte aligned.  One byte per element in the
  *                      OCP FP8 E4M3 encoding (bias 7, no infinities, 0x7F / 0xFF NaN).

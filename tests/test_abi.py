@@ -224,7 +224,8 @@ def test_fp8_forward_checks_its_arguments(lib):
     assert call(ds=(1.0, -1.0, 1.0)) == api.FA_ERR_INVALID_ARG
     assert call(ds=(1.0, 1.0, float("inf"))) == api.FA_ERR_INVALID_ARG
     assert call(ds=(1.0, float("nan"), 1.0)) == api.FA_ERR_INVALID_ARG
-    assert call(p=api.FaAttnProblem(1, 4, 2, 300, 64, 0.125, 1, -1, -1)) == api.FA_ERR_UNSUPPORTED  # d = 128 only
+    assert call(p=api.FaAttnProblem(1, 4, 2, 300, 256, 0.0625, 1, -1, -1)) == api.FA_ERR_UNSUPPORTED  # d = 128, 64
+    assert call(p=api.FaAttnProblem(1, 4, 2, 300, 96, 0.1, 1, -1, -1)) == api.FA_ERR_UNSUPPORTED
     assert call(p=api.FaAttnProblem(1, 6, 4, 300, 128, 0.125, 1, -1, -1)) == api.FA_ERR_INVALID_ARG
     assert call(q=None) == api.FA_ERR_INVALID_ARG
     assert call(ws=None) == api.FA_ERR_INVALID_ARG

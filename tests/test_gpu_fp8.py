@@ -113,10 +113,22 @@ CASES = [  # B, H, H_kv, N, causal, window, spiky
 ]
 
 
-@pytest.mark.parametrize("B,H,Hkv,N,causal,window,spiky", CASES)
-def test_fp8_forward_within_its_rounding_bound(B, H, Hkv, N, causal, window, spiky):
-    x = inputs.make_qkv_fp8(B, H, N, 128, kv_heads=Hkv, spiky_frac=spiky, seed=11 + N, device="cuda")
-    scale = 1.0 / math.sqrt(128)
+# head dim 64: rows of 64 bytes (the 64-byte swizzle), O of 64 TMEM columns per tile
+CASES_D64 = [
+    (1, 2, 2, 256, True, (-1, -1), 0.0),
+    (2, 4, 4, 1000, False, (-1, -1), 0.0),
+    (1, 4, 1, 777, True, (-1, -1), 0.0),
+    (1, 2, 2, 900, False, (100, 50), 0.0),
+    (1, 2, 2, 2048, True, (-1, -1), 0.01),
+    (1, 2, 2, 1, False, (-1, -1), 0.0),
+]
+
+
+@pytest.mark.parametrize("d,B,H,Hkv,N,causal,window,spiky",
+                         [(128,) + c for c in CASES] + [(64,) + c for c in CASES_D64])
+def test_fp8_forward_within_its_rounding_bound(d, B, H, Hkv, N, causal, window, spiky):
+    x = inputs.make_qkv_fp8(B, H, N, d, kv_heads=Hkv, spiky_frac=spiky, seed=11 + N + d, device="cuda")
+    scale = 1.0 / math.sqrt(d)
     o, lse = api.fa_attn_fwd_fp8(x["q"], x["k"], x["v"], x["q_descale"], x["k_descale"], x["v_descale"],
                                  causal=causal, scale=scale, window=window)
     torch.cuda.synchronize()
@@ -124,10 +136,11 @@ def test_fp8_forward_within_its_rounding_bound(B, H, Hkv, N, causal, window, spi
     check_heads(x, o, lse, scale, causal, window, heads, tag=f"N={N}")
 
 
-def test_fp8_exact_probabilities():
+@pytest.mark.parametrize("d", [128, 64])
+def test_fp8_exact_probabilities(d):
     # scale = ln 2 and integer scores in [-4, 4]: every probability the kernel forms is a
     # power of two in [2^-8, 2^8], exact in E4M3, so only fp32 sums and the bf16 output round
-    B, H, N, d = 1, 2, 2048, 128
+    B, H, N = 1, 2, 2048
     g = torch.Generator().manual_seed(5)
     q = torch.zeros(B, H, N, d)
     q[..., 0] = 1.0
@@ -161,6 +174,18 @@ def test_fp8_workload3_shape_sampled_rows():
     check_heads(x, o, lse, w.scale, True, (-1, -1), [(0, 0), (1, 31), (0, 17)], rows=rows, tag="workload 3")
 
 
+def test_fp8_workload4_shape_sampled_heads():
+    # workload 4's shape (B=64, H=16, N=512, d=64, no mask, U(-1, 1)) in E4M3: 512 work units,
+    # several per CTA; every row of a sample of heads
+    w = inputs.workload(4)
+    x = inputs.make_qkv_fp8(w.B, w.H, w.N, w.d, dist=w.dist, seed=w.seed, device="cuda")
+    o, lse = api.fa_attn_fwd_fp8(x["q"], x["k"], x["v"], x["q_descale"], x["k_descale"], x["v_descale"],
+                                 causal=False, scale=w.scale)
+    torch.cuda.synchronize()
+    heads = [(0, 0), (17, 5), (40, 9), (63, 15)]
+    check_heads(x, o, lse, w.scale, False, (-1, -1), heads, tag="workload 4")
+
+
 def test_fp8_argument_checks():
     x = inputs.make_qkv_fp8(1, 2, 64, 128, seed=1, device="cuda")
     with pytest.raises(api.FAError) as e:
@@ -169,7 +194,7 @@ def test_fp8_argument_checks():
     with pytest.raises(api.FAError) as e:
         api.fa_attn_fwd_fp8(x["q"], x["k"], x["v"], 1.0, float("nan"), 1.0)
     assert e.value.status == api.FA_ERR_INVALID_ARG
-    y = inputs.make_qkv_fp8(1, 2, 64, 64, seed=1, device="cuda")
+    y = inputs.make_qkv_fp8(1, 2, 64, 256, seed=1, device="cuda")
     with pytest.raises(api.FAError) as e:
         api.fa_attn_fwd_fp8(y["q"], y["k"], y["v"], 1.0, 1.0, 1.0)
     assert e.value.status == api.FA_ERR_UNSUPPORTED
