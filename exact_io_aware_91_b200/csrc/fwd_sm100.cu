@@ -95,6 +95,12 @@ constexpr int kConvThreads = 64;
 #ifndef FA_EXP_FMA_PER8_F8
 #define FA_EXP_FMA_PER8_F8 2
 #endif
+// The persistent forward hands P to the tensor core in this many parts per 128-key step
+// (2 or 4): the last part's share of P V is what the next S product of the tile waits for.
+#ifndef FA_FWD_PARTS
+#define FA_FWD_PARTS 2
+#endif
+constexpr int kFwdParts = FA_FWD_PARTS;
 // element pairs out of every 8 whose exponentials run on the FMA pipe (even, 0..8)
 constexpr int kExpFmaPer8 = FA_EXP_FMA_PER8;
 constexpr int kExpFmaPer8F8 = FA_EXP_FMA_PER8_F8;
@@ -131,7 +137,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // A tile whose P sum exceeds what valid scores allow (a non-finite input, or a score beyond
 // the fp32 range) is recorded as kDevRange in the error word.
 // Returns false if a bounded wait gave up.
-template <int D, bool F8 = false, bool TILE_EXP = false>
+template <int D, bool F8 = false, bool TILE_EXP = false, int PARTS = 2>
 __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS, uint32_t tO, uint32_t bar_s_full,
                                                  uint32_t s_parity, uint32_t bar_p_half, uint32_t bar_p_full, int j,
                                                  bool first, int q_base, int r, float& m, float& l,
@@ -205,12 +211,17 @@ __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS
     }
   }
   uint64_t sa = 0, sb = 0;  // packed fp32 partial row sums (0.0f, 0.0f)
+  // P goes to TMEM in PARTS parts of 128 / PARTS keys; part h is announced on bar_p_half +
+  // 16 h (with two parts: bar_p_half, then bar_p_full), so its share of P V can start while
+  // the next part is computed
+  static_assert(PARTS == 2 || PARTS == 4, "two halves or four quarters of the 128 keys");
+  constexpr int PER = 128 / PARTS;  // keys per part
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t pk[32];
+  for (int h = 0; h < PARTS; ++h) {
+    uint32_t pk[PER / 2];
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      float* e = &x[64 * h + 2 * i];
+    for (int i = 0; i < PER / 2; i += 2) {
+      float* e = &x[PER * h + 2 * i];
       fma2(e[0], e[1], sl2, neg_m);
       fma2(e[2], e[3], sl2, neg_m);
       // kExpFmaPer8 (kExpFmaPer8F8) of every 8 element pairs take 2^x on the FMA pipe, the
@@ -234,15 +245,19 @@ __device__ __forceinline__ bool fwd_softmax_step(const FwdParams& p, uint32_t tS
       asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sa) : "l"(f2pack(e[0], e[1])));
       asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sb) : "l"(f2pack(e[2], e[3])));
     }
-    if constexpr (F8)
+    if constexpr (F8 && PER == 64)
       tmem_st16(tS + 16 * h, pk);
+    else if constexpr (F8)
+      tmem_st8(tS + 8 * h, pk);
+    else if constexpr (PER == 64)
+      tmem_st32(tS + 32 * h, reinterpret_cast<const uint32_t(&)[32]>(pk));
     else
-      tmem_st32(tS + 32 * h, pk);
-    // first half of P (and any rescale of O) visible to the tensor core: its half of P V
-    // can start while the second half is computed
+      tmem_st16(tS + 16 * h, pk);
+    // this part of P (and any rescale of O) visible to the tensor core: its share of P V
+    // can start while the next part is computed
     tmem_wait_st();
     tc_fence_before();
-    mbar_arrive(h == 0 ? bar_p_half : bar_p_full);
+    mbar_arrive(PARTS == 2 ? (h == 0 ? bar_p_half : bar_p_full) : bar_p_half + 16u * h);
   }
   float s0, s1, s2, s3;
   f2unpack(sa, s0, s1);
@@ -607,7 +622,8 @@ struct FwdPLayout {
   static constexpr int QK_STEPS = ROW_BYTES / 32;      // instructions per Q K^T (32 bytes of K each)
   static constexpr int QK_STEPS_CH = SW / 32;          // of which inside one column chunk
   static constexpr int ATOM = 8 * SW;                  // bytes of an 8-row swizzle atom
-  static constexpr int PV_STEPS_HALF = 64 / K_STEP;    // instructions per half of P V (64 keys)
+  static constexpr int PARTS = kFwdParts;              // P handed to the tensor core in PARTS parts
+  static constexpr int PV_STEPS_PART = 128 / PARTS / K_STEP;  // instructions per part of P V
   static constexpr int PV_B_STEP = K_STEP * SW;        // bytes between the V rows of consecutive steps
   static constexpr int OFF_Q0 = 0;
   static constexpr int OFF_Q1 = TILE;
@@ -618,9 +634,8 @@ struct FwdPLayout {
   static constexpr int BAR_KV_FULL = 2;
   static constexpr int BAR_KV_EMPTY = 2 + STAGES;
   static constexpr int BAR_S_FULL = 2 + 2 * STAGES;  // [2]
-  static constexpr int BAR_P_HALF = BAR_S_FULL + 2;  // [2]
-  static constexpr int BAR_P_FULL = BAR_P_HALF + 2;  // [2]
-  static constexpr int BAR_O_FULL = BAR_P_FULL + 2;  // [2]
+  static constexpr int BAR_P_PART = BAR_S_FULL + 2;  // [PARTS][2]: part h of tile t at BAR_P_PART + t + 2 h
+  static constexpr int BAR_O_FULL = BAR_P_PART + 2 * PARTS;  // [2]
   static constexpr int BAR_O_FREE = BAR_O_FULL + 2;  // [2] a tile's epilogue has read O out of TMEM
   static constexpr int BAR_UNIT_FULL = BAR_O_FREE + 2;   // [2]
   static constexpr int BAR_UNIT_EMPTY = BAR_UNIT_FULL + 2;  // [2]
@@ -686,8 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::BAR_S_FULL + t), 1);
-      mbar_init(bar(L::BAR_P_HALF + t), 128);
-      mbar_init(bar(L::BAR_P_FULL + t), 128);
+      for (int h = 0; h < L::PARTS; ++h) mbar_init(bar(L::BAR_P_PART + t + 2 * h), 128);
       mbar_init(bar(L::BAR_O_FULL + t), 1);
       mbar_init(bar(L::BAR_O_FREE + t), 128);
       mbar_init(bar(L::BAR_UNIT_FULL + t), 1);
@@ -783,11 +797,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     // P for keys [K_STEP k, K_STEP (k + 1)) sits in TMEM columns [8 k, 8 k + 8) in both forms
-    auto issue_pv_half = [&](uint32_t d_tmem, uint32_t p_tmem, int stage, bool acc, int part) {
+    auto issue_pv_part = [&](uint32_t d_tmem, uint32_t p_tmem, int stage, bool acc, int part) {
       const uint64_t v_desc = sdesc_add(dV0, stage * L::TILE);
 #pragma unroll
-      for (int kk = 0; kk < L::PV_STEPS_HALF; ++kk) {
-        const int k = part * L::PV_STEPS_HALF + kk;
+      for (int kk = 0; kk < L::PV_STEPS_PART; ++kk) {
+        const int k = part * L::PV_STEPS_PART + kk;
         if constexpr (F8)
           mma_ts_f8(d_tmem, p_tmem + k * 8, sdesc_add(v_desc, k * L::PV_B_STEP), idesc_pv, (acc || k > 0) ? 1u : 0u,
                     leader);
@@ -806,12 +820,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
       const uint32_t ph = ((t ? G1 : G0) + jt) & 1;
-      if (!mbar_wait(bar(L::BAR_P_HALF + t), ph, wctx)) return false;
-      tc_fence_after();
-      issue_pv_half(tO[t], tS[t], stage, jt > 0, 0);
-      if (!mbar_wait(bar(L::BAR_P_FULL + t), ph, wctx)) return false;
-      tc_fence_after();
-      issue_pv_half(tO[t], tS[t], stage, jt > 0, 1);
+      for (int h = 0; h < L::PARTS; ++h) {
+        if (!mbar_wait(bar(L::BAR_P_PART + t + 2 * h), ph, wctx)) return false;
+        tc_fence_after();
+        issue_pv_part(tO[t], tS[t], stage, jt > 0, h);
+      }
       return true;
     };
     for (int uc = 0; ok; ++uc) {
@@ -895,9 +908,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_t = (t ? x.jhi1 : x.jhi0) - jlo + 1;
       float m = -INFINITY, l = 0.f;
       for (int jj = 0; jj < n_t; ++jj) {
-        if (!(ok = fwd_softmax_step<D, F8>(p, tS, tO, bar(L::BAR_S_FULL + t), (G + jj) & 1, bar(L::BAR_P_HALF + t),
-                                       bar(L::BAR_P_FULL + t), jlo + jj, jj == 0, q_base, r, m,
-                                       l, wctx)))
+        if (!(ok = fwd_softmax_step<D, F8, false, L::PARTS>(p, tS, tO, bar(L::BAR_S_FULL + t), (G + jj) & 1,
+                                                            bar(L::BAR_P_PART + t), bar(L::BAR_P_PART + t + 2),
+                                                            jlo + jj, jj == 0, q_base, r, m, l, wctx)))
           break;
       }
       G += n_t;
