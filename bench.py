@@ -1,7 +1,8 @@
 """Benchmark: exact attention forward + backward on one B200 per process.
 
-A step is one pass of the whole hot path -- forward (fa_fwd) then backward
-(fa_bwd: preprocess, dK/dV kernel, dQ kernel) -- over the causal workload
+A step is one pass of the whole hot path -- forward (fa_fwd_ws: V pass, persistent
+kernel) then backward (fa_bwd_ws: preprocess reusing the forward's fp16 V, dK/dV kernel,
+dQ kernel) -- over the causal workload
 B=2, H=32, N=8192, d=128 (bf16 inputs, 1% of the keys of every head scaled by 8).
 The metric is TFLOPS with 4*B*H*N^2*d forward flops (halved under the causal
 mask) and 2.5x that for the backward.
@@ -456,15 +457,17 @@ def run_ours(args, rank: int, world: int, local: int) -> None:
     dq = torch.empty((B, H, N, d), dtype=torch.float32, device=dev)
     dk = torch.empty((B, Hkv, N, d), dtype=torch.float32, device=dev)
     dv = torch.empty_like(dk)
-    ws = torch.empty(api.fa_bwd_gqa_workspace_size(B, H, Hkv, N, d), dtype=torch.uint8, device=dev)
+    ws_size = (api.fa_bwd_ws_workspace_size if args.window is None else api.fa_bwd_gqa_workspace_size)
+    ws = torch.empty(ws_size(B, H, Hkv, N, d), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     # forward with a workspace: V converted to fp16 in one streaming pass, then the kernel
     fws = torch.empty(api.fa_fwd_workspace_size(B, Hkv, N, d), dtype=torch.uint8, device=dev)
     if args.window is None:
-        bwd_call = api.fa_bwd_gqa  # the backward that takes the forward's residual
-
         def fwd_call(q, k, v, **kw):
             return api.fa_fwd_ws(q, k, v, workspace=fws, **kw)
+
+        def bwd_call(q, k, v, o, do, lse, **kw):  # takes the forward's residual and its fp16 V copy
+            return api.fa_bwd_ws(q, k, v, o, do, lse, fws, **kw)
     else:  # sliding window: the descriptor-based entry points
         def fwd_call(q, k, v, **kw):
             return api.fa_attn_fwd(q, k, v, window=window, workspace=fws, **kw)
@@ -767,13 +770,13 @@ def main() -> None:
     ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[2, 3, 4, 5],
                     help="workload index (3 = the metric's; others for profiling runs)")
     ap.add_argument("--kv-heads", type=int, default=None,
-                    help="grouped-query run: K/V with this many heads (fa_fwd_gqa / fa_bwd_gqa); default H")
+                    help="grouped-query run: K/V with this many heads (fa_fwd_ws / fa_bwd_ws); default H")
     ap.add_argument("--window", type=int, default=None,
                     help="sliding-window run: each query sees the previous WINDOW keys and itself "
                          "(fa_attn_fwd / fa_attn_bwd); default no window")
     ap.add_argument("--head-dim", type=int, default=None, choices=[256],
                     help="head dimension 256 on the workload's B * H * d (B=2, H=16, N=8192): forward + "
-                         "backward (fa_fwd_ws, fa_bwd_gqa); with --fwd-only the forward alone")
+                         "backward (fa_fwd_ws, fa_bwd_ws); with --fwd-only the forward alone")
     ap.add_argument("--fwd-only", action="store_true", help="with --head-dim 256: time the forward alone")
     ap.add_argument("--fp8", action="store_true",
                     help="time the 8-bit forward (E4M3 inputs, fa_attn_fwd_fp8) on the workload's shape")

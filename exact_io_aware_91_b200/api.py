@@ -25,7 +25,7 @@ FA_ERR_TIMEOUT = 5
 FA_ERR_RANGE = 6
 
 EXPORTS = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_workspace_size", "fa_fwd_ws", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_gqa_workspace_size",
-           "fa_bwd_gqa", "fa_attn_fwd_workspace_size", "fa_attn_fwd", "fa_attn_bwd_workspace_size", "fa_attn_bwd",
+           "fa_bwd_gqa", "fa_bwd_ws_workspace_size", "fa_bwd_ws", "fa_attn_fwd_workspace_size", "fa_attn_fwd", "fa_attn_bwd_workspace_size", "fa_attn_bwd",
            "fa_attn_fwd_fp8_workspace_size", "fa_attn_fwd_fp8", "fa_bwd_noalloc", "fa_last_device_status",
            "fa_device_status", "fa_bwd_set_phase_events", "fa_selftest_wait_timeout", "fa_selftest_exp2",
            "fa_status_str")
@@ -81,6 +81,10 @@ def library() -> ctypes.CDLL:
     lib.fa_bwd_gqa_workspace_size.restype = sz
     lib.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_bwd_gqa.restype = i
+    lib.fa_bwd_ws_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_bwd_ws_workspace_size.restype = sz
+    lib.fa_bwd_ws.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp, sz, vp]
+    lib.fa_bwd_ws.restype = i
     pp = ctypes.POINTER(FaAttnProblem)
     lib.fa_attn_fwd_workspace_size.argtypes = [pp]
     lib.fa_attn_fwd_workspace_size.restype = sz
@@ -305,6 +309,43 @@ def fa_bwd_gqa(q, k, v, o, do, lse, causal: bool = False, scale: float | None = 
                               dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N, d, _scale(scale, d),
                               int(bool(causal)), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
     _check("fa_bwd_gqa", st)
+    return dq, dk, dv
+
+
+def fa_bwd_ws_workspace_size(B: int, H: int, H_kv: int, N: int, d: int) -> int:
+    return int(library().fa_bwd_ws_workspace_size(B, H, H_kv, N, d))
+
+
+def fa_bwd_ws(q, k, v, o, do, lse, fwd_workspace, causal: bool = False, scale: float | None = None,
+              workspace=None, dq=None, dk=None, dv=None, o_resid=None, stream=None):
+    """``fa_bwd_gqa`` that takes the fp16 V copy from ``fwd_workspace``, the workspace of the
+    ``fa_fwd_ws`` call that produced o (and lse, o_resid) from this v.  Returns (dq, dk, dv)."""
+    B, H, N, d = _shape(q)
+    H_kv = _gqa_heads(q, k)
+    _same(q, o, do, dtype=torch.bfloat16, shape=(B, H, N, d))
+    _same(k, v, dtype=torch.bfloat16, shape=(B, H_kv, N, d))
+    _same(lse, dtype=torch.float32, shape=(B, H, N))
+    if o_resid is not None:
+        _same(o_resid, dtype=torch.bfloat16, shape=(B, H, N, d))
+    if fwd_workspace is None or fwd_workspace.device != q.device:
+        raise ValueError("fa_bwd_ws needs the forward's workspace on the inputs' device")
+    if dq is None:
+        dq = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    if dk is None:
+        dk = torch.empty((B, H_kv, N, d), dtype=torch.float32, device=q.device)
+    if dv is None:
+        dv = torch.empty_like(dk)
+    _same(dq, dtype=torch.float32, shape=(B, H, N, d))
+    _same(dk, dv, dtype=torch.float32, shape=(B, H_kv, N, d))
+    if workspace is None:
+        workspace = torch.empty(max(fa_bwd_ws_workspace_size(B, H, H_kv, N, d), 1), dtype=torch.uint8,
+                                device=q.device)
+    st = library().fa_bwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             None if o_resid is None else o_resid.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N, d, _scale(scale, d),
+                             int(bool(causal)), fwd_workspace.data_ptr(), fwd_workspace.numel(),
+                             workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    _check("fa_bwd_ws", st)
     return dq, dk, dv
 
 

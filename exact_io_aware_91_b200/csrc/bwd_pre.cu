@@ -27,6 +27,11 @@
 // Non-finite inputs (a largest magnitude of inf or NaN) and a non-finite D are reported as
 // kDevRange in the device error word.
 //
+// fa_bwd_ws reuses the fp16 V copy that fa_fwd_ws left in its workspace (the same V, the
+// same exponent rule for V on its own): the preprocess then reads no V, the fix-up takes
+// max |V| from the forward's V-pass maxima, and V is converted again (into the forward's
+// copy) only when the dS bound asks for another exponent than the copy holds.
+//
 // Each row is read with 16-byte loads by d/8 consecutive lanes; the grid is fixed
 // (kPreBlocks blocks or fewer) and its warps stride over the rows.
 #include "fa_internal.h"
@@ -108,11 +113,13 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
       am_do = amax_bf16x8(am_do, vd);
       if (bh < p.BH_kv) {  // key/value rows share the (head, row) index space of the first BH_kv heads
         const uint4 vk = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.k) + off);
-        const uint4 vv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.v) + off);
         *reinterpret_cast<uint4*>(static_cast<__half*>(p.k16) + off) = bf16x8_to_f16x8(vk, fk);
-        *reinterpret_cast<uint4*>(static_cast<__half*>(p.v16) + off) = bf16x8_to_f16x8(vv, fv);
         am_k = amax_bf16x8(am_k, vk);
-        am_v = amax_bf16x8(am_v, vv);
+        if (p.v_amax_fwd == nullptr) {  // else the forward's V copy is reused
+          const uint4 vv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.v) + off);
+          *reinterpret_cast<uint4*>(static_cast<__half*>(p.v16) + off) = bf16x8_to_f16x8(vv, fv);
+          am_v = amax_bf16x8(am_v, vv);
+        }
       }
       bf16x8_to_f16x8(vo, fo);
       if (p.o_resid != nullptr) {
@@ -167,10 +174,14 @@ __global__ void __launch_bounds__(256) fa_bwd_fixup_kernel(const BwdPreParams p,
   __shared__ uint32_t red[8][4];
   __shared__ int ex[4];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ int ev_copy;  // exponent the V copy holds now (0, or the forward's when it is reused)
+  const bool reuse_v = p.v_amax_fwd != nullptr;
   uint32_t m[4] = {0u, 0u, 0u, 0u};
   for (int i = threadIdx.x; i < n_part; i += blockDim.x)
 #pragma unroll
     for (int t = 0; t < 4; ++t) m[t] = max(m[t], p.amax_part[t * kPreBlocks + i]);
+  if (reuse_v)  // max |V| from the forward's V pass (the preprocess did not read V)
+    for (int i = threadIdx.x; i < p.v_n_part_fwd; i += blockDim.x) m[kExpV] = max(m[kExpV], p.v_amax_fwd[i]);
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
     m[t] = __reduce_max_sync(0xffffffffu, m[t]);
@@ -191,6 +202,7 @@ __global__ void __launch_bounds__(256) fa_bwd_fixup_kernel(const BwdPreParams p,
       e[kExpDO] = target_exponent(a[kExpDO]);
     }
     for (int t = 0; t < 4; ++t) ex[t] = e[t];
+    ev_copy = reuse_v ? *p.v_exp_fwd : 0;
     if (blockIdx.x == 0) {
       for (int t = 0; t < 4; ++t) p.exps[t] = e[t];
       if (a[0] >= kBitsInf || a[1] >= kBitsInf || a[2] >= kBitsInf || a[3] >= kBitsInf) atomicExch(p.err, kDevRange);
@@ -198,7 +210,8 @@ __global__ void __launch_bounds__(256) fa_bwd_fixup_kernel(const BwdPreParams p,
   }
   __syncthreads();
   const int eq = ex[kExpQ], ek = ex[kExpK], ev = ex[kExpV], edo = ex[kExpDO];
-  if ((eq | ek | ev | edo) == 0) return;
+  const bool redo_v = ev != ev_copy;  // the V copy holds 2^ev_copy V: convert again with 2^ev
+  if ((eq | ek | edo) == 0 && !redo_v && ev == 0) return;
   const long long stride = (long long)gridDim.x * blockDim.x;
   const long long first = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long n8 = (long long)p.BH * p.N * p.d / 8, n8kv = (long long)p.BH_kv * p.N * p.d / 8;
@@ -209,7 +222,7 @@ __global__ void __launch_bounds__(256) fa_bwd_fixup_kernel(const BwdPreParams p,
   };
   if (eq != 0) reconvert(p.q, p.q16, n8, eq);
   if (ek != 0) reconvert(p.k, p.k16, n8kv, ek);
-  if (ev != 0) reconvert(p.v, p.v16, n8kv, ev);
+  if (redo_v) reconvert(p.v, p.v16, n8kv, ev);
   if (edo != 0) reconvert(p.dout, p.do16, n8, edo);
   if (ev + edo != 0) {
     const long long rows = (long long)p.BH * p.Np;

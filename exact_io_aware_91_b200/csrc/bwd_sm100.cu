@@ -198,6 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_ABORT);
   const WaitCtx wctx{abort_flag, p.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // fa_bwd_ws: the forward's V copy now holds 2^exps[V] V (the fix-up converted it again if
+  // the exponent changed); record that in the forward's workspace
+  if (p.v_exp_fwd != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.v_exp_fwd = p.exps[kExpV];
 
   // heaviest first within groups of heads (see unit_order): under the causal mask the
   // first key tiles of a head meet the most query tiles
@@ -1009,6 +1012,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_ABORT);
   const WaitCtx wctx{abort_flag, p.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (p.v_exp_fwd != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.v_exp_fwd = p.exps[kExpV];  // as above
 
   const int n_kt = (p.N + 127) / 128;
   const int BH_kv = p.BH / p.H * p.H_kv;

@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/fa.h: argument checks, tensor-map
 // encoding, workspace carving and kernel launches.  No allocation happens here.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -134,7 +135,8 @@ int kv_split_for(int B, int H, int H_kv, int N, int d) {
 // group is split, see kv_split_for) fp32 partial dK and dV per split, then a 256-byte control
 // block (work counters of the persistent kernels, exponents of the copies), then the
 // preprocess's per-block maxima of |Q|, |K|, |V|, |dO|.
-BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d) {
+// Without own_v16 (fa_bwd_ws: the forward's V copy is used) the V copy's space is left out.
+BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d, bool own_v16 = true) {
   BwdLayout w{};
   w.kv_split = kv_split_for(B, H, H_kv, N, d);
   const size_t t16 = align256((size_t)B * H * N * d * 2);
@@ -145,7 +147,7 @@ BwdLayout bwd_layout(int B, int H, int H_kv, int N, int d) {
   w.off_do16 = t16;
   w.off_k16 = 2 * t16;
   w.off_v16 = 2 * t16 + t16kv;
-  w.off_delta = 2 * t16 + 2 * t16kv;
+  w.off_delta = 2 * t16 + (own_v16 ? 2 : 1) * t16kv;
   w.off_lse2 = w.off_delta + rows;
   w.off_dk_part = w.off_lse2 + rows;
   const size_t part = w.kv_split > 1 ? align256((size_t)w.kv_split * B * H_kv * N * d * 4) : 0;
@@ -320,6 +322,12 @@ size_t fa_bwd_gqa_workspace_size(int B, int H, int H_kv, int N, int d) {
   return bwd_layout(B, H, H_kv, N, d).total;
 }
 
+size_t fa_bwd_ws_workspace_size(int B, int H, int H_kv, int N, int d) {
+  bool empty = false;
+  if (check_problem(B, H, H_kv, N, d, 1.0f, 0, &empty, true) != FA_OK || empty) return 0;
+  return bwd_layout(B, H, H_kv, N, d, false).total;
+}
+
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                  float* dq, float* dk, float* dv, int B, int H, int N, int d, float scale, int causal,
                  void* workspace, fa_stream_t stream) {
@@ -332,7 +340,7 @@ namespace {
 fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
                    const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int H_kv, int N,
                    int d, float scale, int causal, int wl, int wr, void* workspace, size_t workspace_bytes,
-                   fa_stream_t stream);
+                   fa_stream_t stream, void* fwd_workspace = nullptr);
 }  // namespace
 
 fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
@@ -343,17 +351,31 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
                   workspace_bytes, stream);
 }
 
+fa_status fa_bwd_ws(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                    const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int H_kv, int N,
+                    int d, float scale, int causal, void* fwd_workspace, size_t fwd_workspace_bytes, void* workspace,
+                    size_t workspace_bytes, fa_stream_t stream) {
+  bool empty = false;
+  const fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty, true);
+  if (st != FA_OK || empty) return st;
+  if (fwd_workspace == nullptr || fwd_workspace_bytes < fwd_layout(B, H_kv, N, d).total) return FA_ERR_INVALID_ARG;
+  if (!aligned(fwd_workspace, 256)) return FA_ERR_MISALIGNED;
+  return bwd_impl(q, k, v, o, o_resid, dout, lse, dq, dk, dv, B, H, H_kv, N, d, scale, causal, -1, -1, workspace,
+                  workspace_bytes, stream, fwd_workspace);
+}
+
 namespace {
 fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
                    const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int H_kv, int N,
                    int d, float scale, int causal, int wl, int wr, void* workspace, size_t workspace_bytes,
-                   fa_stream_t stream) {
+                   fa_stream_t stream, void* fwd_workspace) {
   bool empty = false;
   if (!window_ok(wl, wr)) return FA_ERR_INVALID_ARG;
   fa_status st = check_problem(B, H, H_kv, N, d, scale, causal, &empty, true);  // d in {64, 128, 256}
   if (st != FA_OK || empty) return st;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
-  const BwdLayout w = bwd_layout(B, H, H_kv, N, d);
+  const bool reuse_v = fwd_workspace != nullptr;  // the V copy of fa_fwd_ws's workspace (fa_bwd_ws)
+  const BwdLayout w = bwd_layout(B, H, H_kv, N, d, !reuse_v);
   if (workspace_bytes < w.total) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
       !aligned(o_resid, 16) || !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(workspace, 256))
@@ -374,8 +396,20 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   pp.lse = lse;
   pp.q16 = ws + w.off_q16;
   pp.k16 = ws + w.off_k16;
-  pp.v16 = ws + w.off_v16;
   pp.do16 = ws + w.off_do16;
+  int* v_exp_fwd = nullptr;
+  if (reuse_v) {  // the forward workspace: V copy at 0, its exponent in the control block, V-pass maxima
+    const FwdLayout fl = fwd_layout(B, H_kv, N, d);
+    uint8_t* fws = static_cast<uint8_t*>(fwd_workspace);
+    const long long n8 = (long long)B * H_kv * N * d / 8;
+    pp.v16 = fws;
+    v_exp_fwd = reinterpret_cast<int*>(fws + fl.off_ctrl + 4);
+    pp.v_exp_fwd = v_exp_fwd;
+    pp.v_amax_fwd = reinterpret_cast<const uint32_t*>(fws + fl.off_amax);
+    pp.v_n_part_fwd = (int)std::min<long long>((n8 + 255) / 256, kVPassBlocks);  // the V pass's grid
+  } else {
+    pp.v16 = ws + w.off_v16;
+  }
   pp.delta = reinterpret_cast<float*>(ws + w.off_delta);
   pp.lse2 = reinterpret_cast<float*>(ws + w.off_lse2);
   pp.N = N;
@@ -400,6 +434,7 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
       !make_tmap_3d(&t_v, pp.v16, h, 2, d, N, BH_kv, 64, 128, 128))
     return FA_ERR_CUDA;
   BwdParams bp{};
+  bp.v_exp_fwd = v_exp_fwd;
   bp.delta = pp.delta;
   bp.lse2 = pp.lse2;
   bp.exps = pp.exps;

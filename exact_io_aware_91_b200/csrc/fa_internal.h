@@ -84,9 +84,17 @@ struct BwdPreParams {
   uint32_t* amax_part; // [4][kPreBlocks] partial max |x| (float bits) of Q, K, V, dO per block
   int* exps;         // [4] exponents of the Q, K, V, dO copies (written by the fix-up)
   int* err;          // device error word
+  // Reuse of the forward's V copy (fa_bwd_ws), else null / 0: v16 then points into the
+  // forward's workspace, the preprocess leaves V alone, the fix-up takes max |V| from the V
+  // pass's per-block maxima and re-converts the copy only when the backward's exponent for V
+  // differs from the copy's (*v_exp_fwd; the dK/dV kernel then records the new one).
+  const uint32_t* v_amax_fwd;  // [v_n_part_fwd] the V pass's per-block max |V| (float bits)
+  int v_n_part_fwd;
+  const int* v_exp_fwd;        // exponent of the forward's V copy
 };
 
 struct BwdParams {
+  int* v_exp_fwd;      // fa_bwd_ws: the forward workspace's V exponent, set to exps[kExpV] (else null)
   const float* delta;  // (BH, Np), in the units of the dO and V copies
   const float* lse2;   // (BH, Np)
   const int* exps;     // [4] exponents of the Q, K, V, dO copies (kExpQ ...)

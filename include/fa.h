@@ -214,6 +214,31 @@ FA_API fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const v
                             size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * fa_bwd_ws_workspace_size / fa_bwd_ws -- fa_bwd_gqa that reuses the fp16 copy of V which
+ * fa_fwd_ws left in its workspace, instead of converting V again (the backward's streaming
+ * preprocess then reads and writes 4 bytes fewer per element of V).
+ *   fwd_workspace, fwd_workspace_bytes : the workspace of the fa_fwd_ws call that produced
+ *                             o (and o_resid, lse) from this v, with the same B, H_kv, N,
+ *                             d, unchanged since (no other forward in it); 256-byte
+ *                             aligned, at least fa_fwd_workspace_size(B, H_kv, N, d)
+ *                             bytes.  The backward may rewrite the V copy there (and the
+ *                             exponent recorded with it) when the bound on the fp16 dS
+ *                             asks for another power-of-two scaling of V than the copy
+ *                             holds (see "Value range"): a later fa_bwd_ws on the same
+ *                             forward workspace stays correct.
+ *   workspace                : at least fa_bwd_ws_workspace_size(B, H, H_kv, N, d) bytes
+ *                             (fa_bwd_gqa's workspace without the V copy).
+ * Everything else as fa_bwd_gqa; the gradients are identical to fa_bwd_gqa's.
+ * Errors: FA_ERR_INVALID_ARG for a NULL or too small forward workspace,
+ * FA_ERR_MISALIGNED for one not 256-byte aligned; otherwise as fa_bwd_gqa.
+ */
+FA_API size_t fa_bwd_ws_workspace_size(int B, int H, int H_kv, int N, int d);
+FA_API fa_status fa_bwd_ws(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                           const void* dout, const float* lse, float* dq, float* dk, float* dv, int B, int H, int H_kv,
+                           int N, int d, float scale, int causal, void* fwd_workspace, size_t fwd_workspace_bytes,
+                           void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * Descriptor-based entry points: every option of the library in one problem
  * description, so that later options do not need new signatures.
  *   B, H, H_kv, N, d, scale, causal : as in fa_fwd_gqa / fa_bwd_gqa (H_kv = H for plain

@@ -196,6 +196,30 @@ def test_backward_argument_errors(lib):
     assert bwd(lib, ws=A + 16) == api.FA_ERR_MISALIGNED  # workspace needs 256-byte alignment
 
 
+def bwd_ws(lib, fws=A, fws_bytes=1 << 40, ws_bytes=1 << 40, B=1, H=1, N=16, d=64):
+    return lib.fa_bwd_ws(A, A, A, A, A, A, A, A, A, A, B, H, H, N, d, 0.125, 0, fws, fws_bytes, A, ws_bytes, None)
+
+
+@pytest.mark.parametrize("shape", [(1, 4, 1, 1, 64), (2, 32, 8, 8192, 128), (2, 16, 16, 2048, 128),
+                                   (1, 2, 2, 300, 256), (3, 6, 3, 1000, 64)])
+def test_backward_with_forward_workspace_sizes(lib, shape):
+    # fa_bwd_gqa's workspace without its fp16 copy of V (B * H_kv * N * d halves)
+    B, H, Hkv, N, d = shape
+    assert api.fa_bwd_ws_workspace_size(*shape) == api.fa_bwd_gqa_workspace_size(*shape) - _align256(B * Hkv * N * d * 2)
+
+
+def test_backward_with_forward_workspace_checks_its_arguments(lib):
+    # every call here is rejected on the host (or is empty): nothing reaches a GPU
+    fneed = api.fa_fwd_workspace_size(1, 1, 16, 64)
+    assert bwd_ws(lib, fws=None) == api.FA_ERR_INVALID_ARG
+    assert bwd_ws(lib, fws_bytes=fneed - 1) == api.FA_ERR_INVALID_ARG
+    assert bwd_ws(lib, fws=A + 16) == api.FA_ERR_MISALIGNED
+    assert bwd_ws(lib, ws_bytes=api.fa_bwd_ws_workspace_size(1, 1, 1, 16, 64) - 1) == api.FA_ERR_INVALID_ARG
+    assert bwd_ws(lib, d=512) == api.FA_ERR_UNSUPPORTED
+    assert bwd_ws(lib, d=96) == api.FA_ERR_UNSUPPORTED
+    assert bwd_ws(lib, fws=None, N=0) == api.FA_OK  # empty problem: nothing to do
+
+
 def test_f32_forward_argument_errors(lib):
     assert lib.fa_fwd_f32(None, A, A, A, A, 1, 1, 8, 64, 0.125, 0, None) == api.FA_ERR_INVALID_ARG
     assert lib.fa_fwd_f32(A + 2, A, A, A, A, 1, 1, 8, 64, 0.125, 0, None) == api.FA_ERR_MISALIGNED
