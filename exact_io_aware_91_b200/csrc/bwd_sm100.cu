@@ -128,16 +128,18 @@ __device__ __forceinline__ void warp_store_rows_f32(const float (&v)[NC], float*
   }
 }
 
-// Load 64 fp32 columns of this thread's TMEM lane (two 32-column loads, one wait).
+// Load 64 fp32 columns of this thread's TMEM lane (two 32-column loads, one wait; the
+// destination registers are read only after the wait).
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t u[32];
-  tmem_ld32(taddr, u);
-#pragma unroll
-  for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(u[c]);
-  tmem_ld32(taddr + 32, u);
-#pragma unroll
-  for (int c = 0; c < 32; ++c) v[32 + c] = __uint_as_float(u[c]);
+  uint32_t u0[32], u1[32];
+  tmem_ld32(taddr, u0);
+  tmem_ld32(taddr + 32, u1);
   tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    v[c] = __uint_as_float(u0[c]);
+    v[32 + c] = __uint_as_float(u1[c]);
+  }
 }
 
 // ============================================================================ dK / dV
@@ -1379,13 +1381,14 @@ struct DqWLayout {
   static constexpr int BAR_SLOT_EMPTY = 5;  // [kWSlots]
   static constexpr int BAR_S = 8;
   static constexpr int BAR_DP = 9;
-  static constexpr int BAR_DS = 10;         // dS of a step written over S, dP read
+  static constexpr int BAR_DS = 10;         // dS of a step written over dP
   static constexpr int BAR_ACC = 11;
   static constexpr int BAR_DQ_FREE = 12;
   static constexpr int BAR_UNIT_FULL = 13;   // [2]
   static constexpr int BAR_UNIT_EMPTY = 15;  // [2]
   static constexpr int BAR_DONE = 17;
-  static constexpr int NBAR = 18;
+  static constexpr int BAR_S_LOADED = 18;    // the step's S is in the compute warps' registers
+  static constexpr int NBAR = 19;
   static constexpr int OFF_UNIT = OFF_BAR + NBAR * 8;
   static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
@@ -1459,6 +1462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(L::BAR_ACC), 1);
     mbar_init(bar(L::BAR_DQ_FREE), 256);
     mbar_init(bar(L::BAR_DONE), 1);
+    mbar_init(bar(L::BAR_S_LOADED), 256);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -1470,8 +1474,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_TMEM_SLOT);
 
-  // FIFO order of a unit with n key steps: K0(0) K1(0) V0(0) V1(0), then for it = 0..n-1:
-  // K0(it) K1(it) [dQ], [V0(it+1) V1(it+1) K0(it+1) K1(it+1)]  (bracketed part while it + 1 < n).
+  // dS is written over dP, so S(it + 1) may overwrite S as soon as the compute warps hold S(it)
+  // in registers, while dP(it + 1) follows dQ(it) (which reads dS(it)).  FIFO order of a unit
+  // with n key steps: K0(0) K1(0) V0(0) V1(0), then for it = 0..n-1:
+  // [K0(it+1) K1(it+1)] K0(it) K1(it) [V0(it+1) V1(it+1)]  (bracketed parts while it + 1 < n).
   if (warp == 0) {
     // ===================================================== TMA producer + work distribution
     regs_dec<kRegsLow>();
@@ -1517,10 +1523,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = x.n_it;
       ok = load_half(x, 0, 0, 0) && load_half(x, 0, 1, 0) && load_half(x, 1, 0, 0) && load_half(x, 1, 1, 0);
       for (int it = 0; it < n && ok; ++it) {
-        ok = load_half(x, 0, 0, it) && load_half(x, 0, 1, it);  // K again, for dQ(it)
-        if (ok && it + 1 < n)
-          ok = load_half(x, 1, 0, it + 1) && load_half(x, 1, 1, it + 1) && load_half(x, 0, 0, it + 1) &&
-               load_half(x, 0, 1, it + 1);
+        if (it + 1 < n) ok = load_half(x, 0, 0, it + 1) && load_half(x, 0, 1, it + 1);  // S(it + 1)
+        ok = ok && load_half(x, 0, 0, it) && load_half(x, 0, 1, it);                    // K again, dQ(it)
+        if (ok && it + 1 < n) ok = load_half(x, 1, 0, it + 1) && load_half(x, 1, 1, it + 1);  // dP(it + 1)
       }
       if (!ok) break;
     }
@@ -1572,6 +1577,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (n == 1) mma_commit(bar(L::BAR_Q_EMPTY), leader);
       for (int it = 0; it < n && ok; ++it) {
         const int t = T0 + it;
+        if (it + 1 < n) {  // S(it + 1) once the compute warps hold S(it) in registers
+          if (!(ok = mbar_wait(bar(L::BAR_S_LOADED), t & 1, wctx))) break;
+          tc_fence_after();
+          if (!(ok = issue_full(tmem + L::T_S, dQs, bar(L::BAR_S)))) break;
+        }
         if (!(ok = mbar_wait(bar(L::BAR_DS), t & 1, wctx))) break;
         tc_fence_after();
         if (it == 0 && uc > 0) {
@@ -1581,14 +1591,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hh = 0; hh < 2 && ok; ++hh) {  // dQ[:, 128 hh ..] += dS K_hh
           const int st = take();
           if (!ok) break;
-          issue_ts_split(tmem + L::T_DQ + 128 * hh, tmem + L::T_S, sdesc_add(dRingMN, st * kHalf), idesc_g, it > 0,
-                         leader);
+          issue_ts_split(tmem + L::T_DQ + 128 * hh, tmem + L::T_DP, sdesc_add(dRingMN, st * kHalf), idesc_g,
+                         it > 0, leader);
           mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
         }
         if (!ok) break;
         if (it + 1 < n) {
-          if (!(ok = issue_full(tmem + L::T_DP, dDOs, bar(L::BAR_DP)))) break;  // dP(it + 1)
-          if (!(ok = issue_full(tmem + L::T_S, dQs, bar(L::BAR_S)))) break;     // S(it + 1), after dQ(it)
+          if (!(ok = issue_full(tmem + L::T_DP, dDOs, bar(L::BAR_DP)))) break;  // dP(it + 1), after dQ(it)
           if (it + 2 == n) mma_commit(bar(L::BAR_Q_EMPTY), leader);
         }
       }
@@ -1635,6 +1644,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         float pr[64];
         tmem_ld64(tS, pr);
+        tc_fence_before();
+        mbar_arrive(bar(L::BAR_S_LOADED));  // S(it + 1) may overwrite S
         auto probs = [&](auto masked) {
           const int c_lo = k_vis_lo - k0, c_hi = k_vis_hi - k0;
 #pragma unroll
@@ -1662,7 +1673,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(bar(L::BAR_DP), t & 1, wctx))) break;
         tc_fence_after();
         float dp[64];
-        tmem_ld64(tmem + lane_off + L::T_DP + 64 * w, dp);
+        const uint32_t tDP = tmem + lane_off + L::T_DP + 64 * w;
+        tmem_ld64(tDP, dp);
 #pragma unroll
         for (int g = 0; g < 64; g += 16) {
           uint32_t pk[8];
@@ -1672,7 +1684,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(f2pack(dp[c], dp[c + 1]), dd)), d0, d1);
             pk[(c - g) / 2] = pack_f16(d0, d1);
           }
-          tmem_st8(tS + g / 2, pk);
+          tmem_st8(tDP + g / 2, pk);  // dS over dP
         }
         tmem_wait_st();
         tc_fence_before();
