@@ -579,7 +579,8 @@ struct DqLayout {
   static constexpr int BAR_DQ_FREE = 19; // the epilogue has read a unit's dQ out of TMEM
   static constexpr int BAR_UNIT_FULL = 20;   // [2] next work unit index published
   static constexpr int BAR_UNIT_EMPTY = 22;  // [2] ... and read by the MMA warp and both warpgroups
-  static constexpr int NBAR = 24;
+  static constexpr int BAR_DP_LOADED = 24;   // the step's dP is in the compute warps' registers
+  static constexpr int NBAR = 25;
   static constexpr int OFF_UNIT = OFF_BAR + NBAR * 8;  // int[2]: work unit ring
   static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
@@ -665,6 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(L::BAR_DS + s), 256);
     }
     mbar_init(bar(L::BAR_DP), 1);
+    mbar_init(bar(L::BAR_DP_LOADED), 256);
     mbar_init(bar(L::BAR_ACC), 1);
     mbar_init(bar(L::BAR_DQ_FREE), 256);
     mbar_init(bar(L::BAR_DONE), 1);
@@ -778,6 +780,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < n && ok; ++it) {
         const int t = T0 + it;
         const int b = t & 1;
+        // dP(t + 1) as soon as the compute warps hold dP(t) in registers (dS goes over S)
+        if (it + 1 < n) {
+          if (!(ok = mbar_wait(bar(L::BAR_DP_LOADED), t & 1, wctx))) break;
+          if (!(ok = issue_dp(t + 1))) break;
+        }
         if (!(ok = mbar_wait(bar(L::BAR_DS + b), (t >> 1) & 1, wctx))) break;
         tc_fence_after();
         // the first dQ MMA of a unit overwrites the accumulator: the previous unit's epilogue
@@ -789,7 +796,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_ts_split(tmem + L::T_DQ, tmem + L::T_S + 128 * b, sdesc_add(dKmn, (t % 3) * L::TILE), idesc_g, it > 0,
                        leader);  // dQ += dS K
         mma_commit(bar(L::BAR_K_EMPTY + t % 3), leader);
-        if (it + 1 < n && !(ok = issue_dp(t + 1))) break;
         if (it + 2 < n && !(ok = issue_s(t + 2))) break;
         if (it + 2 == n) mma_commit(bar(L::BAR_Q_EMPTY), leader);  // S(n-1), dP(n-1) issued
       }
@@ -871,6 +877,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         float dp[64];
         tmem_ld64(tmem + lane_off + L::T_DP + 64 * w, dp);
+        tc_fence_before();
+        mbar_arrive(bar(L::BAR_DP_LOADED));  // dP(t + 1) may overwrite dP
 #pragma unroll
         for (int g = 0; g < 64; g += 16) {
           uint32_t pk[8];
