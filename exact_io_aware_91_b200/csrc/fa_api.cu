@@ -268,9 +268,19 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   p.err = g_err_ptr[dev];
   // with a workspace: the persistent kernel (work counter in the workspace); without: one CTA
   // per unit, V converted on chip
-  const cudaError_t e = d == 256 ? launch_fwd_d256_sm100(tq, tk, tv, p, s)
-                        : v16    ? launch_fwd_persist_sm100(tq, tk, tv, p, d, s)
-                                 : launch_fwd_sm100(tq, tk, tv, to, p, d, s);
+  cudaError_t e;
+  if (d == 256) {
+    e = launch_fwd_d256_sm100(tq, tk, tv, p, s);
+  } else if (v16) {
+    // O and the residual in 32-row boxes for the persistent kernel's per-warp bulk stores
+    CUtensorMap to32, tr32;
+    if (!make_tmap_3d(&to32, o, bf, 2, d, N, BH, 64, 32, 128) ||
+        !make_tmap_3d(&tr32, o_resid != nullptr ? o_resid : o, bf, 2, d, N, BH, 64, 32, 128))
+      return FA_ERR_CUDA;
+    e = launch_fwd_persist_sm100(tq, tk, tv, to32, tr32, p, d, s);
+  } else {
+    e = launch_fwd_sm100(tq, tk, tv, to, p, d, s);
+  }
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 }  // namespace
@@ -536,8 +546,10 @@ fa_status fa_attn_fwd_fp8(const fa_attn_problem* pr, const void* q, const void* 
   if (cudaMemsetAsync(counter, 0, sizeof(unsigned), s) != cudaSuccess) return FA_ERR_CUDA;
   CUtensorMap tq, tk, tv;
   const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUtensorMap to32;  // bf16 O in 32-row boxes (the epilogue's bulk stores)
   if (!make_tmap_3d(&tq, q, u8, 1, d, N, BH, d, 128, d) || !make_tmap_3d(&tk, k, u8, 1, d, N, BH_kv, d, 128, d) ||
-      !make_tmap_3d(&tv, v, u8, 1, d, N, BH_kv, d, 128, d))
+      !make_tmap_3d(&tv, v, u8, 1, d, N, BH_kv, d, 128, d) ||
+      !make_tmap_3d(&to32, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, 32, 128))
     return FA_ERR_CUDA;
   FwdParams p{};
   p.lse = lse;
@@ -558,7 +570,7 @@ fa_status fa_attn_fwd_fp8(const fa_attn_problem* pr, const void* q, const void* 
   p.win_left = pr->window_left;
   p.win_right = pr->window_right;
   p.err = g_err_ptr[dev];
-  return launch_fwd_persist_fp8_sm100(tq, tk, tv, p, d, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return launch_fwd_persist_fp8_sm100(tq, tk, tv, to32, p, d, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 void fa_bwd_set_phase_events(void* const* events) { t_phase_events = events; }

@@ -143,12 +143,15 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
 // fix-up that picks the copy's exponent (v_exp) and re-converts V if it is not 0.
 cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, uint32_t* amax_part,
                            int* v_exp, int* err, cudaStream_t s);
+// to32, tr32: O and the residual in 64-column x 32-row boxes (the epilogue's bulk stores)
 cudaError_t launch_fwd_persist_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                     const FwdParams& p, int d, cudaStream_t s);
+                                     const CUtensorMap& to32, const CUtensorMap& tr32, const FwdParams& p, int d,
+                                     cudaStream_t s);
 cudaError_t launch_fwd_d256_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                   const FwdParams& p, cudaStream_t s);  // d = 256, fp16 V in 64 x 64 boxes
 cudaError_t launch_fwd_persist_fp8_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                         const FwdParams& p, int d, cudaStream_t s);  // d = 128 or 64, E4M3
+                                         const CUtensorMap& to32, const FwdParams& p, int d,
+                                         cudaStream_t s);  // d = 128 or 64, E4M3
 cudaError_t launch_selftest_wait(int* err, cudaStream_t s);
 cudaError_t launch_selftest_exp2(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_bwd_kv_reduce(const float* dk_part, const float* dv_part, float* dk, float* dv,

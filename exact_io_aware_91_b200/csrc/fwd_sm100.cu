@@ -103,6 +103,7 @@ constexpr int kConvThreads = 64;
 constexpr int kFwdParts = FA_FWD_PARTS;
 // element pairs out of every 8 whose exponentials run on the FMA pipe (even, 0..8)
 constexpr int kExpFmaPer8 = FA_EXP_FMA_PER8;
+
 constexpr int kExpFmaPer8F8 = FA_EXP_FMA_PER8_F8;
 static_assert(kExpFmaPer8 % 2 == 0 && kExpFmaPer8 >= 0 && kExpFmaPer8 <= 8, "pairs are taken two at a time");
 static_assert(kExpFmaPer8F8 % 2 == 0 && kExpFmaPer8F8 >= 0 && kExpFmaPer8F8 <= 8, "pairs are taken two at a time");
@@ -599,9 +600,9 @@ namespace {
 // overlap the previous unit's last steps and epilogue.  V is fp16 already.  K/V ring
 // positions count loads across units, the per-tile barriers (S_FULL, P_HALF, P_FULL)
 // count that tile's steps across units, and the per-unit barriers (Q_FULL, Q_EMPTY,
-// O_FULL, O_FREE) count units.  O and the residual are stored straight from registers
-// (coalesced by warp_store_rows_128b): the Q buffers are reloaded for the next unit and
-// cannot serve as the output staging tile.
+// O_FULL, O_FREE) count units.  O and the residual leave through a 4 KB staging box per
+// softmax warp (its 32 rows x 64 columns, 128-byte swizzle) and one bulk tensor store per box
+// (the Q buffers are reloaded for the next unit and cannot serve as staging).
 //
 // F8 (8-bit inputs, d = 128 or 64): Q, K and V are E4M3, so a row of d elements is one
 // 128-byte swizzle row (d = 128; 16 KB tiles) or one 64-byte swizzle row (d = 64; 8 KB tiles);
@@ -628,7 +629,9 @@ struct FwdPLayout {
   static constexpr int OFF_Q0 = 0;
   static constexpr int OFF_Q1 = TILE;
   static constexpr int OFF_KV = 2 * TILE;
-  static constexpr int OFF_BAR = OFF_KV + STAGES * TILE;
+  // epilogue staging: one 32-row x 128-byte swizzled box per softmax warp
+  static constexpr int OFF_STG = OFF_KV + STAGES * TILE;
+  static constexpr int OFF_BAR = OFF_STG + 8 * 4096;
   static constexpr int BAR_Q_FULL = 0;
   static constexpr int BAR_Q_EMPTY = 1;
   static constexpr int BAR_KV_FULL = 2;
@@ -645,6 +648,7 @@ struct FwdPLayout {
   static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
   static constexpr int SMEM_ALLOC = OFF_ABORT + 8 + 1024;
+  static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
 };
@@ -652,7 +656,8 @@ struct FwdPLayout {
 template <int D, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_persist_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o32,
+                                const __grid_constant__ CUtensorMap tm_r32, const FwdParams p) {
   using L = FwdPLayout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -915,10 +920,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       G += n_t;
       if (!ok) break;
-      // ---- epilogue: O / l -> bf16 and the bf16 residual, stored from registers
+      // ---- epilogue: O / l -> bf16 and the bf16 residual
       if (!(ok = mbar_wait(bar(L::BAR_O_FULL + t), uc & 1, wctx))) break;
       tc_fence_after();
       const float inv_l = out_scale / l;
+      // this warp's 32 rows through its swizzled staging box, one bulk tensor store per
+      // 64-column chunk (and per residual chunk); a box is rewritten only after the
+      // previous store has read it
+      const uint32_t stg = base + L::OFF_STG + (uint32_t)(warp - 4) * 4096u;
+      auto stage_and_store = [&](const uint32_t (&w)[32], const CUtensorMap* m, int col) {
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          st_shared_v4(stg + sw128_offset(lane, q4), w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(m, col, q_base + wq * 32, x.bh, stg);
+          bulk_commit_group();
+        }
+      };
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t u0[32], u1[32];
@@ -929,33 +951,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(bar(L::BAR_O_FREE + t));
         }
-        uint4 oa[8], ra[8];
+        uint32_t pk[32], rk[32];
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          uint32_t pk[4], rk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 4 * q4 + e;  // packed pair index 0..31 within the chunk
-            const uint32_t* uu = i < 16 ? u0 : u1;
-            const int k = 2 * (i & 15);
-            const float a = __uint_as_float(uu[k]) * inv_l, b = __uint_as_float(uu[k + 1]) * inv_l;
-            pk[e] = pack_bf16(a, b);
-            const float2 ab = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
-            rk[e] = pack_bf16(a - ab.x, b - ab.y);
-          }
-          oa[q4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          ra[q4] = make_uint4(rk[0], rk[1], rk[2], rk[3]);
+        for (int i = 0; i < 32; ++i) {
+          const uint32_t* uu = i < 16 ? u0 : u1;
+          const int k2 = 2 * (i & 15);
+          const float a = __uint_as_float(uu[k2]) * inv_l, b = __uint_as_float(uu[k2 + 1]) * inv_l;
+          pk[i] = pack_bf16(a, b);
+          const float2 ab = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i]));
+          rk[i] = pack_bf16(a - ab.x, b - ab.y);
         }
-        warp_store_rows_128b(oa, reinterpret_cast<uint8_t*>(p.o + (size_t)x.bh * p.N * D + 64 * c), D * 2,
-                             q_base + wq * 32, p.N);
-        if (p.o_resid != nullptr)
-          warp_store_rows_128b(ra, reinterpret_cast<uint8_t*>(p.o_resid + (size_t)x.bh * p.N * D + 64 * c), D * 2,
-                               q_base + wq * 32, p.N);
+        stage_and_store(pk, &tm_o32, 64 * c);
+        if (p.o_resid != nullptr) stage_and_store(rk, &tm_r32, 64 * c);
       }
       if (p.lse != nullptr && r < p.N) p.lse[(size_t)x.bh * p.N + r] = (m + __log2f(l)) * 0.69314718055994531f;
       u = next_unit(uc + 1, ok);
       mbar_arrive(bar(L::BAR_UNIT_EMPTY + ((uc + 1) & 1)));
     }
+    if (lane == 0) bulk_wait_group0();  // this warp's bulk stores are complete
   }
 
   tc_fence_before();
@@ -1318,12 +1331,12 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 template <int D, bool F8>
 cudaError_t launch_persist_t(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const FwdParams& p, cudaStream_t s) {
+                             const CUtensorMap& to32, const CUtensorMap& tr32, const FwdParams& p, cudaStream_t s) {
   using L = FwdPLayout<D, F8>;
   cudaError_t e = cudaFuncSetAttribute(fa_fwd_persist_sm100_kernel<D, F8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  fa_fwd_persist_sm100_kernel<D, F8><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, p);
+  fa_fwd_persist_sm100_kernel<D, F8><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tk, tv, to32, tr32, p);
   return cudaGetLastError();
 }
 
@@ -1400,19 +1413,20 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
 }
 
 cudaError_t launch_fwd_persist_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                     const FwdParams& p, int d, cudaStream_t s) {
+                                     const CUtensorMap& to32, const CUtensorMap& tr32, const FwdParams& p, int d,
+                                     cudaStream_t s) {
   const long long units = (long long)p.n_pairs * p.BH;
   const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
-  return d == 128 ? launch_persist_t<128, false>(grid, tq, tk, tv, p, s)
-                  : launch_persist_t<64, false>(grid, tq, tk, tv, p, s);
+  return d == 128 ? launch_persist_t<128, false>(grid, tq, tk, tv, to32, tr32, p, s)
+                  : launch_persist_t<64, false>(grid, tq, tk, tv, to32, tr32, p, s);
 }
 
 cudaError_t launch_fwd_persist_fp8_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                         const FwdParams& p, int d, cudaStream_t s) {
+                                         const CUtensorMap& to32, const FwdParams& p, int d, cudaStream_t s) {
   const long long units = (long long)p.n_pairs * p.BH;
   const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
-  return d == 128 ? launch_persist_t<128, true>(grid, tq, tk, tv, p, s)
-                  : launch_persist_t<64, true>(grid, tq, tk, tv, p, s);
+  return d == 128 ? launch_persist_t<128, true>(grid, tq, tk, tv, to32, to32, p, s)
+                  : launch_persist_t<64, true>(grid, tq, tk, tv, to32, to32, p, s);
 }
 
 cudaError_t launch_fwd_v16(const void* v, void* v16, long long elems, unsigned* counter, uint32_t* amax_part,
