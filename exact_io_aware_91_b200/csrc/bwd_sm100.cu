@@ -142,6 +142,14 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   }
 }
 
+constexpr int kSmemMax = 232448;  // dynamic shared memory of one CTA on sm_100
+// The kernels declare their shared memory 1024-byte aligned and allocate at most kSmemMax; this
+// checks that the aligned base leaves room for the layout (it always does with an aligned start).
+template <typename L>
+__device__ __forceinline__ bool smem_base_fits(uint32_t raw, uint32_t base) {
+  return base - raw + (uint32_t)L::BYTES <= (uint32_t)L::SMEM_ALLOC;
+}
+
 // ============================================================================ dK / dV
 template <int D>
 struct DkdvLayout {
@@ -152,7 +160,8 @@ struct DkdvLayout {
   static constexpr int OFF_Q = 2 * TILE;        // two Q buffers
   static constexpr int OFF_DO = 4 * TILE;       // two dO buffers
   static constexpr int OFF_LD = 6 * TILE;       // two (lse2[128], delta[128]) pairs, 1 KB each
-  static constexpr int OFF_BAR = OFF_LD + 2048;
+  static constexpr int OFF_STG = OFF_LD + 2048;  // epilogue: a 32-row x 128-byte box per compute warp
+  static constexpr int OFF_BAR = OFF_STG + 8 * 4096;
   static constexpr int BAR_KV = 0;        // a unit's K, V landed
   static constexpr int BAR_Q_FULL = 1;    // [2]
   static constexpr int BAR_Q_EMPTY = 3;   // [2]
@@ -173,10 +182,12 @@ struct DkdvLayout {
   static constexpr int OFF_UNIT = OFF_BAR + NBAR * 8;  // int[2]
   static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
-  static constexpr int SMEM_ALLOC = OFF_ABORT + 8 + 1024;
+  static constexpr int BYTES = OFF_ABORT + 8;
+  static constexpr int SMEM_ALLOC = BYTES + 1024 <= kSmemMax ? BYTES + 1024 : kSmemMax;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
 };
+static_assert(DkdvLayout<128>::BYTES <= kSmemMax, "dK/dV kernel exceeds the shared memory of a CTA");
 
 // Persistent dK/dV kernel: one CTA per SM takes work units (key/value head, 128-key tile,
 // share of the group's query heads) one after another from a work counter in the workspace
@@ -190,11 +201,16 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                              const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                             const __grid_constant__ CUtensorMap tm_dv, const __grid_constant__ CUtensorMap tm_dk,
                              const BwdParams p) {
   using L = DkdvLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
+  if (!smem_base_fits<L>(raw, base)) {  // cannot happen with a 1024-aligned start; report, do nothing
+    if (threadIdx.x == 0) atomicExch(p.err, kDevRange);
+    return;
+  }
   uint8_t* gbase = smem_raw + (base - raw);
   auto bar = [&](int i) -> uint32_t { return base + L::OFF_BAR + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_ABORT);
@@ -523,14 +539,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = mbar_wait(bar(L::BAR_ACC), uc & 1, wctx))) break;
       tc_fence_after();
       // with the group split over several CTAs each writes its partial sums for the reduction
+      // (the host points tm_dv / tm_dk at the partial buffers then)
       const Unit x = unit_of(u);
-      const size_t head_off = p.kv_split == 1 ? (size_t)x.bh * p.N * D
-                                              : ((size_t)x.sp * BH_kv + x.bh) * p.N * D;
-      float* out = (p.kv_split == 1 ? (w == 0 ? p.dv : p.dk) : (w == 0 ? p.dv_part : p.dk_part)) + head_off;
-      // warpgroup 0 writes dV, warpgroup 1 writes scale * dK (rows past N are padding), 64
-      // columns at a time; once the last columns are loaded the next unit may overwrite them
+      const int head = p.kv_split == 1 ? x.bh : x.sp * BH_kv + x.bh;
+      // warpgroup 0 writes dV, warpgroup 1 writes scale * dK (rows past N are padding and are
+      // clipped by the bulk store), 64 columns at a time through this warp's 32-row x 128-byte
+      // staging box, one bulk tensor store per 32 columns; once the last columns are loaded
+      // the next unit may overwrite the accumulators
       const uint32_t t_acc = tmem + lane_off + (w == 0 ? L::T_DV : L::T_DK);
       const Pow2 out_f = pow2_factors(w == 0 ? -p.exps[kExpDO] : -(p.exps[kExpV] + p.exps[kExpDO] + p.exps[kExpQ]));
+      const float mult = w == 0 ? 1.0f : p.scale;
+      auto sc = [&](float v) { return __float_as_uint(v * mult * out_f.a * out_f.b); };
+      const uint32_t stg = base + L::OFF_STG + (uint32_t)(warp - 4) * 4096u;
+      const CUtensorMap* m_out = w == 0 ? &tm_dv : &tm_dk;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         float acc[64];
@@ -539,12 +560,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(bar(L::BAR_ACC_FREE));
         }
-        warp_store_rows_f32<64>(acc, out + 64 * c, D, j * 128 + wq * 32, p.N, w == 0 ? 1.0f : p.scale, out_f);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (lane == 0) bulk_wait_group_read0();  // the box's previous store has read it
+          __syncwarp();
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float* a = acc + 32 * h + 4 * q4;
+            const uint32_t addr = stg + sw128_offset(lane, q4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(sc(a[0])), "r"(sc(a[1])),
+                         "r"(sc(a[2])), "r"(sc(a[3]))
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(m_out, 64 * c + 32 * h, j * 128 + wq * 32, head, stg);
+            bulk_commit_group();
+          }
+        }
       }
       T0 += n_it;
       u = next_unit(uc + 1, ok);
       mbar_arrive(bar(L::BAR_UNIT_EMPTY + ((uc + 1) & 1)));
     }
+    if (lane == 0) bulk_wait_group0();  // this warp's bulk stores are complete
   }
 
   tc_fence_before();
@@ -953,7 +993,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 // masks, grouped heads, windows, work order, coalesced epilogues) is the same.
 constexpr int kHalf = 2 * kBox;  // 128 rows x 128 fp16 columns (two 64-column boxes), 32 KB
 constexpr int kWSlots = 3;       // FIFO slots of one half each
-constexpr int kSmemMax = 232448;  // dynamic shared memory of one CTA on sm_100
 
 // SS product D (+)= A * B^T over K = 128 (one half of d): `first` marks the first product into D.
 __device__ __forceinline__ void issue_ss_half(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -999,10 +1038,6 @@ struct DkdvWLayout {
 };
 static_assert(DkdvWLayout::BYTES <= kSmemMax, "d = 256 dK/dV kernel exceeds the shared memory of a CTA");
 
-template <typename L>
-__device__ __forceinline__ bool smem_base_fits(uint32_t raw, uint32_t base) {
-  return base - raw + (uint32_t)L::BYTES <= (uint32_t)L::SMEM_ALLOC;
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_dkdv_d256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -1746,17 +1781,29 @@ cudaError_t launch_one(Kern kern, dim3 grid, const CUtensorMap& a, const CUtenso
 
 }  // namespace
 
+template <int D>
+cudaError_t launch_dkdv_t(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                          const CUtensorMap& tv, const CUtensorMap& tdv, const CUtensorMap& tdk, const BwdParams& p,
+                          cudaStream_t s) {
+  using L = DkdvLayout<D>;
+  cudaError_t e = cudaFuncSetAttribute(fa_bwd_dkdv_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       L::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  fa_bwd_dkdv_sm100_kernel<D><<<grid, kThreads, L::SMEM_ALLOC, s>>>(tq, tdo, tk, tv, tdv, tdk, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
-                                  const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s) {
+                                  const CUtensorMap& tv, const CUtensorMap& tdv, const CUtensorMap& tdk,
+                                  const BwdParams& p, int d, cudaStream_t s) {
   // persistent: one CTA per SM (at most one per unit: key tile x key/value head x group split,
   // and x the d-half at d = 256)
   const long long units =
       (long long)((p.N + 127) / 128) * (p.BH / p.H * p.H_kv) * p.kv_split * (d == 256 ? 2 : 1);
   const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
   if (d == 256) return launch_one<DkdvWLayout>(fa_bwd_dkdv_d256_kernel, grid, tq, tdo, tk, tv, p, s);
-  if (d == 128)
-    return launch_one<DkdvLayout<128>>(fa_bwd_dkdv_sm100_kernel<128>, grid, tq, tdo, tk, tv, p, s);
-  return launch_one<DkdvLayout<64>>(fa_bwd_dkdv_sm100_kernel<64>, grid, tq, tdo, tk, tv, p, s);
+  if (d == 128) return launch_dkdv_t<128>(grid, tq, tdo, tk, tv, tdv, tdk, p, s);
+  return launch_dkdv_t<64>(grid, tq, tdo, tk, tv, tdv, tdk, p, s);
 }
 
 cudaError_t launch_bwd_dq_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,

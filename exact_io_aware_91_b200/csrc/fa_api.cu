@@ -472,7 +472,14 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   bp.win_left = wl;
   bp.win_right = wr;
   bp.err = g_err_ptr[dev];
-  if (launch_bwd_dkdv_sm100(t_q, t_do, t_k, t_v, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  // dV, dK (or their partial sums per group split) in 32 x 32 fp32 boxes for the dK/dV epilogue
+  CUtensorMap t_dv, t_dk;
+  const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const int out_heads = w.kv_split > 1 ? w.kv_split * BH_kv : BH_kv;
+  if (!make_tmap_3d(&t_dv, w.kv_split > 1 ? static_cast<void*>(bp.dv_part) : dv, f32, 4, d, N, out_heads, 32, 32, 128) ||
+      !make_tmap_3d(&t_dk, w.kv_split > 1 ? static_cast<void*>(bp.dk_part) : dk, f32, 4, d, N, out_heads, 32, 32, 128))
+    return FA_ERR_CUDA;
+  if (launch_bwd_dkdv_sm100(t_q, t_do, t_k, t_v, t_dv, t_dk, bp, d, s) != cudaSuccess) return FA_ERR_CUDA;
   if (w.kv_split > 1 &&
       launch_bwd_kv_reduce(bp.dk_part, bp.dv_part, dk, dv, (long long)BH_kv * N * d, w.kv_split, s) != cudaSuccess)
     return FA_ERR_CUDA;

@@ -161,8 +161,11 @@ cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float
 // Backward preprocess (D, LSE * log2(e), fp16 copies with exponent 0, per-block maxima), then
 // the fix-up that picks the copies' exponents, re-converts where they are not 0 and scales D.
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t s);
+// tdv, tdk: fp32 dV and dK (or, with kv_split > 1, the partial buffers: kv_split * B * H_kv
+// heads) in 32-column x 32-row boxes, for the epilogue's bulk stores (d = 64, 128)
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
-                                  const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s);
+                                  const CUtensorMap& tv, const CUtensorMap& tdv, const CUtensorMap& tdk,
+                                  const BwdParams& p, int d, cudaStream_t s);
 cudaError_t launch_bwd_dq_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                                 const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t s);
 
