@@ -95,3 +95,22 @@ def test_backward_rescales_the_forward_copy_when_needed():
     for ref, got in pairs:
         for name, a, b in zip(("dq", "dk", "dv"), ref, got):
             assert torch.equal(a, b), f"{name} differs"
+
+
+def test_forward_and_backward_allocate_nothing():
+    # with caller workspaces the training path (fa_fwd_ws + fa_bwd_ws) allocates no device memory
+    B, H, N, d = 1, 4, 4096, 128
+    inp = inputs.make_qkv(B, H, N, d, seed=3, device="cuda")
+    q, k, v, do = inp["q"], inp["k"], inp["v"], inp["do"]
+    fws = torch.empty(api.fa_fwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(api.fa_bwd_ws_workspace_size(B, H, H, N, d), dtype=torch.uint8, device="cuda")
+    o, lse, res = torch.empty_like(q), torch.empty((B, H, N), device="cuda"), torch.empty_like(q)
+    dq = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    dk, dv = torch.empty_like(dq), torch.empty_like(dq)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    api.fa_fwd_ws(q, k, v, causal=True, o=o, lse=lse, o_resid=res, workspace=fws)
+    api.fa_bwd_ws(q, k, v, o, do, lse, fws, causal=True, workspace=ws, dq=dq, dk=dk, dv=dv, o_resid=res)
+    torch.cuda.synchronize()
+    assert api.fa_last_device_status() == api.FA_OK
+    assert torch.cuda.mem_get_info()[0] >= free0 - (2 << 20)  # no N x N (or any) device buffer
