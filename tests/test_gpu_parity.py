@@ -137,6 +137,35 @@ def test_forward_with_workspace_matches_on_chip_conversion(B, H, Hkv, N, d, caus
     assert_fwd(o2, l2, O, L, f"fa_fwd_ws B={B} H={H} Hkv={Hkv} N={N} d={d} causal={causal}")
 
 
+# the d = 64 workspace forward (the persistent kernel with the 64-byte rows of one swizzle span):
+# several units per head and per CTA, ragged last units, causal, windows, grouped heads and
+# 2 % spiky keys, with the residual checked where O's bf16 rounding dominates its error
+@pytest.mark.parametrize("B,H,Hkv,N,causal,window", [(2, 4, 2, 2100, True, (-1, -1)),
+                                                     (2, 4, 2, 2100, False, (-1, -1)),
+                                                     (1, 6, 3, 1500, True, (200, -1)),
+                                                     (1, 3, 3, 1300, False, (100, 300)),
+                                                     (3, 2, 1, 130, True, (-1, -1)),
+                                                     (1, 2, 2, 640, False, (0, 0))])
+def test_workspace_forward_d64(B, H, Hkv, N, causal, window):
+    d = 64
+    inp = inputs.make_qkv(B, H, N, d, seed=N + 13 * H + Hkv + causal, spiky_frac=0.02, kv_heads=Hkv,
+                          backward=False, device="cuda")
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    scale = 1.0 / np.sqrt(d)
+    tag = f"d=64 B={B} H={H} Hkv={Hkv} N={N} causal={causal} window={window}"
+    o, lse, res = api.fa_attn_fwd(q, k, v, causal=causal, scale=scale, window=window, save_residual=True)
+    torch.cuda.synchronize()
+    O, L = oracle.attention_forward_gqa(q, k, v, scale, causal, window=window)
+    assert_fwd(o, lse, O, L, tag)
+    err_bf16 = np.abs(f64(o) - O).max()
+    if err_bf16 > 1e-3:  # O's bf16 rounding dominates its error: the residual recovers most of it
+        assert np.abs(f64(o) + f64(res) - O).max() < 0.25 * err_bf16, tag
+    if window == (-1, -1):  # fa_fwd_ws takes the same path: the same bits
+        o2, lse2, r2 = api.fa_fwd_ws(q, k, v, causal=causal, scale=scale, save_residual=True)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o2) and torch.equal(lse, lse2) and torch.equal(res, r2), tag
+
+
 WINDOWS = [(True, (0, -1)), (True, (127, -1)), (True, (128, -1)), (True, (300, -1)), (True, (5, 7)),
            (False, (64, 64)), (False, (0, 0)), (False, (-1, 200)), (False, (333, -1))]
 
