@@ -94,7 +94,9 @@ def recorded_traffic(kernel: str, workload_name: str):
     """DRAM bytes per launch from the committed ncu summary, if the kernel's code is unchanged."""
     short = {"causal_b2_h32_n8192_d128_spiky": "causal_b2_h32_n8192_d128",
              "causal_b2_h32_n8192_d128_spiky_fp8": "causal_b2_h32_n8192_d128_fp8",
-             "causal_b2_h16_n8192_d256_spiky": "causal_b2_h16_n8192_d256"}.get(workload_name)
+             "causal_b2_h16_n8192_d256_spiky": "causal_b2_h16_n8192_d256",
+             "causal_b4_h16_n2048_d128": "causal_b4_h16_n2048_d128",
+             "noncausal_b64_h16_n512_d64": "noncausal_b64_h16_n512_d64"}.get(workload_name)
     if short is None:
         return None
     path = os.path.join(ROOT, "profiles", f"traffic_{short}.json")
