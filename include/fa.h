@@ -43,8 +43,10 @@
  *    not synchronise.  Argument errors are detected on the host before anything
  *    is launched; nothing is written then.
  *  - B, H or N equal to 0 is an empty problem: FA_OK, nothing launched.
- *  - Supported: d in {64, 128}; also d = 256 for the forward with a workspace
- *    (fa_fwd_ws, fa_attn_fwd); a B200-class GPU (compute capability 10.0).
+ *  - Supported: d in {64, 128}; d = 256 also for the forward with a workspace
+ *    (fa_fwd_ws, fa_attn_fwd) and for every backward (fa_bwd, fa_bwd_gqa, fa_bwd_ws,
+ *    fa_attn_bwd, fa_bwd_noalloc); the 8-bit forward takes d = 128 or 64; a
+ *    B200-class GPU (compute capability 10.0).
  *
  * Thread safety: calls may be issued from several host threads; calls whose
  * work overlaps on the GPU must not share output buffers or a workspace.
