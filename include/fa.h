@@ -143,7 +143,7 @@ FA_API fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o
  * fa_fwd_gqa, except that d may also be 256 (the head dimension FlashAttention-2 added:
  * "FlashAttention (EL)", section "FlashAttention-2 (2023)"): a kernel of its own with one
  * 128-row query tile per work unit, because S and a 256-column O of two tiles do not fit in
- * tensor memory.  The backward takes d in {64, 128} only.
+ * tensor memory.  Every backward entry point takes d = 256 as well.
  */
 FA_API size_t fa_fwd_workspace_size(int B, int H_kv, int N, int d);
 FA_API fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, void* o_resid, int B,
