@@ -397,7 +397,7 @@ def fa_attn_fwd_fp8_workspace_size(problem: FaAttnProblem) -> int:
 def fa_attn_fwd_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float, causal: bool = False,
                     scale: float | None = None, window=(-1, -1), o=None, lse=None, workspace=None, stream=None):
     """8-bit forward: q (B, H, N, d), k and v (B, H_kv, N, d) ``torch.float8_e4m3fn`` CUDA
-    tensors holding Q / q_descale etc. (per-tensor descales, d = 128).  Computes the
+    tensors holding Q / q_descale etc. (per-tensor descales, d = 128 or 64).  Computes the
     attention of the dequantized inputs; returns (o bf16, lse fp32)."""
     pr = _problem(q, k, causal, scale, window)
     B, H, N, d = _shape(q)
