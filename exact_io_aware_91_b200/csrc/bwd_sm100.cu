@@ -980,13 +980,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // At d = 256 the accumulators do not fit next to S^T and dP^T in tensor memory (dV and dK of
 // a 128-key tile take 256 columns each), and the tiles do not fit in shared memory (K, V, Q
 // and dO of 128 rows take 64 KB each).  The two kernels below therefore:
-//   * dK/dV: a work unit is (key/value head, 128-key tile, d-half h, share of the group's
-//     query heads).  It recomputes S^T = K Q^T and dP^T = V dO^T over the full d and
-//     accumulates only dV[:, h] += P^T dO[:, h] and dK[:, h] += dS^T Q[:, h]: TMEM holds S^T,
-//     dP^T, dV_h, dK_h (128 columns each).  K and V stay resident (64 KB each); Q and dO
-//     stream as 128-column halves (32 KB) through a 3-slot FIFO, and the half h of each is
-//     loaded a second time for its gradient product, so the FIFO releases slots in the order
-//     it fills them.
+//   * dK/dV: two kernels, one per gradient, each accumulating it over the full d in 256 TMEM
+//     columns; a work unit is (key/value head, 128-key tile, share of the group's query heads).
+//     The dV kernel computes S^T = K Q^T (double-buffered: two 128-column buffers) and
+//     dV += P^T dO; the dK kernel S^T, dP^T = V dO^T and dK += dS^T Q.  Per (key tile, query
+//     tile) pair that is 5 products of 128 x 128 x 256 (S^T in both kernels) where one unit
+//     accumulating half of both gradients needs 6 (S^T and dP^T once per half).  K (and V in the
+//     dK kernel) stay resident (64 KB each); Q and dO stream as 128-column halves (32 KB)
+//     through a FIFO of 3 slots, 5 in the dV kernel (V's space), in the order the products take
+//     them (the dK kernel loads Q a second time for dK), so the FIFO releases slots in the
+//     order it fills them.
 //   * dQ: Q and dO stay resident; S is single-buffered (S, dP 128 columns, dQ 256); K and V
 //     stream as halves through the same kind of FIFO, K's halves a second time for dQ += dS K.
 // Both are persistent like the d = 128 kernels; every other step (recomputed probabilities,
@@ -1004,28 +1007,33 @@ __device__ __forceinline__ void issue_ss_half(uint32_t d_tmem, uint64_t a_desc, 
   }
 }
 
+// One gradient per kernel: KIND 0 = dV, KIND 1 = dK (units of the other kind run in the other
+// launch).  A dV unit needs K but not V, so its Q / dO ring takes V's 64 KB as two more slots.
+template <int KIND>
 struct DkdvWLayout {
+  static constexpr int SLOTS = KIND == 0 ? 5 : 3;  // FIFO slots of one half each
   static constexpr int OFF_K = 0;                      // K: two halves
-  static constexpr int OFF_V = 2 * kHalf;              // V: two halves
-  static constexpr int OFF_RING = 4 * kHalf;           // kWSlots halves of Q or dO
-  static constexpr int OFF_LD = OFF_RING + kWSlots * kHalf;  // two (lse2[128], delta[128]) pairs, 1 KB each
+  static constexpr int OFF_V = 2 * kHalf;              // V: two halves (dK), ring slots 3-4 (dV)
+  static constexpr int OFF_RING = 4 * kHalf;           // ring slots 0-2
+  static constexpr int OFF_LD = OFF_RING + 3 * kHalf;  // two (lse2[128], delta[128]) pairs, 1 KB each
   static constexpr int OFF_BAR = OFF_LD + 2048;
-  static constexpr int BAR_KV = 0;          // a unit's K, V landed
+  static constexpr int BAR_KV = 0;          // a unit's K (and V) landed
   static constexpr int BAR_KV_EMPTY = 1;    // the MMAs reading a unit's K and V have completed
-  static constexpr int BAR_SLOT_FULL = 2;   // [kWSlots]
-  static constexpr int BAR_SLOT_EMPTY = 5;  // [kWSlots]
-  static constexpr int BAR_LD_EMPTY = 8;    // [2] the step whose LSE / D a buffer holds is finished
-  static constexpr int BAR_S = 10;
-  static constexpr int BAR_DP = 11;
-  static constexpr int BAR_P_READY = 12;
-  static constexpr int BAR_P_HALF = 13;
-  static constexpr int BAR_DS_READY = 14;
-  static constexpr int BAR_ACC = 15;
-  static constexpr int BAR_ACC_FREE = 16;
-  static constexpr int BAR_UNIT_FULL = 17;   // [2]
-  static constexpr int BAR_UNIT_EMPTY = 19;  // [2]
-  static constexpr int BAR_DONE = 21;
-  static constexpr int NBAR = 22;
+  static constexpr int BAR_SLOT_FULL = 2;                  // [SLOTS]
+  static constexpr int BAR_SLOT_EMPTY = 2 + SLOTS;         // [SLOTS]
+  static constexpr int BAR_LD_EMPTY = 2 + 2 * SLOTS;       // [2] the step whose LSE / D a buffer holds is finished
+  static constexpr int BAR_S = BAR_LD_EMPTY + 2;           // [2] S^T of a step complete in buffer b (dV: two buffers)
+  static constexpr int BAR_DP = BAR_S + 2;                 // dP^T complete (dK)
+  static constexpr int BAR_S_LOADED = BAR_DP + 1;          // the compute warps hold S^T in registers (dK)
+  static constexpr int BAR_P_HALF = BAR_S_LOADED + 1;      // [2] the first half of P^T is in buffer b (dV)
+  static constexpr int BAR_P_READY = BAR_P_HALF + 2;       // [2] all of P^T is in buffer b (dV)
+  static constexpr int BAR_DS_READY = BAR_P_READY + 2;     // dS^T is in TMEM over dP^T (dK)
+  static constexpr int BAR_ACC = BAR_DS_READY + 1;
+  static constexpr int BAR_ACC_FREE = BAR_ACC + 1;
+  static constexpr int BAR_UNIT_FULL = BAR_ACC_FREE + 1;   // [2]
+  static constexpr int BAR_UNIT_EMPTY = BAR_UNIT_FULL + 2; // [2]
+  static constexpr int BAR_DONE = BAR_UNIT_EMPTY + 2;
+  static constexpr int NBAR = BAR_DONE + 1;
   static constexpr int OFF_UNIT = OFF_BAR + NBAR * 8;  // int[2]
   static constexpr int OFF_TMEM_SLOT = OFF_UNIT + 8;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
@@ -1034,17 +1042,25 @@ struct DkdvWLayout {
   // rounding fits (it does for a 1024-aligned start, which the declaration asks for)
   static constexpr int SMEM_ALLOC = BYTES + 1024 <= kSmemMax ? BYTES + 1024 : kSmemMax;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
+  // dV: S^T buffers at 0 and 128; dK: S^T at 0, dP^T at 128; the gradient (256 columns) at 256
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_ACC = 256;
+  // byte offset of ring slot st from the shared-memory base
+  __device__ static uint32_t slot_off(int st) {
+    return (KIND == 0 && st >= 3) ? (uint32_t)(OFF_V + (st - 3) * kHalf) : (uint32_t)(OFF_RING + st * kHalf);
+  }
 };
-static_assert(DkdvWLayout::BYTES <= kSmemMax, "d = 256 dK/dV kernel exceeds the shared memory of a CTA");
+static_assert(DkdvWLayout<0>::BYTES <= kSmemMax && DkdvWLayout<1>::BYTES <= kSmemMax,
+              "d = 256 dK/dV kernels exceed the shared memory of a CTA");
 
 
+template <int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_dkdv_d256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                             const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                             const BwdParams p) {
-  using L = DkdvWLayout;
+  using L = DkdvWLayout<KIND>;
   constexpr int D = 256;
+  constexpr int SL = L::SLOTS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -1057,24 +1073,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_ABORT);
   const WaitCtx wctx{abort_flag, p.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (p.v_exp_fwd != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.v_exp_fwd = p.exps[kExpV];  // as above
+  if (KIND == 1 && p.v_exp_fwd != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
+    *p.v_exp_fwd = p.exps[kExpV];  // as above
 
   const int n_kt = (p.N + 127) / 128;
   const int BH_kv = p.BH / p.H * p.H_kv;
-  const int per_head = n_kt * 2 * p.kv_split;  // (key tile, d-half, split) per key/value head
+  const int per_head = n_kt * p.kv_split;  // (key tile, split) per key/value head
   const int n_units = per_head * BH_kv;
   const int g_per = p.H / p.H_kv / p.kv_split;
   struct Unit {
-    int bh, j, h, sp, i_start, n_q, n_it;
+    int bh, j, sp, i_start, n_q, n_it;
   };
   auto unit_of = [&](int u) -> Unit {
     Unit x;
     int rank;
     unit_order(u, per_head, BH_kv, p.head_group_kv, x.bh, rank);
-    x.j = rank / (2 * p.kv_split);  // heaviest (first) key tiles first
-    const int rem = rank % (2 * p.kv_split);
-    x.h = rem / p.kv_split;
-    x.sp = rem % p.kv_split;
+    x.j = rank / p.kv_split;  // heaviest (first) key tiles first
+    x.sp = rank % p.kv_split;
     x.i_start = query_lo(x.j * 128, p.causal, p.win_right) / 128;
     x.n_q = query_hi(min(x.j * 128 + 127, p.N - 1), p.N, p.win_left) / 128 - x.i_start + 1;
     x.n_it = g_per * x.n_q;
@@ -1091,19 +1106,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     mbar_init(bar(L::BAR_KV), 1);
     mbar_init(bar(L::BAR_KV_EMPTY), 1);
-    for (int s = 0; s < kWSlots; ++s) {
+    for (int s = 0; s < SL; ++s) {
       mbar_init(bar(L::BAR_SLOT_FULL + s), 1);
       mbar_init(bar(L::BAR_SLOT_EMPTY + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(L::BAR_LD_EMPTY + s), 1);
+      mbar_init(bar(L::BAR_S + s), 1);
+      mbar_init(bar(L::BAR_P_HALF + s), 256);
+      mbar_init(bar(L::BAR_P_READY + s), 256);
       mbar_init(bar(L::BAR_UNIT_FULL + s), 1);
       mbar_init(bar(L::BAR_UNIT_EMPTY + s), 1 + 256);
     }
-    mbar_init(bar(L::BAR_S), 1);
     mbar_init(bar(L::BAR_DP), 1);
-    mbar_init(bar(L::BAR_P_READY), 256);
-    mbar_init(bar(L::BAR_P_HALF), 256);
+    mbar_init(bar(L::BAR_S_LOADED), 256);
     mbar_init(bar(L::BAR_DS_READY), 256);
     mbar_init(bar(L::BAR_ACC), 1);
     mbar_init(bar(L::BAR_ACC_FREE), 256);
@@ -1119,10 +1135,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::OFF_TMEM_SLOT);
 
-  // The FIFO order of a unit with n steps (step t: query tile and head of `it`), which the
-  // producer fills and the MMA warp drains:  Q0(0) Q1(0) dO0(0) dO1(0), then for it = 0..n-1:
-  // dOh(it), [Q0(it+1) Q1(it+1)], Qh(it), [dO0(it+1) dO1(it+1)]  (bracketed parts while
-  // it + 1 < n; Xk = half k of X, h = the unit's half).
+  // The FIFO order of a unit with n steps (Xk(t) = half k of X for step t), which the producer
+  // fills and the MMA warp drains:
+  //   dV: Q0(0) Q1(0) [Q0(1) Q1(1)], then for it = 0..n-1: dO0(it) dO1(it) [Q0(it+2) Q1(it+2)]
+  //   dK: Q0(0) Q1(0) dO0(0) dO1(0), then for it = 0..n-1:
+  //       [Q0(it+1) Q1(it+1)] Q0(it) Q1(it) [dO0(it+1) dO1(it+1)]
+  // (bracketed parts only while those steps exist).  The dK products take Q(it) one half at a
+  // time, so each product holds at most one slot and the loads run ahead of the products.
   if (warp == 0) {
     // ===================================================== TMA producer + work distribution
     regs_dec<kRegsLow>();
@@ -1130,7 +1149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_do);
     prefetch_tmap(&tm_k);
-    prefetch_tmap(&tm_v);
+    if (KIND == 1) prefetch_tmap(&tm_v);
     int F = 0;  // halves put in the FIFO so far (all units)
     int T = 0;  // steps of the previous units
     int kv_issued = 0;
@@ -1138,8 +1157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // half `half` of Q (which = 0) or dO (which = 1) for the unit step `it`; with_ld: also the
     // step's LSE * log2(e) and D rows (global step t) into their buffer
     auto load_half = [&](const Unit& x, int which, int half, int it, bool with_ld) -> bool {
-      const int st = F % kWSlots;
-      if (!mbar_wait(bar(L::BAR_SLOT_EMPTY + st), ((F / kWSlots) & 1) ^ 1u, wctx)) return false;
+      const int st = F % SL;
+      if (!mbar_wait(bar(L::BAR_SLOT_EMPTY + st), ((F / SL) & 1) ^ 1u, wctx)) return false;
       const int t = T + it;
       const int i = x.i_start + it % x.n_q;
       const int bhq = q_head_of(x.bh, x.sp * g_per + it / x.n_q, p.H, p.H_kv);
@@ -1147,7 +1166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t fb = bar(L::BAR_SLOT_FULL + st);
       mbar_arrive_expect_tx(fb, kHalf + (with_ld ? 1024 : 0), leader);
       const CUtensorMap* m = which ? &tm_do : &tm_q;
-      const uint32_t dst = base + L::OFF_RING + st * kHalf;
+      const uint32_t dst = base + L::slot_off(st);
       for (int b = 0; b < 2; ++b) tma_load_3d(dst + b * kBox, m, half * 128 + b * 64, i * 128, bhq, fb, leader);
       if (with_ld) {
         const size_t roff = (size_t)bhq * p.Np + (size_t)i * 128;
@@ -1157,10 +1176,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++F;
       return true;
     };
+    auto load_both = [&](const Unit& x, int which, int it) -> bool {  // both halves; Q's first carries LSE / D
+      return load_half(x, which, 0, it, which == 0) && load_half(x, which, 1, it, false);
+    };
     for (int uc = 0;; ++uc) {
       if (uc >= 2 && !(ok = mbar_wait(bar(L::BAR_UNIT_EMPTY + (uc & 1)), ((uc - 2) >> 1) & 1, wctx))) break;
       int u = 0;
-      if (lane == 0) u = (int)atomicAdd(p.dkdv_counter, 1u);
+      if (lane == 0) u = (int)atomicAdd(KIND == 0 ? p.dkdv_counter : p.dk_counter, 1u);
       u = __shfl_sync(0xffffffffu, u, 0);
       if (lane == 0) {
         unit_ring[uc & 1] = u < n_units ? u : n_units;
@@ -1170,29 +1192,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (u >= n_units) break;
       const Unit x = unit_of(u);
       if (uc > 0 && !(ok = mbar_wait(bar(L::BAR_KV_EMPTY), (uc - 1) & 1, wctx))) break;
-      mbar_arrive_expect_tx(bar(L::BAR_KV), 4 * kHalf, leader);
+      mbar_arrive_expect_tx(bar(L::BAR_KV), (KIND == 1 ? 4 : 2) * kHalf, leader);
       for (int c = 0; c < 4; ++c) {
         const uint32_t off = (c >> 1) * kHalf + (c & 1) * kBox;
         tma_load_3d(base + L::OFF_K + off, &tm_k, c * 64, x.j * 128, x.bh, bar(L::BAR_KV), leader);
-        tma_load_3d(base + L::OFF_V + off, &tm_v, c * 64, x.j * 128, x.bh, bar(L::BAR_KV), leader);
+        if (KIND == 1) tma_load_3d(base + L::OFF_V + off, &tm_v, c * 64, x.j * 128, x.bh, bar(L::BAR_KV), leader);
       }
       ++kv_issued;
       const int n = x.n_it;
-      ok = load_half(x, 0, 0, 0, true) && load_half(x, 0, 1, 0, false) && load_half(x, 1, 0, 0, false) &&
-           load_half(x, 1, 1, 0, false);
-      for (int it = 0; it < n && ok; ++it) {
-        ok = load_half(x, 1, x.h, it, false);  // dO half h for dV(it)
-        if (ok && it + 1 < n) ok = load_half(x, 0, 0, it + 1, true) && load_half(x, 0, 1, it + 1, false);
-        if (ok) ok = load_half(x, 0, x.h, it, false);  // Q half h for dK(it)
-        if (ok && it + 1 < n) ok = load_half(x, 1, 0, it + 1, false) && load_half(x, 1, 1, it + 1, false);
+      if (KIND == 0) {
+        ok = load_both(x, 0, 0) && (n < 2 || load_both(x, 0, 1));
+        for (int it = 0; it < n && ok; ++it) ok = load_both(x, 1, it) && (it + 2 >= n || load_both(x, 0, it + 2));
+      } else {
+        ok = load_both(x, 0, 0) && load_both(x, 1, 0);
+        for (int it = 0; it < n && ok; ++it)
+          ok = (it + 1 >= n || load_both(x, 0, it + 1)) && load_half(x, 0, 0, it, false) &&
+               load_half(x, 0, 1, it, false) && (it + 1 >= n || load_both(x, 1, it + 1));
       }
       if (!ok) break;
       T += n;
     }
     // drain: every issued copy has landed before the CTA may exit
     if (kv_issued > 0) drain_wait(bar(L::BAR_KV), (kv_issued - 1) & 1);
-    for (int f = (F > kWSlots ? F - kWSlots : 0); f < F; ++f)
-      drain_wait(bar(L::BAR_SLOT_FULL + f % kWSlots), (f / kWSlots) & 1);
+    for (int f = (F > SL ? F - SL : 0); f < F; ++f) drain_wait(bar(L::BAR_SLOT_FULL + f % SL), (f / SL) & 1);
   } else if (warp == 1) {
     // ===================================================== MMA issuer
     regs_dec<kRegsLow>();
@@ -1203,13 +1225,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                              make_sdesc_sw128(base + L::OFF_K + kHalf, 16, 1024)};
     const uint64_t dVs[2] = {make_sdesc_sw128(base + L::OFF_V, 16, 1024),
                              make_sdesc_sw128(base + L::OFF_V + kHalf, 16, 1024)};
-    const uint64_t dRingK = make_sdesc_sw128(base + L::OFF_RING, 16, 1024);     // a half as K-major B
-    const uint64_t dRingMN = make_sdesc_sw128(base + L::OFF_RING, kBox, 1024);  // a half as MN-major B
     int C = 0;  // halves taken from the FIFO so far
     bool ok = true;
     auto take = [&]() -> int {
-      const int st = C % kWSlots;
-      ok = mbar_wait(bar(L::BAR_SLOT_FULL + st), (C / kWSlots) & 1, wctx);
+      const int st = C % SL;
+      ok = mbar_wait(bar(L::BAR_SLOT_FULL + st), (C / SL) & 1, wctx);
       ++C;
       if (ok) tc_fence_after();
       return st;
@@ -1219,13 +1239,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int hh = 0; hh < 2; ++hh) {
         const int st = take();
         if (!ok) return false;
-        issue_ss_half(d_tmem, a[hh], sdesc_add(dRingK, st * kHalf), idesc_s, hh == 0, leader);
+        issue_ss_half(d_tmem, a[hh], make_sdesc_sw128(base + L::slot_off(st), 16, 1024), idesc_s, hh == 0, leader);
         mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
       }
       mma_commit(done_bar, leader);
       return true;
     };
+    // a slot's half as the MN-major B operand of a gradient product
+    auto mn_desc = [&](int st) -> uint64_t { return make_sdesc_sw128(base + L::slot_off(st), kBox, 1024); };
     int T0 = 0;
+    int nP[2] = {0, 0};    // dV: steps that used S^T buffer b so far (P_HALF / P_READY phases)
+    int nSL = 0, nDS = 0;  // dK: S_LOADED and DS_READY phases so far
     for (int uc = 0; ok; ++uc) {
       const int u = next_unit(uc, ok);
       if (lane == 0) mbar_arrive(bar(L::BAR_UNIT_EMPTY + (uc & 1)));
@@ -1233,40 +1257,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = unit_of(u).n_it;
       if (!(ok = mbar_wait(bar(L::BAR_KV), uc & 1, wctx))) break;
       tc_fence_after();
-      if (!(ok = issue_full(tmem + L::T_S, dKs, bar(L::BAR_S)))) break;
-      if (!(ok = issue_full(tmem + L::T_DP, dVs, bar(L::BAR_DP)))) break;
-      if (n == 1) mma_commit(bar(L::BAR_KV_EMPTY), leader);
-      for (int it = 0; it < n && ok; ++it) {
-        const int t = T0 + it;
-        // dV_h += P^T dO_h in two halves (the first while the second half of P^T is computed);
-        // the unit's first product overwrites the accumulators, which the previous unit's
-        // epilogue must have read
-        int st = take();
-        if (!ok) break;
-        if (!(ok = mbar_wait(bar(L::BAR_P_HALF), t & 1, wctx))) break;
+      // the unit's first product into the accumulator overwrites it: the previous unit's
+      // epilogue must have read it
+      auto acc_free = [&](int it) -> bool {
+        if (it > 0 || uc == 0) return true;
+        if (!mbar_wait(bar(L::BAR_ACC_FREE), (uc - 1) & 1, wctx)) return false;
         tc_fence_after();
-        if (it == 0 && uc > 0) {
-          if (!(ok = mbar_wait(bar(L::BAR_ACC_FREE), (uc - 1) & 1, wctx))) break;
+        return true;
+      };
+      if constexpr (KIND == 0) {
+        // ---- dV: S^T double-buffered, dV (256 columns) += P^T dO in two d-halves
+        if (!(ok = issue_full(tmem + L::T_S, dKs, bar(L::BAR_S)))) break;
+        if (n > 1 && !(ok = issue_full(tmem + L::T_S + 128, dKs, bar(L::BAR_S + 1)))) break;
+        if (n <= 2) mma_commit(bar(L::BAR_KV_EMPTY), leader);  // the unit's last S^T issued
+        for (int it = 0; it < n && ok; ++it) {
+          const int t = T0 + it, b = it & 1;
+          const uint32_t tP = tmem + L::T_S + 128 * b;
+          const int st0 = take();
+          if (!ok) break;
+          const int st1 = take();
+          if (!ok) break;
+          if (!(ok = mbar_wait(bar(L::BAR_P_HALF + b), nP[b] & 1, wctx))) break;
           tc_fence_after();
+          if (!(ok = acc_free(it))) break;
+          // the first half of P^T (query columns {0..31, 64..95}) while the second is computed
+          issue_ts_split_part(tmem + L::T_ACC, tP, mn_desc(st0), idesc_g, it == 0, 0, leader);
+          issue_ts_split_part(tmem + L::T_ACC + 128, tP, mn_desc(st1), idesc_g, it == 0, 0, leader);
+          if (!(ok = mbar_wait(bar(L::BAR_P_READY + b), nP[b] & 1, wctx))) break;
+          tc_fence_after();
+          ++nP[b];
+          issue_ts_split_part(tmem + L::T_ACC, tP, mn_desc(st0), idesc_g, false, 1, leader);
+          issue_ts_split_part(tmem + L::T_ACC + 128, tP, mn_desc(st1), idesc_g, false, 1, leader);
+          mma_commit(bar(L::BAR_SLOT_EMPTY + st0), leader);
+          mma_commit(bar(L::BAR_SLOT_EMPTY + st1), leader);
+          mma_commit(bar(L::BAR_LD_EMPTY + (t & 1)), leader);  // step t's LSE / D buffer is free after this
+          if (it + 2 < n) {  // S^T(it + 2) into this step's buffer, after the products reading its P^T
+            if (!(ok = issue_full(tP, dKs, bar(L::BAR_S + b)))) break;
+            if (it + 3 == n) mma_commit(bar(L::BAR_KV_EMPTY), leader);
+          }
         }
-        const uint64_t dmn = sdesc_add(dRingMN, st * kHalf);
-        issue_ts_split_part(tmem + L::T_DV, tmem + L::T_S, dmn, idesc_g, it == 0, 0, leader);
-        if (!(ok = mbar_wait(bar(L::BAR_P_READY), t & 1, wctx))) break;
-        tc_fence_after();
-        issue_ts_split_part(tmem + L::T_DV, tmem + L::T_S, dmn, idesc_g, false, 1, leader);
-        mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
-        if (it + 1 < n && !(ok = issue_full(tmem + L::T_S, dKs, bar(L::BAR_S)))) break;  // S^T(it + 1)
-        st = take();
-        if (!ok) break;
-        if (!(ok = mbar_wait(bar(L::BAR_DS_READY), t & 1, wctx))) break;
-        tc_fence_after();
-        issue_ts_split(tmem + L::T_DK, tmem + L::T_DP, sdesc_add(dRingMN, st * kHalf), idesc_g, it > 0,
-                       leader);  // dK_h += dS^T Q_h
-        mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
-        mma_commit(bar(L::BAR_LD_EMPTY + (t & 1)), leader);  // step t's LSE / D buffer is free after this
-        if (it + 1 < n) {
-          if (!(ok = issue_full(tmem + L::T_DP, dVs, bar(L::BAR_DP)))) break;  // dP^T(it + 1)
-          if (it + 2 == n) mma_commit(bar(L::BAR_KV_EMPTY), leader);  // the unit's last S^T, dP^T issued
+      } else {
+        // ---- dK: S^T, dP^T; dK (256 columns) += dS^T Q in two d-halves, one Q half at a time
+        if (!(ok = issue_full(tmem + L::T_S, dKs, bar(L::BAR_S)))) break;
+        if (!(ok = issue_full(tmem + L::T_DP, dVs, bar(L::BAR_DP)))) break;
+        if (n == 1) mma_commit(bar(L::BAR_KV_EMPTY), leader);
+        for (int it = 0; it < n && ok; ++it) {
+          const int t = T0 + it;
+          if (it + 1 < n) {  // S^T(it + 1) once the compute warps hold S^T(it) in registers
+            if (!(ok = mbar_wait(bar(L::BAR_S_LOADED), nSL & 1, wctx))) break;
+            tc_fence_after();
+            ++nSL;
+            if (!(ok = issue_full(tmem + L::T_S, dKs, bar(L::BAR_S)))) break;
+          }
+          if (!(ok = mbar_wait(bar(L::BAR_DS_READY), nDS & 1, wctx))) break;
+          tc_fence_after();
+          ++nDS;
+          if (!(ok = acc_free(it))) break;
+          for (int hh = 0; hh < 2; ++hh) {
+            const int st = take();
+            if (!ok) break;
+            issue_ts_split(tmem + L::T_ACC + 128 * hh, tmem + L::T_DP, mn_desc(st), idesc_g, it > 0, leader);
+            mma_commit(bar(L::BAR_SLOT_EMPTY + st), leader);
+          }
+          if (!ok) break;
+          mma_commit(bar(L::BAR_LD_EMPTY + (t & 1)), leader);
+          if (it + 1 < n) {  // dP^T(it + 1) after the products reading dS^T(it)
+            if (!(ok = issue_full(tmem + L::T_DP, dVs, bar(L::BAR_DP)))) break;
+            if (it + 2 == n) mma_commit(bar(L::BAR_KV_EMPTY), leader);  // the unit's last S^T, dP^T issued
+          }
         }
       }
       if (!ok) break;
@@ -1284,12 +1342,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = (warp - 4) & 3;
     const int row = wq * 32 + lane;  // key row inside the tile
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + L::T_S + 64 * w;
     const uint32_t tDP = tmem + lane_off + L::T_DP + 64 * w;
     const float sl2 = ldexpf(p.scale_log2, -(p.exps[kExpQ] + p.exps[kExpK]));
     const uint64_t sl2x2 = f2pack(sl2, sl2);
     bool ok = true;
     int T0 = 0;
+    int nS[2] = {0, 0}, nDP = 0;  // completions of S^T buffer b and of dP^T waited for so far
     int u = next_unit(0, ok);
     mbar_arrive(bar(L::BAR_UNIT_EMPTY + 0));
     for (int uc = 0; ok && u < n_units; ++uc) {
@@ -1306,10 +1364,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* lse2 = reinterpret_cast<const float*>(gbase + L::OFF_LD + (T & 1) * 1024) + 64 * w;
         const float* delta = lse2 + 128;
         const int q0 = i * 128 + 64 * w;
-        if (!(ok = mbar_wait(bar(L::BAR_S), T & 1, wctx))) break;
+        const int b = KIND == 1 ? 0 : (it & 1);  // S^T buffer of this step
+        const uint32_t tS = tmem + lane_off + L::T_S + 128 * b + 64 * w;
+        if (!(ok = mbar_wait(bar(L::BAR_S + b), nS[b] & 1, wctx))) break;
         tc_fence_after();
+        ++nS[b];
         float pr[64];
         tmem_ld64(tS, pr);
+        if (KIND == 1 && it + 1 < n_it) {  // S^T is in registers: the next S^T may overwrite it
+          tc_fence_before();
+          mbar_arrive(bar(L::BAR_S_LOADED));
+        }
+        // P^T = 2^(S^T scale log2(e) - LSE log2(e)); for dV written to TMEM over S^T as fp16 in
+        // two halves (the first announced on P_HALF), for dK kept in registers
         auto probs = [&](auto masked) {
           const int c_lo = q_vis_lo - q0, c_hi = q_vis_hi - q0;
 #pragma unroll
@@ -1339,14 +1406,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 4; ++e)
                   if (c + e < c_lo || c + e > c_hi) pr[c + e] = 0.f;
               }
-              pk[(c - g) / 2] = pack_f16(pr[c], pr[c + 1]);
-              pk[(c - g) / 2 + 1] = pack_f16(pr[c + 2], pr[c + 3]);
+              if constexpr (KIND == 0) {
+                pk[(c - g) / 2] = pack_f16(pr[c], pr[c + 1]);
+                pk[(c - g) / 2 + 1] = pack_f16(pr[c + 2], pr[c + 3]);
+              }
             }
-            tmem_st8(tS + g / 2, pk);
-            if (g == 16) {
-              tmem_wait_st();
-              tc_fence_before();
-              mbar_arrive(bar(L::BAR_P_HALF));
+            if constexpr (KIND == 0) {
+              tmem_st8(tS + g / 2, pk);
+              if (g == 16) {
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(L::BAR_P_HALF + b));
+              }
             }
           }
         };
@@ -1354,41 +1425,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           probs(std::true_type{});
         else
           probs(std::false_type{});
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(L::BAR_P_READY));
-        if (!(ok = mbar_wait(bar(L::BAR_DP), T & 1, wctx))) break;
-        tc_fence_after();
-        float dp[64];
-        tmem_ld64(tDP, dp);
+        if constexpr (KIND == 0) {
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(L::BAR_P_READY + b));
+        } else {
+          if (!(ok = mbar_wait(bar(L::BAR_DP), nDP & 1, wctx))) break;
+          tc_fence_after();
+          ++nDP;
+          float dp[64];
+          tmem_ld64(tDP, dp);
 #pragma unroll
-        for (int g = 0; g < 64; g += 16) {
-          uint32_t pk[8];
+          for (int g = 0; g < 64; g += 16) {
+            uint32_t pk[8];
 #pragma unroll
-          for (int c = g; c < g + 16; c += 4) {
-            const float4 D4 = *reinterpret_cast<const float4*>(delta + c);
-            float d0, d1, d2, d3;
-            f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(f2pack(dp[c], dp[c + 1]), f2pack(D4.x, D4.y))), d0, d1);
-            f2unpack(fmul2(f2pack(pr[c + 2], pr[c + 3]), fsub2(f2pack(dp[c + 2], dp[c + 3]), f2pack(D4.z, D4.w))), d2,
-                     d3);
-            pk[(c - g) / 2] = pack_f16(d0, d1);
-            pk[(c - g) / 2 + 1] = pack_f16(d2, d3);
+            for (int c = g; c < g + 16; c += 4) {
+              const float4 D4 = *reinterpret_cast<const float4*>(delta + c);
+              float d0, d1, d2, d3;
+              f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(f2pack(dp[c], dp[c + 1]), f2pack(D4.x, D4.y))), d0, d1);
+              f2unpack(fmul2(f2pack(pr[c + 2], pr[c + 3]), fsub2(f2pack(dp[c + 2], dp[c + 3]), f2pack(D4.z, D4.w))),
+                       d2, d3);
+              pk[(c - g) / 2] = pack_f16(d0, d1);
+              pk[(c - g) / 2 + 1] = pack_f16(d2, d3);
+            }
+            tmem_st8(tDP + g / 2, pk);
           }
-          tmem_st8(tDP + g / 2, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(L::BAR_DS_READY));
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(L::BAR_DS_READY));
       }
       if (!ok) break;
       if (!(ok = mbar_wait(bar(L::BAR_ACC), uc & 1, wctx))) break;
       tc_fence_after();
-      // warpgroup 0 writes dV[:, h], warpgroup 1 scale * dK[:, h] (128 columns each)
+      // warpgroup w writes columns [128 w, 128 w + 128) of the kernel's gradient: dV, or scale * dK
       const size_t head_off = p.kv_split == 1 ? (size_t)x.bh * p.N * D : ((size_t)x.sp * BH_kv + x.bh) * p.N * D;
-      float* out = (p.kv_split == 1 ? (w == 0 ? p.dv : p.dk) : (w == 0 ? p.dv_part : p.dk_part)) + head_off +
-                   128 * x.h;
-      const uint32_t t_acc = tmem + lane_off + (w == 0 ? L::T_DV : L::T_DK);
-      const Pow2 out_f = pow2_factors(w == 0 ? -p.exps[kExpDO] : -(p.exps[kExpV] + p.exps[kExpDO] + p.exps[kExpQ]));
+      float* out = (p.kv_split == 1 ? (KIND == 1 ? p.dk : p.dv) : (KIND == 1 ? p.dk_part : p.dv_part)) + head_off +
+                   128 * w;
+      const uint32_t t_acc = tmem + lane_off + L::T_ACC + 128 * w;
+      const Pow2 out_f =
+          pow2_factors(KIND == 1 ? -(p.exps[kExpV] + p.exps[kExpDO] + p.exps[kExpQ]) : -p.exps[kExpDO]);
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         float acc[64];
@@ -1397,7 +1473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(bar(L::BAR_ACC_FREE));
         }
-        warp_store_rows_f32<64>(acc, out + 64 * c, D, j * 128 + wq * 32, p.N, w == 0 ? 1.0f : p.scale, out_f);
+        warp_store_rows_f32<64>(acc, out + 64 * c, D, j * 128 + wq * 32, p.N, KIND == 1 ? p.scale : 1.0f, out_f);
       }
       T0 += n_it;
       u = next_unit(uc + 1, ok);
@@ -1796,12 +1872,15 @@ cudaError_t launch_dkdv_t(dim3 grid, const CUtensorMap& tq, const CUtensorMap& t
 cudaError_t launch_bwd_dkdv_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                                   const CUtensorMap& tv, const CUtensorMap& tdv, const CUtensorMap& tdk,
                                   const BwdParams& p, int d, cudaStream_t s) {
-  // persistent: one CTA per SM (at most one per unit: key tile x key/value head x group split,
-  // and x the d-half at d = 256)
-  const long long units =
-      (long long)((p.N + 127) / 128) * (p.BH / p.H * p.H_kv) * p.kv_split * (d == 256 ? 2 : 1);
+  // persistent: one CTA per SM (at most one per unit: key tile x key/value head x group split;
+  // at d = 256 the same units in each of the two kernels)
+  const long long units = (long long)((p.N + 127) / 128) * (p.BH / p.H * p.H_kv) * p.kv_split;
   const dim3 grid((unsigned)(units < p.num_sms ? units : p.num_sms));
-  if (d == 256) return launch_one<DkdvWLayout>(fa_bwd_dkdv_d256_kernel, grid, tq, tdo, tk, tv, p, s);
+  if (d == 256) {  // the dV kernel, then the dK kernel
+    const cudaError_t e = launch_one<DkdvWLayout<0>>(fa_bwd_dkdv_d256_kernel<0>, grid, tq, tdo, tk, tv, p, s);
+    if (e != cudaSuccess) return e;
+    return launch_one<DkdvWLayout<1>>(fa_bwd_dkdv_d256_kernel<1>, grid, tq, tdo, tk, tv, p, s);
+  }
   if (d == 128) return launch_dkdv_t<128>(grid, tq, tdo, tk, tv, tdv, tdk, p, s);
   return launch_dkdv_t<64>(grid, tq, tdo, tk, tv, tdv, tdk, p, s);
 }

@@ -123,8 +123,8 @@ constexpr size_t kCtrlCounters = 0, kCtrlExps = 16;
 constexpr long long kDkdvMinUnits = 4 * 148;
 int kv_split_for(int B, int H, int H_kv, int N, int d) {
   const int group = H / H_kv;
-  // at d = 256 every key tile is two units (one per d-half of dK, dV)
-  const long long units = (long long)B * H_kv * ((N + 127) / 128) * (d == 256 ? 2 : 1);
+  (void)d;  // one unit per key tile (at d = 256 in each of the two dK/dV kernels)
+  const long long units = (long long)B * H_kv * ((N + 127) / 128);
   for (int s = 1; s < group; ++s)
     if (group % s == 0 && units * s >= kDkdvMinUnits) return s;
   return group;
@@ -464,6 +464,7 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   bp.num_sms = g_num_sms[dev];
   bp.dq_counter = pp.counters;
   bp.dkdv_counter = pp.counters + 1;
+  bp.dk_counter = pp.counters + 2;
   bp.dk_part = w.kv_split > 1 ? reinterpret_cast<float*>(ws + w.off_dk_part) : nullptr;
   bp.dv_part = w.kv_split > 1 ? reinterpret_cast<float*>(ws + w.off_dv_part) : nullptr;
   bp.scale = scale;

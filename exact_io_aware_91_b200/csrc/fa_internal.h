@@ -47,7 +47,7 @@ __host__ __device__ __forceinline__ int query_hi(int k, int N, int wl) {
   return (wl >= 0 && k + wl < N - 1) ? k + wl : N - 1;
 }
 
-constexpr int kNumCounters = 2;  // work counters: [0] dQ kernel, [1] dK/dV kernel
+constexpr int kNumCounters = 3;  // work counters: [0] dQ kernel, [1] dK/dV (d = 256: dV) kernel, [2] d = 256 dK kernel
 
 // Streaming passes that make fp16 copies (the forward's V pass, the backward preprocess)
 // run on a fixed grid and leave one partial maximum |x| per block and tensor (float bits);
@@ -110,7 +110,8 @@ struct BwdParams {
   float* dv_part;      //   summed into dk / dv by launch_bwd_kv_reduce; unused when kv_split == 1
   int num_sms;         // multiprocessors of the device (grid of the persistent kernels)
   unsigned* dq_counter;  // work units handed out so far by the persistent dQ kernel (zeroed by the preprocess)
-  unsigned* dkdv_counter;  // the same for the persistent dK/dV kernel
+  unsigned* dkdv_counter;  // the same for the persistent dK/dV kernel (d = 256: the dV kernel)
+  unsigned* dk_counter;    // the same for the d = 256 dK kernel
   float scale;         // softmax scale (applied to dQ and dK)
   float scale_log2;    // scale * log2(e)
   int causal;
