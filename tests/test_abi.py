@@ -62,7 +62,8 @@ def _ws_expected_gqa(B, H, Hkv, N, d):
     a = lambda x: (x + 255) // 256 * 256  # noqa: E731
     Np = (N + 127) // 128 * 128
     # few key/value tiles: the group's query heads are split over CTAs with fp32 partial dK, dV
-    group, units = H // Hkv, B * Hkv * ((N + 127) // 128) * (2 if d == 256 else 1)
+    # (one unit per key tile; at d = 256 the dV and dK kernels each have that many)
+    group, units = H // Hkv, B * Hkv * ((N + 127) // 128)
     split = next((s for s in range(1, group) if group % s == 0 and units * s >= 4 * 148), group)
     part = 2 * a(split * B * Hkv * N * d * 4) if split > 1 else 0
     return (2 * a(B * H * N * d * 2) + 2 * a(B * Hkv * N * d * 2) + 2 * a(B * H * Np * 4) + part + 256 +
@@ -70,7 +71,7 @@ def _ws_expected_gqa(B, H, Hkv, N, d):
 
 
 @pytest.mark.parametrize("shape", [(1, 4, 1, 1, 64), (2, 32, 8, 8192, 128), (1, 8, 1, 131072, 128),
-                                   (3, 6, 3, 1000, 64), (2, 16, 16, 2048, 128)])
+                                   (3, 6, 3, 1000, 64), (2, 16, 16, 2048, 128), (1, 8, 2, 9472, 256)])
 def test_gqa_workspace_size(lib, shape):
     B, H, Hkv, N, d = shape
     assert api.fa_bwd_gqa_workspace_size(*shape) == _ws_expected_gqa(*shape)
@@ -267,7 +268,7 @@ def test_head_dim_256_is_a_forward_with_workspace(lib):
         _align256(4 * VPASS_BLOCKS)
     pr = api.FaAttnProblem(1, 4, 2, 300, 256, 0.0625, 1, -1, -1)
     assert api.fa_attn_fwd_workspace_size(pr) == api.fa_fwd_workspace_size(1, 2, 300, 256)
-    # the backward takes d = 256 (dK/dV per d-half: twice the key-tile units for the split rule)
+    # the backward takes d = 256 (one kernel per gradient, each with one unit per key tile)
     assert api.fa_bwd_workspace_size(1, 2, 300, 256) == _ws_expected(1, 2, 300, 256)
     assert api.fa_bwd_gqa_workspace_size(1, 4, 2, 300, 256) == _ws_expected_gqa(1, 4, 2, 300, 256)
     assert fwd(lib, d=256) == api.FA_ERR_UNSUPPORTED  # fa_fwd: no workspace, no d = 256 kernel
